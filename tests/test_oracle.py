@@ -1,0 +1,246 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+- E4M3 decoding: all 256 codes against torch.float8_e4m3fn.
+- Router: numpy float64 matmul.
+- Top-k: brute-force enumeration of all K-subsets, and Python's sort for ties.
+- Mixture weights: exact sigmoid values and the unbiased-logit rule under a
+  bias that forces the selection.
+- Permutation: Python's stable sort of (expert, token) pairs.
+- Expert FFN and combine: a hand-computed d = I = 1 layer, numpy float64 SwiGLU
+  on a non-square expert, and the closed forms (x = 0, zero routed down
+  projection, identical experts).
+- FP8 block scales: the E4M3 layer equals the FP32 layer on the decoded weights.
+- Shapes: the weight counts printed on the pages.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fine_grained_sparse_fp32_b200.inputs import CONFIGS, LayerConfig, make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _sig(z):
+    return 1.0 / (1.0 + math.exp(-z))
+
+
+def test_e4m3_all_codes_match_torch():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(256):
+        got = oracle.e4m3_to_double(c)
+        if np.isnan(ref[c]):
+            assert np.isnan(got), c
+        else:
+            assert got == ref[c], (c, got, ref[c])
+    assert oracle.e4m3_to_double(0x7E) == 448.0
+    assert oracle.e4m3_to_double(0x01) == 2.0 ** -9
+
+
+def test_router_matches_numpy_float64():
+    inp = make_inputs(CONFIGS["tiny"], seed=0)
+    l = oracle.router_logits(inp["x"], "f32", inp["w_router"], nthreads=2)
+    ref = inp["x"].double().numpy() @ inp["w_router"].double().numpy().T
+    np.testing.assert_allclose(l, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_router_bf16_input_widened_exactly():
+    cfg = LayerConfig("t", 4, 256, 16, 6, 128, "bf16", "bf16")
+    inp = make_inputs(cfg, seed=3)
+    l = oracle.router_logits(inp["x"], "bf16", inp["w_router"])
+    ref = inp["x"].double().numpy() @ inp["w_router"].double().numpy().T
+    np.testing.assert_allclose(l, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_topk_matches_bruteforce_subsets():
+    rng = np.random.default_rng(1)
+    E, K, N = 10, 6, 200
+    logits = rng.normal(size=(N, E))
+    bias = rng.uniform(-0.5, 0.5, size=E).astype(np.float32)
+    idx, g, margin = oracle.select(logits, bias, K)
+    s = logits + bias.astype(np.float64)
+    for t in range(N):
+        best = max(itertools.combinations(range(E), K), key=lambda c: sum(s[t, list(c)]))
+        assert set(idx[t]) == set(best)
+        assert all(s[t, idx[t, k]] >= s[t, idx[t, k + 1]] for k in range(K - 1))
+        rest = sorted(set(range(E)) - set(best), key=lambda e: -s[t, e])
+        assert margin[t] == pytest.approx(s[t, idx[t, K - 1]] - s[t, rest[0]], abs=1e-15)
+        for k in range(K):
+            assert g[t, k] == pytest.approx(_sig(logits[t, idx[t, k]]), rel=1e-15)
+
+
+def test_topk_ties_go_to_lower_index():
+    E, K = 12, 6
+    rng = np.random.default_rng(2)
+    for _ in range(50):
+        logits = rng.integers(-2, 3, size=(1, E)).astype(np.float64)  # many exact ties
+        bias = np.zeros(E, dtype=np.float32)
+        idx, _, margin = oracle.select(logits, bias, K)
+        order = sorted(range(E), key=lambda e: (-logits[0, e], e))
+        assert list(idx[0]) == order[:K]
+        assert margin[0] == logits[0, order[K - 1]] - logits[0, order[K]]
+
+
+def test_mixture_weights_use_unbiased_logits_without_renormalising():
+    E, K = 16, 6
+    logits = np.zeros((2, E))
+    logits[0, :] = -1.0
+    logits[0, [3, 5, 7, 9, 11, 13]] = [0.0, math.log(3.0), 0.0, math.log(3.0), 0.0, 0.0]
+    logits[1, :] = 2.0                       # best unbiased logits sit on 0..5 ...
+    logits[1, [3, 5, 7, 9, 11, 13]] = 0.0
+    bias = np.zeros(E, dtype=np.float32)
+    bias[[3, 5, 7, 9, 11, 13]] = 30.0       # ... but the bias forces these six
+    idx, g, _ = oracle.select(logits, bias, K)
+    for t in range(2):
+        assert sorted(idx[t]) == [3, 5, 7, 9, 11, 13]
+    # sigmoid(0) = 1/2 and sigmoid(ln 3) = 3/4, from the unbiased logits
+    assert sorted(g[0]) == pytest.approx([0.5, 0.5, 0.5, 0.5, 0.75, 0.75], abs=1e-15)
+    assert list(g[1]) == [0.5] * 6
+    assert abs(g[0].sum() - 1.0) > 1.0       # not renormalised to one
+
+
+def test_permute_matches_stable_sort():
+    rng = np.random.default_rng(4)
+    for N, K, E in [(128, 6, 64), (1, 6, 6), (57, 6, 384), (300, 2, 5)]:
+        idx = np.stack([rng.permutation(E)[:K] for _ in range(N)]).astype(np.int32)
+        counts, offsets, perm, inv = oracle.permute(idx, E)
+        pairs = sorted(((idx[t, k], t, k) for t in range(N) for k in range(K)), key=lambda p: (p[0], p[1]))
+        assert [p[1] for p in pairs] == list(perm)
+        for pos, (e, t, k) in enumerate(pairs):
+            assert inv[t, k] == pos
+        assert counts.sum() == N * K and offsets[0] == 0 and offsets[-1] == N * K
+        assert np.all(np.diff(offsets) == counts)
+        assert sorted(inv.ravel()) == list(range(N * K))          # bijection
+        assert np.all(perm[inv] == np.arange(N)[:, None])          # perm o inv_pos = id
+
+
+def test_permute_rejects_out_of_range():
+    with pytest.raises(ValueError):
+        oracle.permute(np.array([[0, 7]], dtype=np.int32), 4)
+
+
+def _one_by_one_layer():
+    cfg = LayerConfig("hand", 1, 1, 2, 1, 1, "f32", "f32")
+    inp = {
+        "cfg": cfg,
+        "x": torch.tensor([[2.0]]),
+        "w_router": torch.tensor([[0.5], [-0.25]]),
+        "bias": torch.tensor([0.0, 0.0]),
+        # experts 0, 1 routed; index 2 is the shared expert
+        "w_gate": torch.tensor([1.0, 2.0, 0.5]).reshape(3, 1, 1),
+        "w_up": torch.tensor([3.0, 1.0, -1.0]).reshape(3, 1, 1),
+        "w_down": torch.tensor([-1.5, 4.0, 2.0]).reshape(3, 1, 1),
+    }
+    return inp
+
+
+def test_hand_computed_one_by_one_layer():
+    # logits: 0.5*2 = 1 and -0.25*2 = -0.5, so expert 0 is chosen, g = sigmoid(1).
+    # expert 0: SiLU(1*2) * (3*2) = 2*sigmoid(2)*6 = 10.569564935734588; down: * -1.5
+    # shared:   SiLU(0.5*2) * (-1*2) = -1.4621171572600098;         down: * 2
+    # y = -2.9242343145200196 + 0.7310585786300049 * -15.854347403601881
+    out = oracle.layer(_one_by_one_layer())
+    assert list(out["idx"][0]) == [0]
+    assert out["g"][0, 0] == pytest.approx(0.7310585786300049, abs=1e-15)
+    assert out["y"][0, 0] == pytest.approx(-14.51469099250352, abs=1e-13)
+
+
+def test_expert_ffn_matches_numpy_swiglu_non_square():
+    cfg = CONFIGS["tiny"]
+    inp = make_inputs(cfg, seed=5)
+    toks = np.array([0, 17, 127], dtype=np.int32)
+    exps = np.array([3, cfg.E, 63], dtype=np.int32)
+    got = oracle.expert_outputs(inp, toks, exps)
+    x = inp["x"].double().numpy()
+    for p, (t, e) in enumerate(zip(toks, exps)):
+        wg = inp["w_gate"][e].double().numpy()     # [I, d]
+        wu = inp["w_up"][e].double().numpy()       # [I, d]
+        wd = inp["w_down"][e].double().numpy()     # [d, I]
+        a, b = wg @ x[t], wu @ x[t]
+        h = a / (1.0 + np.exp(-a)) * b
+        np.testing.assert_allclose(got[p], wd @ h, rtol=1e-10, atol=1e-13)
+
+
+def test_zero_input_gives_zero_output():
+    inp = make_inputs(CONFIGS["tiny"], seed=6)
+    inp["x"] = torch.zeros_like(inp["x"])
+    out = oracle.layer(inp, rows=np.arange(8))
+    assert np.all(out["y"] == 0.0)
+
+
+def test_zero_routed_down_projection_leaves_shared_expert():
+    cfg = CONFIGS["tiny"]
+    inp = make_inputs(cfg, seed=7)
+    inp["w_down"][: cfg.E].zero_()
+    rows = np.arange(0, cfg.N, 9, dtype=np.int32)
+    out = oracle.layer(inp, rows=rows)
+    shared = oracle.expert_outputs(inp, rows, np.full(len(rows), cfg.E))
+    np.testing.assert_array_equal(out["y"], shared)
+
+
+def test_identical_experts_closed_form():
+    # every expert (routed and shared) is the same F: y = (1 + sum_k g_k) F(x)
+    cfg = CONFIGS["tiny"]
+    inp = make_inputs(cfg, seed=8)
+    for name in ("w_gate", "w_up", "w_down"):
+        inp[name][:] = inp[name][cfg.E].clone()
+    rows = np.arange(0, cfg.N, 5, dtype=np.int32)
+    out = oracle.layer(inp, rows=rows)
+    f = oracle.expert_outputs(inp, rows, np.full(len(rows), cfg.E))
+    scale = 1.0 + out["g"].sum(axis=1)
+    np.testing.assert_allclose(out["y"], scale[:, None] * f, rtol=1e-12, atol=1e-15)
+    assert np.all(out["g"] > 0) and np.all(out["g"] < 1)
+
+
+def test_bias_forcing_selects_the_same_six_everywhere():
+    cfg = CONFIGS["tiny"]
+    inp = make_inputs(cfg, seed=9)
+    forced = [2, 11, 19, 30, 41, 60]
+    inp["bias"][forced] = 30.0
+    l = oracle.router_logits(inp["x"], "f32", inp["w_router"])
+    idx, g, _ = oracle.select(l, inp["bias"], cfg.K)
+    for t in range(cfg.N):
+        assert sorted(idx[t]) == forced
+        np.testing.assert_allclose(g[t], 1.0 / (1.0 + np.exp(-l[t, idx[t]])), rtol=1e-15)
+
+
+def test_fp8_layer_equals_f32_layer_on_decoded_weights():
+    cfg = LayerConfig("q", 16, 256, 8, 6, 128, "f32", "e4m3")
+    q = make_inputs(cfg, seed=10)
+    f = dict(q)
+    f["cfg"] = LayerConfig("f", 16, 256, 8, 6, 128, "f32", "f32")
+    for w, s in (("w_gate", "s_gate"), ("w_up", "s_up"), ("w_down", "s_down")):
+        vals = q[w].view(torch.float8_e4m3fn).to(torch.float64)          # [G, R, C]
+        sc = q[s].double().repeat_interleave(128, 1).repeat_interleave(128, 2)
+        f[w] = (vals * sc).to(torch.float32)
+    a = oracle.layer(q)["y"]
+    b = oracle.layer(f)["y"]
+    np.testing.assert_allclose(a, b, rtol=1e-6, atol=1e-6 * np.abs(b).max())
+    # and the scales really vary from block to block
+    assert q["s_gate"].std() > 0
+
+
+def _golden_counts():
+    vals = {}
+    with open(os.path.join(GOLDEN, "kolibri_shape_counts.txt")) as fh:
+        for line in fh:
+            if line.strip() and not line.startswith("#"):
+                name, value, _ = line.split()
+                vals[name] = float(value)
+    return vals
+
+
+def test_layer_shape_matches_printed_weight_counts():
+    g = _golden_counts()
+    cfg = CONFIGS["decode"]
+    assert cfg.expert_weights == g["weights_per_expert"]
+    assert cfg.E == g["routed_experts"] and cfg.K == g["top_k"]
+    assert cfg.E + 1 == g["experts_total_per_block"]
+    assert round((cfg.K + 1) * cfg.expert_weights / 1e5) / 10 == g["touched_per_token_per_block"] / 1e6
+    assert round((cfg.E + 1) * cfg.expert_weights / 1e7) / 100 == g["all_experts_per_block"] / 1e9
