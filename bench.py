@@ -1,0 +1,372 @@
+"""Benchmark of the fine-grained MoE layer on B200.
+
+One step = one whole-layer call (moe_forward: router + top-6, dispatch,
+grouped SwiGLU experts + shared expert, combine) over one batch of N tokens
+whose inputs already sit in HBM. The headline workload is the Kolibri-shaped
+decode layer (N = 32, d = 2560, E = 384, top-6 + 1 shared, I = 512, BF16
+expert weights, FP32 router); the prefill layer (N = 8192) is reported in the
+same line under "prefill".
+
+Launch: python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+With N > 1 (torchrun), every rank runs an independent replica on its own
+tokens: tokens are independent, so the layer shards with no collective
+(weak scaling); rank 0 prints the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fine_grained_sparse_fp32_b200 import _build, kmoe  # noqa: E402
+from fine_grained_sparse_fp32_b200.inputs import CONFIGS, make_inputs, make_x  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at 1 B200 (decode N=32, prefill N=8192); % of HBM/tensor roofline"
+ROTATE = 8           # distinct token batches cycled through the timed steps
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def bytes_per_weight(cfg):
+    return {"f32": 4, "bf16": 2, "e4m3": 1}[cfg.w_dtype]
+
+
+def algorithmic(cfg, distinct_routed: float):
+    """Algorithmic bytes and FLOPs of one layer call (intermediates excluded)."""
+    per_expert = cfg.expert_weights * bytes_per_weight(cfg)
+    if cfg.w_dtype == "e4m3":
+        per_expert += 3 * (cfg.d // 128) * (cfg.I // 128) * 4
+    xb = 4 if cfg.x_dtype == "f32" else 2
+    weights = (distinct_routed + 1) * per_expert
+    act = cfg.N * cfg.d * xb + cfg.N * cfg.d * 2
+    router = cfg.E * cfg.d * 4 + cfg.E * 4
+    flops = 2 * cfg.N * cfg.d * cfg.E + 2 * cfg.N * (cfg.K + 1) * 3 * cfg.d * cfg.I
+    ffn_bytes = weights + cfg.N * cfg.d * xb + (cfg.N * cfg.K + cfg.N) * cfg.d * 2
+    return {"layer_bytes": weights + act + router, "ffn_bytes": ffn_bytes, "flops": flops,
+            "expert_weight_bytes": weights}
+
+
+def launches_per_step(cfg):
+    # router_logits, topk, permute (1 kernel for N <= 256, else 3), ffn_up, ffn_down, combine
+    return 2 + (1 if cfg.N <= 256 else 3) + 2 + 1
+
+
+# --------------------------------------------------------------- GPU arm
+def run_config(cfg, steps, warmup, rank, world, seed=0, use_graph=True):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    layer = make_inputs(cfg, seed=seed, device=dev)
+    lay = kmoe.Layer(layer, cfg.N)
+    xs = [make_x(cfg, seed=1000 * rank + 17 * i + 1, device=dev) for i in range(ROTATE)]
+    ys = [torch.empty((cfg.N, cfg.d), dtype=torch.bfloat16, device=dev) for _ in range(ROTATE)]
+    counts = [torch.empty(cfg.E, dtype=torch.int32, device=dev) for _ in range(ROTATE)]
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(ROTATE):
+            lay.forward(xs[i], y=ys[i], counts=counts[i], stream=stream)
+    stream.synchronize()
+    distinct = float(np.mean([(c > 0).sum().item() for c in counts]))
+
+    graphs = []
+    if use_graph:
+        for i in range(ROTATE):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                lay.forward(xs[i], y=ys[i], counts=counts[i], stream=stream)
+            graphs.append(g)
+
+    def step(i):
+        if use_graph:
+            graphs[i % ROTATE].replay()
+        else:
+            lay.forward(xs[i % ROTATE], y=ys[i % ROTATE], counts=counts[i % ROTATE], stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    time.sleep(0.3 if clocks else 0)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(steps):
+            step(i)
+        t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    clk = clocks.stop() if clocks else None
+    ms_max = all_max(ms, world)
+
+    # per-kernel-group timing of the dominant step (grouped FFN), decomposed calls
+    ffn_ms = time_grouped_ffn(layer, xs, stream, steps=max(20, min(steps, 400)))
+
+    # end to end: pinned host x -> device, layer, device y -> pinned host
+    e2e_ms = time_e2e(lay, cfg, xs, stream, steps=max(20, min(steps, 400)), warmup=max(3, warmup // 4))
+    alg = algorithmic(cfg, distinct)
+    return {"ms_per_step": ms_max / steps, "clocks": clk, "distinct": distinct, "alg": alg,
+            "ffn_ms": ffn_ms, "e2e_ms": e2e_ms}
+
+
+def time_grouped_ffn(layer, xs, stream, steps):
+    """Average duration of one moe_grouped_ffn call (the expert FFN kernels)."""
+    cfg = layer["cfg"]
+    dev = xs[0].device
+    preps = []
+    with torch.cuda.stream(stream):
+        for x in xs:
+            idx, w = kmoe.moe_router_topk(x, layer["w_router"], layer["bias"], cfg.K, stream=stream)
+            _, offsets, perm, _ = kmoe.moe_permute(idx, cfg.E, stream=stream)
+            preps.append((x, perm, offsets))
+    ws = torch.empty(((cfg.N * cfg.K + cfg.N) * cfg.I * 4), dtype=torch.uint8, device=dev)
+    outs = [kmoe.moe_grouped_ffn(x, layer, p, o, ws=ws, stream=stream) for x, p, o in preps]
+    stream.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            x, p, o = preps[i % len(preps)]
+            ev[i][0].record(stream)
+            kmoe.moe_grouped_ffn(x, layer, p, o, ws=ws, stream=stream)
+            ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    del outs
+    return float(np.mean([a.elapsed_time(b) for a, b in ev]))
+
+
+def time_e2e(lay, cfg, xs, stream, steps, warmup):
+    xb = 4 if cfg.x_dtype == "f32" else 2
+    hx = [x.cpu().pin_memory() for x in xs]
+    hy = torch.empty((cfg.N, cfg.d), dtype=torch.bfloat16).pin_memory()
+    dx = torch.empty_like(xs[0])
+    dy = torch.empty((cfg.N, cfg.d), dtype=torch.bfloat16, device=xs[0].device)
+
+    def one(i):
+        dx.copy_(hx[i % len(hx)], non_blocking=True)
+        lay.forward(dx, y=dy, stream=stream)
+        hy.copy_(dy, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            one(i)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(steps):
+            one(i)
+        t1.record(stream)
+    torch.cuda.synchronize()
+    return {"ms": t0.elapsed_time(t1) / steps, "h2d": cfg.N * cfg.d * xb, "d2h": cfg.N * cfg.d * 2}
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def all_max(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- CPU oracle
+def cpu_baseline(cfg, n_tokens, seed=0, layer_host=None):
+    """The oracle, as it stands, on a bounded token sample of the workload."""
+    import oracle
+    from fine_grained_sparse_fp32_b200.inputs import to_host
+    if layer_host is None:
+        layer_host = to_host(make_inputs(cfg, seed=seed, device="cpu" if not torch.cuda.is_available() else "cuda"))
+    rows = np.arange(min(n_tokens, cfg.N), dtype=np.int32)
+    nt = oracle.max_threads()
+    t = time.perf_counter()
+    oracle.layer(layer_host, rows=rows, nthreads=nt)
+    dt = time.perf_counter() - t
+    return {"value": len(rows) / dt, "unit": "tokens/s", "cores": nt, "kind": "oracle",
+            "sample": f"{len(rows)} of the {cfg.N} tokens of the {cfg.name} layer, whole layer in double"}
+
+
+# ------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="kmoe", choices=["kmoe", "reference"])
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=32)
+    args = ap.parse_args()
+    world, rank, local = dist_env()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    _build.build()
+    kmoe.load()
+
+    hbm, tflops, tflops_sus, peak_kind = peaks()
+    dec = CONFIGS["decode"]
+    r = run_config(dec, args.steps, args.warmup, rank, world, use_graph=not args.no_graph)
+    pre = None
+    if not args.no_prefill:
+        pcfg = CONFIGS["prefill"]
+        psteps = max(10, min(args.steps // 10, 200))
+        pre = run_config(pcfg, psteps, max(3, args.warmup // 10), rank, world, use_graph=not args.no_graph)
+
+    if rank == 0:
+        ms = r["ms_per_step"]
+        value = dec.N * world / (ms / 1e3)
+        alg = r["alg"]
+        ffn_gbs = alg["ffn_bytes"] / (r["ffn_ms"] / 1e3) / 1e9
+        layer_gbs = alg["layer_bytes"] / (ms / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "decode layer N=32 d=2560 E=384 top-6+1 shared I=512, BF16 experts, FP32 router",
+                       "tokens_per_gpu": dec.N, "parallelism": f"replicas x{world} (no collective)",
+                       "l2": "inputs larger than L2: ~%.2f GB of expert weights per step, %d rotating token batches"
+                             % (alg["expert_weight_bytes"] / 1e9, ROTATE),
+                       "cuda_graph": not args.no_graph},
+            "roofline": {"bound": "hbm", "kernel": "moe_grouped_ffn (ffn_up + ffn_down)",
+                         "achieved": ffn_gbs, "peak": hbm, "unit": "GB/s", "frac": ffn_gbs / hbm,
+                         "traffic": None, "peak_kind": peak_kind + " burst",
+                         "layer_achieved": layer_gbs, "layer_frac": layer_gbs / hbm,
+                         "algorithmic_bytes_per_launch": alg["ffn_bytes"], "launch_ms": r["ffn_ms"]},
+            "e2e": {"value": dec.N * world / (r["e2e_ms"]["ms"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["e2e_ms"]["h2d"], "d2h_bytes_per_step": r["e2e_ms"]["d2h"]},
+            "gpu_launches": launches_per_step(dec) * args.steps,
+            "clocks": r["clocks"],
+            "distinct_experts_per_step": r["distinct"],
+        }
+        if pre is not None:
+            pcfg = CONFIGS["prefill"]
+            pms = pre["ms_per_step"]
+            palg = pre["alg"]
+            t_hbm = palg["layer_bytes"] / (hbm * 1e9)
+            t_tc = palg["flops"] / (tflops * 1e12)
+            line["prefill"] = {
+                "value": pcfg.N * world / (pms / 1e3), "unit": "tokens/s", "ms_per_step": pms,
+                "roofline_time_ms": max(t_hbm, t_tc) * 1e3, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                "frac": max(t_hbm, t_tc) * 1e3 / pms,
+                "tflops": palg["flops"] / (pms / 1e3) / 1e12, "tensor_frac": palg["flops"] / (pms / 1e3) / (tflops * 1e12),
+                "ffn_ms": pre["ffn_ms"], "clocks": pre["clocks"],
+                "e2e": {"value": pcfg.N * world / (pre["e2e_ms"]["ms"] / 1e3), "unit": "tokens/s"},
+            }
+        if world == 1:
+            try:
+                line["cpu_baseline"] = cpu_baseline(dec, args.cpu_tokens)
+            except Exception as exc:  # the baseline must never hide the GPU number
+                line["cpu_baseline"] = {"value": None, "error": str(exc)[:200]}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args, world, rank):
+    """The oracle on the host cores, on this arm's metric and workload."""
+    if rank != 0:
+        return
+    import oracle
+    from fine_grained_sparse_fp32_b200.inputs import to_host
+    cfg = CONFIGS["decode"]
+    host = to_host(make_inputs(cfg, seed=0, device="cuda" if torch.cuda.is_available() else "cpu"))
+    sample = args.cpu_tokens if args.cpu_tokens else 4
+    sample = max(1, min(sample, 8))
+    rows = np.arange(sample, dtype=np.int32)
+    nt = oracle.max_threads()
+    for _ in range(min(args.warmup, 1)):
+        oracle.layer(host, rows=rows, nthreads=nt)
+    times = []
+    for _ in range(args.steps if args.steps <= 20 else 20):
+        t = time.perf_counter()
+        oracle.layer(host, rows=rows, nthreads=nt)
+        times.append(time.perf_counter() - t)
+    per_token = float(np.mean(times)) / sample
+    value = 1.0 / per_token
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": len(times), "warmup": args.warmup, "ms_per_step": per_token * cfg.N * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "decode layer N=32 d=2560 E=384 top-6+1 shared I=512, BF16 experts, FP32 router"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nt, "kind": "oracle",
+                             "sample": f"{sample} of the {cfg.N} decode tokens per step, whole layer in double"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

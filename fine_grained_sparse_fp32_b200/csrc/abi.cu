@@ -1,0 +1,287 @@
+// C ABI of the kmoe library: argument checks, workspace layout, dispatch to
+// the kernels, and the whole-layer forward.
+#include "common.cuh"
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+namespace kmoe {
+
+static thread_local char g_err[512] = "";
+
+kmoe_status fail(kmoe_status code, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+void clear_error() { g_err[0] = '\0'; }
+
+kmoe_status check_launch(const char *what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(KMOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return KMOE_OK;
+}
+
+// ------------------------------------------------------------ validation
+
+static kmoe_status check_sizes(int N, int d, int E, int K, int I)
+{
+    if (N < 0) return fail(KMOE_ERR_INVALID_ARG, "N=%d must be >= 0", N);
+    if (K < 1 || K > 8) return fail(KMOE_ERR_UNSUPPORTED, "K=%d: supported 1 <= K <= 8", K);
+    if (E < K) return fail(KMOE_ERR_INVALID_ARG, "E=%d must be >= K=%d", E, K);
+    if (E > 1024) return fail(KMOE_ERR_UNSUPPORTED, "E=%d: supported E <= 1024", E);
+    if (d < 128 || d % 128 || d > 6144)
+        return fail(KMOE_ERR_UNSUPPORTED, "d=%d: must be a multiple of 128 in [128, 6144]", d);
+    if (I >= 0 && (I < 128 || I % 128 || I > 4096))
+        return fail(KMOE_ERR_UNSUPPORTED, "I=%d: must be a multiple of 128 in [128, 4096]", I);
+    if ((long long)N * K > (1LL << 30)) return fail(KMOE_ERR_UNSUPPORTED, "N*K too large");
+    return KMOE_OK;
+}
+
+static kmoe_status check_ptr(const void *p, const char *name, bool nullable = false)
+{
+    if (!p) return nullable ? KMOE_OK : fail(KMOE_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned16(p)) return fail(KMOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return KMOE_OK;
+}
+
+#define KMOE_TRY(expr)                          \
+    do {                                        \
+        kmoe_status s_ = (expr);                \
+        if (s_ != KMOE_OK) return s_;           \
+    } while (0)
+
+static kmoe_status check_act_dtype(int t, const char *name)
+{
+    if (t != KMOE_F32 && t != KMOE_BF16) return fail(KMOE_ERR_UNSUPPORTED, "%s dtype %d: F32 or BF16 only", name, t);
+    return KMOE_OK;
+}
+
+static kmoe_status check_experts(const kmoe_experts *x, const char *name)
+{
+    if (!x) return fail(KMOE_ERR_INVALID_ARG, "%s is NULL", name);
+    if (x->dtype != KMOE_F32 && x->dtype != KMOE_BF16 && x->dtype != KMOE_E4M3_B128)
+        return fail(KMOE_ERR_UNSUPPORTED, "%s dtype %d unknown", name, x->dtype);
+    KMOE_TRY(check_ptr(x->w_gate, "w_gate"));
+    KMOE_TRY(check_ptr(x->w_up, "w_up"));
+    KMOE_TRY(check_ptr(x->w_down, "w_down"));
+    if (x->dtype == KMOE_E4M3_B128) {
+        KMOE_TRY(check_ptr(x->s_gate, "s_gate"));
+        KMOE_TRY(check_ptr(x->s_up, "s_up"));
+        KMOE_TRY(check_ptr(x->s_down, "s_down"));
+    }
+    return KMOE_OK;
+}
+
+static ExpertPtrs ptrs(const kmoe_experts *x)
+{
+    ExpertPtrs p{x->w_gate, x->w_up, x->w_down, nullptr, nullptr, nullptr};
+    if (x->dtype == KMOE_E4M3_B128) {
+        p.sg = x->s_gate;
+        p.su = x->s_up;
+        p.sd = x->s_down;
+    }
+    return p;
+}
+
+static size_t act_bytes(int w_dtype) { return w_dtype == KMOE_F32 ? 4 : 2; }
+
+// Workspace of the whole forward; every entry point uses a prefix-compatible
+// subset (router: logits; permute: chunk histograms; grouped FFN: H).
+struct Layout {
+    float *logits;
+    int32_t *idx;
+    float *w;
+    int32_t *counts, *offsets, *perm, *inv, *hist;
+    void *h, *y_perm, *y_shared;
+    size_t bytes;
+};
+
+static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype)
+{
+    Carver c(ws);
+    Layout L;
+    const size_t R = (size_t)N * K + N;
+    const size_t ab = act_bytes(w_dtype);
+    L.logits = c.take<float>((size_t)N * E);
+    L.idx = c.take<int32_t>((size_t)N * K);
+    L.w = c.take<float>((size_t)N * K);
+    L.counts = c.take<int32_t>(E);
+    L.offsets = c.take<int32_t>(E + 1);
+    L.perm = c.take<int32_t>((size_t)N * K);
+    L.inv = c.take<int32_t>((size_t)N * K);
+    L.hist = reinterpret_cast<int32_t *>(c.take<char>(permute_ws_bytes(N, E)));
+    L.h = c.take<char>(R * I * ab);
+    L.y_perm = c.take<char>((size_t)N * K * d * ab);
+    L.y_shared = c.take<char>((size_t)N * d * ab);
+    L.bytes = c.used + 256;
+    return L;
+}
+
+}  // namespace kmoe
+
+using namespace kmoe;
+
+extern "C" {
+
+int moe_abi_version(void) { return KMOE_ABI_VERSION; }
+
+const char *moe_last_error(void) { return g_err; }
+
+size_t moe_workspace_size(int N, int d, int E, int K, int I, int x_dtype, int w_dtype)
+{
+    if (check_sizes(N, d, E, K, I) != KMOE_OK) return 0;
+    if (check_act_dtype(x_dtype, "x") != KMOE_OK) return 0;
+    if (w_dtype != KMOE_F32 && w_dtype != KMOE_BF16 && w_dtype != KMOE_E4M3_B128) return 0;
+    clear_error();
+    return layout(nullptr, N, d, E, K, I, w_dtype).bytes;
+}
+
+kmoe_status moe_router_topk(const void *x, int x_dtype, const float *w_router, const float *bias,
+                            int N, int d, int E, int K, float *logits, int32_t *topk_idx,
+                            float *topk_w, void *ws, size_t ws_bytes, void *stream)
+{
+    clear_error();
+    KMOE_TRY(check_sizes(N, d, E, K, -1));
+    KMOE_TRY(check_act_dtype(x_dtype, "x"));
+    if (N == 0) return KMOE_OK;
+    KMOE_TRY(check_ptr(x, "x"));
+    KMOE_TRY(check_ptr(w_router, "w_router"));
+    KMOE_TRY(check_ptr(bias, "bias"));
+    KMOE_TRY(check_ptr(topk_idx, "topk_idx"));
+    KMOE_TRY(check_ptr(topk_w, "topk_w"));
+    KMOE_TRY(check_ptr(logits, "logits", true));
+    if (!logits) {
+        KMOE_TRY(check_ptr(ws, "ws"));
+        if (ws_bytes < (size_t)N * E * sizeof(float))
+            return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, (size_t)N * E * sizeof(float));
+        logits = static_cast<float *>(ws);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, logits, st));
+    return launch_topk(logits, bias, N, E, K, topk_idx, topk_w, st);
+}
+
+kmoe_status moe_permute(const int32_t *topk_idx, int N, int K, int E, int32_t *counts,
+                        int32_t *offsets, int32_t *perm_token, int32_t *inv_pos, void *ws,
+                        size_t ws_bytes, void *stream)
+{
+    clear_error();
+    KMOE_TRY(check_sizes(N, 128, E, K, -1));
+    KMOE_TRY(check_ptr(counts, "counts"));
+    KMOE_TRY(check_ptr(offsets, "offsets"));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st) != cudaSuccess ||
+            cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st) != cudaSuccess)
+            return check_launch("permute memset");
+        return KMOE_OK;
+    }
+    KMOE_TRY(check_ptr(topk_idx, "topk_idx"));
+    KMOE_TRY(check_ptr(perm_token, "perm_token"));
+    KMOE_TRY(check_ptr(inv_pos, "inv_pos"));
+    const size_t need = permute_ws_bytes(N, E);
+    if (N > 256) {
+        KMOE_TRY(check_ptr(ws, "ws"));
+        if (ws_bytes < need) return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+    }
+    return launch_permute(topk_idx, N, K, E, counts, offsets, perm_token, inv_pos,
+                          static_cast<int32_t *>(ws), st);
+}
+
+kmoe_status moe_grouped_ffn(const void *x, int x_dtype, int N, int d, int I, int E, int K,
+                            const int32_t *perm_token, const int32_t *offsets,
+                            const kmoe_experts *routed, const kmoe_experts *shared, void *y_perm,
+                            void *y_shared, void *ws, size_t ws_bytes, void *stream)
+{
+    clear_error();
+    KMOE_TRY(check_sizes(N, d, E, K, I));
+    KMOE_TRY(check_act_dtype(x_dtype, "x"));
+    KMOE_TRY(check_experts(routed, "routed"));
+    if (shared) {
+        KMOE_TRY(check_experts(shared, "shared"));
+        if (shared->dtype != routed->dtype) return fail(KMOE_ERR_UNSUPPORTED, "shared and routed dtypes differ");
+    }
+    if (N == 0) return KMOE_OK;
+    KMOE_TRY(check_ptr(x, "x"));
+    KMOE_TRY(check_ptr(perm_token, "perm_token"));
+    KMOE_TRY(check_ptr(offsets, "offsets"));
+    KMOE_TRY(check_ptr(y_perm, "y_perm"));
+    if (shared) KMOE_TRY(check_ptr(y_shared, "y_shared"));
+    KMOE_TRY(check_ptr(ws, "ws"));
+    const size_t need = ((size_t)N * K + N) * I * act_bytes(routed->dtype);
+    if (ws_bytes < need) return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+    const ExpertPtrs r = ptrs(routed);
+    ExpertPtrs s{};
+    if (shared) s = ptrs(shared);
+    return launch_ffn_stream(x, x_dtype, N, d, I, E, K, perm_token, offsets, routed->dtype, r,
+                             shared ? &s : nullptr, ws, y_perm, y_shared, static_cast<cudaStream_t>(stream));
+}
+
+kmoe_status moe_combine(const void *y_perm, const void *y_shared, int y_in_dtype, const float *topk_w,
+                        const int32_t *inv_pos, int N, int K, int d, void *y, int y_dtype, void *stream)
+{
+    clear_error();
+    KMOE_TRY(check_sizes(N, d, K, K, -1));
+    KMOE_TRY(check_act_dtype(y_in_dtype, "y_in"));
+    KMOE_TRY(check_act_dtype(y_dtype, "y"));
+    if (N == 0) return KMOE_OK;
+    KMOE_TRY(check_ptr(y_perm, "y_perm"));
+    KMOE_TRY(check_ptr(y_shared, "y_shared", true));
+    KMOE_TRY(check_ptr(topk_w, "topk_w"));
+    KMOE_TRY(check_ptr(inv_pos, "inv_pos"));
+    KMOE_TRY(check_ptr(y, "y"));
+    return launch_combine(y_perm, y_shared, y_in_dtype, topk_w, inv_pos, N, K, d, y, y_dtype,
+                          static_cast<cudaStream_t>(stream));
+}
+
+kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, int I,
+                        const float *w_router, const float *bias, const kmoe_experts *routed,
+                        const kmoe_experts *shared, void *y, int y_dtype, int32_t *topk_idx_out,
+                        float *topk_w_out, int32_t *counts_out, void *ws, size_t ws_bytes, void *stream)
+{
+    clear_error();
+    KMOE_TRY(check_sizes(N, d, E, K, I));
+    KMOE_TRY(check_act_dtype(x_dtype, "x"));
+    KMOE_TRY(check_act_dtype(y_dtype, "y"));
+    KMOE_TRY(check_experts(routed, "routed"));
+    if (shared) {
+        KMOE_TRY(check_experts(shared, "shared"));
+        if (shared->dtype != routed->dtype) return fail(KMOE_ERR_UNSUPPORTED, "shared and routed dtypes differ");
+    }
+    if (N == 0) return KMOE_OK;
+    KMOE_TRY(check_ptr(x, "x"));
+    KMOE_TRY(check_ptr(w_router, "w_router"));
+    KMOE_TRY(check_ptr(bias, "bias"));
+    KMOE_TRY(check_ptr(y, "y"));
+    KMOE_TRY(check_ptr(topk_idx_out, "topk_idx_out", true));
+    KMOE_TRY(check_ptr(topk_w_out, "topk_w_out", true));
+    KMOE_TRY(check_ptr(counts_out, "counts_out", true));
+    KMOE_TRY(check_ptr(ws, "ws"));
+    const Layout need = layout(nullptr, N, d, E, K, I, routed->dtype);
+    if (ws_bytes < need.bytes) return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need.bytes);
+    // the base the Carver sees is 256-aligned by construction of the pieces
+    const Layout L = layout(ws, N, d, E, K, I, routed->dtype);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t *idx = topk_idx_out ? topk_idx_out : L.idx;
+    float *w = topk_w_out ? topk_w_out : L.w;
+    int32_t *counts = counts_out ? counts_out : L.counts;
+    KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, L.logits, st));
+    KMOE_TRY(launch_topk(L.logits, bias, N, E, K, idx, w, st));
+    KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st));
+    const ExpertPtrs r = ptrs(routed);
+    ExpertPtrs s{};
+    if (shared) s = ptrs(shared);
+    KMOE_TRY(launch_ffn_stream(x, x_dtype, N, d, I, E, K, L.perm, L.offsets, routed->dtype, r,
+                               shared ? &s : nullptr, L.h, L.y_perm, L.y_shared, st));
+    const int yin = routed->dtype == KMOE_F32 ? KMOE_F32 : KMOE_BF16;
+    return launch_combine(L.y_perm, shared ? L.y_shared : nullptr, yin, w, L.inv, N, K, d, y, y_dtype, st);
+}
+
+}  // extern "C"

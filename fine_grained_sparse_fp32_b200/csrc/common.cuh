@@ -1,0 +1,134 @@
+// Shared device helpers and host-side plumbing of the kmoe library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cstdint>
+#include <cstddef>
+
+#include "kmoe.h"
+
+namespace kmoe {
+
+// ---------------------------------------------------------------- host side
+
+// Records a printf-style message as the calling thread's last error and
+// returns `code`, so that call sites can write `return fail(...)`.
+kmoe_status fail(kmoe_status code, const char *fmt, ...);
+void clear_error();
+
+// Checks the last launch; on failure records the CUDA error string.
+kmoe_status check_launch(const char *what);
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Carves 256-byte aligned pieces out of a caller-provided workspace.
+struct Carver {
+    char *base;
+    size_t used = 0;
+    explicit Carver(void *b) : base(static_cast<char *>(b)) {}
+    template <class T>
+    T *take(size_t count) {
+        used = (used + 255) & ~size_t(255);
+        T *p = base ? reinterpret_cast<T *>(base + used) : nullptr;
+        used += count * sizeof(T);
+        return p;
+    }
+};
+
+// Weight pointers of one expert stack, as seen by the kernels.
+struct ExpertPtrs {
+    const void *wg, *wu, *wd;
+    const float *sg, *su, *sd;
+};
+
+// ----------------------------------------------------------- device helpers
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// 16 bytes of weights -> VEC floats, for the three storage types.
+template <class WT> struct WVec;
+
+template <> struct WVec<float> {
+    static constexpr int VEC = 4;
+    __device__ __forceinline__ static void cvt(uint4 r, float *o, float) {
+        o[0] = __uint_as_float(r.x); o[1] = __uint_as_float(r.y);
+        o[2] = __uint_as_float(r.z); o[3] = __uint_as_float(r.w);
+    }
+};
+
+template <> struct WVec<__nv_bfloat16> {
+    static constexpr int VEC = 8;
+    __device__ __forceinline__ static void cvt(uint4 r, float *o, float) {
+        o[0] = bf16_lo(r.x); o[1] = bf16_hi(r.x); o[2] = bf16_lo(r.y); o[3] = bf16_hi(r.y);
+        o[4] = bf16_lo(r.z); o[5] = bf16_hi(r.z); o[6] = bf16_lo(r.w); o[7] = bf16_hi(r.w);
+    }
+};
+
+template <> struct WVec<__nv_fp8_e4m3> {
+    static constexpr int VEC = 16;
+    __device__ __forceinline__ static void cvt2(uint32_t v, float *o, float s) {
+        __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v & 0xffffu), __NV_E4M3);
+        __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v >> 16), __NV_E4M3);
+        float2 a = __half22float2(*reinterpret_cast<__half2 *>(&lo));
+        float2 b = __half22float2(*reinterpret_cast<__half2 *>(&hi));
+        o[0] = a.x * s; o[1] = a.y * s; o[2] = b.x * s; o[3] = b.y * s;
+    }
+    __device__ __forceinline__ static void cvt(uint4 r, float *o, float s) {
+        cvt2(r.x, o, s); cvt2(r.y, o + 4, s); cvt2(r.z, o + 8, s); cvt2(r.w, o + 12, s);
+    }
+};
+
+// Activations: 8 consecutive values -> floats.
+__device__ __forceinline__ void load8(const float *p, float *o) {
+    float4 a = *reinterpret_cast<const float4 *>(p);
+    float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float *o) {
+    uint4 r = *reinterpret_cast<const uint4 *>(p);
+    WVec<__nv_bfloat16>::cvt(r, o, 1.f);
+}
+
+__device__ __forceinline__ void store_val(float *p, float v) { *p = v; }
+__device__ __forceinline__ void store_val(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+__device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+}  // namespace kmoe
+
+// ------------------------------------------------ launchers between units
+
+namespace kmoe {
+
+kmoe_status launch_router_logits(const void *x, int x_dtype, const float *w_router, int N, int d,
+                                 int E, float *logits, cudaStream_t st);
+kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, int K,
+                        int32_t *idx, float *w, cudaStream_t st);
+
+size_t permute_ws_bytes(int N, int E);
+kmoe_status launch_permute(const int32_t *idx, int N, int K, int E, int32_t *counts,
+                           int32_t *offsets, int32_t *perm, int32_t *inv, int32_t *hist,
+                           cudaStream_t st);
+
+kmoe_status launch_ffn_stream(const void *x, int x_dtype, int N, int d, int I, int E, int K,
+                              const int32_t *perm, const int32_t *offsets, int w_dtype,
+                              const ExpertPtrs &routed, const ExpertPtrs *shared,
+                              void *h, void *y_perm, void *y_shared, cudaStream_t st);
+
+kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dtype,
+                           const float *w, const int32_t *inv, int N, int K, int d, void *y,
+                           int y_dtype, cudaStream_t st);
+
+}  // namespace kmoe

@@ -1,0 +1,175 @@
+/*
+ * kmoe — C ABI of the fine-grained sparse MoE feed-forward layer for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The layer (page "Inside Kolibri 1: Hybrid RNoPE Attention, Sparse MoE, and
+ * FP8 Serving", flozi.net, section "Routing: selection bias and mixture
+ * weights are separate"):
+ *   l      = x W_r^T                        FP32 logits [N, E]
+ *   idx    = top-K of (l + b) per token     b: learned expert-correction bias
+ *   g      = sigmoid(l[idx])                unbiased logits, not renormalised
+ *   F_e(x) = W_d,e (SiLU(W_g,e x) * (W_u,e x))   SwiGLU expert, no biases
+ *   y      = F_shared(x) + sum_k g_k F_{idx_k}(x)
+ * With the Kolibri-1 shape: d = 2560, E = 384 routed experts, K = 6, one
+ * shared expert, I = 512. FP8 weights (same page, section "The FP8 path is
+ * explicitly mixed precision") are E4M3 in 128 x 128 blocks with one FP32
+ * scale per block; scales are used as stored (never rounded to 2^k).
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers marked "device" point to GPU global memory owned by the
+ *     caller; the library never allocates or frees device memory and keeps
+ *     no state between calls other than a per-thread error message.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is
+ *     enqueued asynchronously; no entry point synchronises the device.
+ *   - Matrices are dense row-major. Every device pointer must be 16-byte
+ *     aligned.
+ *   - Sizes: 1 <= K <= 8, K <= E <= 1024, d and I multiples of 128 (needed by
+ *     the 128 x 128 FP8 blocks and the tensor-core tiles) with d <= 6144 and
+ *     I <= 4096, N >= 0. N == 0 is a successful no-op.
+ *   - Return value: KMOE_OK, or an error code with a message available from
+ *     moe_last_error(). Argument errors are detected on the host before any
+ *     work is enqueued. KMOE_ERR_CUDA reports a failed launch.
+ *   - Inputs are assumed finite.
+ */
+#ifndef KMOE_H
+#define KMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KMOE_OK = 0,
+    KMOE_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size */
+    KMOE_ERR_UNSUPPORTED = 2,   /* size or dtype combination not compiled */
+    KMOE_ERR_CUDA = 3,          /* a CUDA launch or runtime call failed */
+    KMOE_ERR_WORKSPACE = 4      /* workspace smaller than moe_workspace_size() */
+} kmoe_status;
+
+typedef enum {
+    KMOE_F32 = 0,        /* IEEE binary32 */
+    KMOE_BF16 = 1,       /* bfloat16 */
+    KMOE_E4M3_B128 = 2   /* OCP E4M3 bytes + one FP32 scale per 128x128 block */
+} kmoe_dtype;
+
+/*
+ * One stack of G SwiGLU experts (routed: G = E; shared: G = 1).
+ *   w_gate, w_up : device [G, I, d]  row i = weights of intermediate feature i
+ *   w_down       : device [G, d, I]  row j = weights of output feature j
+ *   s_gate, s_up : device [G, I/128, d/128] FP32 block scales (E4M3 only,
+ *   s_down       : device [G, d/128, I/128]  else ignored and may be NULL)
+ * The weight value of an E4M3 element is decode(q) * scale of its block.
+ */
+typedef struct {
+    const void *w_gate;
+    const void *w_up;
+    const void *w_down;
+    const float *s_gate;
+    const float *s_up;
+    const float *s_down;
+    int dtype;           /* kmoe_dtype of the weights */
+} kmoe_experts;
+
+/*
+ * Bytes of device workspace that any entry point below needs for these
+ * sizes (x_dtype: activations; w_dtype: expert weights). Pass a buffer of at
+ * least this size as `ws` (contents need not be initialised; the library
+ * overwrites what it uses). Returns 0 for unsupported arguments.
+ */
+size_t moe_workspace_size(int N, int d, int E, int K, int I, int x_dtype, int w_dtype);
+
+/*
+ * Router and selection ("Inside Kolibri 1", routing section, steps 1-2):
+ *   logits[t][e] = sum_j x[t][j] * w_router[e][j]        (FP32 accumulate)
+ *   topk_idx[t]  = the K experts with the largest logits[t][e] + bias[e],
+ *                  ordered by that biased score, highest first; on equal
+ *                  scores the lower expert index wins
+ *   topk_w[t][k] = 1 / (1 + exp(-logits[t][topk_idx[t][k]]))
+ * x        device [N, d], x_dtype KMOE_F32 or KMOE_BF16
+ * w_router device [E, d] FP32;   bias device [E] FP32
+ * logits   device [N, E] FP32 output, or NULL to keep it in the workspace
+ * topk_idx device [N, K] int32 output;  topk_w device [N, K] FP32 output
+ */
+kmoe_status moe_router_topk(const void *x, int x_dtype, const float *w_router,
+                            const float *bias, int N, int d, int E, int K,
+                            float *logits, int32_t *topk_idx, float *topk_w,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Dispatch: histogram, exclusive scan and a stable permutation of the N*K
+ * (token, slot) pairs by expert. The pages state only that tokens are sent
+ * to their selected experts (routing section); the order here is grouped by
+ * expert ascending and, inside one expert, by token ascending, which makes
+ * every output a deterministic function of topk_idx (bit-exact).
+ *   counts[e]      = #{(t,k) : topk_idx[t][k] == e}
+ *   offsets[e]     = sum_{e' < e} counts[e'],  offsets[E] = N*K
+ *   perm_token[p]  = token of dispatched row p
+ *   inv_pos[t][k]  = dispatched row of (t, k)
+ * topk_idx device [N, K] int32, each row holding K distinct values in
+ * [0, E); out-of-range values are skipped (outputs then unspecified).
+ * counts device [E], offsets device [E+1], perm_token device [N*K],
+ * inv_pos device [N, K]: int32 outputs.
+ */
+kmoe_status moe_permute(const int32_t *topk_idx, int N, int K, int E,
+                        int32_t *counts, int32_t *offsets, int32_t *perm_token,
+                        int32_t *inv_pos, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Grouped expert FFN (routing section, last paragraph: each routed or
+ * shared expert is a SwiGLU MLP):
+ *   y_perm[p]   = F_e(x[perm_token[p]])  for offsets[e] <= p < offsets[e+1]
+ *   y_shared[t] = F_shared(x[t])         (skipped when shared == NULL)
+ * with F(x) = W_d (SiLU(W_g x) * (W_u x)), FP32 accumulation, and the
+ * intermediate SiLU(.)*up rounded to the output dtype.
+ * x device [N, d] (x_dtype F32 or BF16). perm_token, offsets as produced by
+ * moe_permute. Output dtype: FP32 when the weights are FP32, else BF16.
+ * y_perm device [N*K, d]; y_shared device [N, d].
+ */
+kmoe_status moe_grouped_ffn(const void *x, int x_dtype, int N, int d, int I, int E, int K,
+                            const int32_t *perm_token, const int32_t *offsets,
+                            const kmoe_experts *routed, const kmoe_experts *shared,
+                            void *y_perm, void *y_shared,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Weighted combine ("Kolibri 1 Deep Dive", section 1, the layer-output
+ * formula without its residual term; the shared expert has weight 1):
+ *   y[t] = y_shared[t] + sum_{k<K} topk_w[t][k] * y_perm[inv_pos[t][k]]
+ * summed in slot order k = 0..K-1 in FP32 (deterministic, no atomics).
+ * y_perm device [N*K, d], y_shared device [N, d] (both y_in_dtype: F32 or
+ * BF16; y_shared may be NULL for no shared expert); topk_w device [N, K];
+ * inv_pos device [N, K]; y device [N, d] of y_dtype (F32 or BF16).
+ */
+kmoe_status moe_combine(const void *y_perm, const void *y_shared, int y_in_dtype,
+                        const float *topk_w, const int32_t *inv_pos,
+                        int N, int K, int d, void *y, int y_dtype, void *stream);
+
+/*
+ * The whole layer: moe_router_topk -> moe_permute -> moe_grouped_ffn ->
+ * moe_combine on one stream, with every intermediate in `ws`.
+ * y device [N, d] output of y_dtype (F32 or BF16). topk_idx_out [N, K],
+ * topk_w_out [N, K] and counts_out [E] are optional device outputs (NULL to
+ * skip). `shared` may be NULL (no shared expert).
+ */
+kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, int I,
+                        const float *w_router, const float *bias,
+                        const kmoe_experts *routed, const kmoe_experts *shared,
+                        void *y, int y_dtype,
+                        int32_t *topk_idx_out, float *topk_w_out, int32_t *counts_out,
+                        void *ws, size_t ws_bytes, void *stream);
+
+/* Message of the last error on the calling thread ("" after success). */
+const char *moe_last_error(void);
+
+/* ABI version of this header (bumped on incompatible change). */
+int moe_abi_version(void);
+#define KMOE_ABI_VERSION 1
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KMOE_H */

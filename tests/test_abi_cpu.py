@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI: the library loads, exports what the header
+declares, sizes its workspace, and rejects bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fine_grained_sparse_fp32_b200 import _build, kmoe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return kmoe.load()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "kmoe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_documented_entry_points():
+    assert header_functions() == sorted(kmoe.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(_build.LIB)
+    for name in header_functions():
+        assert hasattr(raw, name), name
+
+
+def test_abi_version(lib):
+    assert lib.moe_abi_version() == 1
+
+
+def test_workspace_size_grows_with_tokens(lib):
+    a = kmoe.moe_workspace_size(32, 2560, 384, 6, 512, kmoe.KMOE_BF16, kmoe.KMOE_BF16)
+    b = kmoe.moe_workspace_size(8192, 2560, 384, 6, 512, kmoe.KMOE_BF16, kmoe.KMOE_BF16)
+    assert 0 < a < b
+    # Y rows (N*K + N) * d * 2 bytes dominate at prefill
+    assert b >= (8192 * 7) * 2560 * 2
+
+
+@pytest.mark.parametrize("args", [
+    (32, 2560, 384, 9, 512),     # K > 8
+    (32, 2560, 4, 6, 512),       # E < K
+    (32, 2500, 384, 6, 512),     # d not a multiple of 128
+    (32, 2560, 384, 6, 500),     # I not a multiple of 128
+    (-1, 2560, 384, 6, 512),     # negative N
+    (32, 2560, 2048, 6, 512),    # E > 1024
+])
+def test_workspace_size_rejects_unsupported(lib, args):
+    assert kmoe.moe_workspace_size(*args, kmoe.KMOE_BF16, kmoe.KMOE_BF16) == 0
+
+
+def test_bad_arguments_fail_on_the_host(lib):
+    vp = ctypes.c_void_p
+    aligned = vp(1 << 20)
+    # K = 9 is not compiled
+    st = lib.moe_router_topk(aligned, kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 9,
+                             None, aligned, aligned, aligned, 1 << 20, None)
+    assert st == kmoe.KMOE_ERR_UNSUPPORTED
+    assert b"K=9" in lib.moe_last_error()
+    # null x
+    st = lib.moe_router_topk(None, kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 6,
+                             None, aligned, aligned, aligned, 1 << 20, None)
+    assert st == kmoe.KMOE_ERR_INVALID_ARG
+    # misaligned pointer
+    st = lib.moe_router_topk(vp((1 << 20) + 4), kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 6,
+                             None, aligned, aligned, aligned, 1 << 20, None)
+    assert st == kmoe.KMOE_ERR_INVALID_ARG and b"aligned" in lib.moe_last_error()
+    # unknown activation dtype
+    st = lib.moe_router_topk(aligned, 7, aligned, aligned, 4, 2560, 384, 6,
+                             None, aligned, aligned, aligned, 1 << 20, None)
+    assert st == kmoe.KMOE_ERR_UNSUPPORTED
+    # workspace too small
+    st = lib.moe_router_topk(aligned, kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 6,
+                             None, aligned, aligned, aligned, 16, None)
+    assert st == kmoe.KMOE_ERR_WORKSPACE
+
+
+def test_forward_rejects_null_experts_and_mixed_dtypes(lib):
+    vp = ctypes.c_void_p
+    a = vp(1 << 20)
+    ex = kmoe.Experts(a, a, a, None, None, None, kmoe.KMOE_BF16)
+    fp8 = kmoe.Experts(a, a, a, None, None, None, kmoe.KMOE_E4M3_B128)   # scales missing
+    args = lambda r, s: (a, kmoe.KMOE_BF16, 32, 2560, 384, 6, 512, a, a, r, s, a, kmoe.KMOE_BF16,
+                         None, None, None, a, 1 << 40, None)
+    assert lib.moe_forward(*args(None, None)) == kmoe.KMOE_ERR_INVALID_ARG
+    assert lib.moe_forward(*args(ctypes.byref(fp8), None)) == kmoe.KMOE_ERR_INVALID_ARG
+    mixed = kmoe.Experts(a, a, a, a, a, a, kmoe.KMOE_E4M3_B128)
+    assert lib.moe_forward(*args(ctypes.byref(ex), ctypes.byref(mixed))) == kmoe.KMOE_ERR_UNSUPPORTED
+
+
+def test_zero_tokens_is_a_host_side_no_op(lib):
+    a = ctypes.c_void_p(1 << 20)
+    ex = kmoe.Experts(a, a, a, None, None, None, kmoe.KMOE_BF16)
+    assert lib.moe_router_topk(None, kmoe.KMOE_BF16, None, None, 0, 2560, 384, 6,
+                               None, None, None, None, 0, None) == kmoe.KMOE_OK
+    assert lib.moe_forward(None, kmoe.KMOE_BF16, 0, 2560, 384, 6, 512, None, None, ctypes.byref(ex),
+                           None, None, kmoe.KMOE_BF16, None, None, None, None, 0, None) == kmoe.KMOE_OK
+    assert lib.moe_last_error() == b""

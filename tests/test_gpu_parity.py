@@ -1,0 +1,200 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Every test here needs a B200. Inputs are drawn on the device by the seeded
+generator and copied to the host for the oracle; no oracle input or expected
+value comes from the CUDA path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fine_grained_sparse_fp32_b200 import _build, kmoe
+from fine_grained_sparse_fp32_b200.inputs import CONFIGS, make_inputs, to_host
+from parity import G_TOL, TOL, biased_scores, check_routing, frob_rel_err, row_rel_err
+
+pytestmark = pytest.mark.gpu
+
+NT = None  # oracle threads: all host cores
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    _build.build()
+    kmoe.load()
+
+
+_CACHE = {}
+
+
+def layer_inputs(name, N=None, seed=0):
+    cfg = CONFIGS[name] if N is None else CONFIGS[name].with_tokens(N)
+    key = (cfg, seed)
+    if key not in _CACHE:
+        if len(_CACHE) >= 2:
+            _CACHE.clear()
+            torch.cuda.empty_cache()
+        dev = make_inputs(cfg, seed, device="cuda")
+        _CACHE[key] = (dev, to_host(dev))
+    return _CACHE[key]
+
+
+def threads():
+    return oracle.max_threads()
+
+
+# ----------------------------------------------------------------- router
+@pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("decode", 300), ("decode", 1),
+                                    ("skew", 2048)])
+def test_router_topk_matches_oracle(name, N):
+    dev, host = layer_inputs(name, N)
+    cfg = host["cfg"]
+    logits = torch.empty((cfg.N, cfg.E), dtype=torch.float32, device="cuda")
+    idx, w = kmoe.moe_router_topk(dev["x"], dev["w_router"], dev["bias"], cfg.K, logits=logits)
+    torch.cuda.synchronize()
+    l_ora = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
+    i_ora, g_ora, _ = oracle.select(l_ora, host["bias"], cfg.K)
+    l_gpu = logits.cpu().double().numpy()
+    assert np.abs(l_gpu - l_ora).max() <= 2e-5
+    s = biased_scores(l_ora, host["bias"])
+    idx_g = idx.cpu().numpy()
+    _, differ = check_routing(idx_g, i_ora, s, cfg.K)
+    w_g = w.cpu().double().numpy()
+    for t in range(cfg.N):
+        if t in differ:
+            continue
+        ora = dict(zip(i_ora[t].tolist(), g_ora[t].tolist()))
+        for k in range(cfg.K):
+            assert abs(w_g[t, k] - ora[int(idx_g[t, k])]) <= G_TOL
+
+
+# ---------------------------------------------------------------- permute
+def _distinct_rows(rng, N, K, E, skew=False):
+    if skew:
+        p = 1.0 / np.arange(1, E + 1) ** 1.1
+        p /= p.sum()
+        return np.stack([rng.choice(E, size=K, replace=False, p=p) for _ in range(N)]).astype(np.int32)
+    return np.argsort(rng.random((N, E)), axis=1)[:, :K].astype(np.int32)
+
+
+@pytest.mark.parametrize("N,E,skew", [(1, 384, False), (31, 64, False), (32, 384, False), (256, 384, False),
+                                      (257, 384, False), (1000, 64, True), (8192, 384, False),
+                                      (65536, 384, True), (300, 6, False)])
+def test_permute_is_bit_exact(N, E, skew):
+    rng = np.random.default_rng(N + E)
+    K = 6
+    idx = _distinct_rows(rng, N, K, E, skew)
+    counts, offsets, perm, inv = kmoe.moe_permute(torch.from_numpy(idx).cuda(), E)
+    c_o, o_o, p_o, i_o = oracle.permute(idx, E)
+    np.testing.assert_array_equal(counts.cpu().numpy(), c_o)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), o_o)
+    np.testing.assert_array_equal(perm.cpu().numpy(), p_o)
+    np.testing.assert_array_equal(inv.cpu().numpy(), i_o)
+
+
+def test_permute_zero_tokens():
+    counts, offsets, _, _ = kmoe.moe_permute(torch.empty((0, 6), dtype=torch.int32, device="cuda"), 384)
+    assert counts.abs().sum().item() == 0 and offsets.abs().sum().item() == 0
+
+
+def test_permute_all_tokens_on_the_same_experts():
+    N, E, K = 4000, 384, 6
+    idx = np.tile(np.array([383, 0, 17, 200, 5, 6], dtype=np.int32), (N, 1))
+    counts, offsets, perm, inv = kmoe.moe_permute(torch.from_numpy(idx).cuda(), E)
+    c_o, o_o, p_o, i_o = oracle.permute(idx, E)
+    np.testing.assert_array_equal(perm.cpu().numpy(), p_o)
+    np.testing.assert_array_equal(inv.cpu().numpy(), i_o)
+    np.testing.assert_array_equal(counts.cpu().numpy(), c_o)
+
+
+# ------------------------------------------------------------ grouped FFN
+@pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("fp8_decode", None), ("decode", 200),
+                                    ("fp8_decode", 130)])
+def test_grouped_ffn_matches_oracle(name, N):
+    dev, host = layer_inputs(name, N)
+    cfg = host["cfg"]
+    l_ora = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
+    i_ora, _, _ = oracle.select(l_ora, host["bias"], cfg.K)
+    counts, offsets, perm, inv = oracle.permute(i_ora, cfg.E)
+    y_perm, y_shared = kmoe.moe_grouped_ffn(dev["x"], dev, torch.from_numpy(perm).cuda(),
+                                            torch.from_numpy(offsets).cuda())
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, cfg.N * cfg.K - 1], rng.integers(0, cfg.N * cfg.K, 48)]))
+    expert_of_row = np.searchsorted(offsets, rows, side="right") - 1
+    ref = oracle.expert_outputs(host, perm[rows], expert_of_row, nthreads=threads())
+    got = y_perm[torch.from_numpy(rows).cuda().long()].float().cpu().numpy()
+    assert row_rel_err(got, ref) <= TOL[cfg.w_dtype]
+    toks = np.unique(np.concatenate([[0, cfg.N - 1], rng.integers(0, cfg.N, 16)]))
+    ref_s = oracle.expert_outputs(host, toks, np.full(len(toks), cfg.E), nthreads=threads())
+    got_s = y_shared[torch.from_numpy(toks).cuda().long()].float().cpu().numpy()
+    assert row_rel_err(got_s, ref_s) <= TOL[cfg.w_dtype]
+
+
+# ----------------------------------------------------------- whole layer
+def _forward_and_compare(name, N=None, rows=None, check_all_routing=True):
+    dev, host = layer_inputs(name, N)
+    cfg = host["cfg"]
+    y_dtype = torch.float32 if cfg.x_dtype == "f32" else torch.bfloat16
+    y, idx, w, counts = kmoe.moe_forward(dev["x"], dev, y_dtype=y_dtype, with_outputs=True)
+    torch.cuda.synchronize()
+    idx_g = idx.cpu().numpy()
+    if rows is None:
+        rows = np.arange(cfg.N, dtype=np.int32)
+    ora = oracle.layer(host, rows=rows, nthreads=threads())
+    # routing on the compared rows (oracle logits recomputed for them)
+    xr = host["x"][torch.from_numpy(rows).long()]
+    l_rows = oracle.router_logits(xr, cfg.x_dtype, host["w_router"], nthreads=threads())
+    s = biased_scores(l_rows, host["bias"])
+    _, differ = check_routing(idx_g[rows], ora["idx"], s, cfg.K)
+    keep = np.array([r not in differ for r in range(len(rows))])
+    got = y[torch.from_numpy(rows).cuda().long()].float().cpu().numpy()
+    err = row_rel_err(got[keep], ora["y"][keep])
+    assert err <= TOL[cfg.w_dtype], (name, err, frob_rel_err(got[keep], ora["y"][keep]))
+    if check_all_routing:
+        l_all = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
+        i_all, _, _ = oracle.select(l_all, host["bias"], cfg.K)
+        _, differ_all = check_routing(idx_g, i_all, biased_scores(l_all, host["bias"]), cfg.K)
+        # counts equal the oracle's counting sort of the GPU's own (validated) indices
+        c_o, _, _, _ = oracle.permute(idx_g, cfg.E)
+        np.testing.assert_array_equal(counts.cpu().numpy(), c_o)
+    assert int(counts.sum().item()) == cfg.N * cfg.K
+    return err
+
+
+@pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("fp8_decode", None),
+                                    ("prefill", 300), ("fp8_prefill", 259), ("decode", 1)])
+def test_forward_matches_oracle_all_tokens(name, N):
+    _forward_and_compare(name, N)
+
+
+@pytest.mark.parametrize("name", ["prefill", "fp8_prefill"])
+def test_forward_full_size_sampled_tokens(name):
+    cfg = CONFIGS[name]
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([[0, cfg.N - 1], rng.integers(0, cfg.N, 30)])).astype(np.int32)
+    _forward_and_compare(name, rows=rows, check_all_routing=True)
+
+
+def test_forward_skew_full_size_sampled_tokens():
+    cfg = CONFIGS["skew"]
+    rng = np.random.default_rng(2)
+    rows = np.unique(np.concatenate([[0, cfg.N - 1], rng.integers(0, cfg.N, 24)])).astype(np.int32)
+    _forward_and_compare("skew", rows=rows, check_all_routing=False)
+
+
+def test_forward_is_deterministic():
+    for name, N in (("decode", None), ("prefill", 300)):
+        dev, _ = layer_inputs(name, N)
+        a = kmoe.moe_forward(dev["x"], dev, with_outputs=True)
+        b = kmoe.moe_forward(dev["x"], dev, with_outputs=True)
+        for u, v in zip(a, b):
+            assert torch.equal(u, v)
+
+
+def test_forward_zero_tokens():
+    dev, _ = layer_inputs("decode")
+    y = kmoe.moe_forward(dev["x"][:0], dev)
+    assert y.shape == (0, 2560)
