@@ -184,7 +184,7 @@ def time_grouped_ffn(layer, xs, stream, steps):
             idx, w = kmoe.moe_router_topk(x, layer["w_router"], layer["bias"], cfg.K, stream=stream)
             _, offsets, perm, _ = kmoe.moe_permute(idx, cfg.E, stream=stream)
             preps.append((x, perm, offsets))
-    ws = torch.empty(((cfg.N * cfg.K + cfg.N) * cfg.I * 4), dtype=torch.uint8, device=dev)
+    ws = torch.empty(256 + (cfg.N * cfg.K + cfg.N) * cfg.I * 4, dtype=torch.uint8, device=dev)
     outs = [kmoe.moe_grouped_ffn(x, layer, p, o, ws=ws, stream=stream) for x, p, o in preps]
     stream.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
@@ -345,18 +345,18 @@ def run_reference(args, world, rank):
     from fine_grained_sparse_fp32_b200.inputs import to_host
     cfg = CONFIGS["decode"]
     host = to_host(make_inputs(cfg, seed=0, device="cuda" if torch.cuda.is_available() else "cpu"))
-    sample = args.cpu_tokens if args.cpu_tokens else 4
-    sample = max(1, min(sample, 8))
+    # each step evaluates a bounded token sample so that K steps stay within a
+    # couple of minutes of host time (about 1600 token evaluations in total)
+    sample = max(1, min(cfg.N, 1600 // max(args.steps, 1)))
     rows = np.arange(sample, dtype=np.int32)
-    nt = oracle.max_threads()
-    for _ in range(min(args.warmup, 1)):
-        oracle.layer(host, rows=rows, nthreads=nt)
+    nt = min(oracle.max_threads(), sample)
+    oracle.layer(host, rows=rows[:1], nthreads=1)
     times = []
-    for _ in range(args.steps if args.steps <= 20 else 20):
+    for _ in range(args.steps):
         t = time.perf_counter()
         oracle.layer(host, rows=rows, nthreads=nt)
         times.append(time.perf_counter() - t)
-    per_token = float(np.mean(times)) / sample
+    per_token = float(np.sum(times)) / (sample * len(times))
     value = 1.0 / per_token
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": len(times), "warmup": args.warmup, "ms_per_step": per_token * cfg.N * 1e3,

@@ -95,6 +95,7 @@ static size_t act_bytes(int w_dtype) { return w_dtype == KMOE_F32 ? 4 : 2; }
 // Workspace of the whole forward; every entry point uses a prefix-compatible
 // subset (router: logits; permute: chunk histograms; grouped FFN: H).
 struct Layout {
+    int *status;
     float *logits;
     int32_t *idx;
     float *w;
@@ -109,6 +110,7 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype)
     Layout L;
     const size_t R = (size_t)N * K + N;
     const size_t ab = act_bytes(w_dtype);
+    L.status = c.take<int>(64);
     L.logits = c.take<float>((size_t)N * E);
     L.idx = c.take<int32_t>((size_t)N * K);
     L.w = c.take<float>((size_t)N * K);
@@ -123,6 +125,30 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype)
     L.bytes = c.used + 256;
     return L;
 }
+
+static bool use_tc(int x_dtype, int w_dtype, int N, int d)
+{
+    return x_dtype == KMOE_BF16 && w_dtype == KMOE_BF16 && N >= kTcMinTokens && d % 256 == 0;
+}
+
+static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int E, int K, const int32_t *perm,
+                           const int32_t *offsets, int w_dtype, const ExpertPtrs &r, const ExpertPtrs *s,
+                           void *h, void *y_perm, void *y_shared, int *status, cudaStream_t st)
+{
+    if (use_tc(x_dtype, w_dtype, N, d))
+        return launch_ffn_tc(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, r, s,
+                             static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
+                             static_cast<__nv_bfloat16 *>(y_shared), status, st);
+    return launch_ffn_stream(x, x_dtype, N, d, I, E, K, perm, offsets, w_dtype, r, s, h, y_perm, y_shared, st);
+}
+
+static kmoe_status clear_status(int *status, cudaStream_t st)
+{
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return check_launch("status memset");
+    return KMOE_OK;
+}
+
+constexpr size_t kStatusBytes = 256;
 
 }  // namespace kmoe
 
@@ -215,13 +241,16 @@ kmoe_status moe_grouped_ffn(const void *x, int x_dtype, int N, int d, int I, int
     KMOE_TRY(check_ptr(y_perm, "y_perm"));
     if (shared) KMOE_TRY(check_ptr(y_shared, "y_shared"));
     KMOE_TRY(check_ptr(ws, "ws"));
-    const size_t need = ((size_t)N * K + N) * I * act_bytes(routed->dtype);
+    const size_t need = kStatusBytes + ((size_t)N * K + N) * I * act_bytes(routed->dtype);
     if (ws_bytes < need) return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
     const ExpertPtrs r = ptrs(routed);
     ExpertPtrs s{};
     if (shared) s = ptrs(shared);
-    return launch_ffn_stream(x, x_dtype, N, d, I, E, K, perm_token, offsets, routed->dtype, r,
-                             shared ? &s : nullptr, ws, y_perm, y_shared, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int *status = static_cast<int *>(ws);
+    KMOE_TRY(clear_status(status, st));
+    return run_ffn(x, x_dtype, N, d, I, E, K, perm_token, offsets, routed->dtype, r, shared ? &s : nullptr,
+                   static_cast<char *>(ws) + kStatusBytes, y_perm, y_shared, status, st);
 }
 
 kmoe_status moe_combine(const void *y_perm, const void *y_shared, int y_in_dtype, const float *topk_w,
@@ -272,16 +301,30 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
     int32_t *idx = topk_idx_out ? topk_idx_out : L.idx;
     float *w = topk_w_out ? topk_w_out : L.w;
     int32_t *counts = counts_out ? counts_out : L.counts;
+    KMOE_TRY(clear_status(L.status, st));
     KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, L.logits, st));
     KMOE_TRY(launch_topk(L.logits, bias, N, E, K, idx, w, st));
     KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st));
     const ExpertPtrs r = ptrs(routed);
     ExpertPtrs s{};
     if (shared) s = ptrs(shared);
-    KMOE_TRY(launch_ffn_stream(x, x_dtype, N, d, I, E, K, L.perm, L.offsets, routed->dtype, r,
-                               shared ? &s : nullptr, L.h, L.y_perm, L.y_shared, st));
+    KMOE_TRY(run_ffn(x, x_dtype, N, d, I, E, K, L.perm, L.offsets, routed->dtype, r, shared ? &s : nullptr,
+                     L.h, L.y_perm, L.y_shared, L.status, st));
     const int yin = routed->dtype == KMOE_F32 ? KMOE_F32 : KMOE_BF16;
     return launch_combine(L.y_perm, shared ? L.y_shared : nullptr, yin, w, L.inv, N, K, d, y, y_dtype, st);
+}
+
+kmoe_status moe_device_status(const void *ws, int *status, void *stream)
+{
+    clear_error();
+    KMOE_TRY(check_ptr(ws, "ws"));
+    if (!status) return fail(KMOE_ERR_INVALID_ARG, "status is NULL");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(status, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return check_launch("device status read");
+    if (*status != 0) return fail(KMOE_ERR_DEVICE, "device status %d: a pipeline wait gave up", *status);
+    return KMOE_OK;
 }
 
 }  // extern "C"

@@ -127,6 +127,15 @@ kmoe_status launch_ffn_stream(const void *x, int x_dtype, int N, int d, int I, i
                               const ExpertPtrs &routed, const ExpertPtrs *shared,
                               void *h, void *y_perm, void *y_shared, cudaStream_t st);
 
+// Tensor-core grouped FFN (BF16 weights and activations, d % 256 == 0).
+kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
+                          const int32_t *offsets, const ExpertPtrs &routed, const ExpertPtrs *shared,
+                          __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err,
+                          cudaStream_t st);
+
+// Batches of at least this many tokens take the tensor-core FFN.
+constexpr int kTcMinTokens = 256;
+
 kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dtype,
                            const float *w, const int32_t *inv, int N, int K, int d, void *y,
                            int y_dtype, cudaStream_t st);

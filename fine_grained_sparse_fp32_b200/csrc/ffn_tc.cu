@@ -1,0 +1,404 @@
+// Grouped SwiGLU expert FFN on the 5th-generation tensor cores (tcgen05),
+// for batches where experts see many tokens (prefill).
+//
+// "Inside Kolibri 1" (flozi.net), routing section: each routed or shared
+// expert is a SwiGLU MLP (two d -> I projections, SiLU(gate) * up, one
+// I -> d projection, no biases). Per expert e with rows X_e (the tokens
+// dispatched to it, gathered through perm_token):
+//   up kernel   : H_e = SiLU(X_e W_g,e^T) * (X_e W_u,e^T)     [rows, I]
+//   down kernel : Y_e = H_e W_d,e^T                           [rows, d]
+// Both are persistent, warp-specialised grouped GEMMs with 128 x 256 x 64
+// tiles (BF16 operands, FP32 accumulation in tensor memory):
+//   warps 0-3  epilogue: tcgen05.ld of the accumulator, SwiGLU (up) or the
+//              BF16 cast (down), stores to global memory;
+//   warp  4    one thread issues tcgen05.mma and tcgen05.commit;
+//   warps 5-8  producers: weight tiles by TMA (128-byte swizzle); the
+//              activation rows of the up kernel are gathered with cp.async
+//              straight into the swizzled layout (no permuted copy of x is
+//              ever written), the down kernel loads H tiles by TMA.
+// The up tile pairs 128 gate features with the same 128 up features (one
+// N = 256 MMA into 256 TMEM columns), so SiLU(g) * u is computed in
+// registers. Two accumulators (512 TMEM columns) let the epilogue of one
+// tile overlap the MMAs of the next. Tiles are enumerated per expert as
+// (n-tile, m-tile) so that CTAs working at the same time read the same
+// weight tile and it crosses HBM once.
+#include "common.cuh"
+#include "sm100.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace kmoe {
+using namespace sm100;
+
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kStages = 4;
+constexpr int kATile = kBM * kBK * 2;        // 16 KB
+constexpr int kBTile = kBN * kBK * 2;        // 32 KB
+constexpr int kStage = kATile + kBTile;
+constexpr int kMmaWarp = 4;
+constexpr int kProdWarp = 5;
+constexpr int kTcThreads = 9 * 32;
+constexpr int kLag = 2;                      // cp.async groups in flight before signalling
+constexpr int kMaxGroups = 1025;
+constexpr long long kWaitLimit = 1LL << 32;  // SM cycles (about 2 s)
+
+struct TcMaps {
+    CUtensorMap b0_routed, b1_routed, b0_shared, b1_shared;   // up: gate, up; down: W_d (b0 only)
+    CUtensorMap a;                                            // down: H [R, I]
+};
+
+struct TcArgs {
+    const int32_t *offsets;
+    const int32_t *perm;
+    const __nv_bfloat16 *x;
+    int N, K, E, groups;
+    int d, I, kblocks, n_tiles;
+    __nv_bfloat16 *out0;      // up: H [R, I]; down: y_perm [N*K, d]
+    __nv_bfloat16 *out1;      // down: y_shared [N, d]
+    int *err;
+};
+
+struct SmemTail {
+    uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], drain;
+    uint32_t tmem_base;
+    int abort;
+    int pre[kMaxGroups + 1];
+};
+
+constexpr size_t kTcSmem = 1024 /*align slack*/ + (size_t)kStages * kStage + sizeof(SmemTail);
+
+struct Tile {
+    int g, row0, rows, n0;
+    bool shared;
+};
+
+__device__ __forceinline__ Tile decode_tile(int t, const int *pre, const TcArgs &a, int bn)
+{
+    int lo = 1, hi = a.groups;            // smallest j with pre[j] * n_tiles > t
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (pre[mid] * a.n_tiles > t) hi = mid;
+        else lo = mid + 1;
+    }
+    Tile T;
+    T.g = lo - 1;
+    T.shared = T.g >= a.E;
+    const int mcount = pre[T.g + 1] - pre[T.g];
+    const int local = t - pre[T.g] * a.n_tiles;
+    const int nt = local / mcount, mt = local - nt * mcount;
+    int start, cnt;
+    if (T.shared) { start = a.N * a.K; cnt = a.N; }
+    else { start = a.offsets[T.g]; cnt = a.offsets[T.g + 1] - start; }
+    T.row0 = start + mt * kBM;
+    T.rows = min(kBM, cnt - mt * kBM);
+    T.n0 = nt * bn;
+    return T;
+}
+
+// m-tile prefix over groups, computed by one warp.
+__device__ __forceinline__ void build_prefix(int *pre, const TcArgs &a)
+{
+    const int lane = threadIdx.x & 31;
+    const int per = (a.groups + 31) / 32;
+    const int g0 = lane * per;
+    int sum = 0;
+    for (int i = 0; i < per; ++i) {
+        const int g = g0 + i;
+        if (g < a.groups) {
+            const int cnt = g < a.E ? a.offsets[g + 1] - a.offsets[g] : a.N;
+            sum += (cnt + kBM - 1) / kBM;
+        }
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+    for (int i = 0; i < per; ++i) {
+        const int g = g0 + i;
+        if (g < a.groups) {
+            pre[g] = run;
+            const int cnt = g < a.E ? a.offsets[g + 1] - a.offsets[g] : a.N;
+            run += (cnt + kBM - 1) / kBM;
+        }
+    }
+    if (lane == 31) pre[a.groups] = incl;
+}
+
+template <bool kUp>
+__global__ void __launch_bounds__(kTcThreads, 1)
+ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    SmemTail *tail = reinterpret_cast<SmemTail *>(smem + (size_t)kStages * kStage);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort = &tail->abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&tail->full[s], kUp ? 128 + 1 : 1);
+            mbar_init(&tail->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tail->tfull[b], 1);
+            mbar_init(&tail->tempty[b], 128);
+        }
+        mbar_init(&tail->drain, 1);
+        tail->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) build_prefix(tail->pre, a);
+    if (warp == 0) {
+        tmem_alloc(&tail->tmem_base, 512);
+        tmem_relinquish();
+    }
+    if (warp == kProdWarp && lane == 0) {
+        prefetch_map(&maps.b0_routed);
+        prefetch_map(&maps.b0_shared);
+        if (kUp) { prefetch_map(&maps.b1_routed); prefetch_map(&maps.b1_shared); }
+        else prefetch_map(&maps.a);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const int bn = kUp ? kBN / 2 : kBN;     // output columns per tile
+    const int total = tail->pre[a.groups] * a.n_tiles;
+    const uint32_t tmem = tail->tmem_base;
+
+    if (warp >= kProdWarp) {
+        // ------------------------------------------------------- producers
+        const int p = threadIdx.x - kProdWarp * 32;
+        const bool leader = p == 0;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile T = decode_tile(t, tail->pre, a, bn);
+            const CUtensorMap *m0 = T.shared ? &maps.b0_shared : &maps.b0_routed;
+            const CUtensorMap *m1 = T.shared ? &maps.b1_shared : &maps.b1_routed;
+            const int gi = T.shared ? 0 : T.g;
+            int tok = -1;
+            if (kUp && p < T.rows) tok = T.shared ? T.row0 + p - a.N * a.K : a.perm[T.row0 + p];
+            const __nv_bfloat16 *src = a.x + (size_t)(tok < 0 ? 0 : tok) * a.d;
+            for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                if (!mbar_wait(&tail->empty[s], ph ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                uint8_t *As = smem + (size_t)s * kStage;
+                uint8_t *Bs = As + kATile;
+                if (kUp) {
+                    if (leader) {
+                        mbar_arrive_expect_tx(&tail->full[s], kBTile);
+                        tma_load_2d(Bs, m0, &tail->full[s], kb * kBK, gi * a.I + T.n0);
+                        tma_load_2d(Bs + kBTile / 2, m1, &tail->full[s], kb * kBK, gi * a.I + T.n0);
+                    }
+                    const uint32_t dst = smem_u32(As) + p * 128;
+                    const __nv_bfloat16 *s_row = src + kb * kBK;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        cp_async16(dst + ((c ^ (p & 7)) << 4), s_row + c * 8, tok >= 0 ? 16u : 0u);
+                    cp_async_commit();
+                    if (it >= kLag) {
+                        cp_async_wait<kLag>();
+                        fence_proxy_async();
+                        mbar_arrive(&tail->full[(it - kLag) % kStages]);
+                    }
+                } else if (leader) {
+                    mbar_arrive_expect_tx(&tail->full[s], kATile + kBTile);
+                    tma_load_2d(As, &maps.a, &tail->full[s], kb * kBK, T.row0);
+                    tma_load_2d(Bs, m0, &tail->full[s], kb * kBK, gi * a.d + T.n0);
+                    tma_load_2d(Bs + kBTile / 2, m0, &tail->full[s], kb * kBK, gi * a.d + T.n0 + kBN / 2);
+                }
+            }
+        }
+        if (kUp) {   // signal the stages still waiting for this thread's copies
+            cp_async_wait<0>();
+            fence_proxy_async();
+            for (uint32_t j = it > (uint32_t)kLag ? it - kLag : 0; j < it; ++j) mbar_arrive(&tail->full[j % kStages]);
+        }
+        if (!ok && leader) {   // let in-flight TMA loads land before the CTA exits
+            for (uint32_t j = it > (uint32_t)kStages ? it - kStages : 0; j < it; ++j)
+                mbar_wait_drain(&tail->full[j % kStages], (j / kStages) & 1, kWaitLimit);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN);
+            uint32_t it = 0, at = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++at) {
+                const int b = at & 1;
+                if (!mbar_wait(&tail->tempty[b], ((at >> 1) & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + b * kBN;
+                for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                    const int s = it % kStages;
+                    if (!mbar_wait(&tail->full[s], (it / kStages) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_kmajor_desc(smem_u32(smem + (size_t)s * kStage));
+                    const uint64_t bd = sw128_kmajor_desc(smem_u32(smem + (size_t)s * kStage + kATile));
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma_bf16(d_tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
+                    umma_commit(&tail->empty[s]);
+                }
+                if (ok) umma_commit(&tail->tfull[b]);
+            }
+            umma_commit(&tail->drain);     // every MMA done before tensor memory is released
+            mbar_wait_drain(&tail->drain, 0, kWaitLimit);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------- epilogue
+        uint32_t at = 0;
+        const int row = warp * 32 + lane;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++at) {
+            const Tile T = decode_tile(t, tail->pre, a, bn);
+            const int b = at & 1;
+            if (!mbar_wait(&tail->tfull[b], (at >> 1) & 1, abort, a.err, kWaitLimit)) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + b * kBN;
+            const bool valid = row < T.rows;
+            const int grow = T.row0 + row;
+            if (kUp) {
+                __nv_bfloat16 *dst = a.out0 + (size_t)grow * a.I + T.n0;
+#pragma unroll 1
+                for (int c = 0; c < kBN / 2; c += 16) {
+                    uint32_t g[16], u[16];
+                    tmem_ld16(tbase + c, g);
+                    tmem_ld16(tbase + kBN / 2 + c, u);
+                    tmem_ld_wait();
+                    uint32_t packed[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float g0 = __uint_as_float(g[2 * q]), g1 = __uint_as_float(g[2 * q + 1]);
+                        const float u0 = __uint_as_float(u[2 * q]), u1 = __uint_as_float(u[2 * q + 1]);
+                        packed[q] = pack_bf16x2(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1);
+                    }
+                    if (valid) {
+                        uint4 *o = reinterpret_cast<uint4 *>(dst + c);
+                        o[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                        o[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                    }
+                }
+            } else {
+                __nv_bfloat16 *dst = T.shared ? a.out1 + (size_t)(grow - a.N * a.K) * a.d + T.n0
+                                              : a.out0 + (size_t)grow * a.d + T.n0;
+#pragma unroll 1
+                for (int c = 0; c < kBN; c += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(tbase + c, v);
+                    tmem_ld_wait();
+                    uint32_t packed[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        packed[q] = pack_bf16x2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
+                    if (valid) {
+                        uint4 *o = reinterpret_cast<uint4 *>(dst + c);
+                        o[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                        o[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tail->tempty[b]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------- host
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2D BF16 map over a row-major [rows, cols] matrix, box 128 rows x 64 columns
+// (128 bytes), 128-byte swizzle; reads outside the matrix return zeros.
+static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {kBK, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int sm_count_tc()
+{
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
+                          const int32_t *offsets, const ExpertPtrs &routed, const ExpertPtrs *shared,
+                          __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err,
+                          cudaStream_t st)
+{
+    if (E + 1 > kMaxGroups) return fail(KMOE_ERR_UNSUPPORTED, "tensor-core FFN: too many experts");
+    const ExpertPtrs sh = shared ? *shared : routed;    // unused maps still need a valid base
+    const long long R = (long long)N * K + N;
+    TcMaps up{}, dn{};
+    bool ok = make_map(&up.b0_routed, routed.wg, (uint64_t)E * I, d) &&
+              make_map(&up.b1_routed, routed.wu, (uint64_t)E * I, d) &&
+              make_map(&up.b0_shared, sh.wg, I, d) && make_map(&up.b1_shared, sh.wu, I, d) &&
+              make_map(&up.a, h, R, I) &&
+              make_map(&dn.b0_routed, routed.wd, (uint64_t)E * d, I) && make_map(&dn.b0_shared, sh.wd, d, I) &&
+              make_map(&dn.b1_routed, routed.wd, (uint64_t)E * d, I) && make_map(&dn.b1_shared, sh.wd, d, I) &&
+              make_map(&dn.a, h, R, I);
+    if (!ok) return fail(KMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    TcArgs a{};
+    a.offsets = offsets;
+    a.perm = perm;
+    a.x = x;
+    a.N = N;
+    a.K = K;
+    a.E = E;
+    a.groups = E + (shared ? 1 : 0);
+    a.d = d;
+    a.I = I;
+    a.err = err;
+    const int grid = sm_count_tc();
+    cudaFuncSetAttribute(ffn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
+    cudaFuncSetAttribute(ffn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
+    a.kblocks = d / kBK;
+    a.n_tiles = I / (kBN / 2);
+    a.out0 = h;
+    ffn_tc_kernel<true><<<grid, kTcThreads, kTcSmem, st>>>(up, a);
+    kmoe_status s = check_launch("ffn_up_tc");
+    if (s != KMOE_OK) return s;
+    a.kblocks = I / kBK;
+    a.n_tiles = d / kBN;
+    a.out0 = y_perm;
+    a.out1 = y_shared;
+    ffn_tc_kernel<false><<<grid, kTcThreads, kTcSmem, st>>>(dn, a);
+    return check_launch("ffn_down_tc");
+}
+
+}  // namespace kmoe

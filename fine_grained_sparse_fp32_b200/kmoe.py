@@ -13,11 +13,11 @@ import torch
 
 from ._build import LIB
 
-KMOE_OK, KMOE_ERR_INVALID_ARG, KMOE_ERR_UNSUPPORTED, KMOE_ERR_CUDA, KMOE_ERR_WORKSPACE = range(5)
+KMOE_OK, KMOE_ERR_INVALID_ARG, KMOE_ERR_UNSUPPORTED, KMOE_ERR_CUDA, KMOE_ERR_WORKSPACE, KMOE_ERR_DEVICE = range(6)
 KMOE_F32, KMOE_BF16, KMOE_E4M3_B128 = 0, 1, 2
 
 EXPORTS = ["moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
-           "moe_combine", "moe_forward", "moe_last_error", "moe_abi_version"]
+           "moe_combine", "moe_forward", "moe_device_status", "moe_last_error", "moe_abi_version"]
 
 
 class KmoeError(RuntimeError):
@@ -57,7 +57,9 @@ def load(path: str | None = None):
     lib.moe_combine.argtypes = [vp, vp, i, vp, vp, i, i, i, vp, i, vp]
     lib.moe_forward.argtypes = [vp, i, i, i, i, i, i, vp, vp, ctypes.POINTER(Experts),
                                 ctypes.POINTER(Experts), vp, i, vp, vp, vp, vp, sz, vp]
-    for f in ("moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward"):
+    lib.moe_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
+    for f in ("moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward",
+              "moe_device_status"):
         getattr(lib, f).restype = i
     if lib.moe_abi_version() != 1:
         raise RuntimeError("libkmoe ABI version mismatch")
@@ -153,7 +155,7 @@ def moe_grouped_ffn(x, layer, perm_token, offsets, with_shared=True, ws=None, st
     y_perm = torch.empty((N * K, d), dtype=adt, device=x.device)
     y_shared = torch.empty((N, d), dtype=adt, device=x.device) if with_shared else None
     if ws is None:
-        ws = torch.empty(max((N * K + N) * I * (4 if adt == torch.float32 else 2), 16), dtype=torch.uint8,
+        ws = torch.empty(256 + (N * K + N) * I * (4 if adt == torch.float32 else 2), dtype=torch.uint8,
                          device=x.device)
     routed = experts_of(layer, "routed")
     shared = experts_of(layer, "shared") if with_shared else None
@@ -161,6 +163,15 @@ def moe_grouped_ffn(x, layer, perm_token, offsets, with_shared=True, ws=None, st
                                   ctypes.byref(routed), ctypes.byref(shared) if shared is not None else None,
                                   _ptr(y_perm), _ptr(y_shared), _ptr(ws), ws.numel(), _stream(stream)))
     return y_perm, y_shared
+
+
+def moe_device_status(ws, stream=None) -> int:
+    """Synchronises `stream` and returns the device status word of workspace `ws` (0 = ok)."""
+    st = ctypes.c_int(-1)
+    rc = load().moe_device_status(_ptr(ws), ctypes.byref(st), _stream(stream))
+    if rc not in (KMOE_OK, KMOE_ERR_DEVICE):
+        _check(rc)
+    return st.value
 
 
 def moe_combine(y_perm, y_shared, topk_w, inv_pos, y_dtype=torch.bfloat16, out=None, stream=None):

@@ -46,7 +46,8 @@ typedef enum {
     KMOE_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size */
     KMOE_ERR_UNSUPPORTED = 2,   /* size or dtype combination not compiled */
     KMOE_ERR_CUDA = 3,          /* a CUDA launch or runtime call failed */
-    KMOE_ERR_WORKSPACE = 4      /* workspace smaller than moe_workspace_size() */
+    KMOE_ERR_WORKSPACE = 4,     /* workspace smaller than moe_workspace_size() */
+    KMOE_ERR_DEVICE = 5         /* a kernel reported a failure in the device status word */
 } kmoe_status;
 
 typedef enum {
@@ -160,6 +161,17 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
                         void *y, int y_dtype,
                         int32_t *topk_idx_out, float *topk_w_out, int32_t *counts_out,
                         void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Device status word. moe_forward and moe_grouped_ffn clear the first 4
+ * bytes of `ws` when they are enqueued; a tensor-core kernel whose pipeline
+ * wait gives up (after about two seconds, which only a fault elsewhere can
+ * cause) writes a non-zero code there and returns early, leaving its outputs
+ * invalid. This call copies the word to *status and synchronises `stream`
+ * (the one exception to the no-synchronisation rule). Returns KMOE_OK when
+ * the word is 0, KMOE_ERR_DEVICE otherwise (1 = a wait timed out).
+ */
+kmoe_status moe_device_status(const void *ws, int *status, void *stream);
 
 /* Message of the last error on the calling thread ("" after success). */
 const char *moe_last_error(void);

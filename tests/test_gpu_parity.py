@@ -111,7 +111,7 @@ def test_permute_all_tokens_on_the_same_experts():
 
 # ------------------------------------------------------------ grouped FFN
 @pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("fp8_decode", None), ("decode", 200),
-                                    ("fp8_decode", 130)])
+                                    ("fp8_decode", 130), ("prefill", 256), ("prefill", 300), ("prefill", 1000)])
 def test_grouped_ffn_matches_oracle(name, N):
     dev, host = layer_inputs(name, N)
     cfg = host["cfg"]
@@ -192,6 +192,15 @@ def test_forward_is_deterministic():
         b = kmoe.moe_forward(dev["x"], dev, with_outputs=True)
         for u, v in zip(a, b):
             assert torch.equal(u, v)
+
+
+def test_device_status_is_clear_after_a_forward():
+    for name, N in (("decode", None), ("prefill", 300)):
+        dev, _ = layer_inputs(name, N)
+        cfg = dev["cfg"]
+        lay = kmoe.Layer(dev, cfg.N)
+        lay.forward(dev["x"])
+        assert kmoe.moe_device_status(lay.ws) == 0
 
 
 def test_forward_zero_tokens():
