@@ -16,7 +16,7 @@ from ._build import LIB
 KMOE_OK, KMOE_ERR_INVALID_ARG, KMOE_ERR_UNSUPPORTED, KMOE_ERR_CUDA, KMOE_ERR_WORKSPACE, KMOE_ERR_DEVICE = range(6)
 KMOE_F32, KMOE_BF16, KMOE_E4M3_B128 = 0, 1, 2
 
-EXPORTS = ["moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
+EXPORTS = ["moe_workspace_size", "moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn",
            "moe_combine", "moe_forward", "moe_device_status", "moe_last_error", "moe_abi_version"]
 
 
@@ -52,14 +52,15 @@ def load(path: str | None = None):
     lib.moe_abi_version.restype = i
     lib.moe_router_topk.argtypes = [vp, i, vp, vp, i, i, i, i, vp, vp, vp, vp, sz, vp]
     lib.moe_permute.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, sz, vp]
+    lib.moe_permute_noalloc.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp]
     lib.moe_grouped_ffn.argtypes = [vp, i, i, i, i, i, i, vp, vp, ctypes.POINTER(Experts),
                                     ctypes.POINTER(Experts), vp, vp, vp, sz, vp]
     lib.moe_combine.argtypes = [vp, vp, i, vp, vp, i, i, i, vp, i, vp]
     lib.moe_forward.argtypes = [vp, i, i, i, i, i, i, vp, vp, ctypes.POINTER(Experts),
                                 ctypes.POINTER(Experts), vp, i, vp, vp, vp, vp, sz, vp]
     lib.moe_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
-    for f in ("moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward",
-              "moe_device_status"):
+    for f in ("moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn", "moe_combine",
+              "moe_forward", "moe_device_status"):
         getattr(lib, f).restype = i
     if lib.moe_abi_version() != 1:
         raise RuntimeError("libkmoe ABI version mismatch")
@@ -144,6 +145,23 @@ def moe_permute(topk_idx, E, ws=None, stream=None):
         ws = torch.empty(max(((N + 255) // 256) * E * 4, 16), dtype=torch.uint8, device=dev)
     _check(load().moe_permute(_ptr(topk_idx), N, K, E, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
                               _ptr(ws), ws.numel(), _stream(stream)))
+    return counts, offsets, perm[: N * K], inv
+
+
+def moe_permute_noalloc(topk_idx, E, counts=None, offsets=None, perm=None, inv=None, stream=None):
+    """moe_permute for callers that cannot hand the library a workspace.
+
+    The library keeps the scratch in its own fixed 1 MiB device array, so the
+    C call allocates nothing; the caller passes every output buffer (any left
+    as None is allocated here by torch, for convenience in tests)."""
+    N, K = topk_idx.shape
+    dev = topk_idx.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev) if counts is None else counts
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev) if offsets is None else offsets
+    perm = torch.empty(max(N * K, 1), dtype=torch.int32, device=dev) if perm is None else perm
+    inv = torch.empty((N, K), dtype=torch.int32, device=dev) if inv is None else inv
+    _check(load().moe_permute_noalloc(_ptr(topk_idx), N, K, E, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
+                                      _stream(stream)))
     return counts, offsets, perm[: N * K], inv
 
 

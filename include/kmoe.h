@@ -119,6 +119,29 @@ kmoe_status moe_permute(const int32_t *topk_idx, int N, int K, int E,
                         int32_t *inv_pos, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * moe_permute without a workspace, for callers that cannot allocate device
+ * memory: for example an engine that has already given almost all of the
+ * GPU's memory to a fixed pool and makes no cudaMalloc calls while serving,
+ * or a host program that loads this library as a plugin and offers it no
+ * allocator. The pages have no counterpart of this call; it exists only for
+ * such callers. Outputs, layout and results are those of moe_permute
+ * (bit-identical). The per-chunk histograms live in a fixed array owned by
+ * the library in device memory: 1 MiB (262144 int32) on every GPU that loads
+ * the library, held until the process exits. Sizes needing more than that,
+ * ceil(N / 256) * E > 262144 (e.g. N > 65536 at E = 1024), are rejected with
+ * KMOE_ERR_UNSUPPORTED. The first call on a device looks up the array's
+ * device address (once per device, with that device current); make that
+ * first call before any stream capture. All calls on a GPU share the array:
+ * calls whose kernels may overlap on the GPU (different streams without
+ * ordering) race and give wrong results, so order them on one stream. The
+ * array keeps the last call's contents; each call overwrites every entry it
+ * reads, so no clearing is needed. No allocation is made by this call.
+ */
+kmoe_status moe_permute_noalloc(const int32_t *topk_idx, int N, int K, int E,
+                                int32_t *counts, int32_t *offsets, int32_t *perm_token,
+                                int32_t *inv_pos, void *stream);
+
+/*
  * Grouped expert FFN (routing section, last paragraph: each routed or
  * shared expert is a SwiGLU MLP):
  *   y_perm[p]   = F_e(x[perm_token[p]])  for offsets[e] <= p < offsets[e+1]
