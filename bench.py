@@ -231,11 +231,19 @@ def barrier(world):
 
 
 def all_max(v, world):
+    """Max of a per-rank value over all ranks (NCCL on GPUs, gloo on CPU)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tokens_per_s(tokens_per_rank, world, ms_max):
+    """Replicas: every rank processes its own tokens; the job's throughput is all
+    ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (ms_max / 1e3)
 
 
 # --------------------------------------------------------------- CPU oracle
@@ -289,7 +297,7 @@ def main():
 
     if rank == 0:
         ms = r["ms_per_step"]
-        value = dec.N * world / (ms / 1e3)
+        value = whole_job_tokens_per_s(dec.N, world, ms)
         alg = r["alg"]
         ffn_gbs = alg["ffn_bytes"] / (r["ffn_ms"] / 1e3) / 1e9
         layer_gbs = alg["layer_bytes"] / (ms / 1e3) / 1e9

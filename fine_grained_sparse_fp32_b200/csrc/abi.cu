@@ -100,6 +100,7 @@ struct Layout {
     int32_t *idx;
     float *w;
     int32_t *counts, *offsets, *perm, *inv, *hist;
+    __nv_bfloat16 *w_split;
     void *h, *y_perm, *y_shared;
     size_t bytes;
 };
@@ -119,6 +120,7 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype)
     L.perm = c.take<int32_t>((size_t)N * K);
     L.inv = c.take<int32_t>((size_t)N * K);
     L.hist = reinterpret_cast<int32_t *>(c.take<char>(permute_ws_bytes(N, E)));
+    L.w_split = c.take<__nv_bfloat16>(router_tc_ws_bytes(d, E) / sizeof(__nv_bfloat16));
     L.h = c.take<char>(R * I * ab);
     L.y_perm = c.take<char>((size_t)N * K * d * ab);
     L.y_shared = c.take<char>((size_t)N * d * ab);
@@ -144,11 +146,13 @@ static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int 
 
 static kmoe_status clear_status(int *status, cudaStream_t st)
 {
-    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return check_launch("status memset");
+    // status word, tickets and counters of this call's kernels
+    if (cudaMemsetAsync(status, 0, 64, st) != cudaSuccess) return check_launch("status memset");
     return KMOE_OK;
 }
 
 constexpr size_t kStatusBytes = 256;
+constexpr int kFusedRouteTokens = 256;   // routing, top-K and dispatch in one launch up to here
 
 }  // namespace kmoe
 
@@ -183,14 +187,26 @@ kmoe_status moe_router_topk(const void *x, int x_dtype, const float *w_router, c
     KMOE_TRY(check_ptr(topk_idx, "topk_idx"));
     KMOE_TRY(check_ptr(topk_w, "topk_w"));
     KMOE_TRY(check_ptr(logits, "logits", true));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    KMOE_TRY(check_ptr(ws, "ws", logits != nullptr));
+    // workspace: [logits if not supplied][status 256 B][three BF16 weight terms]
+    size_t used = 0;
     if (!logits) {
-        KMOE_TRY(check_ptr(ws, "ws"));
         if (ws_bytes < (size_t)N * E * sizeof(float))
             return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, (size_t)N * E * sizeof(float));
         logits = static_cast<float *>(ws);
+        used = ((size_t)N * E * sizeof(float) + 255) & ~size_t(255);
     }
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, logits, st));
+    const size_t tc_need = used + kStatusBytes + router_tc_ws_bytes(d, E);
+    if (x_dtype == KMOE_BF16 && N >= kTcRouterTokens && ws && ws_bytes >= tc_need) {
+        int *status = reinterpret_cast<int *>(static_cast<char *>(ws) + used);
+        KMOE_TRY(clear_status(status, st));
+        KMOE_TRY(launch_router_tc(static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E,
+                                  reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<char *>(status) + kStatusBytes),
+                                  logits, status, st));
+    } else {
+        KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, logits, st));
+    }
     return launch_topk(logits, bias, N, E, K, topk_idx, topk_w, st);
 }
 
@@ -302,9 +318,18 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
     float *w = topk_w_out ? topk_w_out : L.w;
     int32_t *counts = counts_out ? counts_out : L.counts;
     KMOE_TRY(clear_status(L.status, st));
-    KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, L.logits, st));
-    KMOE_TRY(launch_topk(L.logits, bias, N, E, K, idx, w, st));
-    KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st));
+    if (N <= kFusedRouteTokens) {
+        KMOE_TRY(launch_route_small(x, x_dtype, w_router, bias, N, d, E, K, L.logits, idx, w, counts, L.offsets,
+                                    L.perm, L.inv, L.status, st));
+    } else {
+        if (x_dtype == KMOE_BF16 && N >= kTcRouterTokens)
+            KMOE_TRY(launch_router_tc(static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E, L.w_split, L.logits,
+                                      L.status, st));
+        else
+            KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, L.logits, st));
+        KMOE_TRY(launch_topk(L.logits, bias, N, E, K, idx, w, st));
+        KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st));
+    }
     const ExpertPtrs r = ptrs(routed);
     ExpertPtrs s{};
     if (shared) s = ptrs(shared);

@@ -44,16 +44,26 @@ combine_kernel(const YI *__restrict__ y_perm, const YI *__restrict__ y_shared,
     const int t = blockIdx.x;
     const int c = (blockIdx.y * kCombineThreads + threadIdx.x) * 8;
     if (c >= d) return;
+    // all K + 1 row loads are issued before the first FMA (K <= 8)
+    float g[8], v[8][8];
+    int p[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        if (k < K) {
+            g[k] = w[(size_t)t * K + k];
+            p[k] = inv[(size_t)t * K + k];
+        }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        if (k < K) load_vec8(y_perm + (size_t)p[k] * d + c, v[k]);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (y_shared) load_vec8(y_shared + (size_t)t * d + c, acc);
-    for (int k = 0; k < K; ++k) {
-        const float g = w[(size_t)t * K + k];
-        const int p = inv[(size_t)t * K + k];
-        float v[8];
-        load_vec8(y_perm + (size_t)p * d + c, v);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] = fmaf(g, v[q], acc[q]);
-    }
+    for (int k = 0; k < 8; ++k)
+        if (k < K) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = fmaf(g[k], v[k][q], acc[q]);
+        }
     store8(y + (size_t)t * d + c, acc);
 }
 

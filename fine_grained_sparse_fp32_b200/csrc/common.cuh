@@ -117,6 +117,19 @@ kmoe_status launch_router_logits(const void *x, int x_dtype, const float *w_rout
 kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, int K,
                         int32_t *idx, float *w, cudaStream_t st);
 
+// Router + top-K + permutation in one launch for N <= 256 (status[4] is a
+// ticket that must be zero before the launch).
+kmoe_status launch_route_small(const void *x, int x_dtype, const float *w_router, const float *bias, int N,
+                               int d, int E, int K, float *logits, int32_t *idx, float *w, int32_t *counts,
+                               int32_t *offsets, int32_t *perm, int32_t *inv, int *status, cudaStream_t st);
+
+// Tensor-core FP32 router (x in BF16): W_r split into three BF16 terms in
+// `w_split` (router_tc_ws_bytes), logits [N, E] written out.
+size_t router_tc_ws_bytes(int d, int E);
+kmoe_status launch_router_tc(const __nv_bfloat16 *x, const float *w_router, int N, int d, int E,
+                             __nv_bfloat16 *w_split, float *logits, int *err, cudaStream_t st);
+constexpr int kTcRouterTokens = 512;
+
 size_t permute_ws_bytes(int N, int E);
 kmoe_status launch_permute(const int32_t *idx, int N, int K, int E, int32_t *counts,
                            int32_t *offsets, int32_t *perm, int32_t *inv, int32_t *hist,

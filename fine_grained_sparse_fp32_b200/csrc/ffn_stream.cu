@@ -4,14 +4,23 @@
 // expert is a SwiGLU MLP, two d -> I projections combined as SiLU(gate) * up,
 // then an I -> d projection, no biases. At decode a routed expert sees one or
 // two tokens, so the work is a weight-bandwidth-bound GEMV: every weight is
-// read from HBM exactly once and used for the few rows of its expert. The
-// kernels below stream each expert's rows with 16-byte loads (FP32, BF16 or
-// E4M3 + FP32 block scale) and keep the token rows in shared memory.
+// read from HBM once and used for the few rows of its expert. Tensor cores
+// would not help here; what matters is keeping enough bytes in flight.
 //
 // Row space: dispatched rows 0 .. N*K-1 belong to routed experts (group e
 // owns rows offsets[e] .. offsets[e+1]-1, token perm_token[row]); rows
 // N*K .. N*K+N-1 belong to the shared expert (group E, token row - N*K).
 // H (the SwiGLU intermediate) is [N*K + N, I] in that row space.
+//
+// Work decomposition: a unit is (expert, chunk of up to MT rows, slice of
+// output features). Every CTA builds the same prefix over the non-empty
+// experts in shared memory and takes units round-robin from that compacted
+// list, so active work is spread evenly over the grid whatever the routing.
+// Units of one (expert, slice) with several row chunks are adjacent, so
+// their repeated weight reads are served by L2. Each lane streams 16-byte
+// vectors (FP32, BF16, or E4M3 with its FP32 block scale) with two column
+// blocks in flight, token rows sit in shared memory as FP32, and dot
+// products end in warp reductions.
 #include "common.cuh"
 
 #include <algorithm>
@@ -20,7 +29,7 @@ namespace kmoe {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMT = 8;               // token rows per pass over the weights
+constexpr int kMaxGroupsS = 1025;
 
 __device__ __forceinline__ uint4 ld_stream(const void *p)
 {
@@ -31,221 +40,278 @@ __device__ __forceinline__ uint4 ld_stream(const void *p)
     return r;
 }
 
-struct Group {
-    int row0, rows;
+// Groups are visited in the order [shared, 0, 1, ..., E-1].
+struct GroupView {
+    int g, row0, rows;
     bool shared;
 };
 
-__device__ __forceinline__ Group group_of(int g, int N, int K, int E, const int32_t *offsets)
+__device__ __forceinline__ GroupView group_at(int ord, int N, int K, int E, bool has_shared,
+                                              const int32_t *offsets)
 {
-    if (g < E) return {offsets[g], offsets[g + 1] - offsets[g], false};
-    return {N * K, N, true};
+    if (has_shared && ord == 0) return {E, N * K, N, true};
+    const int g = ord - (has_shared ? 1 : 0);
+    return {g, offsets[g], offsets[g + 1] - offsets[g], false};
 }
 
-__device__ __forceinline__ int token_of(const Group &G, int row, int N, int K, const int32_t *perm)
+// unit prefix over groups: pre[o] = sum over earlier groups of chunks * S.
+template <int MT>
+__device__ void build_unit_prefix(int *pre, int n_ord, int S, int N, int K, int E, bool has_shared,
+                                  const int32_t *offsets)
+{
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    const int per = (n_ord + 31) / 32;
+    const int o0 = lane * per;
+    int sum = 0;
+    for (int i = 0; i < per; ++i) {
+        const int o = o0 + i;
+        if (o < n_ord) sum += (group_at(o, N, K, E, has_shared, offsets).rows + MT - 1) / MT * S;
+    }
+    int incl = sum;
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, s);
+        if (lane >= s) incl += v;
+    }
+    int run = incl - sum;
+    for (int i = 0; i < per; ++i) {
+        const int o = o0 + i;
+        if (o < n_ord) {
+            pre[o] = run;
+            run += (group_at(o, N, K, E, has_shared, offsets).rows + MT - 1) / MT * S;
+        }
+    }
+    if (lane == 31) pre[n_ord] = incl;
+}
+
+struct Unit {
+    GroupView G;
+    int m0, mc, slice;
+};
+
+template <int MT>
+__device__ __forceinline__ Unit decode_unit(int u, const int *pre, int n_ord, int S, int N, int K, int E,
+                                            bool has_shared, const int32_t *offsets)
+{
+    int lo = 1, hi = n_ord;      // smallest j with pre[j] > u
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (pre[mid] > u) hi = mid;
+        else lo = mid + 1;
+    }
+    Unit U;
+    U.G = group_at(lo - 1, N, K, E, has_shared, offsets);
+    const int chunks = (U.G.rows + MT - 1) / MT;
+    const int local = u - pre[lo - 1];
+    U.slice = local / chunks;
+    const int c = local - U.slice * chunks;
+    U.m0 = c * MT;
+    U.mc = min(MT, U.G.rows - U.m0);
+    return U;
+}
+
+__device__ __forceinline__ int token_of(const GroupView &G, int row, int N, int K, const int32_t *perm)
 {
     return G.shared ? row - N * K : perm[row];
 }
 
-template <class WT> struct WBytes { static constexpr int v = sizeof(WT); };
-
 // ------------------------------------------------------------------ gate/up
-template <class WT, class HT, int MT>
-__device__ __forceinline__ void up_tile(const float *xs, int d, int I, const WT *wg, const WT *wu,
-                                        const float *sg, const float *su, int f0, int mc,
-                                        HT *H, int row0)
-{
-    constexpr int VEC = WVec<WT>::VEC;
-    constexpr int F = 32 / VEC;                     // features per warp
-    const int lane = threadIdx.x & 31;
-    const int cb = d / 128;
-    float ag[F][MT], au[F][MT];
-#pragma unroll
-    for (int f = 0; f < F; ++f)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) ag[f][m] = au[f][m] = 0.f;
+// Features per warp: enough 16-byte loads per column block to cover 32
+// weights per lane and matrix (BF16: 2 features, E4M3: 1, FP32: 4).
+template <class WT> struct UpF { static constexpr int v = 16 / WVec<WT>::VEC > 0 ? 16 / WVec<WT>::VEC : 1; };
 
-    for (int j = lane * VEC; j < d; j += 32 * VEC) {
-        uint4 rg[F], ru[F];
-#pragma unroll
-        for (int f = 0; f < F; ++f) {
-            rg[f] = ld_stream(wg + (size_t)(f0 + f) * d + j);
-            ru[f] = ld_stream(wu + (size_t)(f0 + f) * d + j);
-        }
-#pragma unroll
-        for (int f = 0; f < F; ++f) {
-            float vg[VEC], vu[VEC];
-            float s_g = 1.f, s_u = 1.f;
-            if (sg) {
-                const int sidx = ((f0 + f) / 128) * cb + j / 128;
-                s_g = sg[sidx];
-                s_u = su[sidx];
-            }
-            WVec<WT>::cvt(rg[f], vg, s_g);
-            WVec<WT>::cvt(ru[f], vu, s_u);
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-#pragma unroll
-                for (int q = 0; q < VEC; q += 4) {
-                    const float4 xv = *reinterpret_cast<const float4 *>(xs + m * d + j + q);
-                    ag[f][m] = fmaf(vg[q], xv.x, ag[f][m]);
-                    ag[f][m] = fmaf(vg[q + 1], xv.y, ag[f][m]);
-                    ag[f][m] = fmaf(vg[q + 2], xv.z, ag[f][m]);
-                    ag[f][m] = fmaf(vg[q + 3], xv.w, ag[f][m]);
-                    au[f][m] = fmaf(vu[q], xv.x, au[f][m]);
-                    au[f][m] = fmaf(vu[q + 1], xv.y, au[f][m]);
-                    au[f][m] = fmaf(vu[q + 2], xv.z, au[f][m]);
-                    au[f][m] = fmaf(vu[q + 3], xv.w, au[f][m]);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int f = 0; f < F; ++f)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            const float a = warp_sum(ag[f][m]);
-            const float b = warp_sum(au[f][m]);
-            if (lane == 0 && m < mc) store_val(H + (size_t)(row0 + m) * I + f0 + f, a * sigmoidf_(a) * b);
-        }
-}
-
-template <class WT, class XT, class HT>
+template <class WT, class XT, class HT, int MT>
 __global__ void __launch_bounds__(kThreads)
 ffn_up_stream_kernel(const XT *__restrict__ x, int N, int d, int I, int E, int K,
                      const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
-                     ExpertPtrs routed, ExpertPtrs shared, int groups, HT *__restrict__ H)
+                     ExpertPtrs routed, ExpertPtrs shared, int has_shared, HT *__restrict__ H)
 {
-    constexpr int F = 32 / WVec<WT>::VEC;
+    constexpr int VEC = WVec<WT>::VEC;
+    constexpr int F = UpF<WT>::v;                   // features per warp
     constexpr int FS = F * kWarps;                  // features per unit
+    __shared__ int pre[kMaxGroupsS + 1];
     extern __shared__ float4 smem_f4[];
-    float *xs = reinterpret_cast<float *>(smem_f4); // [kMT][d]
+    float *xs = reinterpret_cast<float *>(smem_f4); // [MT][d]
     const int S = I / FS;
-    const int warp = threadIdx.x >> 5;
+    const int n_ord = E + (has_shared ? 1 : 0);
+    build_unit_prefix<MT>(pre, n_ord, S, N, K, E, has_shared, offsets);
+    __syncthreads();
+    const int total = pre[n_ord];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t mat = (size_t)I * d;
     const int sb = (I / 128) * (d / 128);
-    for (int u = blockIdx.x; u < groups * S; u += gridDim.x) {
-        const int g = u / S, slice = u - (u / S) * S;
-        const Group G = group_of(g, N, K, E, offsets);
-        if (G.rows == 0) continue;
-        const ExpertPtrs &P = G.shared ? shared : routed;
-        const size_t ge = G.shared ? 0 : (size_t)g;
-        const WT *wg = static_cast<const WT *>(P.wg) + ge * mat;
-        const WT *wu = static_cast<const WT *>(P.wu) + ge * mat;
+    const int cb = d / 128;
+
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        const Unit U = decode_unit<MT>(u, pre, n_ord, S, N, K, E, has_shared, offsets);
+        const ExpertPtrs &P = U.G.shared ? shared : routed;
+        const size_t ge = U.G.shared ? 0 : (size_t)U.G.g;
+        const int f0 = U.slice * FS + warp * F;
+        const WT *wg = static_cast<const WT *>(P.wg) + ge * mat + (size_t)f0 * d;
+        const WT *wu = static_cast<const WT *>(P.wu) + ge * mat + (size_t)f0 * d;
         const float *sg = P.sg ? P.sg + ge * sb : nullptr;
         const float *su = P.su ? P.su + ge * sb : nullptr;
-        const int f0 = slice * FS + warp * F;
-        for (int m0 = 0; m0 < G.rows; m0 += kMT) {
-            const int mc = min(kMT, G.rows - m0);
-            const int mt = mc <= 1 ? 1 : mc <= 2 ? 2 : mc <= 4 ? 4 : 8;
-            __syncthreads();
-            const int vpr = d / 8;
-            for (int i = threadIdx.x; i < mt * vpr; i += kThreads) {
-                const int m = i / vpr, c = (i - m * vpr) * 8;
-                float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                if (m < mc) load8(x + (size_t)token_of(G, G.row0 + m0 + m, N, K, perm) * d + c, v);
-                float4 *dst = reinterpret_cast<float4 *>(xs + m * d + c);
-                dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-                dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-            }
-            __syncthreads();
-            const int r0 = G.row0 + m0;
-            switch (mt) {
-            case 1: up_tile<WT, HT, 1>(xs, d, I, wg, wu, sg, su, f0, mc, H, r0); break;
-            case 2: up_tile<WT, HT, 2>(xs, d, I, wg, wu, sg, su, f0, mc, H, r0); break;
-            case 4: up_tile<WT, HT, 4>(xs, d, I, wg, wu, sg, su, f0, mc, H, r0); break;
-            default: up_tile<WT, HT, 8>(xs, d, I, wg, wu, sg, su, f0, mc, H, r0); break;
+
+        __syncthreads();                            // previous unit done with xs
+        const int vpr = d / 8;
+        for (int i = threadIdx.x; i < MT * vpr; i += kThreads) {
+            const int m = i / vpr, c = (i - m * vpr) * 8;
+            float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (m < U.mc) load8(x + (size_t)token_of(U.G, U.G.row0 + U.m0 + m, N, K, perm) * d + c, v);
+            float4 *dst = reinterpret_cast<float4 *>(xs + m * d + c);
+            dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+            dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+        }
+        __syncthreads();
+
+        float ag[F][MT], au[F][MT];
+#pragma unroll
+        for (int f = 0; f < F; ++f)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) ag[f][m] = au[f][m] = 0.f;
+
+        for (int j0 = lane * VEC; j0 < d; j0 += 64 * VEC) {
+            uint4 rg[2][F], ru[2][F];
+            const bool two = j0 + 32 * VEC < d;
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int f = 0; f < F; ++f) {
+                    if (b == 0 || two) {
+                        rg[b][f] = ld_stream(wg + (size_t)f * d + j0 + b * 32 * VEC);
+                        ru[b][f] = ld_stream(wu + (size_t)f * d + j0 + b * 32 * VEC);
+                    }
+                }
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                if (b == 1 && !two) break;
+                const int j = j0 + b * 32 * VEC;
+#pragma unroll
+                for (int f = 0; f < F; ++f) {
+                    float vg[VEC], vu[VEC];
+                    float s_g = 1.f, s_u = 1.f;
+                    if (sg) {
+                        const int sidx = ((f0 + f) / 128) * cb + j / 128;
+                        s_g = sg[sidx];
+                        s_u = su[sidx];
+                    }
+                    WVec<WT>::cvt(rg[b][f], vg, s_g);
+                    WVec<WT>::cvt(ru[b][f], vu, s_u);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+#pragma unroll
+                        for (int q = 0; q < VEC; q += 4) {
+                            const float4 xv = *reinterpret_cast<const float4 *>(xs + m * d + j + q);
+                            ag[f][m] = fmaf(vg[q], xv.x, ag[f][m]);
+                            ag[f][m] = fmaf(vg[q + 1], xv.y, ag[f][m]);
+                            ag[f][m] = fmaf(vg[q + 2], xv.z, ag[f][m]);
+                            ag[f][m] = fmaf(vg[q + 3], xv.w, ag[f][m]);
+                            au[f][m] = fmaf(vu[q], xv.x, au[f][m]);
+                            au[f][m] = fmaf(vu[q + 1], xv.y, au[f][m]);
+                            au[f][m] = fmaf(vu[q + 2], xv.z, au[f][m]);
+                            au[f][m] = fmaf(vu[q + 3], xv.w, au[f][m]);
+                        }
+                    }
+                }
             }
         }
+        const int r0 = U.G.row0 + U.m0;
+#pragma unroll
+        for (int f = 0; f < F; ++f)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const float a = warp_sum(ag[f][m]);
+                const float b = warp_sum(au[f][m]);
+                if (lane == 0 && m < U.mc) store_val(H + (size_t)(r0 + m) * I + f0 + f, a * sigmoidf_(a) * b);
+            }
     }
 }
 
 // --------------------------------------------------------------------- down
-constexpr int kDownRows = 8;          // output features per warp
+constexpr int kDownRows = 4;          // output features per warp
 constexpr int kDownFS = kDownRows * kWarps;
 
 template <class WT, class HT, int MT>
-__device__ __forceinline__ void down_tile(const float *hs, int d, int I, const WT *wd, const float *sd,
-                                          int j0, int mc, HT *Y)
-{
-    constexpr int VEC = WVec<WT>::VEC;
-    const int lane = threadIdx.x & 31;
-    const int ib = I / 128;
-    float acc[kDownRows][MT];
-#pragma unroll
-    for (int r = 0; r < kDownRows; ++r)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
-    for (int i = lane * VEC; i < I; i += 32 * VEC) {
-        uint4 raw[kDownRows];
-#pragma unroll
-        for (int r = 0; r < kDownRows; ++r) raw[r] = ld_stream(wd + (size_t)(j0 + r) * I + i);
-#pragma unroll
-        for (int r = 0; r < kDownRows; ++r) {
-            float w[VEC];
-            const float s = sd ? sd[((j0 + r) / 128) * ib + i / 128] : 1.f;
-            WVec<WT>::cvt(raw[r], w, s);
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-#pragma unroll
-                for (int q = 0; q < VEC; q += 4) {
-                    const float4 hv = *reinterpret_cast<const float4 *>(hs + m * I + i + q);
-                    acc[r][m] = fmaf(w[q], hv.x, acc[r][m]);
-                    acc[r][m] = fmaf(w[q + 1], hv.y, acc[r][m]);
-                    acc[r][m] = fmaf(w[q + 2], hv.z, acc[r][m]);
-                    acc[r][m] = fmaf(w[q + 3], hv.w, acc[r][m]);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < kDownRows; ++r)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            const float v = warp_sum(acc[r][m]);
-            if (lane == 0 && m < mc) store_val(Y + (size_t)m * d + j0 + r, v);
-        }
-}
-
-template <class WT, class HT>
 __global__ void __launch_bounds__(kThreads)
 ffn_down_stream_kernel(const HT *__restrict__ H, int N, int d, int I, int E, int K,
                        const int32_t *__restrict__ offsets, ExpertPtrs routed, ExpertPtrs shared,
-                       int groups, HT *__restrict__ y_perm, HT *__restrict__ y_shared)
+                       int has_shared, HT *__restrict__ y_perm, HT *__restrict__ y_shared)
 {
+    constexpr int VEC = WVec<WT>::VEC;
+    __shared__ int pre[kMaxGroupsS + 1];
     extern __shared__ float4 smem_f4[];
-    float *hs = reinterpret_cast<float *>(smem_f4);  // [kMT][I]
+    float *hs = reinterpret_cast<float *>(smem_f4);  // [MT][I]
     const int S = d / kDownFS;
-    const int warp = threadIdx.x >> 5;
+    const int n_ord = E + (has_shared ? 1 : 0);
+    build_unit_prefix<MT>(pre, n_ord, S, N, K, E, has_shared, offsets);
+    __syncthreads();
+    const int total = pre[n_ord];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t mat = (size_t)I * d;
     const int sb = (I / 128) * (d / 128);
-    for (int u = blockIdx.x; u < groups * S; u += gridDim.x) {
-        const int g = u / S, slice = u - (u / S) * S;
-        const Group G = group_of(g, N, K, E, offsets);
-        if (G.rows == 0) continue;
-        const ExpertPtrs &P = G.shared ? shared : routed;
-        const size_t ge = G.shared ? 0 : (size_t)g;
-        const WT *wd = static_cast<const WT *>(P.wd) + ge * mat;
+    const int ib = I / 128;
+
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        const Unit U = decode_unit<MT>(u, pre, n_ord, S, N, K, E, has_shared, offsets);
+        const ExpertPtrs &P = U.G.shared ? shared : routed;
+        const size_t ge = U.G.shared ? 0 : (size_t)U.G.g;
+        const int j0 = U.slice * kDownFS + warp * kDownRows;
+        const WT *wd = static_cast<const WT *>(P.wd) + ge * mat + (size_t)j0 * I;
         const float *sd = P.sd ? P.sd + ge * sb : nullptr;
-        const int j0 = slice * kDownFS + warp * kDownRows;
-        for (int m0 = 0; m0 < G.rows; m0 += kMT) {
-            const int mc = min(kMT, G.rows - m0);
-            const int mt = mc <= 1 ? 1 : mc <= 2 ? 2 : mc <= 4 ? 4 : 8;
-            __syncthreads();
-            for (int i = threadIdx.x; i < mt * I; i += kThreads) {
-                const int m = i / I, c = i - m * I;
-                hs[i] = m < mc ? to_f32(H[(size_t)(G.row0 + m0 + m) * I + c]) : 0.f;
-            }
-            __syncthreads();
-            HT *Y = G.shared ? y_shared + (size_t)(G.row0 + m0 - N * K) * d
-                             : y_perm + (size_t)(G.row0 + m0) * d;
-            switch (mt) {
-            case 1: down_tile<WT, HT, 1>(hs, d, I, wd, sd, j0, mc, Y); break;
-            case 2: down_tile<WT, HT, 2>(hs, d, I, wd, sd, j0, mc, Y); break;
-            case 4: down_tile<WT, HT, 4>(hs, d, I, wd, sd, j0, mc, Y); break;
-            default: down_tile<WT, HT, 8>(hs, d, I, wd, sd, j0, mc, Y); break;
+        const int r0 = U.G.row0 + U.m0;
+
+        __syncthreads();
+        for (int i = threadIdx.x; i < MT * I; i += kThreads) {
+            const int m = i / I, c = i - m * I;
+            hs[i] = m < U.mc ? to_f32(H[(size_t)(r0 + m) * I + c]) : 0.f;
+        }
+        __syncthreads();
+
+        float acc[kDownRows][MT];
+#pragma unroll
+        for (int r = 0; r < kDownRows; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
+        for (int i0 = lane * VEC; i0 < I; i0 += 64 * VEC) {
+            uint4 raw[2][kDownRows];
+            const bool two = i0 + 32 * VEC < I;
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int r = 0; r < kDownRows; ++r)
+                    if (b == 0 || two) raw[b][r] = ld_stream(wd + (size_t)r * I + i0 + b * 32 * VEC);
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                if (b == 1 && !two) break;
+                const int i = i0 + b * 32 * VEC;
+#pragma unroll
+                for (int r = 0; r < kDownRows; ++r) {
+                    float w[VEC];
+                    const float s = sd ? sd[((j0 + r) / 128) * ib + i / 128] : 1.f;
+                    WVec<WT>::cvt(raw[b][r], w, s);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+#pragma unroll
+                        for (int q = 0; q < VEC; q += 4) {
+                            const float4 hv = *reinterpret_cast<const float4 *>(hs + m * I + i + q);
+                            acc[r][m] = fmaf(w[q], hv.x, acc[r][m]);
+                            acc[r][m] = fmaf(w[q + 1], hv.y, acc[r][m]);
+                            acc[r][m] = fmaf(w[q + 2], hv.z, acc[r][m]);
+                            acc[r][m] = fmaf(w[q + 3], hv.w, acc[r][m]);
+                        }
+                    }
+                }
             }
         }
+        HT *Y = U.G.shared ? y_shared + (size_t)(r0 - N * K) * d : y_perm + (size_t)r0 * d;
+#pragma unroll
+        for (int r = 0; r < kDownRows; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const float v = warp_sum(acc[r][m]);
+                if (lane == 0 && m < U.mc) store_val(Y + (size_t)m * d + j0 + r, v);
+            }
     }
 }
 
@@ -262,30 +328,50 @@ static int sm_count()
     return n;
 }
 
+template <class Kern>
+static int resident_grid(Kern k, size_t smem)
+{
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    return sm_count() * per_sm;
+}
+
+template <class WT, class XT, class HT, int MT>
+static kmoe_status run_stream_mt(const XT *x, int N, int d, int I, int E, int K, const int32_t *perm,
+                                 const int32_t *offsets, const ExpertPtrs &routed, const ExpertPtrs *shared,
+                                 HT *h, HT *y_perm, HT *y_shared, cudaStream_t st)
+{
+    const int has_shared = shared ? 1 : 0;
+    const ExpertPtrs sh = shared ? *shared : ExpertPtrs{};
+    const size_t up_smem = sizeof(float) * MT * d;
+    const size_t down_smem = sizeof(float) * MT * I;
+    auto upk = ffn_up_stream_kernel<WT, XT, HT, MT>;
+    auto dnk = ffn_down_stream_kernel<WT, HT, MT>;
+    cudaFuncSetAttribute(upk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)up_smem);
+    cudaFuncSetAttribute(dnk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem);
+    upk<<<resident_grid(upk, up_smem), kThreads, up_smem, st>>>(x, N, d, I, E, K, perm, offsets, routed, sh,
+                                                                 has_shared, h);
+    kmoe_status s = check_launch("ffn_up_stream");
+    if (s != KMOE_OK) return s;
+    dnk<<<resident_grid(dnk, down_smem), kThreads, down_smem, st>>>(h, N, d, I, E, K, offsets, routed, sh,
+                                                                     has_shared, y_perm, y_shared);
+    return check_launch("ffn_down_stream");
+}
+
+// Decode batches (a routed expert sees one or two tokens) use 2-row chunks,
+// which keeps registers low enough for three CTAs per SM; larger batches use
+// 8-row chunks so that the weights are re-read from L2 fewer times.
+constexpr int kSmallBatch = 256;
+
 template <class WT, class XT, class HT>
 static kmoe_status run_stream(const XT *x, int N, int d, int I, int E, int K, const int32_t *perm,
                               const int32_t *offsets, const ExpertPtrs &routed, const ExpertPtrs *shared,
                               HT *h, HT *y_perm, HT *y_shared, cudaStream_t st)
 {
-    const int groups = E + (shared ? 1 : 0);
-    const ExpertPtrs sh = shared ? *shared : ExpertPtrs{};
-    constexpr int FS = (32 / WVec<WT>::VEC) * kWarps;
-    const int up_units = groups * (I / FS);
-    const int down_units = groups * (d / kDownFS);
-    const int cap = sm_count() * 4;
-    const size_t up_smem = sizeof(float) * kMT * d;
-    const size_t down_smem = sizeof(float) * kMT * I;
-    auto upk = ffn_up_stream_kernel<WT, XT, HT>;
-    auto dnk = ffn_down_stream_kernel<WT, HT>;
-    cudaFuncSetAttribute(upk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)up_smem);
-    cudaFuncSetAttribute(dnk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem);
-    upk<<<std::min(up_units, cap), kThreads, up_smem, st>>>(x, N, d, I, E, K, perm, offsets, routed, sh,
-                                                             groups, h);
-    kmoe_status s = check_launch("ffn_up_stream");
-    if (s != KMOE_OK) return s;
-    dnk<<<std::min(down_units, cap), kThreads, down_smem, st>>>(h, N, d, I, E, K, offsets, routed, sh,
-                                                                 groups, y_perm, y_shared);
-    return check_launch("ffn_down_stream");
+    if (N < kSmallBatch)
+        return run_stream_mt<WT, XT, HT, 2>(x, N, d, I, E, K, perm, offsets, routed, shared, h, y_perm, y_shared, st);
+    return run_stream_mt<WT, XT, HT, 8>(x, N, d, I, E, K, perm, offsets, routed, shared, h, y_perm, y_shared, st);
 }
 
 kmoe_status launch_ffn_stream(const void *x, int x_dtype, int N, int d, int I, int E, int K,
@@ -294,6 +380,7 @@ kmoe_status launch_ffn_stream(const void *x, int x_dtype, int N, int d, int I, i
                               void *h, void *y_perm, void *y_shared, cudaStream_t st)
 {
     using bf = __nv_bfloat16;
+    if (E + 1 > kMaxGroupsS) return fail(KMOE_ERR_UNSUPPORTED, "streaming FFN: too many experts");
     if (w_dtype == KMOE_F32) {
         float *H = static_cast<float *>(h), *yp = static_cast<float *>(y_perm), *ys = static_cast<float *>(y_shared);
         if (x_dtype == KMOE_F32)

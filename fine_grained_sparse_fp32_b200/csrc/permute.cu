@@ -5,36 +5,12 @@
 // sent to the experts they selected ("Inside Kolibri 1", routing section).
 // The order chosen here (expert ascending, token ascending inside an expert)
 // is a pure function of the indices, so every output is bit-exact and
-// independent of scheduling: no atomics decide a position.
-//
-// Tokens are cut into chunks of 256 (one CTA, 8 warps of 32 tokens). Inside
-// a CTA, bit `lane` of mask[w][e] says "token 32*w + lane of this chunk chose
-// expert e"; popcounts of those masks give the per-chunk histogram and the
-// rank of a token among the earlier tokens of its chunk that chose the same
-// expert. Chunk histograms are scanned per expert in chunk order.
-#include "common.cuh"
+// independent of scheduling: no atomics decide a position. Per-chunk
+// ballot masks (permute_dev.cuh) give chunk histograms and in-chunk ranks;
+// chunk histograms are scanned per expert in chunk order.
+#include "permute_dev.cuh"
 
 namespace kmoe {
-
-constexpr int kChunk = 256;
-constexpr int kChunkWarps = kChunk / 32;
-
-// Builds the 8 x E ballot masks of one chunk in shared memory.
-__device__ __forceinline__ void build_masks(const int32_t *__restrict__ idx, int N, int K, int E,
-                                            int chunk, uint32_t *mask)
-{
-    for (int i = threadIdx.x; i < kChunkWarps * E; i += blockDim.x) mask[i] = 0u;
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = chunk * kChunk + threadIdx.x;
-    if (t < N) {
-        for (int k = 0; k < K; ++k) {
-            const int e = idx[(size_t)t * K + k];
-            if ((unsigned)e < (unsigned)E) atomicOr(&mask[warp * E + e], 1u << lane);
-        }
-    }
-    __syncthreads();
-}
 
 // Pass 1: per-chunk histogram hist[c][e].
 __global__ void __launch_bounds__(kChunk)
@@ -48,34 +24,6 @@ chunk_hist_kernel(const int32_t *__restrict__ idx, int N, int K, int E, int32_t 
         for (int w = 0; w < kChunkWarps; ++w) c += __popc(mask[w * E + e]);
         hist[(size_t)blockIdx.x * E + e] = c;
     }
-}
-
-// Block-wide exclusive scan over threadIdx.x (blockDim.x a multiple of 32).
-__device__ __forceinline__ int block_exclusive_scan(int v, int *tmp)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-    }
-    if (lane == 31) tmp[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const int nw = blockDim.x >> 5;
-        int s = lane < nw ? tmp[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, s, o);
-            if (lane >= o) s += n;
-        }
-        if (lane < nw) tmp[lane] = s;   // inclusive warp totals
-    }
-    __syncthreads();
-    const int before = warp ? tmp[warp - 1] : 0;
-    __syncthreads();
-    return before + incl - v;
 }
 
 // Pass 2 (one CTA, thread e): counts, offsets, and hist[c][e] replaced by
@@ -101,14 +49,6 @@ scan_kernel(int32_t *__restrict__ hist, int chunks, int E, int32_t *__restrict__
             run += v;
         }
     }
-}
-
-// Rank of token (warp, lane) among the earlier tokens of its chunk that chose e.
-__device__ __forceinline__ int rank_in_chunk(const uint32_t *mask, int E, int e, int warp, int lane)
-{
-    int r = __popc(mask[warp * E + e] & ((1u << lane) - 1u));
-    for (int w = 0; w < warp; ++w) r += __popc(mask[w * E + e]);
-    return r;
 }
 
 // Pass 3: scatter perm_token and inv_pos.
@@ -137,43 +77,7 @@ permute_single_kernel(const int32_t *__restrict__ idx, int N, int K, int E,
                       int32_t *__restrict__ perm, int32_t *__restrict__ inv)
 {
     extern __shared__ uint32_t mask[];
-    __shared__ int tmp[32];
-    int *start = reinterpret_cast<int *>(mask + kChunkWarps * E);   // [E]
-    build_masks(idx, N, K, E, 0, mask);
-    // E may exceed the CTA: scan in rounds of blockDim.x experts.
-    int carry = 0;
-    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
-        const int e = e0 + threadIdx.x;
-        int c = 0;
-        if (e < E) {
-#pragma unroll
-            for (int w = 0; w < kChunkWarps; ++w) c += __popc(mask[w * E + e]);
-        }
-        const int excl = block_exclusive_scan(c, tmp);
-        if (e < E) {
-            counts[e] = c;
-            offsets[e] = carry + excl;
-            start[e] = carry + excl;
-        }
-        // total of this round = last thread's exclusive + its count
-        __shared__ int round_total;
-        if (threadIdx.x == blockDim.x - 1) round_total = excl + c;
-        __syncthreads();
-        carry += round_total;
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) offsets[E] = carry;
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = threadIdx.x;
-    if (t >= N) return;
-    for (int k = 0; k < K; ++k) {
-        const int e = idx[(size_t)t * K + k];
-        if ((unsigned)e >= (unsigned)E) continue;
-        const int pos = start[e] + rank_in_chunk(mask, E, e, warp, lane);
-        perm[pos] = t;
-        inv[(size_t)t * K + k] = pos;
-    }
+    permute_small_block(idx, N, K, E, counts, offsets, perm, inv, mask);
 }
 
 size_t permute_ws_bytes(int N, int E)

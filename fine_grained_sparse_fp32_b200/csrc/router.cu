@@ -6,7 +6,10 @@
 // top six experts; the mixture weights are sigmoid of the unbiased logits of
 // those six, not renormalised.
 #include "common.cuh"
+#include "permute_dev.cuh"
+#include "sm100.cuh"
 
+#include <algorithm>
 #include <cfloat>
 #include <climits>
 
@@ -87,21 +90,18 @@ kmoe_status launch_router_logits(const void *x, int x_dtype, const float *w_rout
 // One warp per token. Lane l holds the biased scores s[e] = l[e] + b[e] of
 // experts e = i*32 + l (NPL of them) in registers. K rounds: every lane finds
 // its best remaining candidate, a butterfly reduction picks the warp's best
-// by (score descending, index ascending), and its owner retires it.
+// by (score descending, index ascending), and its owner retires it. Logits
+// are read through L2 (they may come from other CTAs of the same kernel).
 template <int NPL>
-__global__ void __launch_bounds__(256)
-topk_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int N, int E, int K,
-            int32_t *__restrict__ idx, float *__restrict__ wout)
+__device__ __forceinline__ void topk_warp(const float *lr, const float *__restrict__ bias, int E, int K,
+                                          int32_t *idx_row, float *w_row)
 {
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= N) return;
-    const float *lr = logits + (size_t)t * E;
     float s[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = i * 32 + lane;
-        s[i] = e < E ? lr[e] + bias[e] : -FLT_MAX;
+        s[i] = e < E ? __ldcg(lr + e) + bias[e] : -FLT_MAX;
     }
     for (int k = 0; k < K; ++k) {
         float bv = -INFINITY;
@@ -120,10 +120,20 @@ topk_kernel(const float *__restrict__ logits, const float *__restrict__ bias, in
             if (i * 32 + lane == be) s[i] = -INFINITY;
         if (lane == 0) {   // be < E whenever K <= E and the scores are finite
             const int e = be < E ? be : E - 1;
-            idx[(size_t)t * K + k] = e;
-            wout[(size_t)t * K + k] = sigmoidf_(lr[e]);
+            idx_row[k] = e;
+            w_row[k] = sigmoidf_(__ldcg(lr + e));
         }
     }
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(256)
+topk_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int N, int E, int K,
+            int32_t *__restrict__ idx, float *__restrict__ wout)
+{
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= N) return;
+    topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, idx + (size_t)t * K, wout + (size_t)t * K);
 }
 
 kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, int K,
@@ -141,6 +151,135 @@ kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, in
     else KMOE_TOPK(32);
 #undef KMOE_TOPK
     return check_launch("topk");
+}
+
+// ------------------------------------------------ fused small-batch routing
+//
+// For N <= 256 tokens (decode) the router, the top-K selection and the
+// dispatch permutation run as one launch. Each CTA owns kRouteEPC experts:
+// the bulk-copy engine brings their FP32 router rows and the token rows into
+// shared memory, and every warp computes the logits of one token at a time.
+// The last CTA to finish (a ticket in the workspace status area, zeroed by
+// the caller before the launch) then selects the top K of every token and
+// builds the permutation, reusing its shared memory for the ballot masks.
+constexpr int kRouteEPC = 3;
+constexpr int kRouteSmemMax = 200 * 1024;
+constexpr long long kRouteWaitLimit = 1LL << 32;
+
+template <class XT, int NPL>
+__global__ void __launch_bounds__(256, 1)
+route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
+                   int N, int d, int E, int K, int chunk, int x_off, float *__restrict__ logits,
+                   int32_t *__restrict__ idx, float *__restrict__ wout, int32_t *__restrict__ counts,
+                   int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv,
+                   int *status)
+{
+    using namespace sm100;
+    extern __shared__ __align__(128) uint8_t sm_raw[];
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int last, abort_flag;
+    float *wsm = reinterpret_cast<float *>(sm_raw);
+    XT *xsm = reinterpret_cast<XT *>(sm_raw + x_off);
+    const int e0 = blockIdx.x * kRouteEPC;
+    const int ne = min(kRouteEPC, E - e0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int *ticket = status + 4;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    uint32_t phase = 0;
+    for (int c0 = 0; c0 < N; c0 += chunk) {
+        const int nt = min(chunk, N - c0);
+        if (threadIdx.x == 0) {
+            fence_proxy_async();      // earlier generic reads of xsm before the async overwrite
+            const uint32_t xbytes = (uint32_t)nt * d * sizeof(XT);
+            const uint32_t wbytes = c0 == 0 ? (uint32_t)ne * d * 4 : 0u;
+            mbar_arrive_expect_tx(&bar, xbytes + wbytes);
+            if (wbytes) bulk_load(wsm, w + (size_t)e0 * d, wbytes, &bar);
+            bulk_load(xsm, x + (size_t)c0 * d, xbytes, &bar);
+        }
+        mbar_wait(&bar, phase, &abort_flag, status, kRouteWaitLimit);
+        phase ^= 1;
+        __syncthreads();
+        if (abort_flag) break;
+        for (int t = warp; t < nt; t += 8) {
+            float acc[kRouteEPC];
+#pragma unroll
+            for (int e = 0; e < kRouteEPC; ++e) acc[e] = 0.f;
+            const XT *xr = xsm + (size_t)t * d;
+            for (int j = lane * 8; j < d; j += 256) {
+                float xv[8];
+                load8(xr + j, xv);
+#pragma unroll
+                for (int e = 0; e < kRouteEPC; ++e) {
+                    if (e < ne) {
+                        float wv[8];
+                        load8(wsm + e * d + j, wv);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) acc[e] = fmaf(xv[q], wv[q], acc[e]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < kRouteEPC; ++e) {
+                const float v = warp_sum(acc[e]);
+                if (lane == 0 && e < ne) logits[(size_t)(c0 + t) * E + e0 + e] = v;
+            }
+        }
+        __syncthreads();
+    }
+    if (abort_flag) {            // a copy never landed: let it finish (bounded) and leave
+        if (threadIdx.x == 0) mbar_wait_drain(&bar, phase ^ 1, kRouteWaitLimit);
+        return;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    for (int t = warp; t < N; t += 8)
+        topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, idx + (size_t)t * K, wout + (size_t)t * K);
+    __syncthreads();
+    permute_small_block(idx, N, K, E, counts, offsets, perm, inv, reinterpret_cast<uint32_t *>(sm_raw));
+    if (threadIdx.x == 0) *ticket = 0;
+}
+
+kmoe_status launch_route_small(const void *x, int x_dtype, const float *w_router, const float *bias, int N,
+                               int d, int E, int K, float *logits, int32_t *idx, float *w, int32_t *counts,
+                               int32_t *offsets, int32_t *perm, int32_t *inv, int *status, cudaStream_t st)
+{
+    if (N > kChunk) return fail(KMOE_ERR_UNSUPPORTED, "fused routing: N=%d > %d", N, kChunk);
+    const int xb = x_dtype == KMOE_F32 ? 4 : 2;
+    const int w_bytes = ((kRouteEPC * d * 4) + 127) / 128 * 128;
+    const int chunk = std::min(N, std::max(1, (kRouteSmemMax - w_bytes) / (d * xb)));
+    const size_t smem = std::max((size_t)w_bytes + (size_t)chunk * d * xb, (size_t)(kChunkWarps + 1) * E * 4);
+    const int grid = (E + kRouteEPC - 1) / kRouteEPC;
+    const int npl = (E + 31) / 32;
+#define KMOE_ROUTE(XT, n)                                                                                   \
+    do {                                                                                                    \
+        auto k = route_small_kernel<XT, n>;                                                                 \
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                    \
+        k<<<grid, 256, smem, st>>>(static_cast<const XT *>(x), w_router, bias, N, d, E, K, chunk, w_bytes,   \
+                                   logits, idx, w, counts, offsets, perm, inv, status);                     \
+    } while (0)
+#define KMOE_ROUTE_X(n)                                   \
+    do {                                                  \
+        if (x_dtype == KMOE_F32) KMOE_ROUTE(float, n);    \
+        else KMOE_ROUTE(__nv_bfloat16, n);                \
+    } while (0)
+    if (npl <= 2) KMOE_ROUTE_X(2);
+    else if (npl <= 4) KMOE_ROUTE_X(4);
+    else if (npl <= 8) KMOE_ROUTE_X(8);
+    else if (npl <= 12) KMOE_ROUTE_X(12);
+    else if (npl <= 16) KMOE_ROUTE_X(16);
+    else KMOE_ROUTE_X(32);
+#undef KMOE_ROUTE_X
+#undef KMOE_ROUTE
+    return check_launch("route_small");
 }
 
 }  // namespace kmoe

@@ -90,6 +90,21 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// Contiguous global -> shared copy by the bulk-copy engine (16-byte aligned
+// addresses, size a multiple of 16), completing on `bar`. Issued in pieces
+// of at most 32 KB.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    const char *s = static_cast<const char *>(src);
+    char *d = static_cast<char *>(dst);
+    for (uint32_t off = 0; off < bytes; off += 32768u) {
+        const uint32_t n = bytes - off < 32768u ? bytes - off : 32768u;
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                     ::"r"(smem_u32(d + off)), "l"(s + off), "r"(n), "r"(smem_u32(bar))
+                     : "memory");
+    }
+}
+
 __device__ __forceinline__ void prefetch_map(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");

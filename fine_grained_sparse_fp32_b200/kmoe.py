@@ -126,8 +126,9 @@ def moe_router_topk(x, w_router, bias, K, logits=None, topk_idx=None, topk_w=Non
         topk_idx = torch.empty((N, K), dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty((N, K), dtype=torch.float32, device=x.device)
-    if logits is None and ws is None:
-        ws = torch.empty(max(N * E * 4, 16), dtype=torch.uint8, device=x.device)
+    if ws is None:   # logits (if not supplied) + status + the three BF16 router terms
+        ws = torch.empty(((N * E * 4 + 255) // 256) * 256 + 256 + 3 * E * d * 2, dtype=torch.uint8,
+                         device=x.device)
     _check(load().moe_router_topk(_ptr(x), dtype_code(x.dtype), _ptr(w_router), _ptr(bias), N, d, E, K,
                                   _ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(ws),
                                   0 if ws is None else ws.numel(), _stream(stream)))

@@ -93,6 +93,13 @@ size_t moe_workspace_size(int N, int d, int E, int K, int I, int x_dtype, int w_
  * w_router device [E, d] FP32;   bias device [E] FP32
  * logits   device [N, E] FP32 output, or NULL to keep it in the workspace
  * topk_idx device [N, K] int32 output;  topk_w device [N, K] FP32 output
+ * ws       device workspace (may be NULL when logits is given). With BF16 x,
+ *          N >= 512 and a workspace of at least moe_workspace_size() bytes,
+ *          the logits run on the tensor cores: W_r is split into three BF16
+ *          terms (W1 = bf16(W), W2 = bf16(W - W1), W3 = bf16(W - W1 - W2))
+ *          whose exact products accumulate in FP32, otherwise on CUDA cores
+ *          in FP32. Its status word is read by moe_device_status on
+ *          (ws + the logits bytes rounded up to 256 when logits is NULL).
  */
 kmoe_status moe_router_topk(const void *x, int x_dtype, const float *w_router,
                             const float *bias, int N, int d, int E, int K,

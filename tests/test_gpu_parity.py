@@ -47,7 +47,7 @@ def threads():
 
 # ----------------------------------------------------------------- router
 @pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("decode", 300), ("decode", 1),
-                                    ("skew", 2048)])
+                                    ("skew", 2048), ("decode", 513), ("prefill", None)])
 def test_router_topk_matches_oracle(name, N):
     dev, host = layer_inputs(name, N)
     cfg = host["cfg"]
