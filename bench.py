@@ -111,8 +111,11 @@ def algorithmic(cfg, distinct_routed: float):
 
 
 def launches_per_step(cfg):
-    # router_logits, topk, permute (1 kernel for N <= 256, else 3), ffn_up, ffn_down, combine
-    return 2 + (1 if cfg.N <= 256 else 3) + 2 + 1
+    """Kernels of this library that one moe_forward launches (mirrors abi.cu's dispatch)."""
+    if cfg.N <= 256:
+        return 4            # fused router+top-K+permute, ffn up, ffn down, combine
+    router = 2 if (cfg.x_dtype == "bf16" and cfg.N >= 512) else 1   # split + tcgen05 router | SIMT router
+    return router + 1 + 3 + 2 + 1   # + top-K, permute (hist, scan, scatter), ffn up, ffn down, combine
 
 
 # --------------------------------------------------------------- GPU arm
@@ -271,6 +274,7 @@ def main():
     ap.add_argument("--impl", default="kmoe", choices=["kmoe", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the FP8 and skewed-routing layers")
     ap.add_argument("--cpu-tokens", type=int, default=32)
     args = ap.parse_args()
     world, rank, local = dist_env()
@@ -290,10 +294,16 @@ def main():
     dec = CONFIGS["decode"]
     r = run_config(dec, args.steps, args.warmup, rank, world, use_graph=not args.no_graph)
     pre = None
+    extras = {}
     if not args.no_prefill:
         pcfg = CONFIGS["prefill"]
         psteps = max(10, min(args.steps // 10, 200))
         pre = run_config(pcfg, psteps, max(3, args.warmup // 10), rank, world, use_graph=not args.no_graph)
+        torch.cuda.empty_cache()
+        if not args.no_extra:
+            for name, n_steps in (("fp8_decode", max(20, min(args.steps, 1000))), ("fp8_prefill", 50), ("skew", 10)):
+                extras[name] = run_config(CONFIGS[name], n_steps, 3, rank, world, use_graph=not args.no_graph)
+                torch.cuda.empty_cache()
 
     if rank == 0:
         ms = r["ms_per_step"]
@@ -332,8 +342,22 @@ def main():
                 "roofline_time_ms": max(t_hbm, t_tc) * 1e3, "bound": "hbm" if t_hbm >= t_tc else "tensor",
                 "frac": max(t_hbm, t_tc) * 1e3 / pms,
                 "tflops": palg["flops"] / (pms / 1e3) / 1e12, "tensor_frac": palg["flops"] / (pms / 1e3) / (tflops * 1e12),
-                "ffn_ms": pre["ffn_ms"], "clocks": pre["clocks"],
+                "ffn_ms": pre["ffn_ms"], "clocks": pre["clocks"], "gpu_launches_per_step": launches_per_step(pcfg),
                 "e2e": {"value": pcfg.N * world / (pre["e2e_ms"]["ms"] / 1e3), "unit": "tokens/s"},
+            }
+        for name, r_x in extras.items():
+            xcfg = CONFIGS[name]
+            xms = r_x["ms_per_step"]
+            xalg = r_x["alg"]
+            t_hbm = xalg["layer_bytes"] / (hbm * 1e9)
+            t_tc = xalg["flops"] / (tflops * 1e12)
+            line[name] = {
+                "value": whole_job_tokens_per_s(xcfg.N, world, xms), "unit": "tokens/s", "ms_per_step": xms,
+                "N": xcfg.N, "weights": xcfg.w_dtype, "distinct_experts_per_step": r_x["distinct"],
+                "roofline_time_ms": max(t_hbm, t_tc) * 1e3, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                "frac": max(t_hbm, t_tc) * 1e3 / xms, "tflops": xalg["flops"] / (xms / 1e3) / 1e12,
+                "ffn_ms": r_x["ffn_ms"], "ffn_gbs": xalg["ffn_bytes"] / (r_x["ffn_ms"] / 1e3) / 1e9,
+                "gpu_launches_per_step": launches_per_step(xcfg), "clocks": r_x["clocks"],
             }
         if world == 1:
             try:

@@ -130,7 +130,8 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype)
 
 static bool use_tc(int x_dtype, int w_dtype, int N, int d)
 {
-    return x_dtype == KMOE_BF16 && w_dtype == KMOE_BF16 && N >= kTcMinTokens && d % 256 == 0;
+    return x_dtype == KMOE_BF16 && (w_dtype == KMOE_BF16 || w_dtype == KMOE_E4M3_B128) && N >= kTcMinTokens &&
+           d % 256 == 0;
 }
 
 static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int E, int K, const int32_t *perm,
@@ -138,7 +139,7 @@ static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int 
                            void *h, void *y_perm, void *y_shared, int *status, cudaStream_t st)
 {
     if (use_tc(x_dtype, w_dtype, N, d))
-        return launch_ffn_tc(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, r, s,
+        return launch_ffn_tc(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, w_dtype, r, s,
                              static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
                              static_cast<__nv_bfloat16 *>(y_shared), status, st);
     return launch_ffn_stream(x, x_dtype, N, d, I, E, K, perm, offsets, w_dtype, r, s, h, y_perm, y_shared, st);

@@ -229,8 +229,9 @@ ffn_up_stream_kernel(const XT *__restrict__ x, int N, int d, int I, int E, int K
 }
 
 // --------------------------------------------------------------------- down
-constexpr int kDownRows = 4;          // output features per warp
-constexpr int kDownFS = kDownRows * kWarps;
+constexpr int kDownRows = 4;          // output features per warp and pass
+constexpr int kDownPasses = 4;        // passes per unit
+constexpr int kDownFS = kDownRows * kWarps * kDownPasses;   // 128 output features per unit
 
 template <class WT, class HT, int MT>
 __global__ void __launch_bounds__(kThreads)
@@ -256,8 +257,6 @@ ffn_down_stream_kernel(const HT *__restrict__ H, int N, int d, int I, int E, int
         const Unit U = decode_unit<MT>(u, pre, n_ord, S, N, K, E, has_shared, offsets);
         const ExpertPtrs &P = U.G.shared ? shared : routed;
         const size_t ge = U.G.shared ? 0 : (size_t)U.G.g;
-        const int j0 = U.slice * kDownFS + warp * kDownRows;
-        const WT *wd = static_cast<const WT *>(P.wd) + ge * mat + (size_t)j0 * I;
         const float *sd = P.sd ? P.sd + ge * sb : nullptr;
         const int r0 = U.G.row0 + U.m0;
 
@@ -267,7 +266,11 @@ ffn_down_stream_kernel(const HT *__restrict__ H, int N, int d, int I, int E, int
             hs[i] = m < U.mc ? to_f32(H[(size_t)(r0 + m) * I + c]) : 0.f;
         }
         __syncthreads();
+        HT *Y = U.G.shared ? y_shared + (size_t)(r0 - N * K) * d : y_perm + (size_t)r0 * d;
 
+        for (int pass = 0; pass < kDownPasses; ++pass) {
+        const int j0 = U.slice * kDownFS + (pass * kWarps + warp) * kDownRows;
+        const WT *wd = static_cast<const WT *>(P.wd) + ge * mat + (size_t)j0 * I;
         float acc[kDownRows][MT];
 #pragma unroll
         for (int r = 0; r < kDownRows; ++r)
@@ -304,7 +307,6 @@ ffn_down_stream_kernel(const HT *__restrict__ H, int N, int d, int I, int E, int
                 }
             }
         }
-        HT *Y = U.G.shared ? y_shared + (size_t)(r0 - N * K) * d : y_perm + (size_t)r0 * d;
 #pragma unroll
         for (int r = 0; r < kDownRows; ++r)
 #pragma unroll
@@ -312,6 +314,7 @@ ffn_down_stream_kernel(const HT *__restrict__ H, int N, int d, int I, int E, int
                 const float v = warp_sum(acc[r][m]);
                 if (lane == 0 && m < U.mc) store_val(Y + (size_t)m * d + j0 + r, v);
             }
+        }
     }
 }
 

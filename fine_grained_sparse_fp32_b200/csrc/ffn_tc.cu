@@ -22,6 +22,14 @@
 // tile overlap the MMAs of the next. Tiles are enumerated per expert as
 // (n-tile, m-tile) so that CTAs working at the same time read the same
 // weight tile and it crosses HBM once.
+//
+// E4M3 weights ("Inside Kolibri 1", FP8 section: 128 x 128 blocks, one FP32
+// scale per block) take the same kernels with four more warps: the weight
+// tile arrives by TMA as E4M3 bytes in a staging buffer, and converter warps
+// 9-12 decode it (hardware e4m3x2 -> f16x2), multiply by the FP32 scale of
+// its block, round to BF16 and write it in the swizzled layout the MMA reads.
+// Activations stay BF16, so the tensor cores see BF16 x BF16 with FP32
+// accumulation, and the weights cross HBM at one byte each.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -31,14 +39,16 @@ namespace kmoe {
 using namespace sm100;
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kStages = 4;
 constexpr int kATile = kBM * kBK * 2;        // 16 KB
 constexpr int kBTile = kBN * kBK * 2;        // 32 KB
-constexpr int kStage = kATile + kBTile;
+constexpr int kB8Tile = kBN * kBK;           // 16 KB of E4M3 staging
+constexpr int kMaxStages = 4;
+__host__ __device__ constexpr int stages_of(bool fp8) { return fp8 ? 3 : 4; }
+__host__ __device__ constexpr int stage_bytes(bool fp8) { return kATile + kBTile + (fp8 ? kB8Tile : 0); }
 constexpr int kMmaWarp = 4;
 constexpr int kProdWarp = 5;
-constexpr int kTcThreads = 9 * 32;
-constexpr int kLag = 2;                      // cp.async groups in flight before signalling
+constexpr int kConvWarp = 9;                 // E4M3 only: warps 9-12
+__host__ __device__ constexpr int threads_of(bool fp8) { return (fp8 ? 13 : 9) * 32; }
 constexpr int kMaxGroups = 1025;
 constexpr long long kWaitLimit = 1LL << 32;  // SM cycles (about 2 s)
 
@@ -55,17 +65,22 @@ struct TcArgs {
     int d, I, kblocks, n_tiles;
     __nv_bfloat16 *out0;      // up: H [R, I]; down: y_perm [N*K, d]
     __nv_bfloat16 *out1;      // down: y_shared [N, d]
+    // E4M3 block scales (up: s0 = gate, s1 = up; down: s0 = W_d), routed and shared
+    const float *s0_routed, *s1_routed, *s0_shared, *s1_shared;
     int *err;
 };
 
 struct SmemTail {
-    uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], drain;
+    uint64_t full[kMaxStages], empty[kMaxStages], b8full[kMaxStages], tfull[2], tempty[2], drain;
     uint32_t tmem_base;
     int abort;
     int pre[kMaxGroups + 1];
 };
 
-constexpr size_t kTcSmem = 1024 /*align slack*/ + (size_t)kStages * kStage + sizeof(SmemTail);
+constexpr size_t tc_smem(bool fp8)
+{
+    return 1024 /*align slack*/ + (size_t)stages_of(fp8) * stage_bytes(fp8) + sizeof(SmemTail);
+}
 
 struct Tile {
     int g, row0, rows, n0;
@@ -127,10 +142,39 @@ __device__ __forceinline__ void build_prefix(int *pre, const TcArgs &a)
     if (lane == 31) pre[a.groups] = incl;
 }
 
-template <bool kUp>
-__global__ void __launch_bounds__(kTcThreads, 1)
+// Decodes one 64-element E4M3 row of the staging tile, scales it and writes
+// it as BF16 into row r of the 128-byte-swizzled B tile.
+__device__ __forceinline__ void convert_row(const uint8_t *src, uint8_t *dst, int r, float scale)
+{
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+        const int c = (c4 + r) & 3;                  // rotate 16-byte reads across banks
+        const uint4 q = *reinterpret_cast<const uint4 *>(src + c * 16);
+        const uint32_t wds[4] = {q.x, q.y, q.z, q.w};
+        uint32_t out[8];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(wds[h] & 0xffffu), __NV_E4M3);
+            __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(wds[h] >> 16), __NV_E4M3);
+            const float2 a = __half22float2(*reinterpret_cast<__half2 *>(&lo));
+            const float2 b = __half22float2(*reinterpret_cast<__half2 *>(&hi));
+            out[2 * h] = pack_bf16x2(a.x * scale, a.y * scale);
+            out[2 * h + 1] = pack_bf16x2(b.x * scale, b.y * scale);
+        }
+        // elements c*16 .. c*16+15 = 16-byte chunks 2c and 2c+1 of the BF16 row
+        uint8_t *row = dst + r * 128;
+        *reinterpret_cast<uint4 *>(row + (((2 * c) ^ (r & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+        *reinterpret_cast<uint4 *>(row + (((2 * c + 1) ^ (r & 7)) << 4)) = make_uint4(out[4], out[5], out[6], out[7]);
+    }
+}
+
+template <bool kUp, bool kFp8>
+__global__ void __launch_bounds__(threads_of(kFp8), 1)
 ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
 {
+    constexpr int kStages = stages_of(kFp8);
+    constexpr int kStage = stage_bytes(kFp8);
+    constexpr int kLag = kStages - 1;        // cp.async groups in flight before a stage is signalled
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     SmemTail *tail = reinterpret_cast<SmemTail *>(smem + (size_t)kStages * kStage);
@@ -139,8 +183,11 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&tail->full[s], kUp ? 128 + 1 : 1);
+            // arrivals: up = 128 cp.async producers + (TMA expect_tx | 128 converters);
+            //           down = TMA expect_tx (+ 128 converters)
+            mbar_init(&tail->full[s], (kUp ? 128 : 1) + (kFp8 ? 128 : (kUp ? 1 : 0)));
             mbar_init(&tail->empty[s], 1);
+            mbar_init(&tail->b8full[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tail->tfull[b], 1);
@@ -169,10 +216,43 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
     const int total = tail->pre[a.groups] * a.n_tiles;
     const uint32_t tmem = tail->tmem_base;
 
-    if (warp >= kProdWarp) {
+    if (kFp8 && warp >= kConvWarp) {
+        // ------------------------------------------- E4M3 -> BF16 converters
+        const int q = threadIdx.x - kConvWarp * 32;          // rows q and q + 128 of the B tile
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile T = decode_tile(t, tail->pre, a, bn);
+            const size_t ge = T.shared ? 0 : (size_t)T.g;
+            const float *s0 = T.shared ? a.s0_shared : a.s0_routed;
+            const float *s1 = T.shared ? a.s1_shared : a.s1_routed;
+            for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                const int s = it % kStages;
+                if (!mbar_wait(&tail->b8full[s], (it / kStages) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                uint8_t *Bs = smem + (size_t)s * kStage + kATile;
+                const uint8_t *B8 = Bs + kBTile;
+                float sc0, sc1;
+                if (kUp) {     // gate rows n0.., up rows n0..; blocks [G, I/128, d/128]
+                    const size_t si = (ge * (a.I / 128) + T.n0 / 128) * (a.d / 128) + (kb * kBK) / 128;
+                    sc0 = s0[si];
+                    sc1 = s1[si];
+                } else {       // W_d rows n0.. and n0+128..; blocks [G, d/128, I/128]
+                    const size_t si = (ge * (a.d / 128) + T.n0 / 128) * (a.I / 128) + (kb * kBK) / 128;
+                    sc0 = s0[si];
+                    sc1 = s0[si + a.I / 128];
+                }
+                convert_row(B8 + q * kBK, Bs, q, sc0);
+                convert_row(B8 + (q + 128) * kBK, Bs, q + 128, sc1);
+                fence_proxy_async();
+                mbar_arrive(&tail->full[s]);
+            }
+        }
+    } else if (warp >= kProdWarp) {
         // ------------------------------------------------------- producers
         const int p = threadIdx.x - kProdWarp * 32;
         const bool leader = p == 0;
+        const uint64_t pol_w = policy_evict_first();   // weight tiles: streamed
+        const uint64_t pol_a = policy_evict_last();    // token rows / H rows: reused across n-tiles
         uint32_t it = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -189,17 +269,25 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                 if (!mbar_wait(&tail->empty[s], ph ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
                 uint8_t *As = smem + (size_t)s * kStage;
                 uint8_t *Bs = As + kATile;
+                if (kFp8 && leader) {       // E4M3 weight rows into the staging buffer
+                    uint8_t *B8 = Bs + kBTile;
+                    const int r0 = kUp ? gi * a.I + T.n0 : gi * a.d + T.n0;
+                    mbar_arrive_expect_tx(&tail->b8full[s], kB8Tile);
+                    tma_load_2d_hint(B8, m0, &tail->b8full[s], kb * kBK, r0, pol_w);
+                    tma_load_2d_hint(B8 + kB8Tile / 2, kUp ? m1 : m0, &tail->b8full[s], kb * kBK,
+                                     kUp ? r0 : r0 + kBN / 2, pol_w);
+                }
                 if (kUp) {
-                    if (leader) {
+                    if (leader && !kFp8) {
                         mbar_arrive_expect_tx(&tail->full[s], kBTile);
-                        tma_load_2d(Bs, m0, &tail->full[s], kb * kBK, gi * a.I + T.n0);
-                        tma_load_2d(Bs + kBTile / 2, m1, &tail->full[s], kb * kBK, gi * a.I + T.n0);
+                        tma_load_2d_hint(Bs, m0, &tail->full[s], kb * kBK, gi * a.I + T.n0, pol_w);
+                        tma_load_2d_hint(Bs + kBTile / 2, m1, &tail->full[s], kb * kBK, gi * a.I + T.n0, pol_w);
                     }
                     const uint32_t dst = smem_u32(As) + p * 128;
                     const __nv_bfloat16 *s_row = src + kb * kBK;
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
-                        cp_async16(dst + ((c ^ (p & 7)) << 4), s_row + c * 8, tok >= 0 ? 16u : 0u);
+                        cp_async16_hint(dst + ((c ^ (p & 7)) << 4), s_row + c * 8, tok >= 0 ? 16u : 0u, pol_a);
                     cp_async_commit();
                     if (it >= kLag) {
                         cp_async_wait<kLag>();
@@ -207,10 +295,13 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                         mbar_arrive(&tail->full[(it - kLag) % kStages]);
                     }
                 } else if (leader) {
-                    mbar_arrive_expect_tx(&tail->full[s], kATile + kBTile);
-                    tma_load_2d(As, &maps.a, &tail->full[s], kb * kBK, T.row0);
-                    tma_load_2d(Bs, m0, &tail->full[s], kb * kBK, gi * a.d + T.n0);
-                    tma_load_2d(Bs + kBTile / 2, m0, &tail->full[s], kb * kBK, gi * a.d + T.n0 + kBN / 2);
+                    mbar_arrive_expect_tx(&tail->full[s], kATile + (kFp8 ? 0 : kBTile));
+                    tma_load_2d_hint(As, &maps.a, &tail->full[s], kb * kBK, T.row0, pol_a);
+                    if (!kFp8) {
+                        tma_load_2d_hint(Bs, m0, &tail->full[s], kb * kBK, gi * a.d + T.n0, pol_w);
+                        tma_load_2d_hint(Bs + kBTile / 2, m0, &tail->full[s], kb * kBK, gi * a.d + T.n0 + kBN / 2,
+                                         pol_w);
+                    }
                 }
             }
         }
@@ -220,8 +311,10 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             for (uint32_t j = it > (uint32_t)kLag ? it - kLag : 0; j < it; ++j) mbar_arrive(&tail->full[j % kStages]);
         }
         if (!ok && leader) {   // let in-flight TMA loads land before the CTA exits
-            for (uint32_t j = it > (uint32_t)kStages ? it - kStages : 0; j < it; ++j)
-                mbar_wait_drain(&tail->full[j % kStages], (j / kStages) & 1, kWaitLimit);
+            for (uint32_t j = it > (uint32_t)kStages ? it - kStages : 0; j < it; ++j) {
+                if (kFp8) mbar_wait_drain(&tail->b8full[j % kStages], (j / kStages) & 1, kWaitLimit);
+                if (!kFp8 || !kUp) mbar_wait_drain(&tail->full[j % kStages], (j / kStages) & 1, kWaitLimit);
+            }
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA
@@ -344,6 +437,21 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t c
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D byte map (E4M3 weights) over [rows, cols], box 128 rows x 64 bytes, no
+// swizzle (the converter warps read it with plain shared-memory loads).
+static bool make_map_u8(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {kBK, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int sm_count_tc()
 {
     static int n = 0;
@@ -356,21 +464,54 @@ static int sm_count_tc()
     return n;
 }
 
+template <bool kFp8>
+static kmoe_status run_tc(const TcMaps &up, const TcMaps &dn, TcArgs a, int d, int I, __nv_bfloat16 *h,
+                          __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, const ExpertPtrs &routed,
+                          const ExpertPtrs &sh, cudaStream_t st)
+{
+    const int grid = sm_count_tc();
+    constexpr size_t smem = tc_smem(kFp8);
+    cudaFuncSetAttribute(ffn_tc_kernel<true, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(ffn_tc_kernel<false, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    a.kblocks = d / kBK;
+    a.n_tiles = I / (kBN / 2);
+    a.out0 = h;
+    a.s0_routed = routed.sg;
+    a.s1_routed = routed.su;
+    a.s0_shared = sh.sg;
+    a.s1_shared = sh.su;
+    ffn_tc_kernel<true, kFp8><<<grid, threads_of(kFp8), smem, st>>>(up, a);
+    kmoe_status s = check_launch("ffn_up_tc");
+    if (s != KMOE_OK) return s;
+    a.kblocks = I / kBK;
+    a.n_tiles = d / kBN;
+    a.out0 = y_perm;
+    a.out1 = y_shared;
+    a.s0_routed = routed.sd;
+    a.s1_routed = nullptr;
+    a.s0_shared = sh.sd;
+    a.s1_shared = nullptr;
+    ffn_tc_kernel<false, kFp8><<<grid, threads_of(kFp8), smem, st>>>(dn, a);
+    return check_launch("ffn_down_tc");
+}
+
 kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
-                          const int32_t *offsets, const ExpertPtrs &routed, const ExpertPtrs *shared,
+                          const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
                           __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err,
                           cudaStream_t st)
 {
     if (E + 1 > kMaxGroups) return fail(KMOE_ERR_UNSUPPORTED, "tensor-core FFN: too many experts");
+    const bool fp8 = w_dtype == KMOE_E4M3_B128;
     const ExpertPtrs sh = shared ? *shared : routed;    // unused maps still need a valid base
     const long long R = (long long)N * K + N;
+    auto wmap = [&](CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols) {
+        return fp8 ? make_map_u8(m, base, rows, cols) : make_map(m, base, rows, cols);
+    };
     TcMaps up{}, dn{};
-    bool ok = make_map(&up.b0_routed, routed.wg, (uint64_t)E * I, d) &&
-              make_map(&up.b1_routed, routed.wu, (uint64_t)E * I, d) &&
-              make_map(&up.b0_shared, sh.wg, I, d) && make_map(&up.b1_shared, sh.wu, I, d) &&
-              make_map(&up.a, h, R, I) &&
-              make_map(&dn.b0_routed, routed.wd, (uint64_t)E * d, I) && make_map(&dn.b0_shared, sh.wd, d, I) &&
-              make_map(&dn.b1_routed, routed.wd, (uint64_t)E * d, I) && make_map(&dn.b1_shared, sh.wd, d, I) &&
+    bool ok = wmap(&up.b0_routed, routed.wg, (uint64_t)E * I, d) && wmap(&up.b1_routed, routed.wu, (uint64_t)E * I, d) &&
+              wmap(&up.b0_shared, sh.wg, I, d) && wmap(&up.b1_shared, sh.wu, I, d) && make_map(&up.a, h, R, I) &&
+              wmap(&dn.b0_routed, routed.wd, (uint64_t)E * d, I) && wmap(&dn.b0_shared, sh.wd, d, I) &&
+              wmap(&dn.b1_routed, routed.wd, (uint64_t)E * d, I) && wmap(&dn.b1_shared, sh.wd, d, I) &&
               make_map(&dn.a, h, R, I);
     if (!ok) return fail(KMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     TcArgs a{};
@@ -384,21 +525,8 @@ kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, in
     a.d = d;
     a.I = I;
     a.err = err;
-    const int grid = sm_count_tc();
-    cudaFuncSetAttribute(ffn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
-    cudaFuncSetAttribute(ffn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
-    a.kblocks = d / kBK;
-    a.n_tiles = I / (kBN / 2);
-    a.out0 = h;
-    ffn_tc_kernel<true><<<grid, kTcThreads, kTcSmem, st>>>(up, a);
-    kmoe_status s = check_launch("ffn_up_tc");
-    if (s != KMOE_OK) return s;
-    a.kblocks = I / kBK;
-    a.n_tiles = d / kBN;
-    a.out0 = y_perm;
-    a.out1 = y_shared;
-    ffn_tc_kernel<false><<<grid, kTcThreads, kTcSmem, st>>>(dn, a);
-    return check_launch("ffn_down_tc");
+    if (fp8) return run_tc<true>(up, dn, a, d, I, h, y_perm, y_shared, routed, sh, st);
+    return run_tc<false>(up, dn, a, d, I, h, y_perm, y_shared, routed, sh, st);
 }
 
 }  // namespace kmoe

@@ -15,14 +15,16 @@ namespace kmoe {
 constexpr int kChunk = 256;
 constexpr int kChunkWarps = kChunk / 32;
 
-// Builds the 8 x E ballot masks of one chunk in shared memory.
+// Builds the W x E ballot masks of one chunk of W*32 tokens in shared memory
+// (a CTA of W warps, thread i <-> token chunk * W*32 + i).
+template <int W = kChunkWarps>
 __device__ __forceinline__ void build_masks(const int32_t *__restrict__ idx, int N, int K, int E,
                                             int chunk, uint32_t *mask)
 {
-    for (int i = threadIdx.x; i < kChunkWarps * E; i += blockDim.x) mask[i] = 0u;
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) mask[i] = 0u;
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = chunk * kChunk + threadIdx.x;
+    const int t = chunk * W * 32 + threadIdx.x;
     if (t < N) {
         for (int k = 0; k < K; ++k) {
             const int e = idx[(size_t)t * K + k];
@@ -68,8 +70,9 @@ __device__ __forceinline__ int rank_in_chunk(const uint32_t *mask, int E, int e,
     return r;
 }
 
-// Whole permutation of N <= 256 tokens by one CTA of 256 threads.
-// `mask` is shared memory of kChunkWarps * E + E 32-bit words.
+// Whole permutation of N <= W*32 tokens by one CTA of W warps.
+// `mask` is shared memory of W * E + E 32-bit words.
+template <int W = kChunkWarps>
 __device__ __forceinline__ void permute_small_block(const int32_t *__restrict__ idx, int N, int K, int E,
                                                     int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                                                     int32_t *__restrict__ perm, int32_t *__restrict__ inv,
@@ -77,16 +80,16 @@ __device__ __forceinline__ void permute_small_block(const int32_t *__restrict__ 
 {
     __shared__ int tmp[32];
     __shared__ int round_total;
-    int *start = reinterpret_cast<int *>(mask + kChunkWarps * E);   // [E]
-    build_masks(idx, N, K, E, 0, mask);
+    int *start = reinterpret_cast<int *>(mask + W * E);   // [E]
+    build_masks<W>(idx, N, K, E, 0, mask);
     // E may exceed the CTA: scan in rounds of blockDim.x experts.
     int carry = 0;
     for (int e0 = 0; e0 < E; e0 += blockDim.x) {
         const int e = e0 + threadIdx.x;
         int c = 0;
         if (e < E) {
-#pragma unroll
-            for (int w = 0; w < kChunkWarps; ++w) c += __popc(mask[w * E + e]);
+#pragma unroll 8
+            for (int w = 0; w < W; ++w) c += __popc(mask[w * E + e]);
         }
         const int excl = block_exclusive_scan(c, tmp);
         if (e < E) {

@@ -156,18 +156,27 @@ kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, in
 // ------------------------------------------------ fused small-batch routing
 //
 // For N <= 256 tokens (decode) the router, the top-K selection and the
-// dispatch permutation run as one launch. Each CTA owns kRouteEPC experts:
-// the bulk-copy engine brings their FP32 router rows and the token rows into
-// shared memory, and every warp computes the logits of one token at a time.
-// The last CTA to finish (a ticket in the workspace status area, zeroed by
-// the caller before the launch) then selects the top K of every token and
-// builds the permutation, reusing its shared memory for the ballot masks.
+// dispatch permutation run as one launch of CTAs of 32 warps. Each CTA owns
+// kRouteEPC experts: the bulk-copy engine brings their FP32 router rows and a
+// chunk of up to 32 token rows into shared memory. Warp w handles tokens
+// 4*(w%8) .. 4*(w%8)+3 of the chunk over column quarter w/8, so every router
+// weight read from shared memory feeds four tokens; the four quarter sums of
+// a logit are added in a fixed order. The last CTA to finish (a ticket in
+// the workspace status area, zeroed before the launch) then selects the top K
+// of every token (one warp per token) and builds the permutation with 32-warp
+// ballot masks, reusing its shared memory.
 constexpr int kRouteEPC = 3;
+constexpr int kRouteThreads = 1024;
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kRouteTPW = 4;                          // tokens per warp
+constexpr int kRouteTG = 8;                           // token groups per chunk
+constexpr int kRouteCQ = kRouteWarps / kRouteTG;      // column parts (4)
+constexpr int kRouteChunkMax = kRouteTPW * kRouteTG;  // 32 tokens per chunk
 constexpr int kRouteSmemMax = 200 * 1024;
 constexpr long long kRouteWaitLimit = 1LL << 32;
 
 template <class XT, int NPL>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kRouteThreads, 1)
 route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
                    int N, int d, int E, int K, int chunk, int x_off, float *__restrict__ logits,
                    int32_t *__restrict__ idx, float *__restrict__ wout, int32_t *__restrict__ counts,
@@ -178,11 +187,14 @@ route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const 
     extern __shared__ __align__(128) uint8_t sm_raw[];
     __shared__ __align__(8) uint64_t bar;
     __shared__ int last, abort_flag;
+    __shared__ float red[kRouteCQ][kRouteChunkMax][kRouteEPC];
     float *wsm = reinterpret_cast<float *>(sm_raw);
     XT *xsm = reinterpret_cast<XT *>(sm_raw + x_off);
     const int e0 = blockIdx.x * kRouteEPC;
     const int ne = min(kRouteEPC, E - e0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tg = warp % kRouteTG, cq = warp / kRouteTG;
+    const int qd = d / kRouteCQ;                     // columns per part (d % 128 == 0)
     int *ticket = status + 4;
     if (threadIdx.x == 0) {
         mbar_init(&bar, 1);
@@ -205,29 +217,50 @@ route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const 
         phase ^= 1;
         __syncthreads();
         if (abort_flag) break;
-        for (int t = warp; t < nt; t += 8) {
-            float acc[kRouteEPC];
+        const int t0 = tg * kRouteTPW;
+        float acc[kRouteTPW][kRouteEPC];
 #pragma unroll
-            for (int e = 0; e < kRouteEPC; ++e) acc[e] = 0.f;
-            const XT *xr = xsm + (size_t)t * d;
-            for (int j = lane * 8; j < d; j += 256) {
-                float xv[8];
-                load8(xr + j, xv);
+        for (int a = 0; a < kRouteTPW; ++a)
+#pragma unroll
+            for (int e = 0; e < kRouteEPC; ++e) acc[a][e] = 0.f;
+        if (t0 < nt) {
+            for (int j = cq * qd + lane * 8; j < (cq + 1) * qd; j += 256) {
+                float wv[kRouteEPC][8];
 #pragma unroll
                 for (int e = 0; e < kRouteEPC; ++e) {
-                    if (e < ne) {
-                        float wv[8];
-                        load8(wsm + e * d + j, wv);
+                    if (e < ne) load8(wsm + e * d + j, wv[e]);
+                    else {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) acc[e] = fmaf(xv[q], wv[q], acc[e]);
+                        for (int q = 0; q < 8; ++q) wv[e][q] = 0.f;
+                    }
+                }
+#pragma unroll
+                for (int a = 0; a < kRouteTPW; ++a) {
+                    if (t0 + a < nt) {
+                        float xv[8];
+                        load8(xsm + (size_t)(t0 + a) * d + j, xv);
+#pragma unroll
+                        for (int e = 0; e < kRouteEPC; ++e)
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) acc[a][e] = fmaf(xv[q], wv[e][q], acc[a][e]);
                     }
                 }
             }
+        }
+#pragma unroll
+        for (int a = 0; a < kRouteTPW; ++a)
 #pragma unroll
             for (int e = 0; e < kRouteEPC; ++e) {
-                const float v = warp_sum(acc[e]);
-                if (lane == 0 && e < ne) logits[(size_t)(c0 + t) * E + e0 + e] = v;
+                const float v = warp_sum(acc[a][e]);
+                if (lane == 0) red[cq][t0 + a][e] = v;
             }
+        __syncthreads();
+        if (threadIdx.x < nt * ne) {
+            const int t = threadIdx.x / ne, e = threadIdx.x - t * ne;
+            float v = red[0][t][e];
+#pragma unroll
+            for (int q = 1; q < kRouteCQ; ++q) v += red[q][t][e];
+            logits[(size_t)(c0 + t) * E + e0 + e] = v;
         }
         __syncthreads();
     }
@@ -241,10 +274,10 @@ route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const 
     __syncthreads();
     if (!last) return;
     __threadfence();
-    for (int t = warp; t < N; t += 8)
+    for (int t = warp; t < N; t += kRouteWarps)
         topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, idx + (size_t)t * K, wout + (size_t)t * K);
     __syncthreads();
-    permute_small_block(idx, N, K, E, counts, offsets, perm, inv, reinterpret_cast<uint32_t *>(sm_raw));
+    permute_small_block<kRouteWarps>(idx, N, K, E, counts, offsets, perm, inv, reinterpret_cast<uint32_t *>(sm_raw));
     if (threadIdx.x == 0) *ticket = 0;
 }
 
@@ -255,16 +288,16 @@ kmoe_status launch_route_small(const void *x, int x_dtype, const float *w_router
     if (N > kChunk) return fail(KMOE_ERR_UNSUPPORTED, "fused routing: N=%d > %d", N, kChunk);
     const int xb = x_dtype == KMOE_F32 ? 4 : 2;
     const int w_bytes = ((kRouteEPC * d * 4) + 127) / 128 * 128;
-    const int chunk = std::min(N, std::max(1, (kRouteSmemMax - w_bytes) / (d * xb)));
-    const size_t smem = std::max((size_t)w_bytes + (size_t)chunk * d * xb, (size_t)(kChunkWarps + 1) * E * 4);
+    const int chunk = std::min(std::min(N, kRouteChunkMax), std::max(1, (kRouteSmemMax - w_bytes) / (d * xb)));
+    const size_t smem = std::max((size_t)w_bytes + (size_t)chunk * d * xb, (size_t)(kRouteWarps + 1) * E * 4);
     const int grid = (E + kRouteEPC - 1) / kRouteEPC;
     const int npl = (E + 31) / 32;
 #define KMOE_ROUTE(XT, n)                                                                                   \
     do {                                                                                                    \
         auto k = route_small_kernel<XT, n>;                                                                 \
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                    \
-        k<<<grid, 256, smem, st>>>(static_cast<const XT *>(x), w_router, bias, N, d, E, K, chunk, w_bytes,   \
-                                   logits, idx, w, counts, offsets, perm, inv, status);                     \
+        k<<<grid, kRouteThreads, smem, st>>>(static_cast<const XT *>(x), w_router, bias, N, d, E, K, chunk,  \
+                                             w_bytes, logits, idx, w, counts, offsets, perm, inv, status);   \
     } while (0)
 #define KMOE_ROUTE_X(n)                                   \
     do {                                                  \

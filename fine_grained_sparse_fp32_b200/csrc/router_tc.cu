@@ -112,6 +112,7 @@ router_tc_kernel(const __grid_constant__ RouterMaps maps, int N, int d, int E, f
 
     if (warp == kRProdWarp) {
         if (lane == 0) {
+            const uint64_t pol = policy_evict_last();   // x and the weight terms are read by several CTAs
             int i = 0;
             for (; i < iters; ++i) {
                 const int s = i % kRStages;
@@ -119,8 +120,8 @@ router_tc_kernel(const __grid_constant__ RouterMaps maps, int N, int d, int E, f
                 const int kb = i / 3, term = i - kb * 3;
                 uint8_t *As = smem + (size_t)s * kRStage;
                 mbar_arrive_expect_tx(&tail->full[s], kRStage);
-                tma_load_2d(As, &maps.x, &tail->full[s], kb * kRBK, m0);
-                tma_load_2d(As + kRA, &maps.w, &tail->full[s], kb * kRBK, term * E + n0);
+                tma_load_2d_hint(As, &maps.x, &tail->full[s], kb * kRBK, m0, pol);
+                tma_load_2d_hint(As + kRA, &maps.w, &tail->full[s], kb * kRBK, term * E + n0, pol);
             }
             if (i < iters)     // aborted: let the loads already issued land
                 for (int j = i > kRStages ? i - kRStages : 0; j < i; ++j)

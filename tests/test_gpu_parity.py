@@ -111,7 +111,8 @@ def test_permute_all_tokens_on_the_same_experts():
 
 # ------------------------------------------------------------ grouped FFN
 @pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("fp8_decode", None), ("decode", 200),
-                                    ("fp8_decode", 130), ("prefill", 256), ("prefill", 300), ("prefill", 1000)])
+                                    ("fp8_decode", 130), ("prefill", 256), ("prefill", 300), ("prefill", 1000),
+                                    ("fp8_prefill", 300), ("fp8_prefill", 777)])
 def test_grouped_ffn_matches_oracle(name, N):
     dev, host = layer_inputs(name, N)
     cfg = host["cfg"]
