@@ -51,8 +51,11 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 // 16 bytes of weights -> VEC floats, for the three storage types.
 template <class WT> struct WVec;
 
+// cvt_word: one 32-bit word of the vector -> EPW = VEC/4 floats.
 template <> struct WVec<float> {
     static constexpr int VEC = 4;
+    static constexpr int EPW = 1;
+    __device__ __forceinline__ static void cvt_word(uint32_t v, float *o, float) { o[0] = __uint_as_float(v); }
     __device__ __forceinline__ static void cvt(uint4 r, float *o, float) {
         o[0] = __uint_as_float(r.x); o[1] = __uint_as_float(r.y);
         o[2] = __uint_as_float(r.z); o[3] = __uint_as_float(r.w);
@@ -61,6 +64,8 @@ template <> struct WVec<float> {
 
 template <> struct WVec<__nv_bfloat16> {
     static constexpr int VEC = 8;
+    static constexpr int EPW = 2;
+    __device__ __forceinline__ static void cvt_word(uint32_t v, float *o, float) { o[0] = bf16_lo(v); o[1] = bf16_hi(v); }
     __device__ __forceinline__ static void cvt(uint4 r, float *o, float) {
         o[0] = bf16_lo(r.x); o[1] = bf16_hi(r.x); o[2] = bf16_lo(r.y); o[3] = bf16_hi(r.y);
         o[4] = bf16_lo(r.z); o[5] = bf16_hi(r.z); o[6] = bf16_lo(r.w); o[7] = bf16_hi(r.w);
@@ -69,6 +74,7 @@ template <> struct WVec<__nv_bfloat16> {
 
 template <> struct WVec<__nv_fp8_e4m3> {
     static constexpr int VEC = 16;
+    static constexpr int EPW = 4;
     __device__ __forceinline__ static void cvt2(uint32_t v, float *o, float s) {
         __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v & 0xffffu), __NV_E4M3);
         __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v >> 16), __NV_E4M3);
@@ -79,6 +85,7 @@ template <> struct WVec<__nv_fp8_e4m3> {
     __device__ __forceinline__ static void cvt(uint4 r, float *o, float s) {
         cvt2(r.x, o, s); cvt2(r.y, o + 4, s); cvt2(r.z, o + 8, s); cvt2(r.w, o + 12, s);
     }
+    __device__ __forceinline__ static void cvt_word(uint32_t v, float *o, float s) { cvt2(v, o, s); }
 };
 
 // Activations: 8 consecutive values -> floats.
@@ -94,6 +101,8 @@ __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float *o) {
 
 __device__ __forceinline__ void store_val(float *p, float v) { *p = v; }
 __device__ __forceinline__ void store_val(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ uint32_t word_of(const uint4 &r, int w) { return w == 0 ? r.x : w == 1 ? r.y : w == 2 ? r.z : r.w; }
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }

@@ -117,17 +117,20 @@ __device__ __forceinline__ int token_of(const GroupView &G, int row, int N, int 
 }
 
 // ------------------------------------------------------------------ gate/up
-// Features per warp: enough 16-byte loads per column block to cover 32
-// weights per lane and matrix (BF16: 2 features, E4M3: 1, FP32: 4).
-template <class WT> struct UpF { static constexpr int v = 16 / WVec<WT>::VEC > 0 ? 16 / WVec<WT>::VEC : 1; };
+// Features per warp: two 16-byte loads per lane and matrix per column block
+// for the 2-byte and 1-byte weights (so that as many bytes are in flight
+// for E4M3 as for BF16), four for FP32.
+template <class WT> struct UpF { static constexpr int v = WVec<WT>::VEC == 4 ? 4 : 2; };
 
 template <class WT, class XT, class HT, int MT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, MT <= 2 ? 3 : 1)
 ffn_up_stream_kernel(const XT *__restrict__ x, int N, int d, int I, int E, int K,
                      const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
                      ExpertPtrs routed, ExpertPtrs shared, int has_shared, HT *__restrict__ H)
 {
     constexpr int VEC = WVec<WT>::VEC;
+    constexpr int EPW = WVec<WT>::EPW;
+    constexpr int CH = VEC == 16 ? 4 : VEC;         // weights converted at a time
     constexpr int F = UpF<WT>::v;                   // features per warp
     constexpr int FS = F * kWarps;                  // features per unit
     __shared__ int pre[kMaxGroupsS + 1];
@@ -189,28 +192,36 @@ ffn_up_stream_kernel(const XT *__restrict__ x, int N, int d, int I, int E, int K
                 const int j = j0 + b * 32 * VEC;
 #pragma unroll
                 for (int f = 0; f < F; ++f) {
-                    float vg[VEC], vu[VEC];
                     float s_g = 1.f, s_u = 1.f;
                     if (sg) {
                         const int sidx = ((f0 + f) / 128) * cb + j / 128;
                         s_g = sg[sidx];
                         s_u = su[sidx];
                     }
-                    WVec<WT>::cvt(rg[b][f], vg, s_g);
-                    WVec<WT>::cvt(ru[b][f], vu, s_u);
+                    // CH weights at a time (all 8 for BF16, one 32-bit word of 4 for
+                    // E4M3): few values live, x read with 16-byte shared loads
 #pragma unroll
-                    for (int m = 0; m < MT; ++m) {
+                    for (int c = 0; c < VEC / CH; ++c) {
+                        float vg[CH], vu[CH];
 #pragma unroll
-                        for (int q = 0; q < VEC; q += 4) {
-                            const float4 xv = *reinterpret_cast<const float4 *>(xs + m * d + j + q);
-                            ag[f][m] = fmaf(vg[q], xv.x, ag[f][m]);
-                            ag[f][m] = fmaf(vg[q + 1], xv.y, ag[f][m]);
-                            ag[f][m] = fmaf(vg[q + 2], xv.z, ag[f][m]);
-                            ag[f][m] = fmaf(vg[q + 3], xv.w, ag[f][m]);
-                            au[f][m] = fmaf(vu[q], xv.x, au[f][m]);
-                            au[f][m] = fmaf(vu[q + 1], xv.y, au[f][m]);
-                            au[f][m] = fmaf(vu[q + 2], xv.z, au[f][m]);
-                            au[f][m] = fmaf(vu[q + 3], xv.w, au[f][m]);
+                        for (int w = 0; w < CH / EPW; ++w) {
+                            WVec<WT>::cvt_word(word_of(rg[b][f], c * (CH / EPW) + w), vg + w * EPW, s_g);
+                            WVec<WT>::cvt_word(word_of(ru[b][f], c * (CH / EPW) + w), vu + w * EPW, s_u);
+                        }
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) {
+#pragma unroll
+                            for (int q = 0; q < CH; q += 4) {
+                                const float4 xv = *reinterpret_cast<const float4 *>(xs + m * d + j + c * CH + q);
+                                ag[f][m] = fmaf(vg[q], xv.x, ag[f][m]);
+                                ag[f][m] = fmaf(vg[q + 1], xv.y, ag[f][m]);
+                                ag[f][m] = fmaf(vg[q + 2], xv.z, ag[f][m]);
+                                ag[f][m] = fmaf(vg[q + 3], xv.w, ag[f][m]);
+                                au[f][m] = fmaf(vu[q], xv.x, au[f][m]);
+                                au[f][m] = fmaf(vu[q + 1], xv.y, au[f][m]);
+                                au[f][m] = fmaf(vu[q + 2], xv.z, au[f][m]);
+                                au[f][m] = fmaf(vu[q + 3], xv.w, au[f][m]);
+                            }
                         }
                     }
                 }
@@ -234,12 +245,14 @@ constexpr int kDownPasses = 4;        // passes per unit
 constexpr int kDownFS = kDownRows * kWarps * kDownPasses;   // 128 output features per unit
 
 template <class WT, class HT, int MT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, MT <= 2 ? 3 : 1)
 ffn_down_stream_kernel(const HT *__restrict__ H, int N, int d, int I, int E, int K,
                        const int32_t *__restrict__ offsets, ExpertPtrs routed, ExpertPtrs shared,
                        int has_shared, HT *__restrict__ y_perm, HT *__restrict__ y_shared)
 {
     constexpr int VEC = WVec<WT>::VEC;
+    constexpr int EPW = WVec<WT>::EPW;
+    constexpr int CH = VEC == 16 ? 4 : VEC;
     __shared__ int pre[kMaxGroupsS + 1];
     extern __shared__ float4 smem_f4[];
     float *hs = reinterpret_cast<float *>(smem_f4);  // [MT][I]
@@ -290,18 +303,23 @@ ffn_down_stream_kernel(const HT *__restrict__ H, int N, int d, int I, int E, int
                 const int i = i0 + b * 32 * VEC;
 #pragma unroll
                 for (int r = 0; r < kDownRows; ++r) {
-                    float w[VEC];
                     const float s = sd ? sd[((j0 + r) / 128) * ib + i / 128] : 1.f;
-                    WVec<WT>::cvt(raw[b][r], w, s);
 #pragma unroll
-                    for (int m = 0; m < MT; ++m) {
+                    for (int c = 0; c < VEC / CH; ++c) {
+                        float w[CH];
 #pragma unroll
-                        for (int q = 0; q < VEC; q += 4) {
-                            const float4 hv = *reinterpret_cast<const float4 *>(hs + m * I + i + q);
-                            acc[r][m] = fmaf(w[q], hv.x, acc[r][m]);
-                            acc[r][m] = fmaf(w[q + 1], hv.y, acc[r][m]);
-                            acc[r][m] = fmaf(w[q + 2], hv.z, acc[r][m]);
-                            acc[r][m] = fmaf(w[q + 3], hv.w, acc[r][m]);
+                        for (int wi = 0; wi < CH / EPW; ++wi)
+                            WVec<WT>::cvt_word(word_of(raw[b][r], c * (CH / EPW) + wi), w + wi * EPW, s);
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) {
+#pragma unroll
+                            for (int q = 0; q < CH; q += 4) {
+                                const float4 hv = *reinterpret_cast<const float4 *>(hs + m * I + i + c * CH + q);
+                                acc[r][m] = fmaf(w[q], hv.x, acc[r][m]);
+                                acc[r][m] = fmaf(w[q + 1], hv.y, acc[r][m]);
+                                acc[r][m] = fmaf(w[q + 2], hv.z, acc[r][m]);
+                                acc[r][m] = fmaf(w[q + 3], hv.w, acc[r][m]);
+                            }
                         }
                     }
                 }

@@ -7,21 +7,27 @@
 // dispatched to it, gathered through perm_token):
 //   up kernel   : H_e = SiLU(X_e W_g,e^T) * (X_e W_u,e^T)     [rows, I]
 //   down kernel : Y_e = H_e W_d,e^T                           [rows, d]
-// Both are persistent, warp-specialised grouped GEMMs with 128 x 256 x 64
-// tiles (BF16 operands, FP32 accumulation in tensor memory):
-//   warps 0-3  epilogue: tcgen05.ld of the accumulator, SwiGLU (up) or the
-//              BF16 cast (down), stores to global memory;
+// Both are persistent, warp-specialised grouped GEMMs (BF16 operands, FP32
+// accumulation in tensor memory). A CTA tile is up to 256 rows of one
+// expert (two M = 128 m-tiles) by 256 accumulator columns: every 64-column
+// weight tile (N = 256 rows) that lands in shared memory feeds both
+// m-tiles, into the two 256-column halves of tensor memory, so a weight tile
+// crosses HBM and L2 once per expert and n-tile even when the expert's rows
+// spill past 128 (at prefill an expert sees ~128 +- 11 tokens).
+//   warps 0-3  epilogue: tcgen05.ld of each half, SwiGLU (up) or the BF16
+//              cast (down), stores to global memory; a half is handed back
+//              to the MMA as soon as it is drained, so the next tile's first
+//              MMAs overlap the epilogue of the second half;
 //   warp  4    one thread issues tcgen05.mma and tcgen05.commit;
 //   warps 5-8  producers: weight tiles by TMA (128-byte swizzle); the
 //              activation rows of the up kernel are gathered with cp.async
 //              straight into the swizzled layout (no permuted copy of x is
-//              ever written), the down kernel loads H tiles by TMA.
+//              ever written) and complete on the stage barrier without the
+//              producer waiting; the down kernel loads H tiles by TMA.
 // The up tile pairs 128 gate features with the same 128 up features (one
-// N = 256 MMA into 256 TMEM columns), so SiLU(g) * u is computed in
-// registers. Two accumulators (512 TMEM columns) let the epilogue of one
-// tile overlap the MMAs of the next. Tiles are enumerated per expert as
-// (n-tile, m-tile) so that CTAs working at the same time read the same
-// weight tile and it crosses HBM once.
+// N = 256 MMA), so SiLU(g) * u is computed in registers. Tiles are
+// enumerated per expert as (n-tile, row pair), so CTAs running at the same
+// time share the expert's token rows in L2.
 //
 // E4M3 weights ("Inside Kolibri 1", FP8 section: 128 x 128 blocks, one FP32
 // scale per block) take the same kernels with four more warps: the weight
@@ -39,12 +45,13 @@ namespace kmoe {
 using namespace sm100;
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kATile = kBM * kBK * 2;        // 16 KB
+constexpr int kPairRows = 2 * kBM;           // rows of one CTA tile
+constexpr int kATile = kBM * kBK * 2;        // 16 KB per m-tile
 constexpr int kBTile = kBN * kBK * 2;        // 32 KB
 constexpr int kB8Tile = kBN * kBK;           // 16 KB of E4M3 staging
-constexpr int kMaxStages = 4;
-__host__ __device__ constexpr int stages_of(bool fp8) { return fp8 ? 3 : 4; }
-__host__ __device__ constexpr int stage_bytes(bool fp8) { return kATile + kBTile + (fp8 ? kB8Tile : 0); }
+constexpr int kMaxStages = 3;
+__host__ __device__ constexpr int stages_of(bool fp8) { return fp8 ? 2 : 3; }
+__host__ __device__ constexpr int stage_bytes(bool fp8) { return 2 * kATile + kBTile + (fp8 ? kB8Tile : 0); }
 constexpr int kMmaWarp = 4;
 constexpr int kProdWarp = 5;
 constexpr int kConvWarp = 9;                 // E4M3 only: warps 9-12
@@ -71,20 +78,20 @@ struct TcArgs {
 };
 
 struct SmemTail {
-    uint64_t full[kMaxStages], empty[kMaxStages], b8full[kMaxStages], tfull[2], tempty[2], drain;
+    uint64_t full[kMaxStages], empty[kMaxStages], b8full[kMaxStages], tfull, tempty[2], drain;
     uint32_t tmem_base;
     int abort;
     int pre[kMaxGroups + 1];
 };
 
-constexpr size_t tc_smem(bool fp8)
+__host__ __device__ constexpr size_t tc_smem(bool fp8)
 {
     return 1024 /*align slack*/ + (size_t)stages_of(fp8) * stage_bytes(fp8) + sizeof(SmemTail);
 }
 
 struct Tile {
     int g, row0, rows, n0;
-    bool shared;
+    bool shared, two;     // two: rows > 128 (second m-tile present)
 };
 
 __device__ __forceinline__ Tile decode_tile(int t, const int *pre, const TcArgs &a, int bn)
@@ -98,19 +105,20 @@ __device__ __forceinline__ Tile decode_tile(int t, const int *pre, const TcArgs 
     Tile T;
     T.g = lo - 1;
     T.shared = T.g >= a.E;
-    const int mcount = pre[T.g + 1] - pre[T.g];
+    const int pcount = pre[T.g + 1] - pre[T.g];
     const int local = t - pre[T.g] * a.n_tiles;
-    const int nt = local / mcount, mt = local - nt * mcount;
+    const int nt = local / pcount, mp = local - nt * pcount;
     int start, cnt;
     if (T.shared) { start = a.N * a.K; cnt = a.N; }
     else { start = a.offsets[T.g]; cnt = a.offsets[T.g + 1] - start; }
-    T.row0 = start + mt * kBM;
-    T.rows = min(kBM, cnt - mt * kBM);
+    T.row0 = start + mp * kPairRows;
+    T.rows = min(kPairRows, cnt - mp * kPairRows);
+    T.two = T.rows > kBM;
     T.n0 = nt * bn;
     return T;
 }
 
-// m-tile prefix over groups, computed by one warp.
+// row-pair prefix over groups, computed by one warp.
 __device__ __forceinline__ void build_prefix(int *pre, const TcArgs &a)
 {
     const int lane = threadIdx.x & 31;
@@ -121,7 +129,7 @@ __device__ __forceinline__ void build_prefix(int *pre, const TcArgs &a)
         const int g = g0 + i;
         if (g < a.groups) {
             const int cnt = g < a.E ? a.offsets[g + 1] - a.offsets[g] : a.N;
-            sum += (cnt + kBM - 1) / kBM;
+            sum += (cnt + kPairRows - 1) / kPairRows;
         }
     }
     int incl = sum;
@@ -136,7 +144,7 @@ __device__ __forceinline__ void build_prefix(int *pre, const TcArgs &a)
         if (g < a.groups) {
             pre[g] = run;
             const int cnt = g < a.E ? a.offsets[g + 1] - a.offsets[g] : a.N;
-            run += (cnt + kBM - 1) / kBM;
+            run += (cnt + kPairRows - 1) / kPairRows;
         }
     }
     if (lane == 31) pre[a.groups] = incl;
@@ -168,13 +176,61 @@ __device__ __forceinline__ void convert_row(const uint8_t *src, uint8_t *dst, in
     }
 }
 
+// Epilogue of one 128-row half of the accumulator (rows r_base .. r_base+127
+// of the tile). tbase addresses this warp's 32 lanes in that half.
+template <bool kUp>
+__device__ __forceinline__ void epilogue_half(uint32_t tbase, const Tile &T, const TcArgs &a, int row)
+{
+    const bool valid = row < T.rows;
+    const int grow = T.row0 + row;
+    if (kUp) {
+        __nv_bfloat16 *dst = a.out0 + (size_t)grow * a.I + T.n0;
+#pragma unroll 1
+        for (int c = 0; c < kBN / 2; c += 16) {
+            uint32_t g[16], u[16];
+            tmem_ld16(tbase + c, g);
+            tmem_ld16(tbase + kBN / 2 + c, u);
+            tmem_ld_wait();
+            uint32_t packed[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float g0 = __uint_as_float(g[2 * q]), g1 = __uint_as_float(g[2 * q + 1]);
+                const float u0 = __uint_as_float(u[2 * q]), u1 = __uint_as_float(u[2 * q + 1]);
+                packed[q] = pack_bf16x2(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1);
+            }
+            if (valid) {
+                uint4 *o = reinterpret_cast<uint4 *>(dst + c);
+                o[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                o[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            }
+        }
+    } else {
+        __nv_bfloat16 *dst = T.shared ? a.out1 + (size_t)(grow - a.N * a.K) * a.d + T.n0
+                                      : a.out0 + (size_t)grow * a.d + T.n0;
+#pragma unroll 1
+        for (int c = 0; c < kBN; c += 16) {
+            uint32_t v[16];
+            tmem_ld16(tbase + c, v);
+            tmem_ld_wait();
+            uint32_t packed[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                packed[q] = pack_bf16x2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
+            if (valid) {
+                uint4 *o = reinterpret_cast<uint4 *>(dst + c);
+                o[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                o[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            }
+        }
+    }
+}
+
 template <bool kUp, bool kFp8>
 __global__ void __launch_bounds__(threads_of(kFp8), 1)
 ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
 {
     constexpr int kStages = stages_of(kFp8);
     constexpr int kStage = stage_bytes(kFp8);
-    constexpr int kLag = kStages - 1;        // cp.async groups in flight before a stage is signalled
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     SmemTail *tail = reinterpret_cast<SmemTail *>(smem + (size_t)kStages * kStage);
@@ -189,10 +245,9 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             mbar_init(&tail->empty[s], 1);
             mbar_init(&tail->b8full[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tail->tfull[b], 1);
-            mbar_init(&tail->tempty[b], 128);
-        }
+        mbar_init(&tail->tfull, 1);
+        mbar_init(&tail->tempty[0], 128);
+        mbar_init(&tail->tempty[1], 128);
         mbar_init(&tail->drain, 1);
         tail->abort = 0;
         fence_mbar_init();
@@ -229,7 +284,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
                 const int s = it % kStages;
                 if (!mbar_wait(&tail->b8full[s], (it / kStages) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-                uint8_t *Bs = smem + (size_t)s * kStage + kATile;
+                uint8_t *Bs = smem + (size_t)s * kStage + 2 * kATile;
                 const uint8_t *B8 = Bs + kBTile;
                 float sc0, sc1;
                 if (kUp) {     // gate rows n0.., up rows n0..; blocks [G, I/128, d/128]
@@ -260,15 +315,19 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             const CUtensorMap *m0 = T.shared ? &maps.b0_shared : &maps.b0_routed;
             const CUtensorMap *m1 = T.shared ? &maps.b1_shared : &maps.b1_routed;
             const int gi = T.shared ? 0 : T.g;
-            int tok = -1;
-            if (kUp && p < T.rows) tok = T.shared ? T.row0 + p - a.N * a.K : a.perm[T.row0 + p];
-            const __nv_bfloat16 *src = a.x + (size_t)(tok < 0 ? 0 : tok) * a.d;
+            int tok0 = -1, tok1 = -1;
+            if (kUp) {
+                if (p < T.rows) tok0 = T.shared ? T.row0 + p - a.N * a.K : a.perm[T.row0 + p];
+                if (p + kBM < T.rows) tok1 = T.shared ? T.row0 + kBM + p - a.N * a.K : a.perm[T.row0 + kBM + p];
+            }
+            const __nv_bfloat16 *src0 = a.x + (size_t)(tok0 < 0 ? 0 : tok0) * a.d;
+            const __nv_bfloat16 *src1 = a.x + (size_t)(tok1 < 0 ? 0 : tok1) * a.d;
             for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
                 const int s = it % kStages;
                 const uint32_t ph = (it / kStages) & 1;
                 if (!mbar_wait(&tail->empty[s], ph ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-                uint8_t *As = smem + (size_t)s * kStage;
-                uint8_t *Bs = As + kATile;
+                uint8_t *As = smem + (size_t)s * kStage;           // A0 | A1 | B | (B8)
+                uint8_t *Bs = As + 2 * kATile;
                 if (kFp8 && leader) {       // E4M3 weight rows into the staging buffer
                     uint8_t *B8 = Bs + kBTile;
                     const int r0 = kUp ? gi * a.I + T.n0 : gi * a.d + T.n0;
@@ -283,20 +342,23 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                         tma_load_2d_hint(Bs, m0, &tail->full[s], kb * kBK, gi * a.I + T.n0, pol_w);
                         tma_load_2d_hint(Bs + kBTile / 2, m1, &tail->full[s], kb * kBK, gi * a.I + T.n0, pol_w);
                     }
-                    const uint32_t dst = smem_u32(As) + p * 128;
-                    const __nv_bfloat16 *s_row = src + kb * kBK;
+                    const uint32_t dst0 = smem_u32(As) + p * 128;
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
-                        cp_async16_hint(dst + ((c ^ (p & 7)) << 4), s_row + c * 8, tok >= 0 ? 16u : 0u, pol_a);
-                    cp_async_commit();
-                    if (it >= kLag) {
-                        cp_async_wait<kLag>();
-                        fence_proxy_async();
-                        mbar_arrive(&tail->full[(it - kLag) % kStages]);
+                        cp_async16_hint(dst0 + ((c ^ (p & 7)) << 4), src0 + kb * kBK + c * 8, tok0 >= 0 ? 16u : 0u,
+                                        pol_a);
+                    if (T.two) {
+                        const uint32_t dst1 = smem_u32(As + kATile) + p * 128;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            cp_async16_hint(dst1 + ((c ^ (p & 7)) << 4), src1 + kb * kBK + c * 8,
+                                            tok1 >= 0 ? 16u : 0u, pol_a);
                     }
+                    cp_async_arrive_noinc(&tail->full[s]);   // the stage completes when these rows land
                 } else if (leader) {
-                    mbar_arrive_expect_tx(&tail->full[s], kATile + (kFp8 ? 0 : kBTile));
+                    mbar_arrive_expect_tx(&tail->full[s], kATile * (T.two ? 2 : 1) + (kFp8 ? 0 : kBTile));
                     tma_load_2d_hint(As, &maps.a, &tail->full[s], kb * kBK, T.row0, pol_a);
+                    if (T.two) tma_load_2d_hint(As + kATile, &maps.a, &tail->full[s], kb * kBK, T.row0 + kBM, pol_a);
                     if (!kFp8) {
                         tma_load_2d_hint(Bs, m0, &tail->full[s], kb * kBK, gi * a.d + T.n0, pol_w);
                         tma_load_2d_hint(Bs + kBTile / 2, m0, &tail->full[s], kb * kBK, gi * a.d + T.n0 + kBN / 2,
@@ -305,11 +367,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                 }
             }
         }
-        if (kUp) {   // signal the stages still waiting for this thread's copies
-            cp_async_wait<0>();
-            fence_proxy_async();
-            for (uint32_t j = it > (uint32_t)kLag ? it - kLag : 0; j < it; ++j) mbar_arrive(&tail->full[j % kStages]);
-        }
+        if (kUp) cp_async_wait_all();   // this thread's row copies have landed before it leaves
         if (!ok && leader) {   // let in-flight TMA loads land before the CTA exits
             for (uint32_t j = it > (uint32_t)kStages ? it - kStages : 0; j < it; ++j) {
                 if (kFp8) mbar_wait_drain(&tail->b8full[j % kStages], (j / kStages) & 1, kWaitLimit);
@@ -323,22 +381,31 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             uint32_t it = 0, at = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++at) {
-                const int b = at & 1;
-                if (!mbar_wait(&tail->tempty[b], ((at >> 1) & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + b * kBN;
+                const Tile T = decode_tile(t, tail->pre, a, bn);
                 for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
                     const int s = it % kStages;
                     if (!mbar_wait(&tail->full[s], (it / kStages) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                    if (kb == 0 &&   // half 0 drained by the previous tile's epilogue
+                        !mbar_wait(&tail->tempty[0], (at & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t ad = sw128_kmajor_desc(smem_u32(smem + (size_t)s * kStage));
-                    const uint64_t bd = sw128_kmajor_desc(smem_u32(smem + (size_t)s * kStage + kATile));
+                    const uint32_t sa = smem_u32(smem + (size_t)s * kStage);
+                    const uint64_t a0 = sw128_kmajor_desc(sa);
+                    const uint64_t bd = sw128_kmajor_desc(sa + 2 * kATile);
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16(d_tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
+                        umma_bf16(tmem, a0 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
+                    if (kb == 0 &&   // half 1 drained (waited for even when unused, to keep phases)
+                        !mbar_wait(&tail->tempty[1], (at & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                    if (T.two) {
+                        tc_fence_after();
+                        const uint64_t a1 = sw128_kmajor_desc(sa + kATile);
+#pragma unroll
+                        for (int k = 0; k < kBK / 16; ++k)
+                            umma_bf16(tmem + kBN, a1 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
+                    }
                     umma_commit(&tail->empty[s]);
                 }
-                if (ok) umma_commit(&tail->tfull[b]);
+                if (ok) umma_commit(&tail->tfull);
             }
             umma_commit(&tail->drain);     // every MMA done before tensor memory is released
             mbar_wait_drain(&tail->drain, 0, kWaitLimit);
@@ -350,54 +417,17 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         const int row = warp * 32 + lane;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++at) {
             const Tile T = decode_tile(t, tail->pre, a, bn);
-            const int b = at & 1;
-            if (!mbar_wait(&tail->tfull[b], (at >> 1) & 1, abort, a.err, kWaitLimit)) break;
+            if (!mbar_wait(&tail->tfull, at & 1, abort, a.err, kWaitLimit)) break;
             tc_fence_after();
-            const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + b * kBN;
-            const bool valid = row < T.rows;
-            const int grow = T.row0 + row;
-            if (kUp) {
-                __nv_bfloat16 *dst = a.out0 + (size_t)grow * a.I + T.n0;
-#pragma unroll 1
-                for (int c = 0; c < kBN / 2; c += 16) {
-                    uint32_t g[16], u[16];
-                    tmem_ld16(tbase + c, g);
-                    tmem_ld16(tbase + kBN / 2 + c, u);
-                    tmem_ld_wait();
-                    uint32_t packed[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float g0 = __uint_as_float(g[2 * q]), g1 = __uint_as_float(g[2 * q + 1]);
-                        const float u0 = __uint_as_float(u[2 * q]), u1 = __uint_as_float(u[2 * q + 1]);
-                        packed[q] = pack_bf16x2(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1);
-                    }
-                    if (valid) {
-                        uint4 *o = reinterpret_cast<uint4 *>(dst + c);
-                        o[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                        o[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-                    }
-                }
-            } else {
-                __nv_bfloat16 *dst = T.shared ? a.out1 + (size_t)(grow - a.N * a.K) * a.d + T.n0
-                                              : a.out0 + (size_t)grow * a.d + T.n0;
-#pragma unroll 1
-                for (int c = 0; c < kBN; c += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(tbase + c, v);
-                    tmem_ld_wait();
-                    uint32_t packed[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        packed[q] = pack_bf16x2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
-                    if (valid) {
-                        uint4 *o = reinterpret_cast<uint4 *>(dst + c);
-                        o[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                        o[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-                    }
-                }
-            }
+            const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
+            epilogue_half<kUp>(tlane, T, a, row);
             tc_fence_before();
-            mbar_arrive(&tail->tempty[b]);
+            mbar_arrive(&tail->tempty[0]);
+            if (T.two) {
+                epilogue_half<kUp>(tlane + kBN, T, a, row + kBM);
+                tc_fence_before();
+            }
+            mbar_arrive(&tail->tempty[1]);
         }
     }
     tc_fence_before();

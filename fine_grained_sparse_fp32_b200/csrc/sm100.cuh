@@ -148,9 +148,16 @@ __device__ __forceinline__ void cp_async16_hint(uint32_t dst, const void *src, u
                  "r"(src_bytes), "l"(policy)
                  : "memory");
 }
+// Arrives on `bar` (counted as one arrival) once every cp.async issued so
+// far by this thread has landed; the thread itself does not wait.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Makes generic-proxy writes to shared memory visible to the async proxy
 // (TMA, tensor cores).

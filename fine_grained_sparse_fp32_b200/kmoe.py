@@ -166,13 +166,16 @@ def moe_permute_noalloc(topk_idx, E, counts=None, offsets=None, perm=None, inv=N
     return counts, offsets, perm[: N * K], inv
 
 
-def moe_grouped_ffn(x, layer, perm_token, offsets, with_shared=True, ws=None, stream=None):
+def moe_grouped_ffn(x, layer, perm_token, offsets, with_shared=True, ws=None, stream=None, out=None):
     cfg = layer["cfg"]
     N, d = x.shape
     I, E, K = cfg.I, cfg.E, cfg.K
     adt = act_dtype_for(cfg.w_dtype)
-    y_perm = torch.empty((N * K, d), dtype=adt, device=x.device)
-    y_shared = torch.empty((N, d), dtype=adt, device=x.device) if with_shared else None
+    if out is not None:
+        y_perm, y_shared = out
+    else:
+        y_perm = torch.empty((N * K, d), dtype=adt, device=x.device)
+        y_shared = torch.empty((N, d), dtype=adt, device=x.device) if with_shared else None
     if ws is None:
         ws = torch.empty(256 + (N * K + N) * I * (4 if adt == torch.float32 else 2), dtype=torch.uint8,
                          device=x.device)
