@@ -113,6 +113,8 @@ def algorithmic(cfg, distinct_routed: float):
 def launches_per_step(cfg):
     """Kernels of this library that one moe_forward launches (mirrors abi.cu's dispatch)."""
     if cfg.N <= 256:
+        if cfg.x_dtype == "bf16" and cfg.w_dtype in ("bf16", "e4m3"):
+            return 3        # fused router+top-K+permute, swap-AB FFN (up and down), combine
         return 4            # fused router+top-K+permute, ffn up, ffn down, combine
     router = 2 if (cfg.x_dtype == "bf16" and cfg.N >= 512) else 1   # split + tcgen05 router | SIMT router
     return router + 1 + 3 + 2 + 1   # + top-K, permute (hist, scan, scatter), ffn up, ffn down, combine
@@ -187,7 +189,7 @@ def time_grouped_ffn(layer, xs, stream, steps):
             idx, w = kmoe.moe_router_topk(x, layer["w_router"], layer["bias"], cfg.K, stream=stream)
             _, offsets, perm, _ = kmoe.moe_permute(idx, cfg.E, stream=stream)
             preps.append((x, perm, offsets))
-    ws = torch.empty(256 + (cfg.N * cfg.K + cfg.N) * cfg.I * 4, dtype=torch.uint8, device=dev)
+    ws = torch.empty(kmoe.FFN_STATUS_BYTES + (cfg.N * cfg.K + cfg.N) * cfg.I * 4, dtype=torch.uint8, device=dev)
     adt = kmoe.act_dtype_for(cfg.w_dtype)
     y_perm = torch.empty((cfg.N * cfg.K, cfg.d), dtype=adt, device=dev)
     y_shared = torch.empty((cfg.N, cfg.d), dtype=adt, device=dev)
@@ -279,6 +281,9 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the FP8 and skewed-routing layers")
     ap.add_argument("--cpu-tokens", type=int, default=32)
+    ap.add_argument("--capture", default=None, metavar="LAYER",
+                    help="untimed: run --calls whole-layer calls of one workload (for ncu captures) and exit")
+    ap.add_argument("--calls", type=int, default=4)
     args = ap.parse_args()
     world, rank, local = dist_env()
     if args.warmup < 3:
@@ -286,6 +291,8 @@ def main():
 
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.capture:
+        return run_capture(args.capture, args.calls)
 
     if world > 1:
         torch.cuda.set_device(local)
@@ -370,6 +377,26 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
+
+
+def run_capture(name, calls):
+    """A few untimed whole-layer calls of one workload, on rotating token
+    batches: the command that ncu profiles (no number is reported)."""
+    _build.build()
+    kmoe.load()
+    cfg = CONFIGS[name]
+    dev = torch.device("cuda", 0)
+    layer = make_inputs(cfg, seed=0, device=dev)
+    lay = kmoe.Layer(layer, cfg.N)
+    xs = [make_x(cfg, seed=17 * i + 1, device=dev) for i in range(min(calls, ROTATE))]
+    for i in range(calls):
+        y = lay.forward(xs[i % len(xs)])
+    torch.cuda.synchronize()
+    status = kmoe.moe_device_status(lay.ws)
+    print(json.dumps({"capture": name, "calls": calls, "device_status": status,
+                      "y_abs_mean": float(y.float().abs().mean())}), flush=True)
+    if status != 0:
+        raise SystemExit(f"device status {status}")
 
 
 def run_reference(args, world, rank):

@@ -10,6 +10,14 @@ namespace kmoe {
 
 static thread_local char g_err[512] = "";
 
+// Workspace status block: the status word and tickets (ints 0..63), then the
+// grouped FFN's counters (kSyncInts ints). Router-only calls use 256 bytes.
+constexpr int kSyncOffset = 64;                         // ints
+constexpr int kStatusInts = kSyncOffset + kSyncInts;    // status word, tickets, FFN counters
+constexpr size_t kStatusBytes = 256;                    // router-only calls
+constexpr size_t kFfnStatusBytes = kStatusInts * sizeof(int);
+
+
 kmoe_status fail(kmoe_status code, const char *fmt, ...)
 {
     va_list ap;
@@ -111,7 +119,7 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype)
     Layout L;
     const size_t R = (size_t)N * K + N;
     const size_t ab = act_bytes(w_dtype);
-    L.status = c.take<int>(64);
+    L.status = c.take<int>(kStatusInts);
     L.logits = c.take<float>((size_t)N * E);
     L.idx = c.take<int32_t>((size_t)N * K);
     L.w = c.take<float>((size_t)N * K);
@@ -134,10 +142,21 @@ static bool use_tc(int x_dtype, int w_dtype, int N, int d)
            d % 256 == 0;
 }
 
+static bool use_swap(int x_dtype, int w_dtype)
+{
+    return x_dtype == KMOE_BF16 && (w_dtype == KMOE_BF16 || w_dtype == KMOE_E4M3_B128);
+}
+
+// `status` is the workspace status block: the status word, tickets, then
+// kSyncInts counters at kSyncOffset (all zeroed by clear_status).
 static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int E, int K, const int32_t *perm,
                            const int32_t *offsets, int w_dtype, const ExpertPtrs &r, const ExpertPtrs *s,
                            void *h, void *y_perm, void *y_shared, int *status, cudaStream_t st)
 {
+    if (use_swap(x_dtype, w_dtype) && !use_tc(x_dtype, w_dtype, N, d))
+        return launch_ffn_swap(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, w_dtype, r, s,
+                               static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
+                               static_cast<__nv_bfloat16 *>(y_shared), status, status + kSyncOffset, st);
     if (use_tc(x_dtype, w_dtype, N, d))
         return launch_ffn_tc(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, w_dtype, r, s,
                              static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
@@ -145,14 +164,13 @@ static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int 
     return launch_ffn_stream(x, x_dtype, N, d, I, E, K, perm, offsets, w_dtype, r, s, h, y_perm, y_shared, st);
 }
 
-static kmoe_status clear_status(int *status, cudaStream_t st)
+static kmoe_status clear_status(int *status, cudaStream_t st, size_t bytes = kStatusBytes)
 {
     // status word, tickets and counters of this call's kernels
-    if (cudaMemsetAsync(status, 0, 64, st) != cudaSuccess) return check_launch("status memset");
+    if (cudaMemsetAsync(status, 0, bytes, st) != cudaSuccess) return check_launch("status memset");
     return KMOE_OK;
 }
 
-constexpr size_t kStatusBytes = 256;
 constexpr int kFusedRouteTokens = 256;   // routing, top-K and dispatch in one launch up to here
 
 }  // namespace kmoe
@@ -258,16 +276,16 @@ kmoe_status moe_grouped_ffn(const void *x, int x_dtype, int N, int d, int I, int
     KMOE_TRY(check_ptr(y_perm, "y_perm"));
     if (shared) KMOE_TRY(check_ptr(y_shared, "y_shared"));
     KMOE_TRY(check_ptr(ws, "ws"));
-    const size_t need = kStatusBytes + ((size_t)N * K + N) * I * act_bytes(routed->dtype);
+    const size_t need = kFfnStatusBytes + ((size_t)N * K + N) * I * act_bytes(routed->dtype);
     if (ws_bytes < need) return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
     const ExpertPtrs r = ptrs(routed);
     ExpertPtrs s{};
     if (shared) s = ptrs(shared);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int *status = static_cast<int *>(ws);
-    KMOE_TRY(clear_status(status, st));
+    KMOE_TRY(clear_status(status, st, kFfnStatusBytes));
     return run_ffn(x, x_dtype, N, d, I, E, K, perm_token, offsets, routed->dtype, r, shared ? &s : nullptr,
-                   static_cast<char *>(ws) + kStatusBytes, y_perm, y_shared, status, st);
+                   static_cast<char *>(ws) + kFfnStatusBytes, y_perm, y_shared, status, st);
 }
 
 kmoe_status moe_combine(const void *y_perm, const void *y_shared, int y_in_dtype, const float *topk_w,
@@ -318,7 +336,7 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
     int32_t *idx = topk_idx_out ? topk_idx_out : L.idx;
     float *w = topk_w_out ? topk_w_out : L.w;
     int32_t *counts = counts_out ? counts_out : L.counts;
-    KMOE_TRY(clear_status(L.status, st));
+    KMOE_TRY(clear_status(L.status, st, kFfnStatusBytes));
     if (N <= kFusedRouteTokens) {
         KMOE_TRY(launch_route_small(x, x_dtype, w_router, bias, N, d, E, K, L.logits, idx, w, counts, L.offsets,
                                     L.perm, L.inv, L.status, st));

@@ -159,6 +159,15 @@ kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, in
 // Batches of at least this many tokens take the tensor-core FFN.
 constexpr int kTcMinTokens = 256;
 
+// Swap-AB tensor-core FFN for smaller batches (BF16 activations; BF16 or
+// E4M3 + FP32 block-scale weights). `sync` holds kSyncInts counters that
+// must be zero at launch (a unit counter and one counter per expert).
+constexpr int kSyncInts = 1088;
+kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
+                            const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
+                            __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status,
+                            int *sync, cudaStream_t st);
+
 kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dtype,
                            const float *w, const int32_t *inv, int N, int K, int d, void *y,
                            int y_dtype, cudaStream_t st);

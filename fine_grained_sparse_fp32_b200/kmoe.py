@@ -16,6 +16,10 @@ from ._build import LIB
 KMOE_OK, KMOE_ERR_INVALID_ARG, KMOE_ERR_UNSUPPORTED, KMOE_ERR_CUDA, KMOE_ERR_WORKSPACE, KMOE_ERR_DEVICE = range(6)
 KMOE_F32, KMOE_BF16, KMOE_E4M3_B128 = 0, 1, 2
 
+# Bytes at the head of a moe_grouped_ffn workspace: the status word, tickets
+# and the grouped FFN's unit counters (include/kmoe.h).
+FFN_STATUS_BYTES = (64 + 1088) * 4
+
 EXPORTS = ["moe_workspace_size", "moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn",
            "moe_combine", "moe_forward", "moe_device_status", "moe_last_error", "moe_abi_version"]
 
@@ -177,7 +181,7 @@ def moe_grouped_ffn(x, layer, perm_token, offsets, with_shared=True, ws=None, st
         y_perm = torch.empty((N * K, d), dtype=adt, device=x.device)
         y_shared = torch.empty((N, d), dtype=adt, device=x.device) if with_shared else None
     if ws is None:
-        ws = torch.empty(256 + (N * K + N) * I * (4 if adt == torch.float32 else 2), dtype=torch.uint8,
+        ws = torch.empty(FFN_STATUS_BYTES + (N * K + N) * I * (4 if adt == torch.float32 else 2), dtype=torch.uint8,
                          device=x.device)
     routed = experts_of(layer, "routed")
     shared = experts_of(layer, "shared") if with_shared else None

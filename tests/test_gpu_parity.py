@@ -134,6 +134,61 @@ def test_grouped_ffn_matches_oracle(name, N):
     assert row_rel_err(got_s, ref_s) <= TOL[cfg.w_dtype]
 
 
+@pytest.mark.parametrize("name,N", [("decode", 200), ("fp8_decode", 200), ("decode", 33)])
+def test_grouped_ffn_crowded_experts(name, N):
+    """Every token on the same six experts: groups of N rows, several 32-row
+    token chunks per expert on the small-batch path, and 378 empty groups."""
+    dev, host = layer_inputs(name, N)
+    cfg = host["cfg"]
+    idx = np.tile(np.array([383, 0, 17, 200, 5, 6], dtype=np.int32), (cfg.N, 1))
+    counts, offsets, perm, inv = oracle.permute(idx, cfg.E)
+    y_perm, y_shared = kmoe.moe_grouped_ffn(dev["x"], dev, torch.from_numpy(perm).cuda(),
+                                            torch.from_numpy(offsets).cuda())
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([[0, cfg.N * cfg.K - 1], np.arange(0, cfg.N * cfg.K, 7)]))
+    expert_of_row = np.searchsorted(offsets, rows, side="right") - 1
+    ref = oracle.expert_outputs(host, perm[rows], expert_of_row, nthreads=threads())
+    got = y_perm[torch.from_numpy(rows).cuda().long()].float().cpu().numpy()
+    assert row_rel_err(got, ref) <= TOL[cfg.w_dtype]
+    toks = np.arange(cfg.N)
+    ref_s = oracle.expert_outputs(host, toks, np.full(len(toks), cfg.E), nthreads=threads())
+    assert row_rel_err(y_shared.float().cpu().numpy(), ref_s) <= TOL[cfg.w_dtype]
+
+
+@pytest.mark.parametrize("name", ["decode", "fp8_decode", "prefill"])
+def test_grouped_ffn_without_shared_expert(name):
+    dev, host = layer_inputs(name, 40 if name != "prefill" else 300)
+    cfg = host["cfg"]
+    l_ora = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
+    i_ora, _, _ = oracle.select(l_ora, host["bias"], cfg.K)
+    counts, offsets, perm, inv = oracle.permute(i_ora, cfg.E)
+    y_perm, y_shared = kmoe.moe_grouped_ffn(dev["x"], dev, torch.from_numpy(perm).cuda(),
+                                            torch.from_numpy(offsets).cuda(), with_shared=False)
+    torch.cuda.synchronize()
+    assert y_shared is None
+    rows = np.arange(0, cfg.N * cfg.K, 5)
+    expert_of_row = np.searchsorted(offsets, rows, side="right") - 1
+    ref = oracle.expert_outputs(host, perm[rows], expert_of_row, nthreads=threads())
+    got = y_perm[torch.from_numpy(rows).cuda().long()].float().cpu().numpy()
+    assert row_rel_err(got, ref) <= TOL[cfg.w_dtype]
+
+
+def test_fp8_small_batch_flags_activations_outside_f16_range():
+    """The E4M3 small-batch path feeds the tensor cores F16 activations: an
+    |x| beyond the F16 range is reported in the device status word (2)."""
+    dev, host = layer_inputs("fp8_decode", 8)
+    cfg = host["cfg"]
+    x = dev["x"].clone()
+    x[3, 100] = 1.0e6
+    idx = np.tile(np.arange(cfg.K, dtype=np.int32), (cfg.N, 1))
+    _, offsets, perm, _ = oracle.permute(idx, cfg.E)
+    ws = torch.empty(kmoe.FFN_STATUS_BYTES + (cfg.N * cfg.K + cfg.N) * cfg.I * 2, dtype=torch.uint8, device="cuda")
+    kmoe.moe_grouped_ffn(x, dev, torch.from_numpy(perm).cuda(), torch.from_numpy(offsets).cuda(), ws=ws)
+    assert kmoe.moe_device_status(ws) == 2
+    kmoe.moe_grouped_ffn(dev["x"], dev, torch.from_numpy(perm).cuda(), torch.from_numpy(offsets).cuda(), ws=ws)
+    assert kmoe.moe_device_status(ws) == 0
+
+
 # ----------------------------------------------------------- whole layer
 def _forward_and_compare(name, N=None, rows=None, check_all_routing=True):
     dev, host = layer_inputs(name, N)
