@@ -9,9 +9,9 @@
 //
 // Here a 128-row weight tile is the MMA's A operand (M = 128, streamed by
 // TMA in 64-column stages) and the expert's tokens are its B operand
-// (N = 16 or 32 rows), so the tensor cores do the dot products and the SM's
+// (N = 16 rows), so the tensor cores do the dot products and the SM's
 // issue slots stay free: the kernel only moves bytes. Work units:
-//   up unit   (expert, 64 intermediate features, chunk of <= 32 tokens):
+//   up unit   (expert, 64 intermediate features, chunk of <= 16 tokens):
 //             A = [64 gate rows ; 64 up rows] x d, one M = 128 MMA per k16
 //             gives gate in accumulator lanes 0-63 and up in lanes 64-127;
 //             the epilogue pairs them through shared memory and writes
@@ -55,30 +55,31 @@ constexpr int kM = 128;                 // weight rows per unit (MMA M)
 constexpr int kBK = 64;                 // k per BF16 stage: 128 bytes of BF16
 constexpr int kBK8 = 128;               // k per E4M3 stage: one scale block, 128 bytes of E4M3
 __host__ __device__ constexpr int stage_k(bool fp8) { return fp8 ? kBK8 : kBK; }
-constexpr int kNT = 32;                 // tokens per unit at most
-constexpr int kPanel = kNT * 128;       // one 64-element column panel of a B tile (4 KB)
+constexpr int kNT = 16;                 // tokens per unit at most (the MMA's N)
+constexpr int kPanel = kNT * 128;       // one 64-element column panel of a B tile (2 KB)
 constexpr int kUpF = 64;                // intermediate features per up unit
 constexpr int kDnF = 128;               // output features per down unit
 constexpr int kATile = kM * kBK * 2;    // 16 KB
-constexpr int kBTile = kNT * kBK * 2;   // 4 KB
+constexpr int kBTile = kNT * kBK * 2;   // 2 KB
 constexpr int kA8Tile = kM * kBK8;      // 16 KB of E4M3
-constexpr int kB8Tile = kNT * kBK8 * 2;  // 8 KB: two column panels
+constexpr int kB8Tile = kNT * kBK8 * 2;  // 4 KB: two column panels
 constexpr int kNU = 8;                  // unit-info slots
 constexpr int kNAcc = 4;                // accumulators of 32 TMEM columns (N <= 32)
+static_assert(kNT % 16 == 0 && kNT <= 32, "token chunk: a multiple of 16, at most 32");
 constexpr int kAccCols = kNAcc * 32;    // E4M3: A stages follow at this column
 constexpr int kMaxOrd = 1025;
 constexpr long long kWaitLimit = 1LL << 32;   // SM cycles, about 2 s
 
 // BF16 weights: one ring of (A | B) stages.
-constexpr int kStagesBf = 10;
-constexpr int kStageBf = kATile + kBTile;                       // 20 KB
+constexpr int kStagesBf = 11;
+constexpr int kStageBf = kATile + kBTile;                       // 18 KB
 // E4M3 weights: a raw ring (E4M3 A | BF16 B rows) in shared memory and a
 // converted ring: F16 A in tensor memory (64 columns a stage), F16 B in
 // shared memory. Two groups of four converter warps take alternate stages.
-constexpr int kRawStages = 7;
-constexpr int kRawStage = kA8Tile + kB8Tile;                    // 24 KB
+constexpr int kRawStages = 10;
+constexpr int kRawStage = kA8Tile + kB8Tile;                    // 20 KB
 constexpr int kConvStages = 3;
-constexpr int kConvStage = kB8Tile;                             // 8 KB
+constexpr int kConvStage = kB8Tile;                             // 4 KB
 constexpr int kConvGroups = 2;
 __host__ __device__ constexpr int tmem_cols(bool fp8) { return fp8 ? 512 : 128; }
 static_assert(kAccCols + kConvStages * 64 <= 512, "tensor memory columns");
@@ -97,7 +98,7 @@ struct Slot {
     int wrow;                // first weight row in the stacked weight matrix
     int src[kNT];            // B row n: token (up) or dispatched row (down), n < mc
     float ref[2];            // E4M3: largest block scale of the rows (gate or W_d, up)
-    float s[2][64];          // E4M3: block scales of the rows along K
+    float s[2][48];          // E4M3: block scales of the rows along K (d / 128 <= 48)
 };
 
 struct Tail {
@@ -109,8 +110,9 @@ struct Tail {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    int pre[kMaxOrd + 1];        // token-chunk prefix over the group order
     Slot slot[kNU];
+    uint16_t pre[kMaxOrd + 1];   // token-chunk prefix over the group order
+    uint16_t off[kMaxOrd + 1];   // copy of the routed groups' row offsets
     float xch[kUpF][kNT + 1];    // up-unit epilogue: up values handed to the gate warps
 };
 
@@ -120,6 +122,7 @@ __host__ __device__ constexpr size_t ring_bytes(bool fp8)
                : (size_t)kStagesBf * kStageBf;
 }
 __host__ __device__ constexpr size_t smem_bytes(bool fp8) { return 1024 + ring_bytes(fp8) + sizeof(Tail); }
+static_assert(smem_bytes(false) <= 232448 && smem_bytes(true) <= 232448, "227 KB of shared memory per CTA");
 
 struct Maps {
     CUtensorMap g_r, u_r, g_s, u_s;   // up: gate / up rows, box 64 columns x 64 rows
@@ -145,11 +148,13 @@ struct Group {
     bool shared;
 };
 
-__device__ __forceinline__ Group group_at(int o, const Args &a)
+// Batches on this path have N * (K + 1) < 65536, so row offsets and chunk
+// counts fit 16 bits; `off` is the shared-memory copy of `offsets`.
+__device__ __forceinline__ Group group_at(int o, const uint16_t *off, const Args &a)
 {
     if (a.has_shared && o == 0) return {a.E, a.N * a.K, a.N, true};
     const int g = o - a.has_shared;
-    return {g, a.offsets[g], a.offsets[g + 1] - a.offsets[g], false};
+    return {g, off[g], off[g + 1] - off[g], false};
 }
 
 __device__ __forceinline__ int chunks_of(int rows) { return (rows + kNT - 1) / kNT; }
@@ -164,15 +169,17 @@ struct Unit {
     int kb;         // k stages
 };
 
-// pre[o] = token chunks of the groups before o (one warp builds it).
-__device__ void build_prefix(int *pre, const Args &a)
+// off = offsets; pre[o] = token chunks of the groups before o (one warp).
+__device__ void build_prefix(uint16_t *pre, uint16_t *off, const Args &a)
 {
     const int lane = threadIdx.x & 31;
+    for (int i = lane; i <= a.E; i += 32) off[i] = static_cast<uint16_t>(a.offsets[i]);
+    __syncwarp();
     const int per = (a.n_ord + 31) / 32;
     const int o0 = lane * per;
     int sum = 0;
     for (int i = 0; i < per; ++i)
-        if (o0 + i < a.n_ord) sum += chunks_of(group_at(o0 + i, a).rows);
+        if (o0 + i < a.n_ord) sum += chunks_of(group_at(o0 + i, off, a).rows);
     int incl = sum;
 #pragma unroll
     for (int s = 1; s < 32; s <<= 1) {
@@ -182,15 +189,15 @@ __device__ void build_prefix(int *pre, const Args &a)
     int run = incl - sum;
     for (int i = 0; i < per; ++i)
         if (o0 + i < a.n_ord) {
-            pre[o0 + i] = run;
-            run += chunks_of(group_at(o0 + i, a).rows);
+            pre[o0 + i] = static_cast<uint16_t>(run);
+            run += chunks_of(group_at(o0 + i, off, a).rows);
         }
-    if (lane == 31) pre[a.n_ord] = incl;
+    if (lane == 31) pre[a.n_ord] = static_cast<uint16_t>(incl);
 }
 
 // Unit u: up units first (per group: feature tile major, chunk minor), then
 // down units in the same order.
-__device__ __forceinline__ Unit decode(int u, const int *pre, const Args &a)
+__device__ __forceinline__ Unit decode(int u, const uint16_t *pre, const uint16_t *off, const Args &a)
 {
     const int up_tiles = a.I / kUpF, dn_tiles = a.d / kDnF;
     const int total_ch = pre[a.n_ord];
@@ -205,19 +212,19 @@ __device__ __forceinline__ Unit decode(int u, const int *pre, const Args &a)
         else lo = mid + 1;
     }
     U.o = lo - 1;
-    U.G = group_at(U.o, a);
+    U.G = group_at(U.o, off, a);
     const int ch = chunks_of(U.G.rows);
     const int local = v - pre[U.o] * tiles;
     const int tile = local / ch, c = local - tile * ch;
     U.f0 = tile * (U.up ? kUpF : kDnF);
     U.m0 = c * kNT;
     U.mc = min(kNT, U.G.rows - U.m0);
-    U.nmma = U.mc > 16 ? 32 : 16;
+    U.nmma = U.mc > 16 ? 32 : 16;          // <= kNT
     U.kb = (U.up ? a.d : a.I) / a.sk;
     return U;
 }
 
-__device__ __forceinline__ int total_units(const int *pre, const Args &a)
+__device__ __forceinline__ int total_units(const uint16_t *pre, const Args &a)
 {
     return pre[a.n_ord] * (a.I / kUpF + a.d / kDnF);
 }
@@ -249,7 +256,7 @@ __host__ __device__ constexpr uint32_t idesc(int M, int N, bool bf16)
            ((uint32_t)(M >> 4) << 24);
 }
 
-// The block scales of one row block, s[0 .. nkb-1] (nkb <= 64), loaded by a
+// The block scales of one row block, s[0 .. nkb-1] (nkb <= 48), loaded by a
 // whole warp at once: lane l holds s[l] in lo and s[l + 32] in hi (0 past
 // the end). ref() is their maximum (the F16 path's normaliser), at(i) is s[i].
 struct WarpScales {
@@ -341,7 +348,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
         T->abort = 0;
         fence_mbar_init();
     }
-    if (warp == kSchedWarp) build_prefix(T->pre, a);
+    if (warp == kSchedWarp) build_prefix(T->pre, T->off, a);
     if (warp == 0) {
         tmem_alloc(&T->tmem_base, tmem_cols(kFp8));
         tmem_relinquish();
@@ -377,35 +384,39 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 }
                 break;
             }
-            const Unit U = decode(u, T->pre, a);
+            const Unit U = decode(u, T->pre, T->off, a);
             const int row0 = U.G.row0 + U.m0;
-            if (lane < U.mc)
-                sl.src[lane] = U.up ? (U.G.shared ? row0 + lane - a.N * a.K : a.perm[row0 + lane]) : row0 + lane;
             const size_t ge = U.G.shared ? 0 : (size_t)U.G.g;
+            // every global load of the unit is issued before any is used: one round trip
+            int srcv = 0;
+            if (lane < U.mc)
+                srcv = U.up ? (U.G.shared ? row0 + lane - a.N * a.K : a.perm[row0 + lane]) : row0 + lane;
+            WarpScales w0, w1;
+            w0.lo = w0.hi = w1.lo = w1.hi = 0.f;
             if (kFp8) {
-                const float *s0, *s1 = nullptr;
-                int nkb;
                 if (U.up) {
-                    nkb = a.d / 128;
+                    const int nkb = a.d / 128;
                     const size_t off = (ge * (a.I / 128) + U.f0 / 128) * nkb;
-                    s0 = (U.G.shared ? a.sg_s : a.sg_r) + off;
-                    s1 = (U.G.shared ? a.su_s : a.su_r) + off;
+                    w0.load((U.G.shared ? a.sg_s : a.sg_r) + off, nkb);
+                    w1.load((U.G.shared ? a.su_s : a.su_r) + off, nkb);
                 } else {
-                    nkb = a.I / 128;
-                    s0 = (U.G.shared ? a.sd_s : a.sd_r) + (ge * (a.d / 128) + U.f0 / 128) * nkb;
+                    const int nkb = a.I / 128;
+                    w0.load((U.G.shared ? a.sd_s : a.sd_r) + (ge * (a.d / 128) + U.f0 / 128) * nkb, nkb);
                 }
-                WarpScales w0, w1;
-                w0.load(s0, nkb);
-                if (s1) w1.load(s1, nkb);
-                else w1.lo = w1.hi = 0.f;
-                sl.s[0][lane] = w0.lo; sl.s[0][lane + 32] = w0.hi;
-                sl.s[1][lane] = w1.lo; sl.s[1][lane + 32] = w1.hi;
+            }
+            const int need = (a.I / kUpF) * chunks_of(U.G.rows);
+            int done = need;
+            if (!U.up && lane == 0) done = ld_acquire(a.up_done + U.o);
+            if (lane < U.mc) sl.src[lane] = srcv;
+            if (kFp8) {
+                sl.s[0][lane] = w0.lo;
+                sl.s[1][lane] = w1.lo;
+                if (lane < 16) { sl.s[0][lane + 32] = w0.hi; sl.s[1][lane + 32] = w1.hi; }
                 const float r0 = w0.ref(), r1 = w1.ref();
                 if (lane == 0) { sl.ref[0] = r0; sl.ref[1] = r1; }
             }
             bool good = true;
-            if (!U.up && lane == 0) {        // the expert's H rows come from up units of any CTA
-                const int need = (a.I / kUpF) * chunks_of(U.G.rows);
+            if (lane == 0 && done < need) {       // the expert's H rows come from up units of any CTA
                 const long long t0 = clock64();
                 while (ld_acquire(a.up_done + U.o) < need) {
                     if (*abort) { good = false; break; }
@@ -549,23 +560,24 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
             if (!mbar_wait(&T->tfull[acc], (us / kNAcc) & 1, abort, a.err, kWaitLimit)) break;
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + acc * 32;
-            uint32_t v[32];
-            tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(v));
-            if (sl.nmma > 16) tmem_ld16(taddr + 16, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
+            uint32_t v[kNT];
+#pragma unroll
+            for (int c = 0; c < kNT; c += 16)
+                if (c < sl.nmma) tmem_ld16(taddr + c, *reinterpret_cast<uint32_t(*)[16]>(v + c));
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(&T->tempty[acc]);
             if (up) {
                 if (warp >= 2) {
 #pragma unroll
-                    for (int n = 0; n < 32; ++n)
+                    for (int n = 0; n < kNT; ++n)
                         if (n < mc) T->xch[row - kUpF][n] = __uint_as_float(v[n]) * sref;
                 }
                 epi_sync();
                 if (warp < 2) {
                     __nv_bfloat16 *dst = a.h + (size_t)r0 * a.I + f0 + row;
 #pragma unroll
-                    for (int n = 0; n < 32; ++n)
+                    for (int n = 0; n < kNT; ++n)
                         if (n < mc) {
                             const float g = __uint_as_float(v[n]) * sref;
                             dst[(size_t)n * a.I] = __float2bfloat16_rn(g * sigmoidf_(g) * T->xch[row][n]);
@@ -578,7 +590,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 __nv_bfloat16 *dst = shared ? a.y_shared + (size_t)(r0 - a.N * a.K) * a.d : a.y_perm + (size_t)r0 * a.d;
                 dst += f0 + row;
 #pragma unroll
-                for (int n = 0; n < 32; ++n)
+                for (int n = 0; n < kNT; ++n)
                     if (n < mc) dst[(size_t)n * a.d] = __float2bfloat16_rn(__uint_as_float(v[n]) * sref);
                 epi_sync();
             }
@@ -638,11 +650,12 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                     }
                     tmem_st32(tq + half * 32, o);
                 }
-                // B: BF16 token (or H) rows -> F16 at the same swizzled positions
+                // B: BF16 token (or H) rows -> F16 at the same swizzled positions;
+                // a panel holds kNT rows of eight 16-byte chunks
 #pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
+                for (int i4 = 0; i4 < kB8Tile / 16 / 128; ++i4) {
                     const int c16 = q + i4 * 128;
-                    if (((c16 & 255) >> 3) < nmma) {
+                    if (((c16 % (kNT * 8)) >> 3) < nmma) {
                         const uint4 w = *reinterpret_cast<const uint4 *>(Braw + c16 * 16);
                         const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
                         uint32_t p[4];
@@ -726,6 +739,7 @@ kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, 
 {
     if (E + 1 > kMaxOrd || E + 2 > kSyncInts) return fail(KMOE_ERR_UNSUPPORTED, "swap-AB FFN: too many experts");
     if (d % kDnF || I % 128) return fail(KMOE_ERR_UNSUPPORTED, "swap-AB FFN: d, I must be multiples of 128");
+    if ((long long)N * (K + 1) >= 65536) return fail(KMOE_ERR_UNSUPPORTED, "swap-AB FFN: batch too large");
     const bool fp8 = w_dtype == KMOE_E4M3_B128;
     const ExpertPtrs sh = shared ? *shared : routed;     // unused maps still need a valid base
     Maps m{};
