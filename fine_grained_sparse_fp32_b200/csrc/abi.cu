@@ -136,15 +136,16 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype)
     return L;
 }
 
-static bool use_tc(int x_dtype, int w_dtype, int N, int d)
-{
-    return x_dtype == KMOE_BF16 && (w_dtype == KMOE_BF16 || w_dtype == KMOE_E4M3_B128) && N >= kTcMinTokens &&
-           d % 256 == 0;
-}
+// Grouped FFN kernel for a batch (BF16 activations, BF16 or E4M3 weights,
+// d % 256 == 0): below kTcMinTokens tokens the swap-AB tcgen05 kernel
+// (weights as M, 16-token chunks as N), from there the tokens-as-M tcgen05
+// kernel; FP32 activations or weights take the CUDA-core streaming kernel.
+enum FfnPath { kPathStream, kPathSwap, kPathTc };
 
-static bool use_swap(int x_dtype, int w_dtype)
+static FfnPath ffn_path(int x_dtype, int w_dtype, int N, int d)
 {
-    return x_dtype == KMOE_BF16 && (w_dtype == KMOE_BF16 || w_dtype == KMOE_E4M3_B128);
+    if (x_dtype != KMOE_BF16 || (w_dtype != KMOE_BF16 && w_dtype != KMOE_E4M3_B128) || d % 256) return kPathStream;
+    return N < kTcMinTokens ? kPathSwap : kPathTc;
 }
 
 // `status` is the workspace status block: the status word, tickets, then
@@ -153,11 +154,12 @@ static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int 
                            const int32_t *offsets, int w_dtype, const ExpertPtrs &r, const ExpertPtrs *s,
                            void *h, void *y_perm, void *y_shared, int *status, cudaStream_t st)
 {
-    if (use_swap(x_dtype, w_dtype) && !use_tc(x_dtype, w_dtype, N, d))
+    const FfnPath path = ffn_path(x_dtype, w_dtype, N, d);
+    if (path == kPathSwap)
         return launch_ffn_swap(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, w_dtype, r, s,
                                static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
                                static_cast<__nv_bfloat16 *>(y_shared), status, status + kSyncOffset, st);
-    if (use_tc(x_dtype, w_dtype, N, d))
+    if (path == kPathTc)
         return launch_ffn_tc(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, w_dtype, r, s,
                              static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
                              static_cast<__nv_bfloat16 *>(y_shared), status, st);

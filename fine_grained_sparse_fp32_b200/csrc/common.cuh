@@ -159,9 +159,9 @@ kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, in
 // Batches of at least this many tokens take the tensor-core FFN.
 constexpr int kTcMinTokens = 256;
 
-// Swap-AB tensor-core FFN for smaller batches (BF16 activations; BF16 or
-// E4M3 + FP32 block-scale weights). `sync` holds kSyncInts counters that
-// must be zero at launch (a unit counter and one counter per expert).
+// Swap-AB tensor-core FFN for small batches (BF16 activations; BF16 or
+// E4M3 + FP32 block-scale weights; d % 256 == 0). `sync` holds kSyncInts
+// counters that must be zero at launch (a unit counter and one per expert).
 constexpr int kSyncInts = 1088;
 kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
                             const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,

@@ -1,46 +1,49 @@
-// Grouped SwiGLU expert FFN for small batches (decode) on the tcgen05 tensor
-// cores, weights as the M operand ("swap-AB").
+// Grouped SwiGLU expert FFN on the tcgen05 tensor cores with the weights as
+// the M operand ("swap-AB").
 //
 // "Inside Kolibri 1" (flozi.net), routing section: every routed or shared
 // expert is a SwiGLU MLP (two d -> I projections, SiLU(gate) * up, one
-// I -> d projection, no biases). At decode a routed expert sees one or two
-// tokens, so the layer is a weight stream: each selected expert's 3*d*I
-// weights cross HBM once and meet a handful of token rows.
+// I -> d projection, no biases). Each selected expert's 3*d*I weights cross
+// HBM once and meet the expert's token rows; at decode one or two rows, so
+// the layer is a weight stream. This kernel serves batches below 256 tokens
+// (prefill batches take the tokens-as-M kernel in ffn_tc.cu).
 //
-// Here a 128-row weight tile is the MMA's A operand (M = 128, streamed by
-// TMA in 64-column stages) and the expert's tokens are its B operand
-// (N = 16 rows), so the tensor cores do the dot products and the SM's
-// issue slots stay free: the kernel only moves bytes. Work units:
-//   up unit   (expert, 64 intermediate features, chunk of <= 16 tokens):
-//             A = [64 gate rows ; 64 up rows] x d, one M = 128 MMA per k16
-//             gives gate in accumulator lanes 0-63 and up in lanes 64-127;
-//             the epilogue pairs them through shared memory and writes
-//             H = SiLU(gate) * up;
-//   down unit (expert, 128 output features, same token chunk):
-//             A = W_d rows x I, B = the chunk's H rows.
-// One persistent launch runs every up unit, then every down unit: a CTA
-// claims units from a global counter, and the producer of a down unit waits
-// (bounded) until all up units of that expert have published their H rows.
-// Units are small (655 KB / 131 KB of BF16 weights), so the grid finishes
-// within one down unit of the mean.
+// A 128-row weight tile is the MMA's A operand (M = 128, streamed by TMA in
+// 128-byte column stages) and a chunk of the expert's token rows is its B
+// operand, with N = the chunk's rows rounded up to 16 (chunks of at most
+// kNT = 16 rows are compiled). Work units:
+//   up unit   (expert, 128 intermediate features, token chunk): the gate rows
+//             and the up rows of those features are two A tiles multiplied
+//             by the same B; gate and up accumulate side by side in tensor
+//             memory, so the thread holding a feature's accumulator lane
+//             has both and writes H = SiLU(gate) * up;
+//   down unit (expert, 256 output features, token chunk): two A tiles of
+//             128 W_d rows each against the chunk's H rows (B), so a stage
+//             carries as many weight bytes as an up unit's.
+// One persistent launch runs every up unit, then every down unit. A
+// scheduler warp claims units from a global counter, resolves each one into
+// a shared-memory slot (rows, weight rows, scales) and, before a down unit,
+// waits (bounded) until all up units of that expert have published H.
 //
 // Warp roles (one CTA per SM):
-//   warps 0-3  epilogue: tcgen05.ld of the accumulator, SwiGLU or the BF16
-//              cast, global stores; hands the accumulator back to the MMA;
+//   warps 0-3  epilogue: tcgen05.ld of the accumulators, SwiGLU or the BF16
+//              cast, global stores; hands the accumulator back to the MMA
+//              (with chunks above 32 rows, warps 7-10 form a second group);
 //   warp  4    one thread issues tcgen05.mma / tcgen05.commit;
-//   warp  5    producer: claims units, TMA loads of the weight tiles,
-//              cp.async gathers of the token (or H) rows;
-//   warps 6-9  E4M3 weights only: converters.
+//   warp  5    producer: TMA loads of the weight tiles (lane 0), cp.async
+//              gathers of the token (or H) rows (all lanes);
+//   warp  6    scheduler;
+//   warps 7-14 E4M3 weights only: two groups of converters.
 // E4M3 weights ("Inside Kolibri 1", FP8 section: 128 x 128 blocks with one
 // FP32 scale each) arrive by TMA as bytes. Converter warps decode them
 // exactly to F16 (hardware e4m3x2 -> f16x2), multiply each row by
 // s_kb / s_ref (its block's scale over the largest scale of the row block,
-// so the factor is at most 1 and nothing overflows), and write the tile
+// so the factor is at most 1 and nothing overflows), and write the tiles
 // straight into tensor memory with tcgen05.st: the MMA takes A from tensor
-// memory, so the decoded weights never cross shared memory. The token rows
-// are converted to F16 for the B operand, the MMA is F16 x F16 with FP32
-// accumulation, and the epilogue multiplies by s_ref. |x| must stay inside
-// the F16 range (65504); a value outside it sets device status 2.
+// memory. The token rows are converted to F16 for the B operand, the MMA is
+// F16 x F16 with FP32 accumulation, and the epilogue multiplies by s_ref.
+// |x| must stay inside the F16 range (65504); a value outside it sets
+// device status 2.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -51,82 +54,88 @@ using namespace sm100;
 
 namespace swp {
 
-constexpr int kM = 128;                 // weight rows per unit (MMA M)
-constexpr int kBK = 64;                 // k per BF16 stage: 128 bytes of BF16
-constexpr int kBK8 = 128;               // k per E4M3 stage: one scale block, 128 bytes of E4M3
-__host__ __device__ constexpr int stage_k(bool fp8) { return fp8 ? kBK8 : kBK; }
-constexpr int kNT = 16;                 // tokens per unit at most (the MMA's N)
-constexpr int kPanel = kNT * 128;       // one 64-element column panel of a B tile (2 KB)
-constexpr int kUpF = 64;                // intermediate features per up unit
-constexpr int kDnF = 128;               // output features per down unit
-constexpr int kATile = kM * kBK * 2;    // 16 KB
-constexpr int kBTile = kNT * kBK * 2;   // 2 KB
-constexpr int kA8Tile = kM * kBK8;      // 16 KB of E4M3
-constexpr int kB8Tile = kNT * kBK8 * 2;  // 4 KB: two column panels
+constexpr int kM = 128;                 // weight rows per tile (MMA M)
+constexpr int kATile = kM * 128;        // 16 KB: 128 rows x 128 bytes
+constexpr int kF = 128;                 // intermediate features per up unit (gate and up rows)
+constexpr int kFD = 256;                // output features per down unit (two tiles of W_d rows)
 constexpr int kNU = 8;                  // unit-info slots
-constexpr int kNAcc = 4;                // accumulators of 32 TMEM columns (N <= 32)
-static_assert(kNT % 16 == 0 && kNT <= 32, "token chunk: a multiple of 16, at most 32");
-constexpr int kAccCols = kNAcc * 32;    // E4M3: A stages follow at this column
 constexpr int kMaxOrd = 1025;
 constexpr long long kWaitLimit = 1LL << 32;   // SM cycles, about 2 s
+constexpr int kSmemLimit = 232448;            // 227 KB per CTA
 
-// BF16 weights: one ring of (A | B) stages.
-constexpr int kStagesBf = 11;
-constexpr int kStageBf = kATile + kBTile;                       // 18 KB
-// E4M3 weights: a raw ring (E4M3 A | BF16 B rows) in shared memory and a
-// converted ring: F16 A in tensor memory (64 columns a stage), F16 B in
-// shared memory. Two groups of four converter warps take alternate stages.
-constexpr int kRawStages = 10;
-constexpr int kRawStage = kA8Tile + kB8Tile;                    // 20 KB
-constexpr int kConvStages = 3;
-constexpr int kConvStage = kB8Tile;                             // 4 KB
+// Per configuration: kNT = token rows per unit at most (16 at decode, 128 at
+// prefill); E4M3 weights use 128-column stages (one scale block), BF16 64.
+template <bool kFp8, int kNT>
+struct Cfg {
+    static constexpr int BK = kFp8 ? 128 : 64;           // k per stage
+    static constexpr int Panel = kNT * 128;              // one 64-column panel of a B tile
+    static constexpr int BTile = kNT * BK * 2;           // token rows of a stage (16-bit)
+    static constexpr int Stage = 2 * kATile + BTile;     // gate | up (or W_d) | tokens
+    static constexpr int AccW = 2 * kNT;                 // accumulator slot: gate | up
+    static constexpr int NAcc = 256 / kNT < 4 ? 256 / kNT : 4;
+    static constexpr int AccCols = NAcc * AccW;
+    static constexpr int ConvStages = kFp8 ? 3 : 0;      // E4M3: decoded tiles in tensor memory
+    static constexpr int ConvCols = 128;                 // gate | up, 64 columns of F16 each
+    static constexpr int TmemCols = kFp8 ? 512 : (AccCols <= 128 ? 128 : AccCols <= 256 ? 256 : 512);
+    static constexpr int Stages = kFp8 ? 5 : (kNT <= 16 ? 6 : 4);
+    static constexpr int ConvB = ConvStages * BTile;     // E4M3: F16 token tiles
+    static constexpr int Ring = Stages * Stage + ConvB;
+    static constexpr int EpiGroups = kNT > 32 ? 2 : 1;   // groups of four epilogue warps
+    static constexpr int Warps = kFp8 ? 15 : (EpiGroups == 2 ? 11 : 7);
+    static constexpr int EpiThreads = 128 * EpiGroups;
+    static constexpr int W = kNT < 32 ? kNT : 32;        // accumulator columns an epilogue warp loads at once
+    static_assert(kNT % 16 == 0 && kNT >= 16 && kNT <= 128, "token chunk");
+    static_assert(AccCols + ConvStages * ConvCols <= TmemCols && TmemCols <= 512, "tensor memory columns");
+};
+
+// Warps 0-3 (and 7-10 when EpiGroups == 2) run the epilogue; E4M3
+// converters are warps 7-14.
+constexpr int kMmaWarp = 4, kProdWarp = 5, kSchedWarp = 6, kConvWarp = 7, kEpi2Warp = 7;
 constexpr int kConvGroups = 2;
-__host__ __device__ constexpr int tmem_cols(bool fp8) { return fp8 ? 512 : 128; }
-static_assert(kAccCols + kConvStages * 64 <= 512, "tensor memory columns");
-
-constexpr int kEpiWarps = 4, kMmaWarp = 4, kProdWarp = 5, kSchedWarp = 6, kConvWarp = 7;
-__host__ __device__ constexpr int threads_of(bool fp8) { return (fp8 ? kConvWarp + 4 * kConvGroups : kConvWarp) * 32; }
 
 // A unit as the scheduler warp resolved it: everything the other roles need,
 // so that none of them touches global memory to set a unit up.
+template <int kNT>
 struct Slot {
     int u;                   // unit index, -1 = no more work
     int up, shared, o;       // kind, shared expert, position in the group order
-    int g;                   // expert (E = shared)
     int f0, mc, nmma, kb;    // first feature, token rows, MMA N, stages
     int row0;                // first dispatched row of the chunk
     int wrow;                // first weight row in the stacked weight matrix
-    int src[kNT];            // B row n: token (up) or dispatched row (down), n < mc
     float ref[2];            // E4M3: largest block scale of the rows (gate or W_d, up)
     float s[2][48];          // E4M3: block scales of the rows along K (d / 128 <= 48)
+    int src[kNT];            // B row n: token (up) or dispatched row (down), n < mc
 };
 
+template <int kNT>
 struct Tail {
-    uint64_t full[kRawStages > kStagesBf ? kRawStages : kStagesBf];
-    uint64_t empty[kRawStages > kStagesBf ? kRawStages : kStagesBf];
-    uint64_t cfull[kConvStages], cempty[kConvStages];
+    uint64_t full[6], empty[6];          // weight + token ring (Stages <= 6)
+    uint64_t cfull[3], cempty[3];        // E4M3: decoded stages
     uint64_t ufull[kNU], uempty[kNU];
-    uint64_t tfull[kNAcc], tempty[kNAcc];
-    uint64_t drain;
+    uint64_t tfull[4], tempty[4];
+    uint64_t drain, pstart;              // pstart: the producer has started a unit
     uint32_t tmem_base;
     int abort;
-    Slot slot[kNU];
-    uint16_t pre[kMaxOrd + 1];   // token-chunk prefix over the group order
-    uint16_t off[kMaxOrd + 1];   // copy of the routed groups' row offsets
-    float xch[kUpF][kNT + 1];    // up-unit epilogue: up values handed to the gate warps
+    Slot<kNT> slot[kNU];
+    alignas(16) uint16_t stage[8][16][32];   // epilogue transposes (16-byte reads): 16 tokens x 32 features per warp
+    int pre[kMaxOrd + 1];        // token-chunk prefix over the group order
+    int off[kMaxOrd + 1];        // copy of the routed groups' row offsets
 };
 
-__host__ __device__ constexpr size_t ring_bytes(bool fp8)
+static_assert(offsetof(Tail<16>, stage) % 16 == 0 && offsetof(Tail<128>, stage) % 16 == 0, "16-byte staging");
+static_assert(sizeof(Tail<16>) % 16 == 0 && sizeof(Tail<128>) % 16 == 0, "tail size");
+
+template <bool kFp8, int kNT>
+__host__ __device__ constexpr size_t smem_bytes()
 {
-    return fp8 ? (size_t)kRawStages * kRawStage + (size_t)kConvStages * kConvStage
-               : (size_t)kStagesBf * kStageBf;
+    return 1024 + (size_t)Cfg<kFp8, kNT>::Ring + sizeof(Tail<kNT>);
 }
-__host__ __device__ constexpr size_t smem_bytes(bool fp8) { return 1024 + ring_bytes(fp8) + sizeof(Tail); }
-static_assert(smem_bytes(false) <= 232448 && smem_bytes(true) <= 232448, "227 KB of shared memory per CTA");
 
 struct Maps {
-    CUtensorMap g_r, u_r, g_s, u_s;   // up: gate / up rows, box 64 columns x 64 rows
-    CUtensorMap d_r, d_s;             // down: W_d rows, box 64 columns x 128 rows
+    CUtensorMap g_r, u_r, g_s, u_s;   // up: gate / up rows
+    CUtensorMap d_r, d_s;             // down: W_d rows (boxes of 128 rows x 128 bytes)
+    CUtensorMap xg;                   // x [N, d]: boxes of 1 row x 64 columns (gathered four at a time)
+    CUtensorMap hb;                   // H [N*K + N, I]: boxes of kNT rows x 64 columns
 };
 
 struct Args {
@@ -139,25 +148,25 @@ struct Args {
     int *claim;                       // unit counter (zero at launch)
     int *up_done;                     // [groups] finished up units (zero at launch)
     int N, K, E, d, I, has_shared, n_ord;
-    int sk;                           // k per stage (stage_k)
+    int sk;                           // k per stage
+    int nt;                           // token rows per unit at most
 };
 
-// Group order: [shared (if any), routed 0 .. E-1].
+// Group order: [shared (if any), routed 0 .. E-1]; `off` is the
+// shared-memory copy of `offsets`.
 struct Group {
     int g, row0, rows;
     bool shared;
 };
 
-// Batches on this path have N * (K + 1) < 65536, so row offsets and chunk
-// counts fit 16 bits; `off` is the shared-memory copy of `offsets`.
-__device__ __forceinline__ Group group_at(int o, const uint16_t *off, const Args &a)
+__device__ __forceinline__ Group group_at(int o, const int *off, const Args &a)
 {
     if (a.has_shared && o == 0) return {a.E, a.N * a.K, a.N, true};
     const int g = o - a.has_shared;
     return {g, off[g], off[g + 1] - off[g], false};
 }
 
-__device__ __forceinline__ int chunks_of(int rows) { return (rows + kNT - 1) / kNT; }
+__device__ __forceinline__ int chunks_of(int rows, int nt) { return (rows + nt - 1) / nt; }
 
 struct Unit {
     bool up;
@@ -165,21 +174,21 @@ struct Unit {
     int o;          // position in the group order
     int f0;         // first feature (up: intermediate, down: output)
     int m0, mc;     // first row of the chunk inside the group, rows in it
-    int nmma;       // MMA N: 16 or 32
+    int nmma;       // MMA N: mc rounded up to 16
     int kb;         // k stages
 };
 
 // off = offsets; pre[o] = token chunks of the groups before o (one warp).
-__device__ void build_prefix(uint16_t *pre, uint16_t *off, const Args &a)
+__device__ void build_prefix(int *pre, int *off, const Args &a)
 {
     const int lane = threadIdx.x & 31;
-    for (int i = lane; i <= a.E; i += 32) off[i] = static_cast<uint16_t>(a.offsets[i]);
+    for (int i = lane; i <= a.E; i += 32) off[i] = a.offsets[i];
     __syncwarp();
     const int per = (a.n_ord + 31) / 32;
     const int o0 = lane * per;
     int sum = 0;
     for (int i = 0; i < per; ++i)
-        if (o0 + i < a.n_ord) sum += chunks_of(group_at(o0 + i, off, a).rows);
+        if (o0 + i < a.n_ord) sum += chunks_of(group_at(o0 + i, off, a).rows, a.nt);
     int incl = sum;
 #pragma unroll
     for (int s = 1; s < 32; s <<= 1) {
@@ -189,17 +198,18 @@ __device__ void build_prefix(uint16_t *pre, uint16_t *off, const Args &a)
     int run = incl - sum;
     for (int i = 0; i < per; ++i)
         if (o0 + i < a.n_ord) {
-            pre[o0 + i] = static_cast<uint16_t>(run);
-            run += chunks_of(group_at(o0 + i, off, a).rows);
+            pre[o0 + i] = run;
+            run += chunks_of(group_at(o0 + i, off, a).rows, a.nt);
         }
-    if (lane == 31) pre[a.n_ord] = static_cast<uint16_t>(incl);
+    if (lane == 31) pre[a.n_ord] = incl;
 }
 
-// Unit u: up units first (per group: feature tile major, chunk minor), then
+// Unit u: up units first (per group: feature tile major, chunk minor, so the
+// chunks of one weight tile run back to back and share it in L2), then the
 // down units in the same order.
-__device__ __forceinline__ Unit decode(int u, const uint16_t *pre, const uint16_t *off, const Args &a)
+__device__ __forceinline__ Unit decode(int u, const int *pre, const int *off, const Args &a)
 {
-    const int up_tiles = a.I / kUpF, dn_tiles = a.d / kDnF;
+    const int up_tiles = a.I / kF, dn_tiles = a.d / kFD;
     const int total_ch = pre[a.n_ord];
     Unit U;
     U.up = u < up_tiles * total_ch;
@@ -213,20 +223,20 @@ __device__ __forceinline__ Unit decode(int u, const uint16_t *pre, const uint16_
     }
     U.o = lo - 1;
     U.G = group_at(U.o, off, a);
-    const int ch = chunks_of(U.G.rows);
+    const int ch = chunks_of(U.G.rows, a.nt);
     const int local = v - pre[U.o] * tiles;
     const int tile = local / ch, c = local - tile * ch;
-    U.f0 = tile * (U.up ? kUpF : kDnF);
-    U.m0 = c * kNT;
-    U.mc = min(kNT, U.G.rows - U.m0);
-    U.nmma = U.mc > 16 ? 32 : 16;          // <= kNT
+    U.f0 = tile * (U.up ? kF : kFD);
+    U.m0 = c * a.nt;
+    U.mc = min(a.nt, U.G.rows - U.m0);
+    U.nmma = (U.mc + 15) & ~15;
     U.kb = (U.up ? a.d : a.I) / a.sk;
     return U;
 }
 
-__device__ __forceinline__ int total_units(const uint16_t *pre, const Args &a)
+__device__ __forceinline__ int total_units(const int *pre, const Args &a)
 {
-    return pre[a.n_ord] * (a.I / kUpF + a.d / kDnF);
+    return pre[a.n_ord] * (a.I / kF + a.d / kFD);
 }
 
 __device__ __forceinline__ int ld_acquire(const int *p)
@@ -246,7 +256,8 @@ __device__ __forceinline__ void fence_proxy_async_global()
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+template <int kThreads>
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
 
 // Instruction descriptor of tcgen05.mma kind::f16: A and B both BF16 or both
 // F16 (K-major), FP32 accumulator, M x N.
@@ -258,7 +269,7 @@ __host__ __device__ constexpr uint32_t idesc(int M, int N, bool bf16)
 
 // The block scales of one row block, s[0 .. nkb-1] (nkb <= 48), loaded by a
 // whole warp at once: lane l holds s[l] in lo and s[l + 32] in hi (0 past
-// the end). ref() is their maximum (the F16 path's normaliser), at(i) is s[i].
+// the end). ref() is their maximum (the F16 path's normaliser).
 struct WarpScales {
     float lo, hi;
     __device__ __forceinline__ void load(const float *s, int nkb)
@@ -273,10 +284,6 @@ struct WarpScales {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         return m;
-    }
-    __device__ __forceinline__ float at(int i) const
-    {
-        return __shfl_sync(0xffffffffu, i < 32 ? lo : hi, i & 31);
     }
 };
 
@@ -306,33 +313,55 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b)
     return r;
 }
 
+// Decodes one 128-byte E4M3 row (128-byte swizzle, row q of its tile), times
+// r, into 64 columns of tensor memory at `taddr` (this warp's lanes).
+__device__ __forceinline__ void convert_row_tmem(const uint8_t *tile, int q, uint32_t r2, uint32_t taddr)
+{
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t o[32];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+            const int c = half * 4 + c4;
+            const uint4 w = *reinterpret_cast<const uint4 *>(tile + q * 128 + ((c ^ (q & 7)) << 4));
+            const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                uint32_t lo, hi;
+                e4m3x4_to_f16(wd[h], lo, hi);
+                o[c4 * 8 + 2 * h] = hmul2(lo, r2);
+                o[c4 * 8 + 2 * h + 1] = hmul2(hi, r2);
+            }
+        }
+        tmem_st32(taddr + half * 32, o);
+    }
+}
+
 }  // namespace swp
 
 using namespace swp;
 
 enum : int { kErrF16Range = 2 };
 
-template <bool kFp8>
-__global__ void __launch_bounds__(threads_of(kFp8), 1)
+template <bool kFp8, int kNT>
+__global__ void __launch_bounds__(Cfg<kFp8, kNT>::Warps * 32, 1)
 ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
 {
-    constexpr int S = kFp8 ? kRawStages : kStagesBf;     // producer ring
-    constexpr int SB = kFp8 ? kRawStage : kStageBf;
-    constexpr int ABytes = kFp8 ? kA8Tile : kATile;      // A bytes a stage receives by TMA
-    constexpr int BK = stage_k(kFp8);
+    using C = Cfg<kFp8, kNT>;
+    constexpr int SA = C::Stages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *conv = smem + (size_t)kRawStages * kRawStage;   // E4M3 only
-    Tail *T = reinterpret_cast<Tail *>(smem + ring_bytes(kFp8));
+    uint8_t *convb = smem + (size_t)SA * C::Stage;           // E4M3: F16 token tiles
+    Tail<kNT> *T = reinterpret_cast<Tail<kNT> *>(smem + C::Ring);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort = &T->abort;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&T->full[s], 1 + 32);              // TMA expect_tx + 32 cp.async arrivals
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&T->full[s], 1);                   // TMA expect_tx (weights and token rows)
             mbar_init(&T->empty[s], kFp8 ? 128 : 1);     // converters | tcgen05.commit
         }
-        for (int s = 0; s < kConvStages; ++s) {
+        for (int s = 0; s < C::ConvStages; ++s) {
             mbar_init(&T->cfull[s], 128);
             mbar_init(&T->cempty[s], 1);
         }
@@ -340,22 +369,24 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
             mbar_init(&T->ufull[j], 1);
             mbar_init(&T->uempty[j], 1);
         }
-        for (int c = 0; c < kNAcc; ++c) {
+        for (int c = 0; c < C::NAcc; ++c) {
             mbar_init(&T->tfull[c], 1);
-            mbar_init(&T->tempty[c], 128);
+            mbar_init(&T->tempty[c], C::EpiThreads);
         }
         mbar_init(&T->drain, 1);
+        mbar_init(&T->pstart, 1);
         T->abort = 0;
         fence_mbar_init();
     }
     if (warp == kSchedWarp) build_prefix(T->pre, T->off, a);
     if (warp == 0) {
-        tmem_alloc(&T->tmem_base, tmem_cols(kFp8));
+        tmem_alloc(&T->tmem_base, C::TmemCols);
         tmem_relinquish();
     }
     if (warp == kProdWarp && lane == 0) {
         prefetch_map(&maps.g_r); prefetch_map(&maps.u_r); prefetch_map(&maps.d_r);
         if (a.has_shared) { prefetch_map(&maps.g_s); prefetch_map(&maps.u_s); prefetch_map(&maps.d_s); }
+        prefetch_map(&maps.xg); prefetch_map(&maps.hb);
     }
     tc_fence_before();
     __syncthreads();
@@ -364,19 +395,23 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
 
     if (warp == kSchedWarp) {
         // ----------------------------------------------------------- scheduler
-        // Claims units one ahead, resolves each into a slot (rows, weight
-        // rows, E4M3 scales) and, for a down unit, waits until the expert's
-        // up units have published H. Runs up to kNU units ahead of the
-        // epilogue, so these global-memory round trips overlap the stream.
+        // Claims units one ahead, resolves each into a slot and, for a down
+        // unit, waits until the expert's up units have published H. Runs up
+        // to kNU units ahead of the epilogue, so its global-memory round trips
+        // overlap the weight stream.
+        // A unit is claimed only once the producer has started the previous
+        // one, so a CTA never holds work that it will reach much later (a
+        // down unit claimed by anyone waits on the up units the others hold).
         const int total = total_units(T->pre, a);
-        int ahead = lane == 0 ? atomicAdd(a.claim, 1) : 0;
         for (int us = 0;; ++us) {
             const int j = us % kNU;
             if (!mbar_wait(&T->uempty[j], ((us / kNU) & 1) ^ 1, abort, a.err, kWaitLimit)) break;
-            int u = __shfl_sync(0xffffffffu, ahead, 0);
+            if (us > 0 && !mbar_wait(&T->pstart, (us - 1) & 1, abort, a.err, kWaitLimit)) break;
+            int u = 0;
+            if (lane == 0) u = atomicAdd(a.claim, 1);
+            u = __shfl_sync(0xffffffffu, u, 0);
             if (u >= total) u = -1;
-            if (lane == 0 && u >= 0) ahead = atomicAdd(a.claim, 1);
-            Slot &sl = T->slot[j];
+            Slot<kNT> &sl = T->slot[j];
             if (u < 0) {
                 if (lane == 0) {
                     sl.u = -1;
@@ -388,9 +423,15 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
             const int row0 = U.G.row0 + U.m0;
             const size_t ge = U.G.shared ? 0 : (size_t)U.G.g;
             // every global load of the unit is issued before any is used: one round trip
-            int srcv = 0;
-            if (lane < U.mc)
-                srcv = U.up ? (U.G.shared ? row0 + lane - a.N * a.K : a.perm[row0 + lane]) : row0 + lane;
+            constexpr int RPL = (kNT + 31) / 32;         // rows per lane
+            int srcv[RPL];
+#pragma unroll
+            for (int i = 0; i < RPL; ++i) {
+                const int n = lane + 32 * i;
+                srcv[i] = 0;
+                if (n < U.mc)
+                    srcv[i] = U.up ? (U.G.shared ? row0 + n - a.N * a.K : a.perm[row0 + n]) : row0 + n;
+            }
             WarpScales w0, w1;
             w0.lo = w0.hi = w1.lo = w1.hi = 0.f;
             if (kFp8) {
@@ -399,15 +440,19 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                     const size_t off = (ge * (a.I / 128) + U.f0 / 128) * nkb;
                     w0.load((U.G.shared ? a.sg_s : a.sg_r) + off, nkb);
                     w1.load((U.G.shared ? a.su_s : a.su_r) + off, nkb);
-                } else {
+                } else {        // the two row blocks of W_d
                     const int nkb = a.I / 128;
-                    w0.load((U.G.shared ? a.sd_s : a.sd_r) + (ge * (a.d / 128) + U.f0 / 128) * nkb, nkb);
+                    const float *sd = (U.G.shared ? a.sd_s : a.sd_r) + (ge * (a.d / 128) + U.f0 / 128) * nkb;
+                    w0.load(sd, nkb);
+                    w1.load(sd + nkb, nkb);
                 }
             }
-            const int need = (a.I / kUpF) * chunks_of(U.G.rows);
+            const int need = (a.I / kF) * chunks_of(U.G.rows, a.nt);
             int done = need;
             if (!U.up && lane == 0) done = ld_acquire(a.up_done + U.o);
-            if (lane < U.mc) sl.src[lane] = srcv;
+#pragma unroll
+            for (int i = 0; i < RPL; ++i)
+                if (lane + 32 * i < U.mc) sl.src[lane + 32 * i] = srcv[i];
             if (kFp8) {
                 sl.s[0][lane] = w0.lo;
                 sl.s[1][lane] = w1.lo;
@@ -435,7 +480,6 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 sl.up = U.up;
                 sl.shared = U.G.shared;
                 sl.o = U.o;
-                sl.g = U.G.g;
                 sl.f0 = U.f0;
                 sl.mc = U.mc;
                 sl.nmma = U.nmma;
@@ -449,91 +493,103 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
         }
     } else if (warp == kProdWarp) {
         // ------------------------------------------------------------ producer
+        // Weight tiles (lane 0) and token tiles all by TMA: a down unit's H
+        // rows are contiguous (one box of kNT rows per 64-column panel); an
+        // up unit's token rows are gathered four at a time (lane i: rows
+        // 4i .. 4i+3), rows past the chunk repeating its first row.
         const uint64_t pol_w = policy_evict_first();    // weights: streamed once
         const uint64_t pol_a = policy_evict_last();     // token / H rows: reused by many units
+        constexpr int NP = C::BK / 64;                  // 64-column panels per stage
         uint32_t it = 0;
         bool ok = true;
         for (int us = 0;; ++us) {
             const int j = us % kNU;
             if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-            const Slot &sl = T->slot[j];
+            const Slot<kNT> &sl = T->slot[j];
             if (sl.u < 0) break;
             const bool up = sl.up, shared = sl.shared;
-            const int kb_n = sl.kb, wrow = sl.wrow, mc = sl.mc, nmma = sl.nmma;
-            const int n = lane;                         // B row of this lane
-            const bool live = n < nmma, valid = n < mc;
-            const int srow = valid ? sl.src[n] : 0;
+            const int kb_n = sl.kb, wrow = sl.wrow, mc = sl.mc, nmma = sl.nmma, r0 = sl.row0;
+            const bool gl = up && 4 * lane < nmma;       // this lane gathers four token rows
+            int gr[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) gr[q] = 4 * lane + q < mc ? sl.src[4 * lane + q] : sl.src[0];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&T->pstart);
             if (!up) fence_proxy_async_global();        // H written by other CTAs, seen through the scheduler
-            const __nv_bfloat16 *src = up ? a.x + (size_t)srow * a.d : a.h + (size_t)srow * a.I;
             const CUtensorMap *m0 = up ? (shared ? &maps.g_s : &maps.g_r) : (shared ? &maps.d_s : &maps.d_r);
             const CUtensorMap *m1 = shared ? &maps.u_s : &maps.u_r;
+            const uint32_t bbytes = (uint32_t)(up ? nmma : kNT) * 128 * NP;
             for (int kb = 0; kb < kb_n; ++kb, ++it) {
-                const int s = it % S;
-                if (!mbar_wait(&T->empty[s], ((it / S) & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-                uint8_t *A = smem + (size_t)s * SB;
-                uint8_t *B = A + ABytes;
+                const int s = it % SA;
+                if (!mbar_wait(&T->empty[s], ((it / SA) & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                uint8_t *A = smem + (size_t)s * C::Stage;
+                uint8_t *B = A + 2 * kATile;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&T->full[s], ABytes);
-                    if (up) {
-                        tma_load_2d_hint(A, m0, &T->full[s], kb * BK, wrow, pol_w);
-                        tma_load_2d_hint(A + ABytes / 2, m1, &T->full[s], kb * BK, wrow, pol_w);
-                    } else {
-                        tma_load_2d_hint(A, m0, &T->full[s], kb * BK, wrow, pol_w);
-                    }
-                }
-                if (live) {     // 64-element column panels of 128-byte swizzled rows
-                    const uint32_t dst = smem_u32(B) + n * 128;
-                    const __nv_bfloat16 *sp = src + kb * BK;
+                    mbar_arrive_expect_tx(&T->full[s], 2 * kATile + bbytes);
+                    tma_load_2d_hint(A, m0, &T->full[s], kb * C::BK, wrow, pol_w);
+                    // second tile: the up rows of the same features, or the next 128 W_d rows
+                    tma_load_2d_hint(A + kATile, up ? m1 : m0, &T->full[s], kb * C::BK, up ? wrow : wrow + kM, pol_w);
+                    if (!up)
 #pragma unroll
-                    for (int c = 0; c < BK / 8; ++c)
-                        cp_async16_hint(dst + (c >> 3) * kPanel + (((c & 7) ^ (n & 7)) << 4), sp + c * 8,
-                                        valid ? 16u : 0u, pol_a);
+                        for (int p = 0; p < NP; ++p)
+                            tma_load_2d_hint(B + p * C::Panel, &maps.hb, &T->full[s], kb * C::BK + p * 64, r0, pol_a);
                 }
-                cp_async_arrive_noinc(&T->full[s]);
+                __syncwarp();
+                if (gl)
+#pragma unroll
+                    for (int p = 0; p < NP; ++p)
+                        tma_gather4_hint(B + p * C::Panel + lane * 512, &maps.xg, &T->full[s], kb * C::BK + p * 64,
+                                         gr[0], gr[1], gr[2], gr[3], pol_a);
             }
             if (!ok) break;
         }
-        cp_async_wait_all();
         if (!ok && lane == 0)    // let in-flight TMA loads land before the CTA exits
-            for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
-                mbar_wait_drain(&T->full[j % S], (j / S) & 1, kWaitLimit);
+            for (uint32_t j = it > (uint32_t)SA ? it - SA : 0; j < it; ++j)
+                mbar_wait_drain(&T->full[j % SA], (j / SA) & 1, kWaitLimit);
     } else if (warp == kMmaWarp) {
         // ----------------------------------------------------------------- MMA
         if (lane == 0) {
-            constexpr int CS = kFp8 ? kConvStages : kStagesBf;
             uint32_t it = 0;
             for (int us = 0;; ++us) {
                 const int j = us % kNU;
                 if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, kWaitLimit)) break;
-                const Slot &sl = T->slot[j];
+                const Slot<kNT> &sl = T->slot[j];
                 if (sl.u < 0) break;
+                const bool up = sl.up;
                 const int kb_n = sl.kb;
-                const int acc = us % kNAcc;
-                if (!mbar_wait(&T->tempty[acc], ((us / kNAcc) & 1) ^ 1, abort, a.err, kWaitLimit)) break;
+                const int acc = us % C::NAcc;
+                if (!mbar_wait(&T->tempty[acc], ((us / C::NAcc) & 1) ^ 1, abort, a.err, kWaitLimit)) break;
                 tc_fence_after();
-                const uint32_t dcol = tmem + acc * 32;
+                const uint32_t dg = tmem + acc * C::AccW;          // gate (or W_d) accumulator
+                const uint32_t du = dg + kNT;                      // up accumulator
                 const uint32_t id = idesc(kM, sl.nmma, !kFp8);
                 bool ok = true;
                 for (int kb = 0; kb < kb_n; ++kb, ++it) {
-                    const int s = it % CS;
-                    uint64_t *fullb = kFp8 ? &T->cfull[s] : &T->full[s];
-                    if (!mbar_wait(fullb, (it / CS) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-                    tc_fence_after();
-                    if (kFp8) {       // A: F16 in tensor memory (8 columns per k16); B: F16 panels in shared memory
-                        const uint32_t at = tmem + kAccCols + s * 64;
-                        const uint64_t bd = sw128_kmajor_desc(smem_u32(conv + (size_t)s * kConvStage));
+                    if (kFp8) {       // A: F16 in tensor memory (8 columns per k16); B: F16 panels
+                        const int cs = it % C::ConvStages;
+                        if (!mbar_wait(&T->cfull[cs], (it / C::ConvStages) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t at = tmem + C::AccCols + cs * C::ConvCols;
+                        const uint64_t bd = sw128_kmajor_desc(smem_u32(convb + (size_t)cs * C::BTile));
 #pragma unroll
-                        for (int k = 0; k < kBK8 / 16; ++k)
-                            umma_f16_tmem_a(dcol, at + k * 8, bd + (uint64_t)(((k >> 2) * kPanel + (k & 3) * 32) >> 4), id,
-                                            (kb | k) != 0);
-                        umma_commit(&T->cempty[s]);
+                        for (int k = 0; k < C::BK / 16; ++k) {
+                            const uint64_t bk = bd + (uint64_t)(((k >> 2) * C::Panel + (k & 3) * 32) >> 4);
+                            umma_f16_tmem_a(dg, at + k * 8, bk, id, (kb | k) != 0);
+                            umma_f16_tmem_a(du, at + 64 + k * 8, bk, id, (kb | k) != 0);
+                        }
+                        umma_commit(&T->cempty[cs]);
                     } else {
-                        const uint32_t sa = smem_u32(smem + (size_t)s * kStageBf);
-                        const uint64_t ad = sw128_kmajor_desc(sa);
-                        const uint64_t bd = sw128_kmajor_desc(sa + kATile);
+                        const int s = it % SA;
+                        if (!mbar_wait(&T->full[s], (it / SA) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t sa = smem_u32(smem + (size_t)s * C::Stage);
+                        const uint64_t a0 = sw128_kmajor_desc(sa), a1 = sw128_kmajor_desc(sa + kATile);
+                        const uint64_t bd = sw128_kmajor_desc(sa + 2 * kATile);
 #pragma unroll
-                        for (int k = 0; k < kBK / 16; ++k)
-                            umma_bf16(dcol, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), id, (kb | k) != 0);
+                        for (int k = 0; k < C::BK / 16; ++k) {
+                            umma_bf16(dg, a0 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), id, (kb | k) != 0);
+                            umma_bf16(du, a1 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), id, (kb | k) != 0);
+                        }
                         umma_commit(&T->empty[s]);
                     }
                 }
@@ -544,126 +600,126 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
             mbar_wait_drain(&T->drain, 0, kWaitLimit);
         }
         __syncwarp();
-    } else if (warp < kEpiWarps) {
+    } else if (warp < 4 || (C::EpiGroups == 2 && warp >= kEpi2Warp)) {
         // ------------------------------------------------------------ epilogue
-        const int row = warp * 32 + lane;              // accumulator lane = weight row of the unit
+        // A warp reads its quadrant of accumulator lanes (32 features of the
+        // unit), W token columns at a time; group eg takes every EpiGroups-th
+        // block. Results go through a 16 x 32 shared-memory transpose so that
+        // each global store writes 16 bytes (8 features of one token).
+        constexpr int W = C::W;
+        const int quad = warp & 3, eg = warp < 4 ? 0 : 1;
+        uint16_t *stg = &T->stage[eg * 4 + quad][0][0];
         for (int us = 0;; ++us) {
             const int j = us % kNU;
             if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, kWaitLimit)) break;
-            const Slot &sl = T->slot[j];
+            const Slot<kNT> &sl = T->slot[j];
             if (sl.u < 0) break;
             const bool up = sl.up, shared = sl.shared;
-            const int mc = sl.mc, f0 = sl.f0, r0 = sl.row0, o = sl.o;
-            // E4M3: rows 0-63 of an up unit are gate rows, 64-127 up rows
-            const float sref = kFp8 ? sl.ref[(up && warp >= 2) ? 1 : 0] : 1.f;
-            const int acc = us % kNAcc;
-            if (!mbar_wait(&T->tfull[acc], (us / kNAcc) & 1, abort, a.err, kWaitLimit)) break;
+            const int mc = sl.mc, nmma = sl.nmma, f0 = sl.f0, r0 = sl.row0, o = sl.o;
+            const float s0 = kFp8 ? sl.ref[0] : 1.f, s1 = kFp8 ? sl.ref[1] : 1.f;
+            const int acc = us % C::NAcc;
+            if (!mbar_wait(&T->tfull[acc], (us / C::NAcc) & 1, abort, a.err, kWaitLimit)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + acc * 32;
-            uint32_t v[kNT];
+            const uint32_t tg = tmem + ((uint32_t)(quad * 32) << 16) + acc * C::AccW;
+            const int ld = up ? a.I : a.d;               // row stride of the output
+            __nv_bfloat16 *dst = up ? a.h + (size_t)r0 * a.I
+                                    : (shared ? a.y_shared + (size_t)(r0 - a.N * a.K) * a.d : a.y_perm + (size_t)r0 * a.d);
+            dst += f0 + quad * 32;
+            // up: one pass, gate and up accumulators combined; down: the two
+            // W_d tiles (features f0 .. f0+127 and f0+128 .. f0+255) in turn
+#pragma unroll 1
+            for (int t = 0; t < (up ? 1 : 2); ++t)
+#pragma unroll 1
+            for (int c = eg * W; c < nmma; c += W * C::EpiGroups) {
+                uint32_t g[W], u[W];
+                const uint32_t ta = tg + t * kNT + c;
+                if (W == 32) {
+                    tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(g));
+                    if (up) tmem_ld32(tg + kNT + c, *reinterpret_cast<uint32_t(*)[32]>(u));
+                } else {
+                    tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(g));
+                    if (up) tmem_ld16(tg + kNT + c, *reinterpret_cast<uint32_t(*)[16]>(u));
+                }
+                tmem_ld_wait();
+                const float sa = t ? s1 : s0;
+                __nv_bfloat16 *dt = dst + t * kM;
 #pragma unroll
-            for (int c = 0; c < kNT; c += 16)
-                if (c < sl.nmma) tmem_ld16(taddr + c, *reinterpret_cast<uint32_t(*)[16]>(v + c));
-            tmem_ld_wait();
+                for (int half = 0; half < W / 16; ++half) {
+#pragma unroll
+                    for (int n = 0; n < 16; ++n) {
+                        const float gv = __uint_as_float(g[half * 16 + n]) * sa;
+                        const float val = up ? gv * sigmoidf_(gv) * __uint_as_float(u[half * 16 + n]) * s1 : gv;
+                        stg[n * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int idx = lane + 32 * hh, n = idx >> 2, p = idx & 3;
+                        const int tok = c + half * 16 + n;
+                        if (tok < mc)
+                            *reinterpret_cast<uint4 *>(dt + (size_t)tok * ld + p * 8) =
+                                *reinterpret_cast<const uint4 *>(stg + n * 32 + p * 8);
+                    }
+                    __syncwarp();
+                }
+            }
             tc_fence_before();
             mbar_arrive(&T->tempty[acc]);
-            if (up) {
-                if (warp >= 2) {
-#pragma unroll
-                    for (int n = 0; n < kNT; ++n)
-                        if (n < mc) T->xch[row - kUpF][n] = __uint_as_float(v[n]) * sref;
-                }
-                epi_sync();
-                if (warp < 2) {
-                    __nv_bfloat16 *dst = a.h + (size_t)r0 * a.I + f0 + row;
-#pragma unroll
-                    for (int n = 0; n < kNT; ++n)
-                        if (n < mc) {
-                            const float g = __uint_as_float(v[n]) * sref;
-                            dst[(size_t)n * a.I] = __float2bfloat16_rn(g * sigmoidf_(g) * T->xch[row][n]);
-                        }
-                    __threadfence();
-                }
-                epi_sync();
-                if (threadIdx.x == 0) red_release_add(a.up_done + o, 1);
-            } else {
-                __nv_bfloat16 *dst = shared ? a.y_shared + (size_t)(r0 - a.N * a.K) * a.d : a.y_perm + (size_t)r0 * a.d;
-                dst += f0 + row;
-#pragma unroll
-                for (int n = 0; n < kNT; ++n)
-                    if (n < mc) dst[(size_t)n * a.d] = __float2bfloat16_rn(__uint_as_float(v[n]) * sref);
-                epi_sync();
+            if (up) __threadfence();                   // H visible before the expert's count is raised
+            epi_sync<C::EpiThreads>();
+            if (threadIdx.x == 0) {
+                if (up) red_release_add(a.up_done + o, 1);
+                mbar_arrive(&T->uempty[j]);
             }
-            if (threadIdx.x == 0) mbar_arrive(&T->uempty[j]);
         }
     } else if (kFp8 && warp >= kConvWarp) {
         // ---------------------------------------------------------- converters
         // A warp reaches only its own quadrant of tensor-memory lanes, so the
-        // A row a thread converts is its lane in that quadrant. Group `grp`
-        // takes the stages it with it % kConvGroups == grp.
+        // rows a thread converts are its lane in that quadrant (of the gate and
+        // of the up tile). Group `grp` takes the stages it with it % 2 == grp.
         const int quad = warp & 3, grp = (warp - kConvWarp) / 4;
-        const int q = quad * 32 + lane;                 // A row; B chunks q + 128 i
+        const int q = quad * 32 + lane;
         uint32_t it = 0;
         bool ok = true;
         for (int us = 0; ok; ++us) {
             const int j = us % kNU;
             if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, kWaitLimit)) break;
-            const Slot &sl = T->slot[j];
+            const Slot<kNT> &sl = T->slot[j];
             if (sl.u < 0) break;
+            const bool up = sl.up;
             const int kb_n = sl.kb, nmma = sl.nmma;
-            // this row's scales: up units = gate (rows 0-63) or up (64-127); down = W_d
-            const int which = (sl.up && quad >= 2) ? 1 : 0;
-            const float ref = sl.ref[which];
-            const float inv = ref > 0.f ? 1.f / ref : 0.f;
-            const float *srow = sl.s[which];
+            const float inv0 = sl.ref[0] > 0.f ? 1.f / sl.ref[0] : 0.f;
+            const float inv1 = sl.ref[1] > 0.f ? 1.f / sl.ref[1] : 0.f;
             bool range_ok = true;
             for (int kb = 0; kb < kb_n; ++kb, ++it) {
                 if ((int)(it % kConvGroups) != grp) continue;
-                const int rs = it % kRawStages, cs = it % kConvStages;
-                const float r = srow[kb] * inv;                      // in [0, 1]
-                if (!mbar_wait(&T->full[rs], (it / kRawStages) & 1, abort, a.err, kWaitLimit) ||
-                    !mbar_wait(&T->cempty[cs], ((it / kConvStages) & 1) ^ 1, abort, a.err, kWaitLimit)) {
+                const int s = it % SA, cs = it % C::ConvStages;
+                const float r0 = sl.s[0][kb] * inv0, r1 = sl.s[1][kb] * inv1;     // in [0, 1]
+                if (!mbar_wait(&T->full[s], (it / SA) & 1, abort, a.err, kWaitLimit) ||
+                    !mbar_wait(&T->cempty[cs], ((it / C::ConvStages) & 1) ^ 1, abort, a.err, kWaitLimit)) {
                     ok = false;
                     break;
                 }
-                const uint8_t *A8 = smem + (size_t)rs * kRawStage;
-                const uint8_t *Braw = A8 + kA8Tile;
-                uint8_t *B = conv + (size_t)cs * kConvStage;
-                // A row q: 128 E4M3 bytes (128-byte swizzle) -> 128 F16 * r -> 64 columns of tensor memory
-                const uint32_t r2 = pack_f16x2(r, r);
-                const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16) + kAccCols + cs * 64;
+                const uint8_t *A8 = smem + (size_t)s * C::Stage;
+                const uint8_t *Braw = A8 + 2 * kATile;
+                uint8_t *B = convb + (size_t)cs * C::BTile;
+                const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16) + C::AccCols + cs * C::ConvCols;
+                convert_row_tmem(A8, q, pack_f16x2(r0, r0), tq);
+                convert_row_tmem(A8 + kATile, q, pack_f16x2(r1, r1), tq + 64);
+                // B: BF16 token (or H) rows -> F16 at the same swizzled positions
+                // (a panel holds kNT rows of eight 16-byte chunks)
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t o[32];
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const int c = half * 4 + c4;
-                        const uint4 w = *reinterpret_cast<const uint4 *>(A8 + q * 128 + ((c ^ (q & 7)) << 4));
-                        const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            uint32_t lo, hi;
-                            e4m3x4_to_f16(wd[h], lo, hi);
-                            o[c4 * 8 + 2 * h] = hmul2(lo, r2);
-                            o[c4 * 8 + 2 * h + 1] = hmul2(hi, r2);
-                        }
-                    }
-                    tmem_st32(tq + half * 32, o);
-                }
-                // B: BF16 token (or H) rows -> F16 at the same swizzled positions;
-                // a panel holds kNT rows of eight 16-byte chunks
-#pragma unroll
-                for (int i4 = 0; i4 < kB8Tile / 16 / 128; ++i4) {
-                    const int c16 = q + i4 * 128;
+                for (int i = 0; i < C::BTile / 16 / 128; ++i) {
+                    const int c16 = q + i * 128;
                     if (((c16 % (kNT * 8)) >> 3) < nmma) {
                         const uint4 w = *reinterpret_cast<const uint4 *>(Braw + c16 * 16);
                         const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
                         uint32_t p[4];
                         float mx = 0.f;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float f0 = bf16_lo(wd[i]), f1 = bf16_hi(wd[i]);
-                            p[i] = pack_f16x2(f0, f1);
+                        for (int e = 0; e < 4; ++e) {
+                            const float f0 = bf16_lo(wd[e]), f1 = bf16_hi(wd[e]);
+                            p[e] = pack_f16x2(f0, f1);
                             mx = fmaxf(mx, fmaxf(fabsf(f0), fabsf(f1)));
                         }
                         if (!(mx <= 65504.f)) range_ok = false;
@@ -674,7 +730,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 fence_proxy_async();
                 tc_fence_before();
                 mbar_arrive(&T->cfull[cs]);
-                mbar_arrive(&T->empty[rs]);
+                mbar_arrive(&T->empty[s]);
             }
             if (!range_ok) atomicCAS(a.err, kErrNone, kErrF16Range);
         }
@@ -683,7 +739,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, tmem_cols(kFp8));
+        tmem_dealloc(tmem, C::TmemCols);
     }
 }
 
@@ -701,22 +757,35 @@ static PFN_cuTensorMapEncodeTiled_v12000 swap_encode_fn()
     return fn;
 }
 
-// Weight map over a row-major [rows, cols] matrix, box of 128-byte rows
-// (64 BF16 or 128 E4M3 columns) x box_rows, 128-byte swizzle: the layout
-// the MMA reads (BF16), and one the converters read without bank conflicts
-// (E4M3).
-static bool weight_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, int box_rows, bool fp8)
+// Weight map over a row-major [rows, cols] matrix, box of 128 rows x 128
+// bytes (64 BF16 or 128 E4M3 columns), 128-byte swizzle: the layout the MMA
+// reads (BF16), and one the converters read without bank conflicts (E4M3).
+static bool weight_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, bool fp8)
 {
     auto fn = swap_encode_fn();
     if (!fn) return false;
     const uint64_t es = fp8 ? 1 : 2;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * es};
-    cuuint32_t box[2] = {(cuuint32_t)(fp8 ? kBK8 : kBK), (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / es), (cuuint32_t)kM};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base),
-              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// BF16 activation map over [rows, cols], box of box_rows x 64 columns,
+// 128-byte swizzle (the layout of a B tile panel).
+static bool act_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, int box_rows)
+{
+    auto fn = swap_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -732,22 +801,33 @@ static int swap_sm_count()
     return n;
 }
 
+template <bool kFp8, int kNT>
+static void launch_cfg(const Maps &m, const Args &a, cudaStream_t st)
+{
+    using C = Cfg<kFp8, kNT>;
+    constexpr size_t smem = smem_bytes<kFp8, kNT>();
+    static_assert(smem <= (size_t)kSmemLimit, "shared memory per CTA");
+    auto k = ffn_swap_kernel<kFp8, kNT>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<swap_sm_count(), C::Warps * 32, smem, st>>>(m, a);
+}
+
 kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
                             const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
                             __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status,
                             int *sync, cudaStream_t st)
 {
+    constexpr int token_chunk = 16;
     if (E + 1 > kMaxOrd || E + 2 > kSyncInts) return fail(KMOE_ERR_UNSUPPORTED, "swap-AB FFN: too many experts");
-    if (d % kDnF || I % 128) return fail(KMOE_ERR_UNSUPPORTED, "swap-AB FFN: d, I must be multiples of 128");
-    if ((long long)N * (K + 1) >= 65536) return fail(KMOE_ERR_UNSUPPORTED, "swap-AB FFN: batch too large");
+    if (d % kFD || I % kF) return fail(KMOE_ERR_UNSUPPORTED, "swap-AB FFN: d %% 256, I %% 128 must be 0");
     const bool fp8 = w_dtype == KMOE_E4M3_B128;
     const ExpertPtrs sh = shared ? *shared : routed;     // unused maps still need a valid base
     Maps m{};
-    const bool ok = weight_map(&m.g_r, routed.wg, (uint64_t)E * I, d, kUpF, fp8) &&
-                    weight_map(&m.u_r, routed.wu, (uint64_t)E * I, d, kUpF, fp8) &&
-                    weight_map(&m.g_s, sh.wg, I, d, kUpF, fp8) && weight_map(&m.u_s, sh.wu, I, d, kUpF, fp8) &&
-                    weight_map(&m.d_r, routed.wd, (uint64_t)E * d, I, kDnF, fp8) &&
-                    weight_map(&m.d_s, sh.wd, d, I, kDnF, fp8);
+    const bool ok = weight_map(&m.g_r, routed.wg, (uint64_t)E * I, d, fp8) &&
+                    weight_map(&m.u_r, routed.wu, (uint64_t)E * I, d, fp8) &&
+                    weight_map(&m.g_s, sh.wg, I, d, fp8) && weight_map(&m.u_s, sh.wu, I, d, fp8) &&
+                    weight_map(&m.d_r, routed.wd, (uint64_t)E * d, I, fp8) && weight_map(&m.d_s, sh.wd, d, I, fp8) &&
+                    act_map(&m.xg, x, N, d, 1) && act_map(&m.hb, h, (uint64_t)N * K + N, I, token_chunk);
     if (!ok) return fail(KMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     Args a{};
     a.x = x;
@@ -764,17 +844,10 @@ kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, 
     a.N = N; a.K = K; a.E = E; a.d = d; a.I = I;
     a.has_shared = shared ? 1 : 0;
     a.n_ord = E + a.has_shared;
-    a.sk = stage_k(fp8);
-    const int grid = swap_sm_count();
-    if (fp8) {
-        constexpr size_t smem = smem_bytes(true);
-        cudaFuncSetAttribute(ffn_swap_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        ffn_swap_kernel<true><<<grid, threads_of(true), smem, st>>>(m, a);
-    } else {
-        constexpr size_t smem = smem_bytes(false);
-        cudaFuncSetAttribute(ffn_swap_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        ffn_swap_kernel<false><<<grid, threads_of(false), smem, st>>>(m, a);
-    }
+    a.sk = fp8 ? Cfg<true, 16>::BK : Cfg<false, 16>::BK;
+    a.nt = token_chunk;
+    if (fp8) launch_cfg<true, token_chunk>(m, a, st);
+    else launch_cfg<false, token_chunk>(m, a, st);
     return check_launch("ffn_swap");
 }
 
