@@ -35,6 +35,28 @@ METRIC = "MoE-layer tokens/s at 1 B200 (decode N=32, prefill N=8192); % of HBM/t
 ROTATE = 8           # distinct token batches cycled through the timed steps
 
 
+# DRAM bytes (read + write) per launch of the dominant decode kernel
+# (ffn_swap_kernel), from one ncu capture of `bench.py --capture <layer>`
+# (dram__bytes_read.sum + dram__bytes_write.sum, mean over 6 launches). They
+# hold only for the kernel sources they were measured on: the key is a hash
+# of those files, and a changed kernel reports no traffic until re-measured.
+TRAFFIC_SOURCES = ("fine_grained_sparse_fp32_b200/csrc/ffn_swap.cu", "fine_grained_sparse_fp32_b200/csrc/sm100.cuh",
+                   "fine_grained_sparse_fp32_b200/csrc/common.cuh")
+TRAFFIC = {"5211395fdc28e5a0": {"decode": (1206.1 + 1.0) * 1e6, "fp8_decode": (603.4 + 1.64) * 1e6}}
+
+
+def kernel_traffic(layer):
+    import hashlib
+    h = hashlib.sha256()
+    try:
+        for f in TRAFFIC_SOURCES:
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return TRAFFIC.get(h.hexdigest()[:16], {}).get(layer)
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -330,9 +352,9 @@ def main():
                        "l2": "inputs larger than L2: ~%.2f GB of expert weights per step, %d rotating token batches"
                              % (alg["expert_weight_bytes"] / 1e9, ROTATE),
                        "cuda_graph": not args.no_graph},
-            "roofline": {"bound": "hbm", "kernel": "moe_grouped_ffn (ffn_up + ffn_down)",
+            "roofline": {"bound": "hbm", "kernel": "moe_grouped_ffn: ffn_swap_kernel (up and down units, one launch)",
                          "achieved": ffn_gbs, "peak": hbm, "unit": "GB/s", "frac": ffn_gbs / hbm,
-                         "traffic": None, "peak_kind": peak_kind + " burst",
+                         "traffic": kernel_traffic("decode"), "peak_kind": peak_kind + " burst",
                          "layer_achieved": layer_gbs, "layer_frac": layer_gbs / hbm,
                          "algorithmic_bytes_per_launch": alg["ffn_bytes"], "launch_ms": r["ffn_ms"]},
             "e2e": {"value": dec.N * world / (r["e2e_ms"]["ms"] / 1e3), "unit": "tokens/s",
@@ -368,6 +390,7 @@ def main():
                 "frac": max(t_hbm, t_tc) * 1e3 / xms, "tflops": xalg["flops"] / (xms / 1e3) / 1e12,
                 "ffn_ms": r_x["ffn_ms"], "ffn_gbs": xalg["ffn_bytes"] / (r_x["ffn_ms"] / 1e3) / 1e9,
                 "gpu_launches_per_step": launches_per_step(xcfg), "clocks": r_x["clocks"],
+                "traffic": kernel_traffic(name),
             }
         if world == 1:
             try:
