@@ -109,6 +109,13 @@ __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162flo
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
 
+// SiLU(z) * u for the tensor-core FFN epilogues: z / (1 + e^-z) with the
+// hardware exponential and reciprocal (__expf, __fdividef; a few ulp of
+// FP32, far below the BF16 rounding of the result). z -> -inf gives 0
+// (e^-z overflows to inf and __fdividef returns 0). The router's mixture
+// weights use the IEEE sigmoidf_ above.
+__device__ __forceinline__ float silu_mul(float z, float u) { return __fdividef(z, 1.f + __expf(-z)) * u; }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

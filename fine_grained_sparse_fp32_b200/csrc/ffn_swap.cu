@@ -648,7 +648,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
 #pragma unroll
                     for (int n = 0; n < 16; ++n) {
                         const float gv = __uint_as_float(g[half * 16 + n]) * sa;
-                        const float val = up ? gv * sigmoidf_(gv) * __uint_as_float(u[half * 16 + n]) * s1 : gv;
+                        const float val = up ? silu_mul(gv, __uint_as_float(u[half * 16 + n]) * s1) : gv;
                         stg[n * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
                     }
                     __syncwarp();

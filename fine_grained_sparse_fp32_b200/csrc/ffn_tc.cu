@@ -196,7 +196,7 @@ __device__ __forceinline__ void epilogue_half(uint32_t tbase, const Tile &T, con
             for (int q = 0; q < 8; ++q) {
                 const float g0 = __uint_as_float(g[2 * q]), g1 = __uint_as_float(g[2 * q + 1]);
                 const float u0 = __uint_as_float(u[2 * q]), u1 = __uint_as_float(u[2 * q + 1]);
-                packed[q] = pack_bf16x2(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1);
+                packed[q] = pack_bf16x2(silu_mul(g0, u0), silu_mul(g1, u1));
             }
             if (valid) {
                 uint4 *o = reinterpret_cast<uint4 *>(dst + c);
@@ -378,34 +378,46 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN);
-            uint32_t it = 0, at = 0;
+            // Tensor memory holds two 256-column halves. A tile with one
+            // m-tile takes the half that the previous single tile did not,
+            // so its MMAs overlap that tile's epilogue; a tile with two
+            // m-tiles takes both (starting with the half drained first).
+            uint32_t it = 0, use0 = 0, use1 = 0;     // uses of half 0 / half 1 so far
+            int hn = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++at) {
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 const Tile T = decode_tile(t, tail->pre, a, bn);
+                const int h0 = hn, h1 = hn ^ 1;
+                const uint32_t c0 = h0 ? use1 : use0, c1 = h0 ? use0 : use1;
                 for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
                     const int s = it % kStages;
                     if (!mbar_wait(&tail->full[s], (it / kStages) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-                    if (kb == 0 &&   // half 0 drained by the previous tile's epilogue
-                        !mbar_wait(&tail->tempty[0], (at & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                    if (kb == 0 &&   // half h0 drained by the epilogue of its last use
+                        !mbar_wait(&tail->tempty[h0], (c0 & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + (size_t)s * kStage);
                     const uint64_t a0 = sw128_kmajor_desc(sa);
                     const uint64_t bd = sw128_kmajor_desc(sa + 2 * kATile);
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16(tmem, a0 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
-                    if (kb == 0 &&   // half 1 drained (waited for even when unused, to keep phases)
-                        !mbar_wait(&tail->tempty[1], (at & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                        umma_bf16(tmem + h0 * kBN, a0 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
                     if (T.two) {
+                        if (kb == 0 &&
+                            !mbar_wait(&tail->tempty[h1], (c1 & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
                         tc_fence_after();
                         const uint64_t a1 = sw128_kmajor_desc(sa + kATile);
 #pragma unroll
                         for (int k = 0; k < kBK / 16; ++k)
-                            umma_bf16(tmem + kBN, a1 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
+                            umma_bf16(tmem + h1 * kBN, a1 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc,
+                                      (kb | k) != 0);
                     }
                     umma_commit(&tail->empty[s]);
                 }
-                if (ok) umma_commit(&tail->tfull);
+                if (!ok) break;
+                umma_commit(&tail->tfull);
+                const uint32_t inc1 = T.two ? 1u : 0u;    // half h0 always, h1 for two m-tiles
+                if (h0) { ++use1; use0 += inc1; } else { ++use0; use1 += inc1; }
+                hn = T.two ? h0 : h1;
             }
             umma_commit(&tail->drain);     // every MMA done before tensor memory is released
             mbar_wait_drain(&tail->drain, 0, kWaitLimit);
@@ -414,20 +426,23 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
     } else {
         // ------------------------------------------------------- epilogue
         uint32_t at = 0;
+        int hn = 0;                       // the half rotation of the MMA thread, replayed
         const int row = warp * 32 + lane;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++at) {
             const Tile T = decode_tile(t, tail->pre, a, bn);
+            const int h0 = hn, h1 = hn ^ 1;
             if (!mbar_wait(&tail->tfull, at & 1, abort, a.err, kWaitLimit)) break;
             tc_fence_after();
             const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
-            epilogue_half<kUp>(tlane, T, a, row);
+            epilogue_half<kUp>(tlane + h0 * kBN, T, a, row);
             tc_fence_before();
-            mbar_arrive(&tail->tempty[0]);
+            mbar_arrive(&tail->tempty[h0]);
             if (T.two) {
-                epilogue_half<kUp>(tlane + kBN, T, a, row + kBM);
+                epilogue_half<kUp>(tlane + h1 * kBN, T, a, row + kBM);
                 tc_fence_before();
+                mbar_arrive(&tail->tempty[h1]);
             }
-            mbar_arrive(&tail->tempty[1]);
+            hn = T.two ? h0 : h1;
         }
     }
     tc_fence_before();
