@@ -303,7 +303,7 @@ kmoe_status moe_combine(const void *y_perm, const void *y_shared, int y_in_dtype
     KMOE_TRY(check_ptr(topk_w, "topk_w"));
     KMOE_TRY(check_ptr(inv_pos, "inv_pos"));
     KMOE_TRY(check_ptr(y, "y"));
-    return launch_combine(y_perm, y_shared, y_in_dtype, topk_w, inv_pos, N, K, d, y, y_dtype,
+    return launch_combine(y_perm, y_shared, y_in_dtype, topk_w, inv_pos, N, K, d, y, y_dtype, nullptr,
                           static_cast<cudaStream_t>(stream));
 }
 
@@ -357,7 +357,7 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
     KMOE_TRY(run_ffn(x, x_dtype, N, d, I, E, K, L.perm, L.offsets, routed->dtype, r, shared ? &s : nullptr,
                      L.h, L.y_perm, L.y_shared, L.status, st));
     const int yin = routed->dtype == KMOE_F32 ? KMOE_F32 : KMOE_BF16;
-    return launch_combine(L.y_perm, shared ? L.y_shared : nullptr, yin, w, L.inv, N, K, d, y, y_dtype, st);
+    return launch_combine(L.y_perm, shared ? L.y_shared : nullptr, yin, w, L.inv, N, K, d, y, y_dtype, L.status, st);
 }
 
 kmoe_status moe_device_status(const void *ws, int *status, void *stream)

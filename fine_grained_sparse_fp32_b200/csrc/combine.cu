@@ -6,6 +6,7 @@
 // unnormalised sigmoid weights. A gather in fixed slot order, FP32
 // accumulation, 16-byte vector loads and stores: deterministic, no atomics.
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace kmoe {
 
@@ -67,11 +68,102 @@ combine_kernel(const YI *__restrict__ y_perm, const YI *__restrict__ y_shared,
     store8(y + (size_t)t * d + c, acc);
 }
 
+// BF16 inputs: a persistent kernel that streams whole token rows into shared
+// memory with the bulk-copy engine (K routed rows and the shared row, d * 2
+// bytes each) two tokens ahead, so each SM keeps ~140 KB of reads in flight;
+// the threads then form the same fixed-order FP32 sum from shared memory.
+constexpr int kBulkThreads = 320;
+constexpr int kBulkStages = 2;
+constexpr long long kBulkWaitLimit = 1LL << 32;
+
+template <class YO>
+__global__ void __launch_bounds__(kBulkThreads)
+combine_bulk_kernel(const __nv_bfloat16 *__restrict__ y_perm, const __nv_bfloat16 *__restrict__ y_shared,
+                    const float *__restrict__ w, const int32_t *__restrict__ inv, int N, int K, int d,
+                    YO *__restrict__ y, int *err)
+{
+    using namespace sm100;
+    extern __shared__ __align__(128) uint8_t cb_smem[];
+    __shared__ __align__(8) uint64_t full[kBulkStages];
+    __shared__ int abort_flag;
+    const int R = K + (y_shared ? 1 : 0);                 // rows per token
+    const size_t row_bytes = (size_t)d * sizeof(__nv_bfloat16);
+    const size_t stage_bytes = (size_t)R * row_bytes;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kBulkStages; ++s) mbar_init(&full[s], 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // thread 0 issues the rows of this block's i-th token into stage i % kBulkStages
+    auto issue = [&](int i) {
+        const int t = blockIdx.x + i * gridDim.x;
+        if (t >= N) return;
+        const int s = i % kBulkStages;
+        uint8_t *dst = cb_smem + (size_t)s * stage_bytes;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
+        for (int k = 0; k < K; ++k)
+            bulk_load(dst + (size_t)k * row_bytes, y_perm + (size_t)inv[(size_t)t * K + k] * d, (uint32_t)row_bytes,
+                      &full[s]);
+        if (y_shared) bulk_load(dst + (size_t)K * row_bytes, y_shared + (size_t)t * d, (uint32_t)row_bytes, &full[s]);
+    };
+    if (threadIdx.x == 0)
+        for (int i = 0; i < kBulkStages; ++i) issue(i);
+    for (int i = 0;; ++i) {
+        const int t = blockIdx.x + i * gridDim.x;
+        if (t >= N) break;
+        const int s = i % kBulkStages;
+        // every thread reaches the vote each round, so a give-up is a uniform exit
+        const bool ok = mbar_wait(&full[s], (i / kBulkStages) & 1, &abort_flag, err, kBulkWaitLimit);
+        if (!__syncthreads_and(ok)) break;
+        const uint8_t *rows = cb_smem + (size_t)s * stage_bytes;
+        float g[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) g[k] = k < K ? w[(size_t)t * K + k] : 0.f;
+        for (int c = threadIdx.x * 8; c < d; c += kBulkThreads * 8) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (y_shared) load8(reinterpret_cast<const __nv_bfloat16 *>(rows + (size_t)K * row_bytes) + c, acc);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k < K) {
+                    float v[8];
+                    load8(reinterpret_cast<const __nv_bfloat16 *>(rows + (size_t)k * row_bytes) + c, v);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) acc[q] = fmaf(g[k], v[q], acc[q]);
+                }
+            store8(y + (size_t)t * d + c, acc);
+        }
+        __syncthreads();                                  // every thread is done with stage s
+        if (threadIdx.x == 0) issue(i + kBulkStages);
+    }
+    if (abort_flag && threadIdx.x == 0)                   // a copy never landed: let the others finish
+        for (int s = 0; s < kBulkStages; ++s) mbar_wait_drain(&full[s], 0, kBulkWaitLimit);
+}
+
+static size_t bulk_smem(int K, int d, bool shared) { return (size_t)kBulkStages * (K + (shared ? 1 : 0)) * d * 2; }
+
 kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dtype,
                            const float *w, const int32_t *inv, int N, int K, int d, void *y,
-                           int y_dtype, cudaStream_t st)
+                           int y_dtype, int *err, cudaStream_t st)
 {
     using bf = __nv_bfloat16;
+    const size_t bsm = bulk_smem(K, d, y_shared != nullptr);
+    if (y_in_dtype == KMOE_BF16 && bsm <= 100 * 1024) {
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int per_sm = (int)((220 * 1024) / bsm) < 3 ? (int)((220 * 1024) / bsm) : 3;
+        const int grid = N < sms * per_sm ? N : sms * per_sm;
+        const bf *yp = static_cast<const bf *>(y_perm), *ys = static_cast<const bf *>(y_shared);
+        if (y_dtype == KMOE_F32) {
+            cudaFuncSetAttribute(combine_bulk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsm);
+            combine_bulk_kernel<float><<<grid, kBulkThreads, bsm, st>>>(yp, ys, w, inv, N, K, d, static_cast<float *>(y), err);
+        } else {
+            cudaFuncSetAttribute(combine_bulk_kernel<bf>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsm);
+            combine_bulk_kernel<bf><<<grid, kBulkThreads, bsm, st>>>(yp, ys, w, inv, N, K, d, static_cast<bf *>(y), err);
+        }
+        return check_launch("combine");
+    }
     dim3 grid(N, (d / 8 + kCombineThreads - 1) / kCombineThreads);
 #define KMOE_COMB(YI, YO)                                                                            \
     combine_kernel<YI, YO><<<grid, kCombineThreads, 0, st>>>(                                        \

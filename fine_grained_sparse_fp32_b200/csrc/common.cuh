@@ -175,8 +175,9 @@ kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, 
                             __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status,
                             int *sync, cudaStream_t st);
 
+// err: device status word for a bounded wait that gives up (may be NULL).
 kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dtype,
                            const float *w, const int32_t *inv, int N, int K, int d, void *y,
-                           int y_dtype, cudaStream_t st);
+                           int y_dtype, int *err, cudaStream_t st);
 
 }  // namespace kmoe

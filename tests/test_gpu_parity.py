@@ -189,6 +189,28 @@ def test_fp8_small_batch_flags_activations_outside_f16_range():
     assert kmoe.moe_device_status(ws) == 0
 
 
+@pytest.mark.parametrize("N,d,with_shared,y_dtype", [(1, 2560, True, torch.bfloat16), (32, 2560, True, torch.bfloat16),
+                                                       (777, 2560, False, torch.bfloat16), (300, 512, True, torch.float32),
+                                                       (8192, 2560, True, torch.bfloat16)])
+def test_combine_matches_float64(N, d, with_shared, y_dtype):
+    """y[t] = y_shared[t] + sum_k g[t,k] y_perm[inv_pos[t,k]] against a float64 sum of the same BF16 inputs."""
+    K = 6
+    gen = torch.Generator(device="cuda").manual_seed(N + d)
+    y_perm = torch.randn((N * K, d), generator=gen, device="cuda").bfloat16()
+    y_sh = torch.randn((N, d), generator=gen, device="cuda").bfloat16() if with_shared else None
+    w = torch.rand((N, K), generator=gen, device="cuda")
+    inv = torch.randperm(N * K, generator=gen, device="cuda").int().reshape(N, K)
+    y = kmoe.moe_combine(y_perm, y_sh, w, inv, y_dtype=y_dtype)
+    torch.cuda.synchronize()
+    yp, wv, iv = y_perm.double().cpu().numpy(), w.double().cpu().numpy(), inv.long().cpu().numpy()
+    ref = np.einsum("tk,tkj->tj", wv, yp[iv])
+    if with_shared:
+        ref = ref + y_sh.double().cpu().numpy()
+    got = y.double().cpu().numpy()
+    tol = 1e-5 if y_dtype == torch.float32 else 2 ** -8
+    assert np.abs(got - ref).max() <= tol * max(1.0, np.abs(ref).max())
+
+
 # ----------------------------------------------------------- whole layer
 def _forward_and_compare(name, N=None, rows=None, check_all_routing=True):
     dev, host = layer_inputs(name, N)
