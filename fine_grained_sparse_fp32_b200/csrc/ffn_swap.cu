@@ -36,12 +36,13 @@
 //   warps 7-14 E4M3 weights only: two groups of converters.
 // E4M3 weights ("Inside Kolibri 1", FP8 section: 128 x 128 blocks with one
 // FP32 scale each) arrive by TMA as bytes. Converter warps decode them
-// exactly to F16 (hardware e4m3x2 -> f16x2), multiply each row by
-// s_kb / s_ref (its block's scale over the largest scale of the row block,
-// so the factor is at most 1 and nothing overflows), and write the tiles
-// straight into tensor memory with tcgen05.st: the MMA takes A from tensor
-// memory. The token rows are converted to F16 for the B operand, the MMA is
-// F16 x F16 with FP32 accumulation, and the epilogue multiplies by s_ref.
+// exactly to F16 (hardware e4m3x2 -> f16x2) and write the tiles straight
+// into tensor memory with tcgen05.st: the MMA takes A from tensor memory.
+// The block scale of a stage is one number per weight tile, so it goes on
+// the token tile instead: each weight tile gets its own F16 copy of the
+// token rows times s_kb / s_ref (its block's scale over the largest scale
+// of the row block, at most 1, so nothing overflows). The MMA is F16 x F16
+// with FP32 accumulation, and the epilogue multiplies by s_ref.
 // |x| must stay inside the F16 range (65504); a value outside it sets
 // device status 2.
 #include "common.cuh"
@@ -78,7 +79,7 @@ struct Cfg {
     static constexpr int ConvCols = 128;                 // gate | up, 64 columns of F16 each
     static constexpr int TmemCols = kFp8 ? 512 : (AccCols <= 128 ? 128 : AccCols <= 256 ? 256 : 512);
     static constexpr int Stages = kFp8 ? 5 : (kNT <= 16 ? 6 : 4);
-    static constexpr int ConvB = ConvStages * BTile;     // E4M3: F16 token tiles
+    static constexpr int ConvB = ConvStages * 2 * BTile; // E4M3: F16 token tiles, one per weight tile
     static constexpr int Ring = Stages * Stage + ConvB;
     static constexpr int EpiGroups = kNT > 32 ? 2 : 1;   // groups of four epilogue warps
     static constexpr int Warps = kFp8 ? 15 : (EpiGroups == 2 ? 11 : 7);
@@ -306,16 +307,10 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
     return r;
 }
 
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b)
-{
-    uint32_t r;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-
-// Decodes one 128-byte E4M3 row (128-byte swizzle, row q of its tile), times
-// r, into 64 columns of tensor memory at `taddr` (this warp's lanes).
-__device__ __forceinline__ void convert_row_tmem(const uint8_t *tile, int q, uint32_t r2, uint32_t taddr)
+// Decodes one 128-byte E4M3 row (128-byte swizzle, row q of its tile)
+// exactly into 64 columns of F16 in tensor memory at `taddr` (this warp's
+// lanes).
+__device__ __forceinline__ void convert_row_tmem(const uint8_t *tile, int q, uint32_t taddr)
 {
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -328,9 +323,7 @@ __device__ __forceinline__ void convert_row_tmem(const uint8_t *tile, int q, uin
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
                 uint32_t lo, hi;
-                e4m3x4_to_f16(wd[h], lo, hi);
-                o[c4 * 8 + 2 * h] = hmul2(lo, r2);
-                o[c4 * 8 + 2 * h + 1] = hmul2(hi, r2);
+                e4m3x4_to_f16(wd[h], o[c4 * 8 + 2 * h], o[c4 * 8 + 2 * h + 1]);
             }
         }
         tmem_st32(taddr + half * 32, o);
@@ -570,12 +563,14 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                         if (!mbar_wait(&T->cfull[cs], (it / C::ConvStages) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t at = tmem + C::AccCols + cs * C::ConvCols;
-                        const uint64_t bd = sw128_kmajor_desc(smem_u32(convb + (size_t)cs * C::BTile));
+                        // token tile 0 carries the first weight tile's block scale, tile 1 the second's
+                        const uint64_t b0 = sw128_kmajor_desc(smem_u32(convb + (size_t)cs * 2 * C::BTile));
+                        const uint64_t b1 = sw128_kmajor_desc(smem_u32(convb + (size_t)(cs * 2 + 1) * C::BTile));
 #pragma unroll
                         for (int k = 0; k < C::BK / 16; ++k) {
-                            const uint64_t bk = bd + (uint64_t)(((k >> 2) * C::Panel + (k & 3) * 32) >> 4);
-                            umma_f16_tmem_a(dg, at + k * 8, bk, id, (kb | k) != 0);
-                            umma_f16_tmem_a(du, at + 64 + k * 8, bk, id, (kb | k) != 0);
+                            const uint64_t ko = (uint64_t)(((k >> 2) * C::Panel + (k & 3) * 32) >> 4);
+                            umma_f16_tmem_a(dg, at + k * 8, b0 + ko, id, (kb | k) != 0);
+                            umma_f16_tmem_a(du, at + 64 + k * 8, b1 + ko, id, (kb | k) != 0);
                         }
                         umma_commit(&T->cempty[cs]);
                     } else {
@@ -702,28 +697,32 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 }
                 const uint8_t *A8 = smem + (size_t)s * C::Stage;
                 const uint8_t *Braw = A8 + 2 * kATile;
-                uint8_t *B = convb + (size_t)cs * C::BTile;
+                uint8_t *B0 = convb + (size_t)cs * 2 * C::BTile, *B1 = B0 + C::BTile;
                 const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16) + C::AccCols + cs * C::ConvCols;
-                convert_row_tmem(A8, q, pack_f16x2(r0, r0), tq);
-                convert_row_tmem(A8 + kATile, q, pack_f16x2(r1, r1), tq + 64);
-                // B: BF16 token (or H) rows -> F16 at the same swizzled positions
-                // (a panel holds kNT rows of eight 16-byte chunks)
+                convert_row_tmem(A8, q, tq);
+                convert_row_tmem(A8 + kATile, q, tq + 64);
+                // B: BF16 token (or H) rows times each weight tile's s_kb / s_ref, as F16
+                // at the same swizzled positions (a panel holds kNT rows of eight
+                // 16-byte chunks): the block scale rides on the small token tile
+                // instead of on every weight
 #pragma unroll
                 for (int i = 0; i < C::BTile / 16 / 128; ++i) {
                     const int c16 = q + i * 128;
                     if (((c16 % (kNT * 8)) >> 3) < nmma) {
                         const uint4 w = *reinterpret_cast<const uint4 *>(Braw + c16 * 16);
                         const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-                        uint32_t p[4];
+                        uint32_t p0[4], p1[4];
                         float mx = 0.f;
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float f0 = bf16_lo(wd[e]), f1 = bf16_hi(wd[e]);
-                            p[e] = pack_f16x2(f0, f1);
+                            p0[e] = pack_f16x2(f0 * r0, f1 * r0);
+                            p1[e] = pack_f16x2(f0 * r1, f1 * r1);
                             mx = fmaxf(mx, fmaxf(fabsf(f0), fabsf(f1)));
                         }
                         if (!(mx <= 65504.f)) range_ok = false;
-                        *reinterpret_cast<uint4 *>(B + c16 * 16) = make_uint4(p[0], p[1], p[2], p[3]);
+                        *reinterpret_cast<uint4 *>(B0 + c16 * 16) = make_uint4(p0[0], p0[1], p0[2], p0[3]);
+                        *reinterpret_cast<uint4 *>(B1 + c16 * 16) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
                     }
                 }
                 tmem_st_wait();
