@@ -83,15 +83,21 @@ def router_logits(x, x_dtype: str, w_router, nthreads: int = 1) -> np.ndarray:
     return out
 
 
-def select(logits: np.ndarray, bias, K: int):
-    """(idx [N,K] int32, g [N,K] double, margin [N] double) for given logits."""
+SCORES = {"sigmoid": 0, "softmax": 1}
+
+
+def select(logits: np.ndarray, bias, K: int, score: str = "sigmoid"):
+    """(idx [N,K] int32, g [N,K] double, margin [N] double) for given logits.
+
+    score "sigmoid": g = sigmoid of the unbiased logit; "softmax": g = softmax
+    over the K selected unbiased logits."""
     l = np.ascontiguousarray(logits, dtype=np.float64)
     b = np.ascontiguousarray(_bits(bias), dtype=np.float32)
     N, E = l.shape
     idx = np.empty((N, K), dtype=np.int32)
     g = np.empty((N, K), dtype=np.float64)
     margin = np.empty(N, dtype=np.float64)
-    lib().oracle_select(N, E, K, _p(l), _p(b), _p(idx), _p(g), _p(margin))
+    lib().oracle_select_score(N, E, K, _p(l), _p(b), SCORES[score], _p(idx), _p(g), _p(margin))
     return idx, g, margin
 
 
@@ -133,8 +139,8 @@ def expert_outputs(inp, tokens, experts, nthreads: int = 1) -> np.ndarray:
     return out
 
 
-def layer(inp, rows=None, nthreads: int = 1):
-    """The whole layer for tokens `rows` (default: all).
+def layer(inp, rows=None, nthreads: int = 1, score: str = "sigmoid"):
+    """The whole layer for tokens `rows` (default: all), mixture weights by `score`.
 
     Returns dict(y [n,d] double, idx [n,K], g [n,K], margin [n])."""
     cfg = inp["cfg"]
@@ -149,9 +155,9 @@ def layer(inp, rows=None, nthreads: int = 1):
     idx = np.empty((n, cfg.K), dtype=np.int32)
     g = np.empty((n, cfg.K), dtype=np.float64)
     margin = np.empty(n, dtype=np.float64)
-    lib().oracle_layer(N, cfg.d, cfg.E, cfg.K, cfg.I, _p(xb), _DT[cfg.x_dtype], _p(wr), _p(b),
-                       _p(wg), _p(wu), _p(wd), _p(sg), _p(su), _p(sd), _DT[cfg.w_dtype],
-                       n, _p(rows), _p(y), _p(idx), _p(g), _p(margin), nthreads)
+    lib().oracle_layer_score(N, cfg.d, cfg.E, cfg.K, cfg.I, _p(xb), _DT[cfg.x_dtype], _p(wr), _p(b),
+                             _p(wg), _p(wu), _p(wd), _p(sg), _p(su), _p(sd), _DT[cfg.w_dtype],
+                             n, _p(rows), SCORES[score], _p(y), _p(idx), _p(g), _p(margin), nthreads)
     return {"y": y, "idx": idx, "g": g, "margin": margin, "rows": rows}
 
 

@@ -125,11 +125,16 @@ static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
 /* Selection and mixture weights for every token:
  *   s[e] = l[e] + b[e];
  *   idx  = the first K experts of 0..E-1 ordered by (s descending, e ascending);
- *   g[k] = sigmoid(l[idx[k]])   (unbiased logit, no renormalisation);
+ *   score 0 ("Inside Kolibri 1", routing section):
+ *     g[k] = sigmoid(l[idx[k]])   (unbiased logit, no renormalisation);
+ *   score 1 ("Kolibri 1 Deep Dive", "Mathematical Routing & Load Balancing
+ *   Formulation": a softmax over the selected experts' logits):
+ *     g[k] = exp(l[idx[k]]) / sum_j exp(l[idx[j]])   (unbiased logits;
+ *     evaluated with the largest selected logit subtracted first);
  *   margin = s of the K-th choice minus s of the (K+1)-th (HUGE_VAL if E == K).
  * K passes of "take the best remaining" give exactly that ordered prefix. */
-void oracle_select(int N, int E, int K, const double *logits, const float *bias,
-                   int32_t *idx, double *g, double *margin)
+void oracle_select_score(int N, int E, int K, const double *logits, const float *bias, int score,
+                         int32_t *idx, double *g, double *margin)
 {
     unsigned char *taken = (unsigned char *)malloc((size_t)E);
     for (int t = 0; t < N; ++t) {
@@ -159,8 +164,25 @@ void oracle_select(int N, int E, int K, const double *logits, const float *bias,
         }
         if (E == K)
             margin[t] = HUGE_VAL;
+        if (score == 1) {
+            double *gt = g + (int64_t)t * K, mx = -HUGE_VAL, sum = 0.0;
+            for (int k = 0; k < K; ++k)
+                mx = fmax(mx, l[idx[(int64_t)t * K + k]]);
+            for (int k = 0; k < K; ++k) {
+                gt[k] = exp(l[idx[(int64_t)t * K + k]] - mx);
+                sum += gt[k];
+            }
+            for (int k = 0; k < K; ++k)
+                gt[k] /= sum;
+        }
     }
     free(taken);
+}
+
+void oracle_select(int N, int E, int K, const double *logits, const float *bias,
+                   int32_t *idx, double *g, double *margin)
+{
+    oracle_select_score(N, E, K, logits, bias, 0, idx, g, margin);
 }
 
 /* Dispatch by counting sort.
@@ -248,13 +270,13 @@ void oracle_expert_outputs(int d, int I, const void *x, int x_dtype, int w_dtype
  * with the shared expert stored at index E of the stacked weight tensors.
  * Writes y [n_rows, d], and the selection idx/g [n_rows, K] and margin
  * [n_rows] of those tokens. */
-void oracle_layer(int N, int d, int E, int K, int I,
-                  const void *x, int x_dtype, const float *w_router, const float *bias,
-                  const void *wg, const void *wu, const void *wd,
-                  const float *sg, const float *su, const float *sd, int w_dtype,
-                  int n_rows, const int32_t *rows,
-                  double *y, int32_t *idx_out, double *g_out, double *margin_out,
-                  int nthreads)
+void oracle_layer_score(int N, int d, int E, int K, int I,
+                        const void *x, int x_dtype, const float *w_router, const float *bias,
+                        const void *wg, const void *wu, const void *wd,
+                        const float *sg, const float *su, const float *sd, int w_dtype,
+                        int n_rows, const int32_t *rows, int score,
+                        double *y, int32_t *idx_out, double *g_out, double *margin_out,
+                        int nthreads)
 {
     int r;
     (void)N;
@@ -274,8 +296,8 @@ void oracle_layer(int N, int d, int E, int K, int I,
                 acc += xrow[j] * (double)w_router[(int64_t)e * d + j];
             l[e] = acc;
         }
-        oracle_select(1, E, K, l, bias, idx_out + (int64_t)r * K, g_out + (int64_t)r * K,
-                      margin_out + r);
+        oracle_select_score(1, E, K, l, bias, score, idx_out + (int64_t)r * K, g_out + (int64_t)r * K,
+                            margin_out + r);
         expert_ffn(d, I, xrow, E, w_dtype, wg, wu, wd, sg, su, sd, h, yr);
         for (int k = 0; k < K; ++k) {
             int e = idx_out[(int64_t)r * K + k];
@@ -289,6 +311,18 @@ void oracle_layer(int N, int d, int E, int K, int I,
         free(l);
         free(xrow);
     }
+}
+
+void oracle_layer(int N, int d, int E, int K, int I,
+                  const void *x, int x_dtype, const float *w_router, const float *bias,
+                  const void *wg, const void *wu, const void *wd,
+                  const float *sg, const float *su, const float *sd, int w_dtype,
+                  int n_rows, const int32_t *rows,
+                  double *y, int32_t *idx_out, double *g_out, double *margin_out,
+                  int nthreads)
+{
+    oracle_layer_score(N, d, E, K, I, x, x_dtype, w_router, bias, wg, wu, wd, sg, su, sd, w_dtype, n_rows, rows, 0,
+                       y, idx_out, g_out, margin_out, nthreads);
 }
 
 int oracle_max_threads(void)

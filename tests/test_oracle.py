@@ -105,6 +105,40 @@ def test_mixture_weights_use_unbiased_logits_without_renormalising():
     assert abs(g[0].sum() - 1.0) > 1.0       # not renormalised to one
 
 
+def test_softmax_score_closed_form_on_the_forced_six():
+    """Softmax over the selected experts ("Kolibri 1 Deep Dive", routing formulation)
+    on a forced selection: unbiased logits (0, ln3, 0, ln3, 0, 0) have exponentials
+    1, 3, 1, 3, 1, 1 (sum 10), so the weights are 1/10 and 3/10."""
+    E, K = 16, 6
+    logits = np.full((1, E), 5.0)            # the best unbiased logits are elsewhere ...
+    logits[0, [3, 5, 7, 9, 11, 13]] = [0.0, math.log(3.0), 0.0, math.log(3.0), 0.0, 0.0]
+    bias = np.zeros(E, dtype=np.float32)
+    bias[[3, 5, 7, 9, 11, 13]] = 30.0        # ... the bias forces these six
+    idx, g, _ = oracle.select(logits, bias, K, score="softmax")
+    assert sorted(idx[0]) == [3, 5, 7, 9, 11, 13]
+    by_e = dict(zip(idx[0].tolist(), g[0].tolist()))
+    for e in (3, 7, 11, 13):
+        assert by_e[e] == pytest.approx(0.1, abs=1e-15)
+    for e in (5, 9):
+        assert by_e[e] == pytest.approx(0.3, abs=1e-15)
+
+
+def test_softmax_score_keeps_selection_and_is_a_distribution():
+    rng = np.random.default_rng(5)
+    logits = rng.normal(0.0, 3.0, (50, 40))
+    bias = rng.uniform(-0.1, 0.1, 40).astype(np.float32)
+    i_sig, g_sig, m_sig = oracle.select(logits, bias, 6)
+    i_soft, g_soft, m_soft = oracle.select(logits, bias, 6, score="softmax")
+    np.testing.assert_array_equal(i_sig, i_soft)          # the score only changes the weights
+    np.testing.assert_array_equal(m_sig, m_soft)
+    assert np.all(g_soft > 0) and np.allclose(g_soft.sum(axis=1), 1.0, atol=1e-14)
+    # two-expert special case against the logistic function: softmax(a, b)[0] = sigmoid(a - b)
+    l2 = rng.normal(0.0, 2.0, (20, 2))
+    i2, g2, _ = oracle.select(l2, np.zeros(2, dtype=np.float32), 2, score="softmax")
+    first = np.take_along_axis(l2, i2, axis=1)
+    np.testing.assert_allclose(g2[:, 0], 1.0 / (1.0 + np.exp(first[:, 1] - first[:, 0])), rtol=1e-13)
+
+
 def test_permute_matches_stable_sort():
     rng = np.random.default_rng(4)
     for N, K, E in [(128, 6, 64), (1, 6, 6), (57, 6, 384), (300, 2, 5)]:
