@@ -194,12 +194,20 @@ size_t moe_workspace_size(int N, int d, int E, int K, int I, int x_dtype, int w_
     return layout(nullptr, N, d, E, K, I, w_dtype).bytes;
 }
 
+static kmoe_status check_score(int score)
+{
+    if (score != KMOE_SCORE_SIGMOID && score != KMOE_SCORE_SOFTMAX)
+        return fail(KMOE_ERR_INVALID_ARG, "score %d: KMOE_SCORE_SIGMOID or KMOE_SCORE_SOFTMAX", score);
+    return KMOE_OK;
+}
+
 kmoe_status moe_router_topk(const void *x, int x_dtype, const float *w_router, const float *bias,
-                            int N, int d, int E, int K, float *logits, int32_t *topk_idx,
+                            int N, int d, int E, int K, int score, float *logits, int32_t *topk_idx,
                             float *topk_w, void *ws, size_t ws_bytes, void *stream)
 {
     clear_error();
     KMOE_TRY(check_sizes(N, d, E, K, -1));
+    KMOE_TRY(check_score(score));
     KMOE_TRY(check_act_dtype(x_dtype, "x"));
     if (N == 0) return KMOE_OK;
     KMOE_TRY(check_ptr(x, "x"));
@@ -228,7 +236,7 @@ kmoe_status moe_router_topk(const void *x, int x_dtype, const float *w_router, c
     } else {
         KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, logits, st));
     }
-    return launch_topk(logits, bias, N, E, K, topk_idx, topk_w, st);
+    return launch_topk(logits, bias, N, E, K, score, topk_idx, topk_w, st);
 }
 
 kmoe_status moe_permute(const int32_t *topk_idx, int N, int K, int E, int32_t *counts,
@@ -307,7 +315,7 @@ kmoe_status moe_combine(const void *y_perm, const void *y_shared, int y_in_dtype
                           static_cast<cudaStream_t>(stream));
 }
 
-kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, int I,
+kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, int I, int score,
                         const float *w_router, const float *bias, const kmoe_experts *routed,
                         const kmoe_experts *shared, void *y, int y_dtype, int32_t *topk_idx_out,
                         float *topk_w_out, int32_t *counts_out, void *ws, size_t ws_bytes, void *stream)
@@ -316,6 +324,7 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
     KMOE_TRY(check_sizes(N, d, E, K, I));
     KMOE_TRY(check_act_dtype(x_dtype, "x"));
     KMOE_TRY(check_act_dtype(y_dtype, "y"));
+    KMOE_TRY(check_score(score));
     KMOE_TRY(check_experts(routed, "routed"));
     if (shared) {
         KMOE_TRY(check_experts(shared, "shared"));
@@ -340,7 +349,7 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
     int32_t *counts = counts_out ? counts_out : L.counts;
     KMOE_TRY(clear_status(L.status, st, kFfnStatusBytes));
     if (N <= kFusedRouteTokens) {
-        KMOE_TRY(launch_route_small(x, x_dtype, w_router, bias, N, d, E, K, L.logits, idx, w, counts, L.offsets,
+        KMOE_TRY(launch_route_small(x, x_dtype, w_router, bias, N, d, E, K, score, L.logits, idx, w, counts, L.offsets,
                                     L.perm, L.inv, L.status, st));
     } else {
         if (x_dtype == KMOE_BF16 && N >= kTcRouterTokens)
@@ -348,7 +357,7 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
                                       L.status, st));
         else
             KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, L.logits, st));
-        KMOE_TRY(launch_topk(L.logits, bias, N, E, K, idx, w, st));
+        KMOE_TRY(launch_topk(L.logits, bias, N, E, K, score, idx, w, st));
         KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st));
     }
     const ExpertPtrs r = ptrs(routed);

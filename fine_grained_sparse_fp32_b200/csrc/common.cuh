@@ -130,13 +130,13 @@ namespace kmoe {
 
 kmoe_status launch_router_logits(const void *x, int x_dtype, const float *w_router, int N, int d,
                                  int E, float *logits, cudaStream_t st);
-kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, int K,
+kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, int K, int score,
                         int32_t *idx, float *w, cudaStream_t st);
 
 // Router + top-K + permutation in one launch for N <= 256 (status[4] is a
 // ticket that must be zero before the launch).
 kmoe_status launch_route_small(const void *x, int x_dtype, const float *w_router, const float *bias, int N,
-                               int d, int E, int K, float *logits, int32_t *idx, float *w, int32_t *counts,
+                               int d, int E, int K, int score, float *logits, int32_t *idx, float *w, int32_t *counts,
                                int32_t *offsets, int32_t *perm, int32_t *inv, int *status, cudaStream_t st);
 
 // Tensor-core FP32 router (x in BF16): W_r split into three BF16 terms in

@@ -92,10 +92,14 @@ kmoe_status launch_router_logits(const void *x, int x_dtype, const float *w_rout
 // its best remaining candidate, a butterfly reduction picks the warp's best
 // by (score descending, index ascending), and its owner retires it. Logits
 // are read through L2 (they may come from other CTAs of the same kernel).
+// Mixture weights from the unbiased logits of the K chosen experts: sigmoid
+// of each ("Inside Kolibri 1", routing section) or, with KMOE_SCORE_SOFTMAX,
+// a softmax over the K ("Kolibri 1 Deep Dive", routing formulation).
 template <int NPL>
-__device__ __forceinline__ void topk_warp(const float *lr, const float *__restrict__ bias, int E, int K,
+__device__ __forceinline__ void topk_warp(const float *lr, const float *__restrict__ bias, int E, int K, int score,
                                           int32_t *idx_row, float *w_row)
 {
+    float lsel[8];                    // lane 0: unbiased logits of the chosen experts (K <= 8)
     const int lane = threadIdx.x & 31;
     float s[NPL];
 #pragma unroll
@@ -121,28 +125,41 @@ __device__ __forceinline__ void topk_warp(const float *lr, const float *__restri
         if (lane == 0) {   // be < E whenever K <= E and the scores are finite
             const int e = be < E ? be : E - 1;
             idx_row[k] = e;
-            w_row[k] = sigmoidf_(__ldcg(lr + e));
+            lsel[k] = __ldcg(lr + e);
+        }
+    }
+    if (lane == 0) {
+        if (score == KMOE_SCORE_SOFTMAX) {
+            float mx = -INFINITY, sum = 0.f;
+            for (int k = 0; k < K; ++k) mx = fmaxf(mx, lsel[k]);
+            for (int k = 0; k < K; ++k) {
+                lsel[k] = expf(lsel[k] - mx);
+                sum += lsel[k];
+            }
+            for (int k = 0; k < K; ++k) w_row[k] = lsel[k] / sum;
+        } else {
+            for (int k = 0; k < K; ++k) w_row[k] = sigmoidf_(lsel[k]);
         }
     }
 }
 
 template <int NPL>
 __global__ void __launch_bounds__(256)
-topk_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int N, int E, int K,
+topk_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int N, int E, int K, int score,
             int32_t *__restrict__ idx, float *__restrict__ wout)
 {
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= N) return;
-    topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, idx + (size_t)t * K, wout + (size_t)t * K);
+    topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, score, idx + (size_t)t * K, wout + (size_t)t * K);
 }
 
-kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, int K,
+kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, int K, int score,
                         int32_t *idx, float *w, cudaStream_t st)
 {
     const int warps = 8;
     dim3 grid((N + warps - 1) / warps);
     const int npl = (E + 31) / 32;
-#define KMOE_TOPK(n) topk_kernel<n><<<grid, warps * 32, 0, st>>>(logits, bias, N, E, K, idx, w)
+#define KMOE_TOPK(n) topk_kernel<n><<<grid, warps * 32, 0, st>>>(logits, bias, N, E, K, score, idx, w)
     if (npl <= 2) KMOE_TOPK(2);
     else if (npl <= 4) KMOE_TOPK(4);
     else if (npl <= 8) KMOE_TOPK(8);
@@ -178,7 +195,7 @@ constexpr long long kRouteWaitLimit = 1LL << 32;
 template <class XT, int NPL>
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
-                   int N, int d, int E, int K, int chunk, int x_off, float *__restrict__ logits,
+                   int N, int d, int E, int K, int score, int chunk, int x_off, float *__restrict__ logits,
                    int32_t *__restrict__ idx, float *__restrict__ wout, int32_t *__restrict__ counts,
                    int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv,
                    int *status)
@@ -275,14 +292,14 @@ route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const 
     if (!last) return;
     __threadfence();
     for (int t = warp; t < N; t += kRouteWarps)
-        topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, idx + (size_t)t * K, wout + (size_t)t * K);
+        topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, score, idx + (size_t)t * K, wout + (size_t)t * K);
     __syncthreads();
     permute_small_block<kRouteWarps>(idx, N, K, E, counts, offsets, perm, inv, reinterpret_cast<uint32_t *>(sm_raw));
     if (threadIdx.x == 0) *ticket = 0;
 }
 
 kmoe_status launch_route_small(const void *x, int x_dtype, const float *w_router, const float *bias, int N,
-                               int d, int E, int K, float *logits, int32_t *idx, float *w, int32_t *counts,
+                               int d, int E, int K, int score, float *logits, int32_t *idx, float *w, int32_t *counts,
                                int32_t *offsets, int32_t *perm, int32_t *inv, int *status, cudaStream_t st)
 {
     if (N > kChunk) return fail(KMOE_ERR_UNSUPPORTED, "fused routing: N=%d > %d", N, kChunk);
@@ -296,7 +313,8 @@ kmoe_status launch_route_small(const void *x, int x_dtype, const float *w_router
     do {                                                                                                    \
         auto k = route_small_kernel<XT, n>;                                                                 \
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                    \
-        k<<<grid, kRouteThreads, smem, st>>>(static_cast<const XT *>(x), w_router, bias, N, d, E, K, chunk,  \
+        k<<<grid, kRouteThreads, smem, st>>>(static_cast<const XT *>(x), w_router, bias, N, d, E, K, score,   \
+                                             chunk,                                                          \
                                              w_bytes, logits, idx, w, counts, offsets, perm, inv, status);   \
     } while (0)
 #define KMOE_ROUTE_X(n)                                   \

@@ -15,6 +15,7 @@ from ._build import LIB
 
 KMOE_OK, KMOE_ERR_INVALID_ARG, KMOE_ERR_UNSUPPORTED, KMOE_ERR_CUDA, KMOE_ERR_WORKSPACE, KMOE_ERR_DEVICE = range(6)
 KMOE_F32, KMOE_BF16, KMOE_E4M3_B128 = 0, 1, 2
+SCORES = {"sigmoid": 0, "softmax": 1}     # kmoe_score
 
 # Bytes at the head of a moe_grouped_ffn workspace: the status word, tickets
 # and the grouped FFN's unit counters (include/kmoe.h).
@@ -54,19 +55,19 @@ def load(path: str | None = None):
     lib.moe_workspace_size.argtypes = [i, i, i, i, i, i, i]
     lib.moe_last_error.restype = ctypes.c_char_p
     lib.moe_abi_version.restype = i
-    lib.moe_router_topk.argtypes = [vp, i, vp, vp, i, i, i, i, vp, vp, vp, vp, sz, vp]
+    lib.moe_router_topk.argtypes = [vp, i, vp, vp, i, i, i, i, i, vp, vp, vp, vp, sz, vp]
     lib.moe_permute.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_permute_noalloc.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp]
     lib.moe_grouped_ffn.argtypes = [vp, i, i, i, i, i, i, vp, vp, ctypes.POINTER(Experts),
                                     ctypes.POINTER(Experts), vp, vp, vp, sz, vp]
     lib.moe_combine.argtypes = [vp, vp, i, vp, vp, i, i, i, vp, i, vp]
-    lib.moe_forward.argtypes = [vp, i, i, i, i, i, i, vp, vp, ctypes.POINTER(Experts),
+    lib.moe_forward.argtypes = [vp, i, i, i, i, i, i, i, vp, vp, ctypes.POINTER(Experts),
                                 ctypes.POINTER(Experts), vp, i, vp, vp, vp, vp, sz, vp]
     lib.moe_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
     for f in ("moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn", "moe_combine",
               "moe_forward", "moe_device_status"):
         getattr(lib, f).restype = i
-    if lib.moe_abi_version() != 1:
+    if lib.moe_abi_version() != 2:
         raise RuntimeError("libkmoe ABI version mismatch")
     _lib = lib
     return lib
@@ -123,7 +124,8 @@ def workspace(N, d, E, K, I, x_dtype: int, w_dtype: int, device="cuda") -> torch
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-def moe_router_topk(x, w_router, bias, K, logits=None, topk_idx=None, topk_w=None, ws=None, stream=None):
+def moe_router_topk(x, w_router, bias, K, logits=None, topk_idx=None, topk_w=None, ws=None, stream=None,
+                    score="sigmoid"):
     N, d = x.shape
     E = w_router.shape[0]
     if topk_idx is None:
@@ -134,7 +136,7 @@ def moe_router_topk(x, w_router, bias, K, logits=None, topk_idx=None, topk_w=Non
         ws = torch.empty(((N * E * 4 + 255) // 256) * 256 + 256 + 3 * E * d * 2, dtype=torch.uint8,
                          device=x.device)
     _check(load().moe_router_topk(_ptr(x), dtype_code(x.dtype), _ptr(w_router), _ptr(bias), N, d, E, K,
-                                  _ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(ws),
+                                  SCORES[score], _ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(ws),
                                   0 if ws is None else ws.numel(), _stream(stream)))
     return topk_idx, topk_w
 
@@ -215,7 +217,7 @@ class Layer:
     `forward(x)` is one moe_forward call; outputs are written into tensors
     owned here (or passed in)."""
 
-    def __init__(self, layer: dict, max_tokens: int, y_dtype=torch.bfloat16):
+    def __init__(self, layer: dict, max_tokens: int, y_dtype=torch.bfloat16, score: str = "sigmoid"):
         self.layer = layer
         cfg = self.cfg = layer["cfg"]
         self.routed = experts_of(layer, "routed")
@@ -225,6 +227,7 @@ class Layer:
         self.ws = workspace(max_tokens, cfg.d, cfg.E, cfg.K, cfg.I, self.x_code, w_dtype_code(cfg.w_dtype), dev)
         self.y_dtype = y_dtype
         self.max_tokens = max_tokens
+        self.score = SCORES[score]
 
     def forward(self, x, y=None, topk_idx=None, topk_w=None, counts=None, stream=None):
         cfg = self.cfg
@@ -234,18 +237,18 @@ class Layer:
         if y is None:
             y = torch.empty((N, cfg.d), dtype=self.y_dtype, device=x.device)
         L = self.layer
-        _check(load().moe_forward(_ptr(x), dtype_code(x.dtype), N, cfg.d, cfg.E, cfg.K, cfg.I,
+        _check(load().moe_forward(_ptr(x), dtype_code(x.dtype), N, cfg.d, cfg.E, cfg.K, cfg.I, self.score,
                                   _ptr(L["w_router"]), _ptr(L["bias"]), ctypes.byref(self.routed),
                                   ctypes.byref(self.shared), _ptr(y), dtype_code(y.dtype), _ptr(topk_idx),
                                   _ptr(topk_w), _ptr(counts), _ptr(self.ws), self.ws.numel(), _stream(stream)))
         return y
 
 
-def moe_forward(x, layer, y_dtype=torch.bfloat16, with_outputs=False, stream=None):
+def moe_forward(x, layer, y_dtype=torch.bfloat16, with_outputs=False, stream=None, score="sigmoid"):
     """One whole-layer call; with_outputs also returns (topk_idx, topk_w, counts)."""
     cfg = layer["cfg"]
     N = x.shape[0]
-    lay = Layer(layer, N, y_dtype)
+    lay = Layer(layer, N, y_dtype, score)
     if not with_outputs:
         return lay.forward(x, stream=stream)
     idx = torch.empty((N, cfg.K), dtype=torch.int32, device=x.device)

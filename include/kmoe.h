@@ -50,6 +50,20 @@ typedef enum {
     KMOE_ERR_DEVICE = 5         /* a kernel reported a failure in the device status word */
 } kmoe_status;
 
+/*
+ * Mixture weights of the K chosen experts, from their unbiased logits l:
+ *   KMOE_SCORE_SIGMOID  g_k = 1 / (1 + exp(-l_k)), not renormalised
+ *                       ("Inside Kolibri 1", routing section; the default);
+ *   KMOE_SCORE_SOFTMAX  g_k = exp(l_k) / sum_j exp(l_j) over the K chosen
+ *                       ("Kolibri 1 Deep Dive", section "Mathematical Routing
+ *                       & Load Balancing Formulation"). The selection itself
+ *                       (top-K of l + bias) is the same for both.
+ */
+typedef enum {
+    KMOE_SCORE_SIGMOID = 0,
+    KMOE_SCORE_SOFTMAX = 1
+} kmoe_score;
+
 typedef enum {
     KMOE_F32 = 0,        /* IEEE binary32 */
     KMOE_BF16 = 1,       /* bfloat16 */
@@ -88,7 +102,8 @@ size_t moe_workspace_size(int N, int d, int E, int K, int I, int x_dtype, int w_
  *   topk_idx[t]  = the K experts with the largest logits[t][e] + bias[e],
  *                  ordered by that biased score, highest first; on equal
  *                  scores the lower expert index wins
- *   topk_w[t][k] = 1 / (1 + exp(-logits[t][topk_idx[t][k]]))
+ *   topk_w[t][k] = 1 / (1 + exp(-logits[t][topk_idx[t][k]]))   (score KMOE_SCORE_SIGMOID),
+ *                  or the softmax of the K chosen logits      (score KMOE_SCORE_SOFTMAX)
  * x        device [N, d], x_dtype KMOE_F32 or KMOE_BF16
  * w_router device [E, d] FP32;   bias device [E] FP32
  * logits   device [N, E] FP32 output, or NULL to keep it in the workspace
@@ -102,7 +117,7 @@ size_t moe_workspace_size(int N, int d, int E, int K, int I, int x_dtype, int w_
  *          (ws + the logits bytes rounded up to 256 when logits is NULL).
  */
 kmoe_status moe_router_topk(const void *x, int x_dtype, const float *w_router,
-                            const float *bias, int N, int d, int E, int K,
+                            const float *bias, int N, int d, int E, int K, int score,
                             float *logits, int32_t *topk_idx, float *topk_w,
                             void *ws, size_t ws_bytes, void *stream);
 
@@ -180,12 +195,13 @@ kmoe_status moe_combine(const void *y_perm, const void *y_shared, int y_in_dtype
 
 /*
  * The whole layer: moe_router_topk -> moe_permute -> moe_grouped_ffn ->
- * moe_combine on one stream, with every intermediate in `ws`.
+ * moe_combine on one stream, with every intermediate in `ws`; `score`
+ * (kmoe_score) picks the mixture weights.
  * y device [N, d] output of y_dtype (F32 or BF16). topk_idx_out [N, K],
  * topk_w_out [N, K] and counts_out [E] are optional device outputs (NULL to
  * skip). `shared` may be NULL (no shared expert).
  */
-kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, int I,
+kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, int I, int score,
                         const float *w_router, const float *bias,
                         const kmoe_experts *routed, const kmoe_experts *shared,
                         void *y, int y_dtype,
@@ -208,7 +224,7 @@ const char *moe_last_error(void);
 
 /* ABI version of this header (bumped on incompatible change). */
 int moe_abi_version(void);
-#define KMOE_ABI_VERSION 1
+#define KMOE_ABI_VERSION 2
 
 #ifdef __cplusplus
 }

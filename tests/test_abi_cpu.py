@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
 
 
 def test_workspace_size_grows_with_tokens(lib):
@@ -61,26 +61,32 @@ def test_bad_arguments_fail_on_the_host(lib):
     vp = ctypes.c_void_p
     aligned = vp(1 << 20)
     # K = 9 is not compiled
-    st = lib.moe_router_topk(aligned, kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 9,
+    st = lib.moe_router_topk(aligned, kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 9, 0,
                              None, aligned, aligned, aligned, 1 << 20, None)
     assert st == kmoe.KMOE_ERR_UNSUPPORTED
     assert b"K=9" in lib.moe_last_error()
     # null x
-    st = lib.moe_router_topk(None, kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 6,
+    st = lib.moe_router_topk(None, kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 6, 0,
                              None, aligned, aligned, aligned, 1 << 20, None)
     assert st == kmoe.KMOE_ERR_INVALID_ARG
     # misaligned pointer
-    st = lib.moe_router_topk(vp((1 << 20) + 4), kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 6,
+    st = lib.moe_router_topk(vp((1 << 20) + 4), kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 6, 0,
                              None, aligned, aligned, aligned, 1 << 20, None)
     assert st == kmoe.KMOE_ERR_INVALID_ARG and b"aligned" in lib.moe_last_error()
     # unknown activation dtype
-    st = lib.moe_router_topk(aligned, 7, aligned, aligned, 4, 2560, 384, 6,
+    st = lib.moe_router_topk(aligned, 7, aligned, aligned, 4, 2560, 384, 6, 0,
                              None, aligned, aligned, aligned, 1 << 20, None)
     assert st == kmoe.KMOE_ERR_UNSUPPORTED
     # workspace too small
-    st = lib.moe_router_topk(aligned, kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 6,
+    st = lib.moe_router_topk(aligned, kmoe.KMOE_BF16, aligned, aligned, 4, 2560, 384, 6, 0,
                              None, aligned, aligned, aligned, 16, None)
     assert st == kmoe.KMOE_ERR_WORKSPACE
+
+
+def test_unknown_score_function_is_rejected(lib):
+    a = ctypes.c_void_p(1 << 20)
+    st = lib.moe_router_topk(a, kmoe.KMOE_BF16, a, a, 4, 2560, 384, 6, 7, None, a, a, a, 1 << 20, None)
+    assert st == kmoe.KMOE_ERR_INVALID_ARG and b"score" in lib.moe_last_error()
 
 
 def test_forward_rejects_null_experts_and_mixed_dtypes(lib):
@@ -88,7 +94,7 @@ def test_forward_rejects_null_experts_and_mixed_dtypes(lib):
     a = vp(1 << 20)
     ex = kmoe.Experts(a, a, a, None, None, None, kmoe.KMOE_BF16)
     fp8 = kmoe.Experts(a, a, a, None, None, None, kmoe.KMOE_E4M3_B128)   # scales missing
-    args = lambda r, s: (a, kmoe.KMOE_BF16, 32, 2560, 384, 6, 512, a, a, r, s, a, kmoe.KMOE_BF16,
+    args = lambda r, s: (a, kmoe.KMOE_BF16, 32, 2560, 384, 6, 512, 0, a, a, r, s, a, kmoe.KMOE_BF16,
                          None, None, None, a, 1 << 40, None)
     assert lib.moe_forward(*args(None, None)) == kmoe.KMOE_ERR_INVALID_ARG
     assert lib.moe_forward(*args(ctypes.byref(fp8), None)) == kmoe.KMOE_ERR_INVALID_ARG
@@ -99,8 +105,8 @@ def test_forward_rejects_null_experts_and_mixed_dtypes(lib):
 def test_zero_tokens_is_a_host_side_no_op(lib):
     a = ctypes.c_void_p(1 << 20)
     ex = kmoe.Experts(a, a, a, None, None, None, kmoe.KMOE_BF16)
-    assert lib.moe_router_topk(None, kmoe.KMOE_BF16, None, None, 0, 2560, 384, 6,
+    assert lib.moe_router_topk(None, kmoe.KMOE_BF16, None, None, 0, 2560, 384, 6, 0,
                                None, None, None, None, 0, None) == kmoe.KMOE_OK
-    assert lib.moe_forward(None, kmoe.KMOE_BF16, 0, 2560, 384, 6, 512, None, None, ctypes.byref(ex),
+    assert lib.moe_forward(None, kmoe.KMOE_BF16, 0, 2560, 384, 6, 512, 0, None, None, ctypes.byref(ex),
                            None, None, kmoe.KMOE_BF16, None, None, None, None, 0, None) == kmoe.KMOE_OK
     assert lib.moe_last_error() == b""

@@ -70,6 +70,26 @@ def test_router_topk_matches_oracle(name, N):
             assert abs(w_g[t, k] - ora[int(idx_g[t, k])]) <= G_TOL
 
 
+@pytest.mark.parametrize("name,N", [("decode", None), ("prefill", 1024), ("tiny", None)])
+def test_router_topk_softmax_score_matches_oracle(name, N):
+    """KMOE_SCORE_SOFTMAX: same selection, weights = softmax over the K chosen unbiased logits."""
+    dev, host = layer_inputs(name, N)
+    cfg = host["cfg"]
+    idx, w = kmoe.moe_router_topk(dev["x"], dev["w_router"], dev["bias"], cfg.K, score="softmax")
+    torch.cuda.synchronize()
+    l_ora = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
+    i_ora, g_ora, _ = oracle.select(l_ora, host["bias"], cfg.K, score="softmax")
+    idx_g, w_g = idx.cpu().numpy(), w.cpu().double().numpy()
+    _, differ = check_routing(idx_g, i_ora, biased_scores(l_ora, host["bias"]), cfg.K)
+    assert np.allclose(w_g.sum(axis=1), 1.0, atol=1e-5)
+    for t in range(cfg.N):
+        if t in differ:
+            continue
+        ora = dict(zip(i_ora[t].tolist(), g_ora[t].tolist()))
+        for k in range(cfg.K):
+            assert abs(w_g[t, k] - ora[int(idx_g[t, k])]) <= G_TOL
+
+
 # ---------------------------------------------------------------- permute
 def _distinct_rows(rng, N, K, E, skew=False):
     if skew:
@@ -261,6 +281,20 @@ def test_forward_skew_full_size_sampled_tokens():
     rng = np.random.default_rng(2)
     rows = np.unique(np.concatenate([[0, cfg.N - 1], rng.integers(0, cfg.N, 24)])).astype(np.int32)
     _forward_and_compare("skew", rows=rows, check_all_routing=False)
+
+
+@pytest.mark.parametrize("name,N", [("decode", None), ("prefill", 300), ("fp8_decode", 64)])
+def test_forward_softmax_score_matches_oracle(name, N):
+    dev, host = layer_inputs(name, N)
+    cfg = host["cfg"]
+    y, idx, w, counts = kmoe.moe_forward(dev["x"], dev, with_outputs=True, score="softmax")
+    torch.cuda.synchronize()
+    ora = oracle.layer(host, nthreads=threads(), score="softmax")
+    l_all = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
+    _, differ = check_routing(idx.cpu().numpy(), ora["idx"], biased_scores(l_all, host["bias"]), cfg.K)
+    keep = np.array([t not in differ for t in range(cfg.N)])
+    got = y.float().cpu().numpy()
+    assert row_rel_err(got[keep], ora["y"][keep]) <= TOL[cfg.w_dtype]
 
 
 def test_forward_is_deterministic():
