@@ -161,5 +161,30 @@ def layer(inp, rows=None, nthreads: int = 1, score: str = "sigmoid"):
     return {"y": y, "idx": idx, "g": g, "margin": margin, "rows": rows}
 
 
+def rmsnorm_bf16(h, gamma, eps: float) -> np.ndarray:
+    """x = bf16(h / sqrt(mean(h^2) + eps) * gamma) row by row, as uint16 BF16 bits."""
+    hb = np.ascontiguousarray(_bits(h), dtype=np.uint16)
+    gb = np.ascontiguousarray(_bits(gamma), dtype=np.uint16)
+    N, d = hb.shape
+    x = np.empty((N, d), dtype=np.uint16)
+    lib().oracle_rmsnorm_bf16(N, d, _p(hb), _p(gb), ctypes.c_double(eps), _p(x))
+    return x
+
+
+def block(inp, h, gamma_pre, gamma_post, eps: float, rows=None, nthreads: int = 1, score: str = "sigmoid"):
+    """The sandwich block around the layer for tokens `rows`: x = bf16(RMSNorm(h) * g_pre),
+    m = layer(x), h_out = h + RMSNorm(m) * g_post. Returns dict(h_out, x, m, idx, g, margin)."""
+    hb = np.ascontiguousarray(_bits(h), dtype=np.uint16)
+    N, d = hb.shape
+    x = rmsnorm_bf16(hb, gamma_pre, eps)
+    ora = layer(dict(inp, x=x), rows=rows, nthreads=nthreads, score=score)
+    m = np.ascontiguousarray(ora["y"], dtype=np.float64)
+    rws = ora["rows"]
+    gp = np.ascontiguousarray(_bits(gamma_post), dtype=np.uint16)
+    h_out = np.empty_like(m)
+    lib().oracle_post_residual(N, d, len(rws), _p(rws), _p(hb), _p(m), _p(gp), ctypes.c_double(eps), _p(h_out))
+    return {"h_out": h_out, "x": x, "m": m, "idx": ora["idx"], "g": ora["g"], "margin": ora["margin"], "rows": rws}
+
+
 __all__ = ["build", "lib", "max_threads", "e4m3_to_double", "router_logits", "select",
-           "permute", "expert_outputs", "layer", "F32", "BF16", "E4M3"]
+           "permute", "expert_outputs", "layer", "rmsnorm_bf16", "block", "F32", "BF16", "E4M3"]

@@ -333,3 +333,63 @@ int oracle_max_threads(void)
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------
+ * Sandwich block around the MoE sublayer ("Inside Kolibri 1", section "The
+ * released stack": RMSNorm before and after the MoE, a residual addition
+ * after it). The pages give no epsilon; it is an argument.
+ *   x     = bf16( h / sqrt(mean_j h_j^2 + eps) * g_pre )
+ *   m     = the MoE layer on x (oracle_layer_score, in double)
+ *   h_out = h + m / sqrt(mean_j m_j^2 + eps) * g_post     (in double)
+ * The layer input x is stored in BF16, as the CUDA path stores it, so that
+ * the top-K is decided on the same input; bf16() rounds to nearest, ties to
+ * even, directly from double.
+ * ---------------------------------------------------------------------- */
+static uint16_t double_to_bf16_rne(double v)
+{
+    if (v == 0.0 || !isfinite(v)) {
+        float f = (float)v;
+        uint32_t u;
+        memcpy(&u, &f, 4);
+        return (uint16_t)(u >> 16);
+    }
+    int e;
+    frexp(v, &e);                                    /* v = f * 2^e, 0.5 <= |f| < 1 */
+    const double q = ldexp(nearbyint(ldexp(v, 8 - e)), e - 8);   /* 8 significant bits, ties to even */
+    const float f = (float)q;                        /* exact: q has 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);
+}
+
+/* x[t] = bf16(h[t] / sqrt(mean(h[t]^2) + eps) * gamma) for N rows of BF16 h. */
+void oracle_rmsnorm_bf16(int N, int d, const uint16_t *h, const uint16_t *gamma, double eps, uint16_t *x)
+{
+    for (int64_t t = 0; t < N; ++t) {
+        double ss = 0.0;
+        for (int j = 0; j < d; ++j) {
+            const double v = bf16_bits_to_double(h[t * d + j]);
+            ss += v * v;
+        }
+        const double r = 1.0 / sqrt(ss / d + eps);
+        for (int j = 0; j < d; ++j)
+            x[t * d + j] = double_to_bf16_rne(bf16_bits_to_double(h[t * d + j]) * r * bf16_bits_to_double(gamma[j]));
+    }
+}
+
+/* h_out[r] = h[rows[r]] + m[r] / sqrt(mean(m[r]^2) + eps) * g_post, with m the
+ * MoE output rows already computed (oracle_layer_score on the normalised x). */
+void oracle_post_residual(int N, int d, int n_rows, const int32_t *rows, const uint16_t *h, const double *m,
+                          const uint16_t *g_post, double eps, double *h_out)
+{
+    (void)N;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        double ss = 0.0;
+        for (int j = 0; j < d; ++j)
+            ss += m[r * d + j] * m[r * d + j];
+        const double s = 1.0 / sqrt(ss / d + eps);
+        for (int j = 0; j < d; ++j)
+            h_out[r * d + j] = bf16_bits_to_double(h[(int64_t)rows[r] * d + j]) + m[r * d + j] * s *
+                               bf16_bits_to_double(g_post[j]);
+    }
+}

@@ -13,6 +13,7 @@
 - Shapes: the weight counts printed on the pages.
 """
 import itertools
+import ctypes
 import math
 import os
 
@@ -137,6 +138,55 @@ def test_softmax_score_keeps_selection_and_is_a_distribution():
     i2, g2, _ = oracle.select(l2, np.zeros(2, dtype=np.float32), 2, score="softmax")
     first = np.take_along_axis(l2, i2, axis=1)
     np.testing.assert_allclose(g2[:, 0], 1.0 / (1.0 + np.exp(first[:, 1] - first[:, 0])), rtol=1e-13)
+
+
+def _bf16_bits(a):
+    return torch.tensor(np.asarray(a, dtype=np.float64)).to(torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _bf16_values(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+def test_rmsnorm_closed_forms():
+    """RMSNorm ("Inside Kolibri 1", section "The released stack"): a row of one repeated value c
+    normalises to sign(c) * gamma; the row (3, 4) has mean square 12.5."""
+    gamma = _bf16_bits([1.0, 1.0, 1.0, 1.0])
+    x = oracle.rmsnorm_bf16(_bf16_bits([[2.5, 2.5, 2.5, 2.5], [-0.75, -0.75, -0.75, -0.75]]), gamma, 0.0)
+    np.testing.assert_array_equal(_bf16_values(x), [[1, 1, 1, 1], [-1, -1, -1, -1]])
+    g2 = _bf16_bits([1.0, 2.0])
+    x2 = _bf16_values(oracle.rmsnorm_bf16(_bf16_bits([[3.0, 4.0]]), g2, 0.0))
+    ref = torch.tensor([3.0 / math.sqrt(12.5), 2 * 4.0 / math.sqrt(12.5)]).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(x2[0], ref)
+
+
+def test_rmsnorm_matches_torch_and_is_scale_invariant():
+    rng = np.random.default_rng(11)
+    h = _bf16_bits(rng.normal(0.0, 3.0, (16, 256)))
+    gamma = _bf16_bits(rng.uniform(0.5, 1.5, 256))
+    eps = 1e-6
+    x = _bf16_values(oracle.rmsnorm_bf16(h, gamma, eps))
+    hv, gv = _bf16_values(h), _bf16_values(gamma)
+    ref = hv / np.sqrt((hv ** 2).mean(axis=1, keepdims=True) + eps) * gv
+    ref_b = torch.tensor(ref).to(torch.bfloat16).double().numpy()   # one rounding from double
+    assert (x != ref_b).mean() < 1e-3                                  # ties of a double -> float -> bf16 path aside
+    assert np.abs(x - ref).max() <= 2.0 ** -8 * np.abs(ref).max()
+    # scaling the row by 4 (exact in BF16) leaves the normalised row unchanged (eps = 0)
+    x1 = oracle.rmsnorm_bf16(h, gamma, 0.0)
+    x4 = oracle.rmsnorm_bf16(_bf16_bits(4.0 * hv), gamma, 0.0)
+    np.testing.assert_array_equal(x1, x4)
+
+
+def test_post_norm_residual_closed_form():
+    """h_out = h + m / rms(m) * g_post: a constant m row adds sign(m) * g_post to h."""
+    h = _bf16_bits([[0.5, -1.0, 2.0], [1.0, 1.0, 1.0]])
+    gp = _bf16_bits([1.0, 2.0, 0.5])
+    m = np.array([[3.0, 3.0, 3.0], [-0.25, -0.25, -0.25]])
+    rows = np.array([0, 1], dtype=np.int32)
+    out = np.empty_like(m)
+    oracle.lib().oracle_post_residual(2, 3, 2, oracle._p(rows), oracle._p(h), oracle._p(m), oracle._p(gp),
+                                      ctypes.c_double(0.0), oracle._p(out))
+    np.testing.assert_allclose(out, [[1.5, 1.0, 2.5], [0.0, -1.0, 0.5]], atol=1e-15)
 
 
 def test_permute_matches_stable_sort():
