@@ -29,7 +29,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from fine_grained_sparse_fp32_b200 import _build, kmoe  # noqa: E402
-from fine_grained_sparse_fp32_b200.inputs import CONFIGS, make_inputs, make_x  # noqa: E402
+from fine_grained_sparse_fp32_b200.inputs import CONFIGS, make_block_inputs, make_inputs, make_x  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at 1 B200 (decode N=32, prefill N=8192); % of HBM/tensor roofline"
 ROTATE = 8           # distinct token batches cycled through the timed steps
@@ -201,6 +201,44 @@ def run_config(cfg, steps, warmup, rank, world, seed=0, use_graph=True):
             "ffn_ms": ffn_ms, "e2e_ms": e2e_ms}
 
 
+def time_block(cfg, steps, warmup, seed=0):
+    """Average step of the sandwich block (pre-norm, layer, post-norm + residual) on
+    rotating residual streams, in CUDA graphs; h_out is written in place."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    layer = make_inputs(cfg, seed=seed, device=dev)
+    lay = kmoe.Layer(layer, cfg.N, block=True)
+    blks = [make_block_inputs(cfg, seed=31 * i + 7, device=dev) for i in range(ROTATE)]
+    stream = torch.cuda.Stream(device=dev)
+    eps = 1e-6
+
+    def call(i):
+        b = blks[i % ROTATE]
+        lay.block_forward(b["h"], b["gamma_pre"], b["gamma_post"], eps, h_out=b["h"], stream=stream)
+
+    with torch.cuda.stream(stream):
+        call(0)
+    stream.synchronize()
+    graphs = []
+    for i in range(ROTATE):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            call(i)
+        graphs.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            graphs[i % ROTATE].replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(steps):
+            graphs[i % ROTATE].replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    status = kmoe.moe_device_status(lay.ws)
+    return {"ms_per_step": t0.elapsed_time(t1) / steps, "status": status}
+
+
 def time_grouped_ffn(layer, xs, stream, steps):
     """Average duration of one moe_grouped_ffn call (the expert FFN kernels)."""
     cfg = layer["cfg"]
@@ -327,6 +365,7 @@ def main():
     r = run_config(dec, args.steps, args.warmup, rank, world, use_graph=not args.no_graph)
     pre = None
     extras = {}
+    blocks = {}
     if not args.no_prefill:
         pcfg = CONFIGS["prefill"]
         psteps = max(10, min(args.steps // 10, 200))
@@ -335,6 +374,10 @@ def main():
         if not args.no_extra:
             for name, n_steps in (("fp8_decode", max(20, min(args.steps, 1000))), ("fp8_prefill", 50), ("skew", 10)):
                 extras[name] = run_config(CONFIGS[name], n_steps, 3, rank, world, use_graph=not args.no_graph)
+                torch.cuda.empty_cache()
+            if not args.no_graph:
+                blocks = {"decode": time_block(dec, max(20, min(args.steps, 1000)), 10),
+                          "prefill": time_block(CONFIGS["prefill"], 50, 3)}
                 torch.cuda.empty_cache()
 
     if rank == 0:
@@ -391,6 +434,14 @@ def main():
                 "ffn_ms": r_x["ffn_ms"], "ffn_gbs": xalg["ffn_bytes"] / (r_x["ffn_ms"] / 1e3) / 1e9,
                 "gpu_launches_per_step": launches_per_step(xcfg), "clocks": r_x["clocks"],
                 "traffic": kernel_traffic(name),
+            }
+        if blocks:
+            base = {"decode": ms, "prefill": pre["ms_per_step"] if pre else None}
+            line["block"] = {
+                "what": "RMSNorm -> layer -> RMSNorm + residual, BF16 residual stream updated in place",
+                **{k: {"ms_per_step": v["ms_per_step"], "layer_ms_per_step": base[k],
+                       "value": CONFIGS[k].N * world / (v["ms_per_step"] / 1e3), "unit": "tokens/s",
+                       "device_status": v["status"]} for k, v in blocks.items()},
             }
         if world == 1:
             try:

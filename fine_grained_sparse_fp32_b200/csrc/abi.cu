@@ -110,10 +110,11 @@ struct Layout {
     int32_t *counts, *offsets, *perm, *inv, *hist;
     __nv_bfloat16 *w_split;
     void *h, *y_perm, *y_shared;
+    __nv_bfloat16 *x_norm;   // sandwich block only: the normalised layer input
     size_t bytes;
 };
 
-static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype)
+static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype, bool block = false)
 {
     Carver c(ws);
     Layout L;
@@ -132,6 +133,7 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype)
     L.h = c.take<char>(R * I * ab);
     L.y_perm = c.take<char>((size_t)N * K * d * ab);
     L.y_shared = c.take<char>((size_t)N * d * ab);
+    L.x_norm = block ? c.take<__nv_bfloat16>((size_t)N * d) : nullptr;
     L.bytes = c.used + 256;
     return L;
 }
@@ -175,6 +177,68 @@ static kmoe_status clear_status(int *status, cudaStream_t st, size_t bytes = kSt
 
 constexpr int kFusedRouteTokens = 256;   // routing, top-K and dispatch in one launch up to here
 
+static kmoe_status check_score(int score)
+{
+    if (score != KMOE_SCORE_SIGMOID && score != KMOE_SCORE_SOFTMAX)
+        return fail(KMOE_ERR_INVALID_ARG, "score %d: KMOE_SCORE_SIGMOID or KMOE_SCORE_SOFTMAX", score);
+    return KMOE_OK;
+}
+
+// Validation shared by moe_forward and moe_block_forward.
+static kmoe_status check_forward(int N, int d, int E, int K, int I, int score, const kmoe_experts *routed,
+                                 const kmoe_experts *shared, const float *w_router, const float *bias,
+                                 int32_t *topk_idx_out, float *topk_w_out, int32_t *counts_out, void *ws)
+{
+    KMOE_TRY(check_sizes(N, d, E, K, I));
+    KMOE_TRY(check_score(score));
+    KMOE_TRY(check_experts(routed, "routed"));
+    if (shared) {
+        KMOE_TRY(check_experts(shared, "shared"));
+        if (shared->dtype != routed->dtype) return fail(KMOE_ERR_UNSUPPORTED, "shared and routed dtypes differ");
+    }
+    if (N == 0) return KMOE_OK;
+    KMOE_TRY(check_ptr(w_router, "w_router"));
+    KMOE_TRY(check_ptr(bias, "bias"));
+    KMOE_TRY(check_ptr(topk_idx_out, "topk_idx_out", true));
+    KMOE_TRY(check_ptr(topk_w_out, "topk_w_out", true));
+    KMOE_TRY(check_ptr(counts_out, "counts_out", true));
+    return check_ptr(ws, "ws");
+}
+
+// Routing, dispatch, expert FFNs and combine of one layer call on laid-out
+// workspace L; with h_res set the combine also applies the post-norm and the
+// residual addition of the sandwich block.
+static kmoe_status forward_path(const void *x, int x_dtype, int N, int d, int E, int K, int I, int score,
+                                const float *w_router, const float *bias, const kmoe_experts *routed,
+                                const kmoe_experts *shared, void *y, int y_dtype, int32_t *topk_idx_out,
+                                float *topk_w_out, int32_t *counts_out, const Layout &L, const void *h_res,
+                                const void *g_post, float eps, cudaStream_t st)
+{
+    int32_t *idx = topk_idx_out ? topk_idx_out : L.idx;
+    float *w = topk_w_out ? topk_w_out : L.w;
+    int32_t *counts = counts_out ? counts_out : L.counts;
+    if (N <= kFusedRouteTokens) {
+        KMOE_TRY(launch_route_small(x, x_dtype, w_router, bias, N, d, E, K, score, L.logits, idx, w, counts, L.offsets,
+                                    L.perm, L.inv, L.status, st));
+    } else {
+        if (x_dtype == KMOE_BF16 && N >= kTcRouterTokens)
+            KMOE_TRY(launch_router_tc(static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E, L.w_split, L.logits,
+                                      L.status, st));
+        else
+            KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, L.logits, st));
+        KMOE_TRY(launch_topk(L.logits, bias, N, E, K, score, idx, w, st));
+        KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st));
+    }
+    const ExpertPtrs r = ptrs(routed);
+    ExpertPtrs s{};
+    if (shared) s = ptrs(shared);
+    KMOE_TRY(run_ffn(x, x_dtype, N, d, I, E, K, L.perm, L.offsets, routed->dtype, r, shared ? &s : nullptr,
+                     L.h, L.y_perm, L.y_shared, L.status, st));
+    const int yin = routed->dtype == KMOE_F32 ? KMOE_F32 : KMOE_BF16;
+    return launch_combine(L.y_perm, shared ? L.y_shared : nullptr, yin, w, L.inv, N, K, d, y, y_dtype, L.status, st,
+                          h_res, g_post, eps);
+}
+
 }  // namespace kmoe
 
 using namespace kmoe;
@@ -194,12 +258,6 @@ size_t moe_workspace_size(int N, int d, int E, int K, int I, int x_dtype, int w_
     return layout(nullptr, N, d, E, K, I, w_dtype).bytes;
 }
 
-static kmoe_status check_score(int score)
-{
-    if (score != KMOE_SCORE_SIGMOID && score != KMOE_SCORE_SOFTMAX)
-        return fail(KMOE_ERR_INVALID_ARG, "score %d: KMOE_SCORE_SIGMOID or KMOE_SCORE_SOFTMAX", score);
-    return KMOE_OK;
-}
 
 kmoe_status moe_router_topk(const void *x, int x_dtype, const float *w_router, const float *bias,
                             int N, int d, int E, int K, int score, float *logits, int32_t *topk_idx,
@@ -321,52 +379,63 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
                         float *topk_w_out, int32_t *counts_out, void *ws, size_t ws_bytes, void *stream)
 {
     clear_error();
-    KMOE_TRY(check_sizes(N, d, E, K, I));
     KMOE_TRY(check_act_dtype(x_dtype, "x"));
     KMOE_TRY(check_act_dtype(y_dtype, "y"));
-    KMOE_TRY(check_score(score));
-    KMOE_TRY(check_experts(routed, "routed"));
-    if (shared) {
-        KMOE_TRY(check_experts(shared, "shared"));
-        if (shared->dtype != routed->dtype) return fail(KMOE_ERR_UNSUPPORTED, "shared and routed dtypes differ");
-    }
+    KMOE_TRY(check_forward(N, d, E, K, I, score, routed, shared, w_router, bias, topk_idx_out, topk_w_out, counts_out,
+                           ws));
     if (N == 0) return KMOE_OK;
     KMOE_TRY(check_ptr(x, "x"));
-    KMOE_TRY(check_ptr(w_router, "w_router"));
-    KMOE_TRY(check_ptr(bias, "bias"));
     KMOE_TRY(check_ptr(y, "y"));
-    KMOE_TRY(check_ptr(topk_idx_out, "topk_idx_out", true));
-    KMOE_TRY(check_ptr(topk_w_out, "topk_w_out", true));
-    KMOE_TRY(check_ptr(counts_out, "counts_out", true));
-    KMOE_TRY(check_ptr(ws, "ws"));
     const Layout need = layout(nullptr, N, d, E, K, I, routed->dtype);
     if (ws_bytes < need.bytes) return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need.bytes);
     // the base the Carver sees is 256-aligned by construction of the pieces
     const Layout L = layout(ws, N, d, E, K, I, routed->dtype);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    int32_t *idx = topk_idx_out ? topk_idx_out : L.idx;
-    float *w = topk_w_out ? topk_w_out : L.w;
-    int32_t *counts = counts_out ? counts_out : L.counts;
     KMOE_TRY(clear_status(L.status, st, kFfnStatusBytes));
-    if (N <= kFusedRouteTokens) {
-        KMOE_TRY(launch_route_small(x, x_dtype, w_router, bias, N, d, E, K, score, L.logits, idx, w, counts, L.offsets,
-                                    L.perm, L.inv, L.status, st));
-    } else {
-        if (x_dtype == KMOE_BF16 && N >= kTcRouterTokens)
-            KMOE_TRY(launch_router_tc(static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E, L.w_split, L.logits,
-                                      L.status, st));
-        else
-            KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, L.logits, st));
-        KMOE_TRY(launch_topk(L.logits, bias, N, E, K, score, idx, w, st));
-        KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st));
-    }
-    const ExpertPtrs r = ptrs(routed);
-    ExpertPtrs s{};
-    if (shared) s = ptrs(shared);
-    KMOE_TRY(run_ffn(x, x_dtype, N, d, I, E, K, L.perm, L.offsets, routed->dtype, r, shared ? &s : nullptr,
-                     L.h, L.y_perm, L.y_shared, L.status, st));
-    const int yin = routed->dtype == KMOE_F32 ? KMOE_F32 : KMOE_BF16;
-    return launch_combine(L.y_perm, shared ? L.y_shared : nullptr, yin, w, L.inv, N, K, d, y, y_dtype, L.status, st);
+    return forward_path(x, x_dtype, N, d, E, K, I, score, w_router, bias, routed, shared, y, y_dtype, topk_idx_out,
+                        topk_w_out, counts_out, L, nullptr, nullptr, 0.f, st);
+}
+
+size_t moe_block_workspace_size(int N, int d, int E, int K, int I, int w_dtype)
+{
+    if (check_sizes(N, d, E, K, I) != KMOE_OK) return 0;
+    if (w_dtype != KMOE_BF16 && w_dtype != KMOE_E4M3_B128) return 0;
+    clear_error();
+    return layout(nullptr, N, d, E, K, I, w_dtype, true).bytes;
+}
+
+kmoe_status moe_block_forward(const void *h, int N, int d, int E, int K, int I, int score, const void *gamma_pre,
+                              const void *gamma_post, float eps, const float *w_router, const float *bias,
+                              const kmoe_experts *routed, const kmoe_experts *shared, void *h_out,
+                              void *x_out, int32_t *topk_idx_out, float *topk_w_out, int32_t *counts_out, void *ws,
+                              size_t ws_bytes, void *stream)
+{
+    clear_error();
+    KMOE_TRY(check_forward(N, d, E, K, I, score, routed, shared, w_router, bias, topk_idx_out, topk_w_out, counts_out,
+                           ws));
+    if (routed->dtype != KMOE_BF16 && routed->dtype != KMOE_E4M3_B128)
+        return fail(KMOE_ERR_UNSUPPORTED, "block: routed weights must be BF16 or E4M3 with 128x128 scales");
+    if (!(eps >= 0.f) || eps > 1.f) return fail(KMOE_ERR_INVALID_ARG, "eps=%g: must be in [0, 1]", (double)eps);
+    const size_t row_smem = (size_t)(K + (shared ? 1 : 0)) * d * 2;
+    if (2 * row_smem > 100 * 1024)
+        return fail(KMOE_ERR_UNSUPPORTED, "block: (K + 1) * d = %zu BF16 values per token exceed the combine's "
+                    "staging buffer", row_smem / 2);
+    if (N == 0) return KMOE_OK;
+    KMOE_TRY(check_ptr(h, "h"));
+    KMOE_TRY(check_ptr(gamma_pre, "gamma_pre"));
+    KMOE_TRY(check_ptr(gamma_post, "gamma_post"));
+    KMOE_TRY(check_ptr(h_out, "h_out"));
+    KMOE_TRY(check_ptr(x_out, "x_out", true));
+    const Layout need = layout(nullptr, N, d, E, K, I, routed->dtype, true);
+    if (ws_bytes < need.bytes) return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need.bytes);
+    const Layout L = layout(ws, N, d, E, K, I, routed->dtype, true);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    KMOE_TRY(clear_status(L.status, st, kFfnStatusBytes));
+    __nv_bfloat16 *x = x_out ? static_cast<__nv_bfloat16 *>(x_out) : L.x_norm;
+    KMOE_TRY(launch_rmsnorm(static_cast<const __nv_bfloat16 *>(h), static_cast<const __nv_bfloat16 *>(gamma_pre), eps,
+                            N, d, x, st));
+    return forward_path(x, KMOE_BF16, N, d, E, K, I, score, w_router, bias, routed, shared, h_out, KMOE_BF16,
+                        topk_idx_out, topk_w_out, counts_out, L, h, gamma_post, eps, st);
 }
 
 kmoe_status moe_device_status(const void *ws, int *status, void *stream)

@@ -72,6 +72,12 @@ combine_kernel(const YI *__restrict__ y_perm, const YI *__restrict__ y_shared,
 // memory with the bulk-copy engine (K routed rows and the shared row, d * 2
 // bytes each) two tokens ahead, so each SM keeps ~140 KB of reads in flight;
 // the threads then form the same fixed-order FP32 sum from shared memory.
+// With h_res set it finishes the sandwich block ("Inside Kolibri 1", "The
+// released stack": RMSNorm after the MoE, then the residual addition):
+//     y[t] = h_res[t] + m[t] / sqrt(mean_j m[t][j]^2 + eps) * g_post
+// where m[t] is the combined row in FP32; its sum of squares is reduced in a
+// fixed order and m is formed twice (once for the norm, once for the output)
+// from the rows in shared memory.
 constexpr int kBulkThreads = 320;
 constexpr int kBulkStages = 2;
 constexpr long long kBulkWaitLimit = 1LL << 32;
@@ -80,12 +86,15 @@ template <class YO>
 __global__ void __launch_bounds__(kBulkThreads)
 combine_bulk_kernel(const __nv_bfloat16 *__restrict__ y_perm, const __nv_bfloat16 *__restrict__ y_shared,
                     const float *__restrict__ w, const int32_t *__restrict__ inv, int N, int K, int d,
-                    YO *__restrict__ y, int *err)
+                    YO *y, int *err, const __nv_bfloat16 *h_res,
+                    const __nv_bfloat16 *__restrict__ g_post, float eps)
 {
     using namespace sm100;
     extern __shared__ __align__(128) uint8_t cb_smem[];
     __shared__ __align__(8) uint64_t full[kBulkStages];
     __shared__ int abort_flag;
+    __shared__ float red[kBulkThreads / 32];
+    __shared__ float post_scale;
     const int R = K + (y_shared ? 1 : 0);                 // rows per token
     const size_t row_bytes = (size_t)d * sizeof(__nv_bfloat16);
     const size_t stage_bytes = (size_t)R * row_bytes;
@@ -120,8 +129,9 @@ combine_bulk_kernel(const __nv_bfloat16 *__restrict__ y_perm, const __nv_bfloat1
         float g[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) g[k] = k < K ? w[(size_t)t * K + k] : 0.f;
-        for (int c = threadIdx.x * 8; c < d; c += kBulkThreads * 8) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        auto combined = [&](int c, float (&acc)[8]) {       // m[t][c .. c+7], fixed slot order
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = 0.f;
             if (y_shared) load8(reinterpret_cast<const __nv_bfloat16 *>(rows + (size_t)K * row_bytes) + c, acc);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
@@ -131,7 +141,40 @@ combine_bulk_kernel(const __nv_bfloat16 *__restrict__ y_perm, const __nv_bfloat1
 #pragma unroll
                     for (int q = 0; q < 8; ++q) acc[q] = fmaf(g[k], v[q], acc[q]);
                 }
-            store8(y + (size_t)t * d + c, acc);
+        };
+        if (!h_res) {
+            for (int c = threadIdx.x * 8; c < d; c += kBulkThreads * 8) {
+                float acc[8];
+                combined(c, acc);
+                store8(y + (size_t)t * d + c, acc);
+            }
+        } else {
+            float ss = 0.f;
+            for (int c = threadIdx.x * 8; c < d; c += kBulkThreads * 8) {
+                float acc[8];
+                combined(c, acc);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) ss = fmaf(acc[q], acc[q], ss);
+            }
+            ss = warp_sum(ss);
+            if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                float tot = 0.f;
+                for (int wq = 0; wq < kBulkThreads / 32; ++wq) tot += red[wq];
+                post_scale = 1.f / sqrtf(tot / (float)d + eps);
+            }
+            __syncthreads();
+            const float sc = post_scale;
+            for (int c = threadIdx.x * 8; c < d; c += kBulkThreads * 8) {
+                float acc[8], hv[8], gv[8];
+                combined(c, acc);
+                load8(h_res + (size_t)t * d + c, hv);
+                load8(g_post + c, gv);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] = fmaf(acc[q] * sc, gv[q], hv[q]);
+                store8(y + (size_t)t * d + c, acc);
+            }
         }
         __syncthreads();                                  // every thread is done with stage s
         if (threadIdx.x == 0) issue(i + kBulkStages);
@@ -144,10 +187,13 @@ static size_t bulk_smem(int K, int d, bool shared) { return (size_t)kBulkStages 
 
 kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dtype,
                            const float *w, const int32_t *inv, int N, int K, int d, void *y,
-                           int y_dtype, int *err, cudaStream_t st)
+                           int y_dtype, int *err, cudaStream_t st, const void *h_res, const void *g_post, float eps)
 {
     using bf = __nv_bfloat16;
     const size_t bsm = bulk_smem(K, d, y_shared != nullptr);
+    const bf *hr = static_cast<const bf *>(h_res), *gp = static_cast<const bf *>(g_post);
+    if (h_res && !(y_in_dtype == KMOE_BF16 && y_dtype == KMOE_BF16 && bsm <= 100 * 1024))
+        return fail(KMOE_ERR_UNSUPPORTED, "post-norm combine: BF16 rows with K + 1 rows of d in 100 KB");
     if (y_in_dtype == KMOE_BF16 && bsm <= 100 * 1024) {
         int dev = 0, sms = 148;
         cudaGetDevice(&dev);
@@ -157,10 +203,12 @@ kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dt
         const bf *yp = static_cast<const bf *>(y_perm), *ys = static_cast<const bf *>(y_shared);
         if (y_dtype == KMOE_F32) {
             cudaFuncSetAttribute(combine_bulk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsm);
-            combine_bulk_kernel<float><<<grid, kBulkThreads, bsm, st>>>(yp, ys, w, inv, N, K, d, static_cast<float *>(y), err);
+            combine_bulk_kernel<float><<<grid, kBulkThreads, bsm, st>>>(yp, ys, w, inv, N, K, d, static_cast<float *>(y), err,
+                                                                        hr, gp, eps);
         } else {
             cudaFuncSetAttribute(combine_bulk_kernel<bf>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsm);
-            combine_bulk_kernel<bf><<<grid, kBulkThreads, bsm, st>>>(yp, ys, w, inv, N, K, d, static_cast<bf *>(y), err);
+            combine_bulk_kernel<bf><<<grid, kBulkThreads, bsm, st>>>(yp, ys, w, inv, N, K, d, static_cast<bf *>(y), err,
+                                                                     hr, gp, eps);
         }
         return check_launch("combine");
     }

@@ -176,8 +176,14 @@ kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, 
                             int *sync, cudaStream_t st);
 
 // err: device status word for a bounded wait that gives up (may be NULL).
+// h_res / g_post (BF16, NULL for the plain combine): y = h_res + RMSNorm(m) * g_post.
 kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dtype,
                            const float *w, const int32_t *inv, int N, int K, int d, void *y,
-                           int y_dtype, int *err, cudaStream_t st);
+                           int y_dtype, int *err, cudaStream_t st, const void *h_res = nullptr,
+                           const void *g_post = nullptr, float eps = 0.f);
+
+// x = bf16(h / sqrt(mean(h^2) + eps) * gamma), row by row.
+kmoe_status launch_rmsnorm(const __nv_bfloat16 *h, const __nv_bfloat16 *gamma, float eps, int N, int d,
+                           __nv_bfloat16 *x, cudaStream_t st);
 
 }  // namespace kmoe

@@ -153,6 +153,23 @@ def make_x(cfg: LayerConfig, seed: int, device="cpu") -> torch.Tensor:
     return x.to(_TORCH_DTYPES[cfg.x_dtype])
 
 
+def make_block_inputs(cfg: LayerConfig, seed: int, device="cpu") -> dict:
+    """Residual stream and norm gains of the sandwich block around the layer.
+
+    One generator seeded with `seed`; draw order h, gamma_pre, gamma_post.
+    h ~ N(0, 2) (a residual stream that has grown past unit scale); each gain
+    ~ 1 + N(0, 0.1), the spread of trained RMSNorm gains around their
+    initial value 1. All three in BF16: h [N, d], gains [d]."""
+    gen = torch.Generator(device=torch.device(device))
+    gen.manual_seed(seed)
+    d = cfg.d
+    h = torch.empty((cfg.N, d), device=device, dtype=torch.float32).normal_(0.0, 2.0, generator=gen)
+    g_pre = torch.empty(d, device=device, dtype=torch.float32).normal_(1.0, 0.1, generator=gen)
+    g_post = torch.empty(d, device=device, dtype=torch.float32).normal_(1.0, 0.1, generator=gen)
+    return {"h": h.to(torch.bfloat16), "gamma_pre": g_pre.to(torch.bfloat16),
+            "gamma_post": g_post.to(torch.bfloat16)}
+
+
 def expected_distinct_experts(cfg: LayerConfig) -> float:
     """Mean number of distinct routed experts hit by N uniform top-K draws."""
     return cfg.E * (1.0 - (1.0 - cfg.K / cfg.E) ** cfg.N)
@@ -163,5 +180,5 @@ def to_host(inputs: dict) -> dict:
     return {k: (v.detach().to("cpu").contiguous() if torch.is_tensor(v) else v) for k, v in inputs.items()}
 
 
-__all__ = ["LayerConfig", "CONFIGS", "make_inputs", "make_x", "to_host",
+__all__ = ["LayerConfig", "CONFIGS", "make_inputs", "make_x", "make_block_inputs", "to_host",
            "expected_distinct_experts", "E4M3_MAX", "FP8_BLOCK", "SKEW_BETA", "SKEW_EMPTY"]

@@ -22,7 +22,8 @@ SCORES = {"sigmoid": 0, "softmax": 1}     # kmoe_score
 FFN_STATUS_BYTES = (64 + 1088) * 4
 
 EXPORTS = ["moe_workspace_size", "moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn",
-           "moe_combine", "moe_forward", "moe_device_status", "moe_last_error", "moe_abi_version"]
+           "moe_combine", "moe_forward", "moe_block_workspace_size", "moe_block_forward", "moe_device_status",
+           "moe_last_error", "moe_abi_version"]
 
 
 class KmoeError(RuntimeError):
@@ -63,9 +64,13 @@ def load(path: str | None = None):
     lib.moe_combine.argtypes = [vp, vp, i, vp, vp, i, i, i, vp, i, vp]
     lib.moe_forward.argtypes = [vp, i, i, i, i, i, i, i, vp, vp, ctypes.POINTER(Experts),
                                 ctypes.POINTER(Experts), vp, i, vp, vp, vp, vp, sz, vp]
+    lib.moe_block_workspace_size.restype = sz
+    lib.moe_block_workspace_size.argtypes = [i, i, i, i, i, i]
+    lib.moe_block_forward.argtypes = [vp, i, i, i, i, i, i, vp, vp, ctypes.c_float, vp, vp,
+                                      ctypes.POINTER(Experts), ctypes.POINTER(Experts), vp, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
     for f in ("moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn", "moe_combine",
-              "moe_forward", "moe_device_status"):
+              "moe_forward", "moe_block_forward", "moe_device_status"):
         getattr(lib, f).restype = i
     if lib.moe_abi_version() != 2:
         raise RuntimeError("libkmoe ABI version mismatch")
@@ -211,20 +216,32 @@ def moe_combine(y_perm, y_shared, topk_w, inv_pos, y_dtype=torch.bfloat16, out=N
     return y
 
 
+def moe_block_workspace_size(N, d, E, K, I, w_dtype: int) -> int:
+    return int(load().moe_block_workspace_size(N, d, E, K, I, w_dtype))
+
+
 class Layer:
     """Device-resident weights of one layer plus a reusable workspace.
 
-    `forward(x)` is one moe_forward call; outputs are written into tensors
-    owned here (or passed in)."""
+    `forward(x)` is one moe_forward call and `block_forward(h, ...)` one
+    moe_block_forward call (workspace sized for it when `block` is set);
+    outputs are written into tensors owned here (or passed in)."""
 
-    def __init__(self, layer: dict, max_tokens: int, y_dtype=torch.bfloat16, score: str = "sigmoid"):
+    def __init__(self, layer: dict, max_tokens: int, y_dtype=torch.bfloat16, score: str = "sigmoid",
+                 block: bool = False):
         self.layer = layer
         cfg = self.cfg = layer["cfg"]
         self.routed = experts_of(layer, "routed")
         self.shared = experts_of(layer, "shared")
         dev = layer["w_gate"].device
         self.x_code = w_dtype_code(cfg.x_dtype)
-        self.ws = workspace(max_tokens, cfg.d, cfg.E, cfg.K, cfg.I, self.x_code, w_dtype_code(cfg.w_dtype), dev)
+        if block:
+            n = moe_block_workspace_size(max_tokens, cfg.d, cfg.E, cfg.K, cfg.I, w_dtype_code(cfg.w_dtype))
+            if n == 0:
+                _check(KMOE_ERR_UNSUPPORTED)
+            self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        else:
+            self.ws = workspace(max_tokens, cfg.d, cfg.E, cfg.K, cfg.I, self.x_code, w_dtype_code(cfg.w_dtype), dev)
         self.y_dtype = y_dtype
         self.max_tokens = max_tokens
         self.score = SCORES[score]
@@ -243,6 +260,24 @@ class Layer:
                                   _ptr(topk_w), _ptr(counts), _ptr(self.ws), self.ws.numel(), _stream(stream)))
         return y
 
+    def block_forward(self, h, gamma_pre, gamma_post, eps: float, h_out=None, topk_idx=None, topk_w=None,
+                      counts=None, x_out=None, stream=None):
+        """h_out = h + RMSNorm(layer(x)) * gamma_post with x = bf16(RMSNorm(h) * gamma_pre); h_out may
+        be h; x_out (optional) receives x."""
+        cfg = self.cfg
+        N = h.shape[0]
+        if N > self.max_tokens:
+            raise ValueError("more tokens than the workspace was sized for")
+        if h_out is None:
+            h_out = torch.empty_like(h)
+        L = self.layer
+        _check(load().moe_block_forward(_ptr(h), N, cfg.d, cfg.E, cfg.K, cfg.I, self.score, _ptr(gamma_pre),
+                                        _ptr(gamma_post), float(eps), _ptr(L["w_router"]), _ptr(L["bias"]),
+                                        ctypes.byref(self.routed), ctypes.byref(self.shared), _ptr(h_out),
+                                        _ptr(x_out), _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(self.ws),
+                                        self.ws.numel(), _stream(stream)))
+        return h_out
+
 
 def moe_forward(x, layer, y_dtype=torch.bfloat16, with_outputs=False, stream=None, score="sigmoid"):
     """One whole-layer call; with_outputs also returns (topk_idx, topk_w, counts)."""
@@ -256,3 +291,20 @@ def moe_forward(x, layer, y_dtype=torch.bfloat16, with_outputs=False, stream=Non
     counts = torch.empty(cfg.E, dtype=torch.int32, device=x.device)
     y = lay.forward(x, topk_idx=idx, topk_w=w, counts=counts, stream=stream)
     return y, idx, w, counts
+
+
+def moe_block_forward(h, layer, gamma_pre, gamma_post, eps: float, with_outputs=False, stream=None,
+                      score="sigmoid", h_out=None):
+    """One sandwich-block call; with_outputs also returns (x, topk_idx, topk_w, counts)."""
+    cfg = layer["cfg"]
+    N = h.shape[0]
+    lay = Layer(layer, N, torch.bfloat16, score, block=True)
+    if not with_outputs:
+        return lay.block_forward(h, gamma_pre, gamma_post, eps, h_out=h_out, stream=stream)
+    idx = torch.empty((N, cfg.K), dtype=torch.int32, device=h.device)
+    w = torch.empty((N, cfg.K), dtype=torch.float32, device=h.device)
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=h.device)
+    x = torch.empty_like(h)
+    out = lay.block_forward(h, gamma_pre, gamma_post, eps, h_out=h_out, topk_idx=idx, topk_w=w, counts=counts,
+                            x_out=x, stream=stream)
+    return out, x, idx, w, counts

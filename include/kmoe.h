@@ -209,7 +209,37 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
                         void *ws, size_t ws_bytes, void *stream);
 
 /*
- * Device status word. moe_forward and moe_grouped_ffn clear the first 4
+ * The sandwich block around the layer ("Inside Kolibri 1", section "The
+ * released stack": RMSNorm before and after the MoE sublayer, residual added
+ * after the second norm):
+ *   x[t]     = bf16( h[t] / sqrt(mean_j h[t][j]^2 + eps) * gamma_pre )
+ *   m        = the layer of moe_forward applied to x (FP32 combine)
+ *   h_out[t] = bf16( h[t] + m[t] / sqrt(mean_j m[t][j]^2 + eps) * gamma_post )
+ * Both sums of squares are FP32 in a fixed order (deterministic). The pages
+ * give neither eps nor the dtype of the residual stream; this call takes eps
+ * (0 <= eps <= 1) and keeps the residual stream in BF16.
+ * h device [N, d] BF16; gamma_pre, gamma_post device [d] BF16; h_out device
+ * [N, d] BF16, which may be the same buffer as h (each element of h is read
+ * before its h_out element is written, by the same thread) but must not
+ * overlap it otherwise. x_out: optional device [N, d] BF16 output of the
+ * normalised layer input x (NULL keeps it in the workspace). Routed (and shared) weights must be BF16 or E4M3
+ * with 128 x 128 scales (KMOE_ERR_UNSUPPORTED otherwise), and
+ * (K + 1) * d <= 25600 BF16 values must fit the combine's staging buffer
+ * (K + 1 counts the shared expert). Other arguments and outputs as in
+ * moe_forward. ws: at least moe_block_workspace_size() bytes; its first 4
+ * bytes are the status word read by moe_device_status.
+ */
+size_t moe_block_workspace_size(int N, int d, int E, int K, int I, int w_dtype);
+kmoe_status moe_block_forward(const void *h, int N, int d, int E, int K, int I, int score,
+                              const void *gamma_pre, const void *gamma_post, float eps,
+                              const float *w_router, const float *bias,
+                              const kmoe_experts *routed, const kmoe_experts *shared,
+                              void *h_out, void *x_out,
+                              int32_t *topk_idx_out, float *topk_w_out, int32_t *counts_out,
+                              void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Device status word. moe_forward, moe_block_forward and moe_grouped_ffn clear the first 4
  * bytes of `ws` when they are enqueued; a tensor-core kernel whose pipeline
  * wait gives up (after about two seconds, which only a fault elsewhere can
  * cause) writes a non-zero code there and returns early, leaving its outputs

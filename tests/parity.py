@@ -23,9 +23,11 @@ def biased_scores(logits: np.ndarray, bias) -> np.ndarray:
     return logits + b[None, :]
 
 
-def check_routing(gpu_idx: np.ndarray, ora_idx: np.ndarray, s: np.ndarray, K: int):
+def check_routing(gpu_idx: np.ndarray, ora_idx: np.ndarray, s: np.ndarray, K: int, margin: float | None = None):
     """Returns (n_flagged, mismatch_rows) where mismatch_rows are flagged tokens whose
-    GPU set differs from the oracle's (valid tie resolutions)."""
+    GPU set differs from the oracle's (valid tie resolutions). `margin` replaces
+    TIE_MARGIN where the two sides route slightly different inputs."""
+    TIE_MARGIN = globals()["TIE_MARGIN"] if margin is None else margin
     gpu_idx = np.asarray(gpu_idx)
     N = gpu_idx.shape[0]
     order = np.argsort(-s, axis=1, kind="stable")

@@ -110,3 +110,36 @@ def test_zero_tokens_is_a_host_side_no_op(lib):
     assert lib.moe_forward(None, kmoe.KMOE_BF16, 0, 2560, 384, 6, 512, 0, None, None, ctypes.byref(ex),
                            None, None, kmoe.KMOE_BF16, None, None, None, None, 0, None) == kmoe.KMOE_OK
     assert lib.moe_last_error() == b""
+
+
+def test_block_workspace_adds_the_normalised_input(lib):
+    for w in (kmoe.KMOE_BF16, kmoe.KMOE_E4M3_B128):
+        base = lib.moe_workspace_size(64, 2560, 384, 6, 512, kmoe.KMOE_BF16, w)
+        blk = lib.moe_block_workspace_size(64, 2560, 384, 6, 512, w)
+        assert blk >= base + 64 * 2560 * 2
+    assert lib.moe_block_workspace_size(64, 2560, 384, 6, 512, kmoe.KMOE_F32) == 0
+
+
+def test_block_forward_checks_arguments_on_the_host(lib):
+    vp = ctypes.c_void_p
+    a = vp(1 << 20)
+    bf = kmoe.Experts(a, a, a, None, None, None, kmoe.KMOE_BF16)
+    f32 = kmoe.Experts(a, a, a, None, None, None, kmoe.KMOE_F32)
+
+    def call(N=32, d=2560, K=6, g_pre=a, g_post=a, eps=1e-6, routed=bf, shared=bf, score=0):
+        return lib.moe_block_forward(a, N, d, 384, K, 512, score, g_pre, g_post, eps, a, a, ctypes.byref(routed),
+                                     ctypes.byref(shared) if shared is not None else None, a, None, None, None, None, a,
+                                     1 << 40, None)
+
+    assert call(routed=f32, shared=f32) == kmoe.KMOE_ERR_UNSUPPORTED and b"BF16" in lib.moe_last_error()
+    assert call(eps=-1.0) == kmoe.KMOE_ERR_INVALID_ARG and b"eps" in lib.moe_last_error()
+    assert call(eps=float("nan")) == kmoe.KMOE_ERR_INVALID_ARG
+    assert call(g_pre=None) == kmoe.KMOE_ERR_INVALID_ARG and b"gamma_pre" in lib.moe_last_error()
+    assert call(g_post=None) == kmoe.KMOE_ERR_INVALID_ARG and b"gamma_post" in lib.moe_last_error()
+    assert call(score=5) == kmoe.KMOE_ERR_INVALID_ARG
+    # K routed rows plus the shared row of d = 6144 do not fit the combine's staging buffer
+    assert call(d=6144, K=8) == kmoe.KMOE_ERR_UNSUPPORTED and b"staging" in lib.moe_last_error()
+    assert call(N=0, g_pre=None, g_post=None) == kmoe.KMOE_OK
+    small = lib.moe_block_forward(a, 32, 2560, 384, 6, 512, 0, a, a, 1e-6, a, a, ctypes.byref(bf), None, a,
+                                  None, None, None, None, a, 1024, None)
+    assert small == kmoe.KMOE_ERR_WORKSPACE

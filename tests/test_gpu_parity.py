@@ -10,7 +10,7 @@ import torch
 
 import oracle
 from fine_grained_sparse_fp32_b200 import _build, kmoe
-from fine_grained_sparse_fp32_b200.inputs import CONFIGS, make_inputs, to_host
+from fine_grained_sparse_fp32_b200.inputs import CONFIGS, make_block_inputs, make_inputs, to_host
 from parity import G_TOL, TOL, biased_scores, check_routing, frob_rel_err, row_rel_err
 
 pytestmark = pytest.mark.gpu
@@ -319,3 +319,83 @@ def test_forward_zero_tokens():
     dev, _ = layer_inputs("decode")
     y = kmoe.moe_forward(dev["x"][:0], dev)
     assert y.shape == (0, 2560)
+
+
+# ------------------------------------------------------- sandwich block
+BLOCK_EPS = 1e-6
+# The two sides route their own normalised inputs, which may differ by one
+# BF16 ulp in a few elements (~1e-4 change of a logit at these weight scales).
+BLOCK_TIE = 1e-3
+
+
+def _bf16_bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().astype(np.int32) & 0xFFFF
+
+
+def _check_block(name, N, rows=None, score="sigmoid"):
+    dev, host = layer_inputs(name, N)
+    cfg = host["cfg"]
+    blk = make_block_inputs(cfg, seed=11, device="cuda")
+    hb = {k: v.cpu() for k, v in blk.items()}
+    out, x, idx, w, counts = kmoe.moe_block_forward(blk["h"], dev, blk["gamma_pre"], blk["gamma_post"], BLOCK_EPS,
+                                                    with_outputs=True, score=score)
+    torch.cuda.synchronize()
+    ora = oracle.block(host, hb["h"], hb["gamma_pre"], hb["gamma_post"], BLOCK_EPS, rows=rows, nthreads=threads(),
+                       score=score)
+    # pre-norm: BF16 bits equal except rare one-ulp flips of values on a rounding boundary
+    xg, xo = _bf16_bits(x), ora["x"].astype(np.int32)
+    diff = xg != xo
+    assert diff.mean() <= 1e-3
+    assert np.all(np.abs(xg[diff] - xo[diff]) == 1)
+    rws = ora["rows"]
+    l_all = oracle.router_logits(ora["x"][rws], "bf16", host["w_router"], nthreads=threads())
+    _, differ = check_routing(idx.cpu().numpy()[rws], ora["idx"], biased_scores(l_all, host["bias"]), cfg.K,
+                              margin=BLOCK_TIE)
+    assert counts.sum().item() == cfg.N * cfg.K
+    keep = np.array([t not in differ for t in range(len(rws))])
+    got = out.float().cpu().numpy()[rws][keep]
+    ref = ora["h_out"][keep]
+    h = hb["h"].float().numpy()[rws][keep]
+    # error against the size of the normalised MoE term, plus BF16 rounding of h_out
+    n_max = np.abs(ref - h).max(axis=1)
+    allow = TOL[cfg.w_dtype] * n_max + 2.0 ** -8 * np.abs(ref).max(axis=1)
+    assert np.all(np.abs(got - ref).max(axis=1) <= allow)
+    return out
+
+
+@pytest.mark.parametrize("name,N", [("decode", None), ("decode", 1), ("decode", 300), ("fp8_decode", None),
+                                    ("fp8_decode", 200), ("prefill", 1024)])
+def test_block_forward_matches_oracle(name, N):
+    _check_block(name, N)
+
+
+def test_block_forward_full_prefill_sampled_rows():
+    rows = np.random.default_rng(5).choice(8192, 192, replace=False).astype(np.int32)
+    rows[:2] = [0, 8191]
+    _check_block("prefill", None, rows=np.sort(rows))
+
+
+def test_block_forward_softmax_score():
+    _check_block("decode", 300, score="softmax")
+
+
+def test_block_forward_in_place_equals_out_of_place():
+    dev, _ = layer_inputs("decode", 300)
+    cfg = dev["cfg"]
+    blk = make_block_inputs(cfg, seed=3, device="cuda")
+    lay = kmoe.Layer(dev, cfg.N, block=True)
+    ref = lay.block_forward(blk["h"], blk["gamma_pre"], blk["gamma_post"], BLOCK_EPS)
+    again = lay.block_forward(blk["h"], blk["gamma_pre"], blk["gamma_post"], BLOCK_EPS)
+    h = blk["h"].clone()
+    lay.block_forward(h, blk["gamma_pre"], blk["gamma_post"], BLOCK_EPS, h_out=h)
+    torch.cuda.synchronize()
+    assert torch.equal(ref, again)
+    assert torch.equal(h, ref)
+    assert kmoe.moe_device_status(lay.ws) == 0
+
+
+def test_block_forward_zero_tokens():
+    dev, _ = layer_inputs("decode")
+    blk = make_block_inputs(dev["cfg"], seed=3, device="cuda")
+    out = kmoe.moe_block_forward(blk["h"][:0], dev, blk["gamma_pre"], blk["gamma_post"], BLOCK_EPS)
+    assert out.shape == (0, 2560)
