@@ -19,23 +19,28 @@
 //              to the MMA as soon as it is drained, so the next tile's first
 //              MMAs overlap the epilogue of the second half;
 //   warp  4    one thread issues tcgen05.mma and tcgen05.commit;
-//   warps 5-8  producers: weight tiles by TMA (128-byte swizzle); the
-//              activation rows of the up kernel are gathered with cp.async
-//              straight into the swizzled layout (no permuted copy of x is
-//              ever written) and complete on the stage barrier without the
-//              producer waiting; the down kernel loads H tiles by TMA.
+//   warps 5-8  token producers: the activation rows of the up kernel are
+//              gathered with cp.async straight into the swizzled layout (no
+//              permuted copy of x is ever written) and complete on the slot
+//              barrier without the producer waiting; the down kernel loads H
+//              tiles by TMA;
+//   warp  9    weight producer: weight tiles by TMA (128-byte swizzle).
+// Token tiles (16 KB per m-tile and k-block) and weight tiles (32 KB per
+// k-block) sit in two separate rings, so the weight stream from HBM runs up
+// to four k-blocks ahead of the MMA (128 KB in flight per SM) whatever the
+// token gather is doing.
 // The up tile pairs 128 gate features with the same 128 up features (one
 // N = 256 MMA), so SiLU(g) * u is computed in registers. Tiles are
 // enumerated per expert as (n-tile, row pair), so CTAs running at the same
 // time share the expert's token rows in L2.
 //
 // E4M3 weights ("Inside Kolibri 1", FP8 section: 128 x 128 blocks, one FP32
-// scale per block) take the same kernels with four more warps: the weight
-// tile arrives by TMA as E4M3 bytes in a staging buffer, and converter warps
-// 9-12 decode it (hardware e4m3x2 -> f16x2), multiply by the FP32 scale of
-// its block, round to BF16 and write it in the swizzled layout the MMA reads.
-// Activations stay BF16, so the tensor cores see BF16 x BF16 with FP32
-// accumulation, and the weights cross HBM at one byte each.
+// scale per block) take the same kernels with four more warps: warp 9 brings
+// the E4M3 bytes by TMA into a five-deep staging ring (16 KB per k-block),
+// and converter warps 10-13 decode them (hardware e4m3x2 -> f16x2), multiply
+// by the FP32 scale of the block, round to BF16 and write the swizzled tile
+// the MMA reads. Activations stay BF16, so the tensor cores see BF16 x BF16
+// with FP32 accumulation, and the weights cross HBM at one byte each.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -46,18 +51,37 @@ using namespace sm100;
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kPairRows = 2 * kBM;           // rows of one CTA tile
-constexpr int kATile = kBM * kBK * 2;        // 16 KB per m-tile
+constexpr int kATile = kBM * kBK * 2;        // 16 KB: one m-tile of one k-block
 constexpr int kBTile = kBN * kBK * 2;        // 32 KB
 constexpr int kB8Tile = kBN * kBK;           // 16 KB of E4M3 staging
-constexpr int kMaxStages = 3;
-__host__ __device__ constexpr int stages_of(bool fp8) { return fp8 ? 2 : 3; }
-__host__ __device__ constexpr int stage_bytes(bool fp8) { return 2 * kATile + kBTile + (fp8 ? kB8Tile : 0); }
+constexpr int kMaxRing = 6;
+constexpr int kSStages = 4;                  // E4M3 staging ring
+constexpr int kEpiStage = 4 * 32 * 128;      // epilogue: 32 rows x 128 bytes per warp
+__host__ __device__ constexpr int a_stages(bool fp8) { return fp8 ? 4 : 6; }
+__host__ __device__ constexpr int b_stages(bool fp8) { return fp8 ? 2 : 3; }
+__host__ __device__ constexpr int ring_bytes(bool fp8)
+{
+    return a_stages(fp8) * kATile + b_stages(fp8) * kBTile + (fp8 ? kSStages * kB8Tile : 0);
+}
 constexpr int kMmaWarp = 4;
-constexpr int kProdWarp = 5;
-constexpr int kConvWarp = 9;                 // E4M3 only: warps 9-12
-__host__ __device__ constexpr int threads_of(bool fp8) { return (fp8 ? 13 : 9) * 32; }
+constexpr int kProdWarp = 5;                 // token producers: warps 5-8
+constexpr int kWProdWarp = 9;                // weight producer
+constexpr int kConvWarp = 10;                // E4M3 only: warps 10-13
+__host__ __device__ constexpr int threads_of(bool fp8) { return (fp8 ? 14 : 10) * 32; }
 constexpr int kMaxGroups = 1025;
 constexpr long long kWaitLimit = 1LL << 32;  // SM cycles (about 2 s)
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
 
 struct TcMaps {
     CUtensorMap b0_routed, b1_routed, b0_shared, b1_shared;   // up: gate, up; down: W_d (b0 only)
@@ -78,7 +102,8 @@ struct TcArgs {
 };
 
 struct SmemTail {
-    uint64_t full[kMaxStages], empty[kMaxStages], b8full[kMaxStages], tfull, tempty[2], drain;
+    uint64_t afull[kMaxRing], aempty[kMaxRing], bfull[kMaxRing], bempty[kMaxRing];
+    uint64_t sfull[kSStages], sempty[kSStages], tfull, tempty[2], drain;
     uint32_t tmem_base;
     int abort;
     int pre[kMaxGroups + 1];
@@ -86,8 +111,9 @@ struct SmemTail {
 
 __host__ __device__ constexpr size_t tc_smem(bool fp8)
 {
-    return 1024 /*align slack*/ + (size_t)stages_of(fp8) * stage_bytes(fp8) + sizeof(SmemTail);
+    return 1024 /*align slack*/ + (size_t)ring_bytes(fp8) + kEpiStage + sizeof(SmemTail);
 }
+static_assert(tc_smem(false) <= 227 * 1024 && tc_smem(true) <= 227 * 1024, "shared memory budget");
 
 struct Tile {
     int g, row0, rows, n0;
@@ -176,52 +202,60 @@ __device__ __forceinline__ void convert_row(const uint8_t *src, uint8_t *dst, in
     }
 }
 
-// Epilogue of one 128-row half of the accumulator (rows r_base .. r_base+127
-// of the tile). tbase addresses this warp's 32 lanes in that half.
+// Epilogue of one 128-row half of the accumulator (tile rows rbase ..
+// rbase + 127); warp w owns rows rbase + 32w .. + 31, its lane quarter of
+// tensor memory, and tbase addresses that quarter in the half. Every 64
+// output columns are first written row by row into the warp's 4 KB staging
+// area (16-byte pieces XOR-swizzled by row, so neither side has bank
+// conflicts) and then stored with 8 lanes per row: each store instruction
+// writes four whole 128-byte row segments.
 template <bool kUp>
-__device__ __forceinline__ void epilogue_half(uint32_t tbase, const Tile &T, const TcArgs &a, int row)
+__device__ __forceinline__ void epilogue_half(uint32_t tbase, const Tile &T, const TcArgs &a, int rbase,
+                                              uint32_t stage)
 {
-    const bool valid = row < T.rows;
-    const int grow = T.row0 + row;
-    if (kUp) {
-        __nv_bfloat16 *dst = a.out0 + (size_t)grow * a.I + T.n0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wrow0 = rbase + warp * 32;
+    constexpr int kCols = kUp ? kBN / 2 : kBN;       // output columns of the tile
+    const uint32_t mine = stage + lane * 128;        // this thread's staging row
+    for (int c0 = 0; c0 < kCols; c0 += 64) {
 #pragma unroll 1
-        for (int c = 0; c < kBN / 2; c += 16) {
-            uint32_t g[16], u[16];
-            tmem_ld16(tbase + c, g);
-            tmem_ld16(tbase + kBN / 2 + c, u);
-            tmem_ld_wait();
+        for (int q = 0; q < 4; ++q) {                // columns c0 + 16q .. + 15: pieces 2q, 2q + 1
             uint32_t packed[8];
+            if (kUp) {
+                uint32_t g[16], u[16];
+                tmem_ld16(tbase + c0 + 16 * q, g);
+                tmem_ld16(tbase + kBN / 2 + c0 + 16 * q, u);
+                tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float g0 = __uint_as_float(g[2 * q]), g1 = __uint_as_float(g[2 * q + 1]);
-                const float u0 = __uint_as_float(u[2 * q]), u1 = __uint_as_float(u[2 * q + 1]);
-                packed[q] = pack_bf16x2(silu_mul(g0, u0), silu_mul(g1, u1));
+                for (int e = 0; e < 8; ++e)
+                    packed[e] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * e]), __uint_as_float(u[2 * e])),
+                                            silu_mul(__uint_as_float(g[2 * e + 1]), __uint_as_float(u[2 * e + 1])));
+            } else {
+                uint32_t v[16];
+                tmem_ld16(tbase + c0 + 16 * q, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    packed[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
             }
-            if (valid) {
-                uint4 *o = reinterpret_cast<uint4 *>(dst + c);
-                o[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                o[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            st_shared_v4(mine + (((2 * q) ^ (lane & 7)) << 4), packed[0], packed[1], packed[2], packed[3]);
+            st_shared_v4(mine + (((2 * q + 1) ^ (lane & 7)) << 4), packed[4], packed[5], packed[6], packed[7]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {                // rows 4j .. 4j + 3 of the warp, 8 lanes each
+            const int r = 4 * j + (lane >> 3), pc = lane & 7;
+            const uint4 v = ld_shared_v4(stage + r * 128 + ((pc ^ (r & 7)) << 4));
+            const int trow = wrow0 + r;
+            if (trow < T.rows) {
+                const size_t grow = (size_t)T.row0 + trow;
+                __nv_bfloat16 *dst = kUp      ? a.out0 + grow * a.I
+                                     : T.shared ? a.out1 + (grow - (size_t)a.N * a.K) * a.d
+                                                : a.out0 + grow * a.d;
+                *reinterpret_cast<uint4 *>(dst + T.n0 + c0 + pc * 8) = v;
             }
         }
-    } else {
-        __nv_bfloat16 *dst = T.shared ? a.out1 + (size_t)(grow - a.N * a.K) * a.d + T.n0
-                                      : a.out0 + (size_t)grow * a.d + T.n0;
-#pragma unroll 1
-        for (int c = 0; c < kBN; c += 16) {
-            uint32_t v[16];
-            tmem_ld16(tbase + c, v);
-            tmem_ld_wait();
-            uint32_t packed[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                packed[q] = pack_bf16x2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
-            if (valid) {
-                uint4 *o = reinterpret_cast<uint4 *>(dst + c);
-                o[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                o[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-            }
-        }
+        __syncwarp();                                // staging free for the next 64 columns
     }
 }
 
@@ -229,21 +263,29 @@ template <bool kUp, bool kFp8>
 __global__ void __launch_bounds__(threads_of(kFp8), 1)
 ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
 {
-    constexpr int kStages = stages_of(kFp8);
-    constexpr int kStage = stage_bytes(kFp8);
+    constexpr int kAS = a_stages(kFp8), kBS = b_stages(kFp8);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    SmemTail *tail = reinterpret_cast<SmemTail *>(smem + (size_t)kStages * kStage);
+    uint8_t *ring_a = smem;                                   // kAS x 16 KB token tiles
+    uint8_t *ring_b = ring_a + (size_t)kAS * kATile;          // kBS x 32 KB BF16 weight tiles
+    uint8_t *ring_s = ring_b + (size_t)kBS * kBTile;          // E4M3: kSStages x 16 KB staging
+    uint8_t *epi = smem + ring_bytes(kFp8);                   // epilogue staging, 4 KB per warp
+    SmemTail *tail = reinterpret_cast<SmemTail *>(epi + kEpiStage);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort = &tail->abort;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            // arrivals: up = 128 cp.async producers + (TMA expect_tx | 128 converters);
-            //           down = TMA expect_tx (+ 128 converters)
-            mbar_init(&tail->full[s], (kUp ? 128 : 1) + (kFp8 ? 128 : (kUp ? 1 : 0)));
-            mbar_init(&tail->empty[s], 1);
-            mbar_init(&tail->b8full[s], 1);
+        for (int s = 0; s < kAS; ++s) {
+            mbar_init(&tail->afull[s], kUp ? 128 : 1);    // up: 128 cp.async arrivals; down: TMA expect_tx
+            mbar_init(&tail->aempty[s], 1);
+        }
+        for (int s = 0; s < kBS; ++s) {
+            mbar_init(&tail->bfull[s], kFp8 ? 128 : 1);   // E4M3: the 128 converter threads
+            mbar_init(&tail->bempty[s], 1);
+        }
+        for (int s = 0; s < kSStages; ++s) {
+            mbar_init(&tail->sfull[s], 1);
+            mbar_init(&tail->sempty[s], 128);
         }
         mbar_init(&tail->tfull, 1);
         mbar_init(&tail->tempty[0], 128);
@@ -257,7 +299,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         tmem_alloc(&tail->tmem_base, 512);
         tmem_relinquish();
     }
-    if (warp == kProdWarp && lane == 0) {
+    if (warp == kWProdWarp && lane == 0) {
         prefetch_map(&maps.b0_routed);
         prefetch_map(&maps.b0_shared);
         if (kUp) { prefetch_map(&maps.b1_routed); prefetch_map(&maps.b1_shared); }
@@ -282,10 +324,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             const float *s0 = T.shared ? a.s0_shared : a.s0_routed;
             const float *s1 = T.shared ? a.s1_shared : a.s1_routed;
             for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
-                const int s = it % kStages;
-                if (!mbar_wait(&tail->b8full[s], (it / kStages) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-                uint8_t *Bs = smem + (size_t)s * kStage + 2 * kATile;
-                const uint8_t *B8 = Bs + kBTile;
+                const int ss = it % kSStages, sb = it % kBS;
                 float sc0, sc1;
                 if (kUp) {     // gate rows n0.., up rows n0..; blocks [G, I/128, d/128]
                     const size_t si = (ge * (a.I / 128) + T.n0 / 128) * (a.d / 128) + (kb * kBK) / 128;
@@ -296,83 +335,115 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                     sc0 = s0[si];
                     sc1 = s0[si + a.I / 128];
                 }
+                if (!mbar_wait(&tail->sfull[ss], (it / kSStages) & 1, abort, a.err, kWaitLimit) ||
+                    !mbar_wait(&tail->bempty[sb], ((it / kBS) & 1) ^ 1, abort, a.err, kWaitLimit)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *B8 = ring_s + (size_t)ss * kB8Tile;
+                uint8_t *Bs = ring_b + (size_t)sb * kBTile;
                 convert_row(B8 + q * kBK, Bs, q, sc0);
                 convert_row(B8 + (q + 128) * kBK, Bs, q + 128, sc1);
-                fence_proxy_async();
-                mbar_arrive(&tail->full[s]);
+                mbar_arrive(&tail->sempty[ss]);      // staging slot read
+                fence_proxy_async();                 // converted rows visible to the tensor cores
+                mbar_arrive(&tail->bfull[sb]);
             }
+        }
+    } else if (warp == kWProdWarp) {
+        // ------------------------------------------------- weight producer
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();   // weight tiles: streamed once
+            constexpr int S = kFp8 ? kSStages : kBS;
+            uint64_t *full = kFp8 ? tail->sfull : tail->bfull;
+            uint64_t *empty = kFp8 ? tail->sempty : tail->bempty;
+            uint8_t *ring = kFp8 ? ring_s : ring_b;
+            constexpr uint32_t bytes = kFp8 ? kB8Tile : kBTile;
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const Tile T = decode_tile(t, tail->pre, a, bn);
+                const CUtensorMap *m0 = T.shared ? &maps.b0_shared : &maps.b0_routed;
+                const CUtensorMap *m1 = T.shared ? &maps.b1_shared : &maps.b1_routed;
+                const int gi = T.shared ? 0 : T.g;
+                const int r0 = kUp ? gi * a.I + T.n0 : gi * a.d + T.n0;
+                for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                    const int s = it % S;
+                    if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                    uint8_t *dst = ring + (size_t)s * bytes;
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    // rows 0-127: gate (up) or W_d rows n0..; rows 128-255: up rows n0.. or W_d rows n0+128..
+                    tma_load_2d_hint(dst, m0, &full[s], kb * kBK, r0, pol_w);
+                    tma_load_2d_hint(dst + bytes / 2, kUp ? m1 : m0, &full[s], kb * kBK, kUp ? r0 : r0 + kBN / 2,
+                                     pol_w);
+                }
+            }
+            if (!ok)   // let in-flight loads land before the CTA exits
+                for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
+                    mbar_wait_drain(&full[j % S], (j / S) & 1, kWaitLimit);
         }
     } else if (warp >= kProdWarp) {
-        // ------------------------------------------------------- producers
+        // -------------------------------------------------- token producers
         const int p = threadIdx.x - kProdWarp * 32;
-        const bool leader = p == 0;
-        const uint64_t pol_w = policy_evict_first();   // weight tiles: streamed
         const uint64_t pol_a = policy_evict_last();    // token rows / H rows: reused across n-tiles
-        uint32_t it = 0;
+        uint32_t ia = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Tile T = decode_tile(t, tail->pre, a, bn);
-            const CUtensorMap *m0 = T.shared ? &maps.b0_shared : &maps.b0_routed;
-            const CUtensorMap *m1 = T.shared ? &maps.b1_shared : &maps.b1_routed;
-            const int gi = T.shared ? 0 : T.g;
-            int tok0 = -1, tok1 = -1;
-            if (kUp) {
-                if (p < T.rows) tok0 = T.shared ? T.row0 + p - a.N * a.K : a.perm[T.row0 + p];
-                if (p + kBM < T.rows) tok1 = T.shared ? T.row0 + kBM + p - a.N * a.K : a.perm[T.row0 + kBM + p];
-            }
-            const __nv_bfloat16 *src0 = a.x + (size_t)(tok0 < 0 ? 0 : tok0) * a.d;
-            const __nv_bfloat16 *src1 = a.x + (size_t)(tok1 < 0 ? 0 : tok1) * a.d;
-            for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
-                if (!mbar_wait(&tail->empty[s], ph ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-                uint8_t *As = smem + (size_t)s * kStage;           // A0 | A1 | B | (B8)
-                uint8_t *Bs = As + 2 * kATile;
-                if (kFp8 && leader) {       // E4M3 weight rows into the staging buffer
-                    uint8_t *B8 = Bs + kBTile;
-                    const int r0 = kUp ? gi * a.I + T.n0 : gi * a.d + T.n0;
-                    mbar_arrive_expect_tx(&tail->b8full[s], kB8Tile);
-                    tma_load_2d_hint(B8, m0, &tail->b8full[s], kb * kBK, r0, pol_w);
-                    tma_load_2d_hint(B8 + kB8Tile / 2, kUp ? m1 : m0, &tail->b8full[s], kb * kBK,
-                                     kUp ? r0 : r0 + kBN / 2, pol_w);
+        if (kUp) {
+            // 8 lanes per row: thread p copies 16-byte piece pc of rows
+            // 32 * (p / 32) + 4j + (p % 32) / 8, j = 0..7, so every cp.async
+            // instruction of a warp reads four whole 128-byte row segments.
+            const int pw = p >> 5, pl = p & 31, pc = pl & 7;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const Tile T = decode_tile(t, tail->pre, a, bn);
+                int tok0[8], tok1[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int r = pw * 32 + 4 * j + (pl >> 3);
+                    tok0[j] = r >= T.rows ? -1 : T.shared ? T.row0 + r - a.N * a.K : a.perm[T.row0 + r];
+                    tok1[j] = r + kBM >= T.rows ? -1
+                              : T.shared        ? T.row0 + kBM + r - a.N * a.K
+                                                : a.perm[T.row0 + kBM + r];
                 }
-                if (kUp) {
-                    if (leader && !kFp8) {
-                        mbar_arrive_expect_tx(&tail->full[s], kBTile);
-                        tma_load_2d_hint(Bs, m0, &tail->full[s], kb * kBK, gi * a.I + T.n0, pol_w);
-                        tma_load_2d_hint(Bs + kBTile / 2, m1, &tail->full[s], kb * kBK, gi * a.I + T.n0, pol_w);
-                    }
-                    const uint32_t dst0 = smem_u32(As) + p * 128;
+                const int mt = T.two ? 2 : 1;
+                for (int kb = 0; kb < a.kblocks && ok; ++kb) {
+                    for (int m = 0; m < mt; ++m, ++ia) {
+                        const int sa = ia % kAS;
+                        if (!mbar_wait(&tail->aempty[sa], ((ia / kAS) & 1) ^ 1, abort, a.err, kWaitLimit)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t dst = smem_u32(ring_a + (size_t)sa * kATile);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        cp_async16_hint(dst0 + ((c ^ (p & 7)) << 4), src0 + kb * kBK + c * 8, tok0 >= 0 ? 16u : 0u,
-                                        pol_a);
-                    if (T.two) {
-                        const uint32_t dst1 = smem_u32(As + kATile) + p * 128;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            cp_async16_hint(dst1 + ((c ^ (p & 7)) << 4), src1 + kb * kBK + c * 8,
-                                            tok1 >= 0 ? 16u : 0u, pol_a);
-                    }
-                    cp_async_arrive_noinc(&tail->full[s]);   // the stage completes when these rows land
-                } else if (leader) {
-                    mbar_arrive_expect_tx(&tail->full[s], kATile * (T.two ? 2 : 1) + (kFp8 ? 0 : kBTile));
-                    tma_load_2d_hint(As, &maps.a, &tail->full[s], kb * kBK, T.row0, pol_a);
-                    if (T.two) tma_load_2d_hint(As + kATile, &maps.a, &tail->full[s], kb * kBK, T.row0 + kBM, pol_a);
-                    if (!kFp8) {
-                        tma_load_2d_hint(Bs, m0, &tail->full[s], kb * kBK, gi * a.d + T.n0, pol_w);
-                        tma_load_2d_hint(Bs + kBTile / 2, m0, &tail->full[s], kb * kBK, gi * a.d + T.n0 + kBN / 2,
-                                         pol_w);
+                        for (int j = 0; j < 8; ++j) {
+                            const int r = pw * 32 + 4 * j + (pl >> 3);
+                            const int tk = m ? tok1[j] : tok0[j];
+                            const __nv_bfloat16 *src = a.x + (size_t)(tk < 0 ? 0 : tk) * a.d + kb * kBK + pc * 8;
+                            cp_async16_hint(dst + r * 128 + ((pc ^ (r & 7)) << 4), src, tk >= 0 ? 16u : 0u, pol_a);
+                        }
+                        cp_async_arrive_noinc(&tail->afull[sa]);   // the slot completes when these rows land
                     }
                 }
             }
-        }
-        if (kUp) cp_async_wait_all();   // this thread's row copies have landed before it leaves
-        if (!ok && leader) {   // let in-flight TMA loads land before the CTA exits
-            for (uint32_t j = it > (uint32_t)kStages ? it - kStages : 0; j < it; ++j) {
-                if (kFp8) mbar_wait_drain(&tail->b8full[j % kStages], (j / kStages) & 1, kWaitLimit);
-                if (!kFp8 || !kUp) mbar_wait_drain(&tail->full[j % kStages], (j / kStages) & 1, kWaitLimit);
+            cp_async_wait_all();   // this thread's row copies have landed before it leaves
+        } else if (p == 0) {
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const Tile T = decode_tile(t, tail->pre, a, bn);
+                const int mt = T.two ? 2 : 1;
+                for (int kb = 0; kb < a.kblocks && ok; ++kb) {
+                    for (int m = 0; m < mt; ++m, ++ia) {
+                        const int sa = ia % kAS;
+                        if (!mbar_wait(&tail->aempty[sa], ((ia / kAS) & 1) ^ 1, abort, a.err, kWaitLimit)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&tail->afull[sa], kATile);
+                        tma_load_2d_hint(ring_a + (size_t)sa * kATile, &maps.a, &tail->afull[sa], kb * kBK,
+                                         T.row0 + m * kBM, pol_a);
+                    }
+                }
             }
+            if (!ok)
+                for (uint32_t j = ia > (uint32_t)kAS ? ia - kAS : 0; j < ia; ++j)
+                    mbar_wait_drain(&tail->afull[j % kAS], (j / kAS) & 1, kWaitLimit);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA
@@ -382,36 +453,35 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             // m-tile takes the half that the previous single tile did not,
             // so its MMAs overlap that tile's epilogue; a tile with two
             // m-tiles takes both (starting with the half drained first).
-            uint32_t it = 0, use0 = 0, use1 = 0;     // uses of half 0 / half 1 so far
+            uint32_t ia = 0, ib = 0, use0 = 0, use1 = 0;     // uses of half 0 / half 1 so far
             int hn = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 const Tile T = decode_tile(t, tail->pre, a, bn);
                 const int h0 = hn, h1 = hn ^ 1;
                 const uint32_t c0 = h0 ? use1 : use0, c1 = h0 ? use0 : use1;
-                for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
-                    const int s = it % kStages;
-                    if (!mbar_wait(&tail->full[s], (it / kStages) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-                    if (kb == 0 &&   // half h0 drained by the epilogue of its last use
-                        !mbar_wait(&tail->tempty[h0], (c0 & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t sa = smem_u32(smem + (size_t)s * kStage);
-                    const uint64_t a0 = sw128_kmajor_desc(sa);
-                    const uint64_t bd = sw128_kmajor_desc(sa + 2 * kATile);
-#pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16(tmem + h0 * kBN, a0 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
-                    if (T.two) {
-                        if (kb == 0 &&
-                            !mbar_wait(&tail->tempty[h1], (c1 & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                const int mt = T.two ? 2 : 1;
+                for (int kb = 0; kb < a.kblocks && ok; ++kb, ++ib) {
+                    const int sb = ib % kBS;
+                    if (!mbar_wait(&tail->bfull[sb], (ib / kBS) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                    const uint64_t bd = sw128_kmajor_desc(smem_u32(ring_b + (size_t)sb * kBTile));
+                    for (int m = 0; m < mt; ++m, ++ia) {
+                        const int sa = ia % kAS, h = m ? h1 : h0;
+                        if (!mbar_wait(&tail->afull[sa], (ia / kAS) & 1, abort, a.err, kWaitLimit) ||
+                            (kb == 0 &&   // half h drained by the epilogue of its last use
+                             !mbar_wait(&tail->tempty[h], ((m ? c1 : c0) & 1) ^ 1, abort, a.err, kWaitLimit))) {
+                            ok = false;
+                            break;
+                        }
                         tc_fence_after();
-                        const uint64_t a1 = sw128_kmajor_desc(sa + kATile);
+                        const uint64_t ad = sw128_kmajor_desc(smem_u32(ring_a + (size_t)sa * kATile));
 #pragma unroll
                         for (int k = 0; k < kBK / 16; ++k)
-                            umma_bf16(tmem + h1 * kBN, a1 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc,
+                            umma_bf16(tmem + h * kBN, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc,
                                       (kb | k) != 0);
+                        umma_commit(&tail->aempty[sa]);
                     }
-                    umma_commit(&tail->empty[s]);
+                    if (ok) umma_commit(&tail->bempty[sb]);
                 }
                 if (!ok) break;
                 umma_commit(&tail->tfull);
@@ -427,18 +497,18 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         // ------------------------------------------------------- epilogue
         uint32_t at = 0;
         int hn = 0;                       // the half rotation of the MMA thread, replayed
-        const int row = warp * 32 + lane;
+        const uint32_t stage = smem_u32(epi) + warp * 4096;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++at) {
             const Tile T = decode_tile(t, tail->pre, a, bn);
             const int h0 = hn, h1 = hn ^ 1;
             if (!mbar_wait(&tail->tfull, at & 1, abort, a.err, kWaitLimit)) break;
             tc_fence_after();
             const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
-            epilogue_half<kUp>(tlane + h0 * kBN, T, a, row);
+            epilogue_half<kUp>(tlane + h0 * kBN, T, a, 0, stage);
             tc_fence_before();
             mbar_arrive(&tail->tempty[h0]);
             if (T.two) {
-                epilogue_half<kUp>(tlane + h1 * kBN, T, a, row + kBM);
+                epilogue_half<kUp>(tlane + h1 * kBN, T, a, kBM, stage);
                 tc_fence_before();
                 mbar_arrive(&tail->tempty[h1]);
             }
