@@ -164,7 +164,7 @@ static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int 
     if (path == kPathTc)
         return launch_ffn_tc(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, w_dtype, r, s,
                              static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
-                             static_cast<__nv_bfloat16 *>(y_shared), status, st);
+                             static_cast<__nv_bfloat16 *>(y_shared), status, status + kSyncOffset, st);
     return launch_ffn_stream(x, x_dtype, N, d, I, E, K, perm, offsets, w_dtype, r, s, h, y_perm, y_shared, st);
 }
 

@@ -157,10 +157,10 @@ kmoe_status launch_ffn_stream(const void *x, int x_dtype, int N, int d, int I, i
                               void *h, void *y_perm, void *y_shared, cudaStream_t st);
 
 // Tensor-core grouped FFN (BF16 activations; BF16 or E4M3 + FP32 block-scale
-// weights; d % 256 == 0).
+// weights; d % 256 == 0). `sync` holds two tile counters, zero at launch.
 kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
                           const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
-                          __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err,
+                          __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err, int *sync,
                           cudaStream_t st);
 
 // Batches of at least this many tokens take the tensor-core FFN.

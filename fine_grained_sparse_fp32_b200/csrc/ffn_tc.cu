@@ -24,11 +24,16 @@
 //              permuted copy of x is ever written) and complete on the slot
 //              barrier without the producer waiting; the down kernel loads H
 //              tiles by TMA;
-//   warp  9    weight producer: weight tiles by TMA (128-byte swizzle).
+//   warp  9    weight producer: claims the CTA's next tile from a global
+//              counter, publishes it to the other roles through a small
+//              shared-memory queue, and streams its weight tiles by TMA
+//              (128-byte swizzle).
 // Token tiles (16 KB per m-tile and k-block) and weight tiles (32 KB per
-// k-block) sit in two separate rings, so the weight stream from HBM runs up
-// to four k-blocks ahead of the MMA (128 KB in flight per SM) whatever the
-// token gather is doing.
+// k-block) sit in two separate rings (six and three deep), so the weight
+// stream runs ahead of the MMA whatever the token gather is doing. Token rows
+// are gathered with 8 lanes per 128-byte row segment, and the epilogue goes
+// through a per-warp staging area so that its stores also cover whole
+// 128-byte segments.
 // The up tile pairs 128 gate features with the same 128 up features (one
 // N = 256 MMA), so SiLU(g) * u is computed in registers. Tiles are
 // enumerated per expert as (n-tile, row pair), so CTAs running at the same
@@ -36,7 +41,7 @@
 //
 // E4M3 weights ("Inside Kolibri 1", FP8 section: 128 x 128 blocks, one FP32
 // scale per block) take the same kernels with four more warps: warp 9 brings
-// the E4M3 bytes by TMA into a five-deep staging ring (16 KB per k-block),
+// the E4M3 bytes by TMA into a four-deep staging ring (16 KB per k-block),
 // and converter warps 10-13 decode them (hardware e4m3x2 -> f16x2), multiply
 // by the FP32 scale of the block, round to BF16 and write the swizzled tile
 // the MMA reads. Activations stay BF16, so the tensor cores see BF16 x BF16
@@ -69,6 +74,7 @@ constexpr int kWProdWarp = 9;                // weight producer
 constexpr int kConvWarp = 10;                // E4M3 only: warps 10-13
 __host__ __device__ constexpr int threads_of(bool fp8) { return (fp8 ? 14 : 10) * 32; }
 constexpr int kMaxGroups = 1025;
+constexpr int kTQ = 4;                       // tile queue depth
 constexpr long long kWaitLimit = 1LL << 32;  // SM cycles (about 2 s)
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w)
@@ -99,11 +105,14 @@ struct TcArgs {
     // E4M3 block scales (up: s0 = gate, s1 = up; down: s0 = W_d), routed and shared
     const float *s0_routed, *s1_routed, *s0_shared, *s1_shared;
     int *err;
+    int *tile_ctr;            // tiles claimed so far by all CTAs (zero at launch)
 };
 
 struct SmemTail {
     uint64_t afull[kMaxRing], aempty[kMaxRing], bfull[kMaxRing], bempty[kMaxRing];
     uint64_t sfull[kSStages], sempty[kSStages], tfull, tempty[2], drain;
+    uint64_t tqfull[kTQ], tqempty[kTQ];
+    int tq[kTQ];
     uint32_t tmem_base;
     int abort;
     int pre[kMaxGroups + 1];
@@ -142,6 +151,29 @@ __device__ __forceinline__ Tile decode_tile(int t, const int *pre, const TcArgs 
     T.two = T.rows > kBM;
     T.n0 = nt * bn;
     return T;
+}
+
+// Claim order -> tile index. Tiles are claimed dynamically from a global
+// counter; the shared expert's tiles (indices routed .. total - 1) are spread
+// evenly among the routed ones, so the CTAs running at any time mix
+// weight-streaming routed tiles with the shared expert's compute-heavy ones.
+__device__ __forceinline__ int claim_to_tile(int c, int routed, int total)
+{
+    const int S = total - routed;
+    const int before = (int)((long long)c * S / total);       // shared tiles among claims 0 .. c-1
+    const int upto = (int)((long long)(c + 1) * S / total);
+    return upto > before ? routed + before : c - before;
+}
+
+// The next tile of this CTA (or -1: no more, -2: a wait gave up), published
+// by the weight producer in the tile queue.
+__device__ __forceinline__ int tq_take(SmemTail *tail, uint32_t q, volatile int *abort, int *err)
+{
+    const int s = q % kTQ;
+    if (!mbar_wait(&tail->tqfull[s], (q / kTQ) & 1, abort, err, kWaitLimit)) return -2;
+    const int t = reinterpret_cast<volatile int *>(tail->tq)[s];
+    mbar_arrive(&tail->tqempty[s]);
+    return t;
 }
 
 // row-pair prefix over groups, computed by one warp.
@@ -291,6 +323,11 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         mbar_init(&tail->tempty[0], 128);
         mbar_init(&tail->tempty[1], 128);
         mbar_init(&tail->drain, 1);
+        for (int s = 0; s < kTQ; ++s) {
+            mbar_init(&tail->tqfull[s], 1);
+            // readers: token producers (up: 128, down: 1), the MMA thread, 128 epilogue threads, converters
+            mbar_init(&tail->tqempty[s], (kUp ? 128 : 1) + 1 + 128 + (kFp8 ? 128 : 0));
+        }
         tail->abort = 0;
         fence_mbar_init();
     }
@@ -318,7 +355,9 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         const int q = threadIdx.x - kConvWarp * 32;          // rows q and q + 128 of the B tile
         uint32_t it = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (uint32_t tq = 0; ok; ++tq) {
+            const int t = tq_take(tail, tq, abort, a.err);
+            if (t < 0) break;
             const Tile T = decode_tile(t, tail->pre, a, bn);
             const size_t ge = T.shared ? 0 : (size_t)T.g;
             const float *s0 = T.shared ? a.s0_shared : a.s0_routed;
@@ -352,7 +391,9 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
     } else if (warp == kWProdWarp) {
         // ------------------------------------------------- weight producer
         if (lane == 0) {
-            const uint64_t pol_w = policy_evict_first();   // weight tiles: streamed once
+            const uint64_t pol_w = policy_evict_first();   // routed weight tiles: streamed once
+            const uint64_t pol_s = policy_evict_last();    // shared expert: reused by every row pair
+            const int routed_tiles = tail->pre[a.E] * a.n_tiles;
             constexpr int S = kFp8 ? kSStages : kBS;
             uint64_t *full = kFp8 ? tail->sfull : tail->bfull;
             uint64_t *empty = kFp8 ? tail->sempty : tail->bempty;
@@ -360,8 +401,19 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             constexpr uint32_t bytes = kFp8 ? kB8Tile : kBTile;
             uint32_t it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (uint32_t tq = 0; ok; ++tq) {
+                const int c = atomicAdd(a.tile_ctr, 1);
+                const int t = c < total ? claim_to_tile(c, routed_tiles, total) : -1;
+                const int qs = tq % kTQ;
+                if (!mbar_wait(&tail->tqempty[qs], ((tq / kTQ) & 1) ^ 1, abort, a.err, kWaitLimit)) {
+                    ok = false;
+                    break;
+                }
+                reinterpret_cast<volatile int *>(tail->tq)[qs] = t;
+                mbar_arrive(&tail->tqfull[qs]);
+                if (t < 0) break;
                 const Tile T = decode_tile(t, tail->pre, a, bn);
+                const uint64_t pol = T.shared ? pol_s : pol_w;
                 const CUtensorMap *m0 = T.shared ? &maps.b0_shared : &maps.b0_routed;
                 const CUtensorMap *m1 = T.shared ? &maps.b1_shared : &maps.b1_routed;
                 const int gi = T.shared ? 0 : T.g;
@@ -372,9 +424,9 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                     uint8_t *dst = ring + (size_t)s * bytes;
                     mbar_arrive_expect_tx(&full[s], bytes);
                     // rows 0-127: gate (up) or W_d rows n0..; rows 128-255: up rows n0.. or W_d rows n0+128..
-                    tma_load_2d_hint(dst, m0, &full[s], kb * kBK, r0, pol_w);
+                    tma_load_2d_hint(dst, m0, &full[s], kb * kBK, r0, pol);
                     tma_load_2d_hint(dst + bytes / 2, kUp ? m1 : m0, &full[s], kb * kBK, kUp ? r0 : r0 + kBN / 2,
-                                     pol_w);
+                                     pol);
                 }
             }
             if (!ok)   // let in-flight loads land before the CTA exits
@@ -392,7 +444,9 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             // 32 * (p / 32) + 4j + (p % 32) / 8, j = 0..7, so every cp.async
             // instruction of a warp reads four whole 128-byte row segments.
             const int pw = p >> 5, pl = p & 31, pc = pl & 7;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (uint32_t tq = 0; ok; ++tq) {
+                const int t = tq_take(tail, tq, abort, a.err);
+                if (t < 0) break;
                 const Tile T = decode_tile(t, tail->pre, a, bn);
                 int tok0[8], tok1[8];
 #pragma unroll
@@ -425,7 +479,9 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             }
             cp_async_wait_all();   // this thread's row copies have landed before it leaves
         } else if (p == 0) {
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (uint32_t tq = 0; ok; ++tq) {
+                const int t = tq_take(tail, tq, abort, a.err);
+                if (t < 0) break;
                 const Tile T = decode_tile(t, tail->pre, a, bn);
                 const int mt = T.two ? 2 : 1;
                 for (int kb = 0; kb < a.kblocks && ok; ++kb) {
@@ -456,7 +512,9 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             uint32_t ia = 0, ib = 0, use0 = 0, use1 = 0;     // uses of half 0 / half 1 so far
             int hn = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (uint32_t tq = 0; ok; ++tq) {
+                const int t = tq_take(tail, tq, abort, a.err);
+                if (t < 0) break;
                 const Tile T = decode_tile(t, tail->pre, a, bn);
                 const int h0 = hn, h1 = hn ^ 1;
                 const uint32_t c0 = h0 ? use1 : use0, c1 = h0 ? use0 : use1;
@@ -498,7 +556,9 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         uint32_t at = 0;
         int hn = 0;                       // the half rotation of the MMA thread, replayed
         const uint32_t stage = smem_u32(epi) + warp * 4096;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++at) {
+        for (;; ++at) {
+            const int t = tq_take(tail, at, abort, a.err);
+            if (t < 0) break;
             const Tile T = decode_tile(t, tail->pre, a, bn);
             const int h0 = hn, h1 = hn ^ 1;
             if (!mbar_wait(&tail->tfull, at & 1, abort, a.err, kWaitLimit)) break;
@@ -580,7 +640,7 @@ static int sm_count_tc()
 }
 
 template <bool kFp8>
-static kmoe_status run_tc(const TcMaps &up, const TcMaps &dn, TcArgs a, int d, int I, __nv_bfloat16 *h,
+static kmoe_status run_tc(const TcMaps &up, const TcMaps &dn, TcArgs a, int d, int I, int *sync, __nv_bfloat16 *h,
                           __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, const ExpertPtrs &routed,
                           const ExpertPtrs &sh, cudaStream_t st)
 {
@@ -595,6 +655,7 @@ static kmoe_status run_tc(const TcMaps &up, const TcMaps &dn, TcArgs a, int d, i
     a.s1_routed = routed.su;
     a.s0_shared = sh.sg;
     a.s1_shared = sh.su;
+    a.tile_ctr = sync;
     ffn_tc_kernel<true, kFp8><<<grid, threads_of(kFp8), smem, st>>>(up, a);
     kmoe_status s = check_launch("ffn_up_tc");
     if (s != KMOE_OK) return s;
@@ -606,13 +667,14 @@ static kmoe_status run_tc(const TcMaps &up, const TcMaps &dn, TcArgs a, int d, i
     a.s1_routed = nullptr;
     a.s0_shared = sh.sd;
     a.s1_shared = nullptr;
+    a.tile_ctr = sync + 1;
     ffn_tc_kernel<false, kFp8><<<grid, threads_of(kFp8), smem, st>>>(dn, a);
     return check_launch("ffn_down_tc");
 }
 
 kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
                           const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
-                          __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err,
+                          __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err, int *sync,
                           cudaStream_t st)
 {
     if (E + 1 > kMaxGroups) return fail(KMOE_ERR_UNSUPPORTED, "tensor-core FFN: too many experts");
@@ -640,8 +702,8 @@ kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, in
     a.d = d;
     a.I = I;
     a.err = err;
-    if (fp8) return run_tc<true>(up, dn, a, d, I, h, y_perm, y_shared, routed, sh, st);
-    return run_tc<false>(up, dn, a, d, I, h, y_perm, y_shared, routed, sh, st);
+    if (fp8) return run_tc<true>(up, dn, a, d, I, sync, h, y_perm, y_shared, routed, sh, st);
+    return run_tc<false>(up, dn, a, d, I, sync, h, y_perm, y_shared, routed, sh, st);
 }
 
 }  // namespace kmoe
