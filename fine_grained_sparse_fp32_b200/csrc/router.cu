@@ -85,13 +85,23 @@ kmoe_status launch_router_logits(const void *x, int x_dtype, const float *w_rout
     return check_launch("router_logits");
 }
 
+// Order-preserving integer key of a finite score (-0 and +0 map to the same
+// key, so they tie like equal floats do).
+__device__ __forceinline__ int score_key(float s)
+{
+    const int b = __float_as_int(s + 0.f);
+    return b < 0 ? b ^ 0x7fffffff : b;
+}
+
 // ------------------------------------------------------------------- top-K
 //
 // One warp per token. Lane l holds the biased scores s[e] = l[e] + b[e] of
-// experts e = i*32 + l (NPL of them) in registers. K rounds: every lane finds
-// its best remaining candidate, a butterfly reduction picks the warp's best
-// by (score descending, index ascending), and its owner retires it. Logits
-// are read through L2 (they may come from other CTAs of the same kernel).
+// experts e = i*32 + l (NPL of them) in registers, as order-preserving
+// integer keys. K rounds: every lane finds its best remaining candidate, the
+// warp's largest key and then the lowest expert index holding it are found
+// with one reduce instruction each (score descending, index ascending), and
+// the owner retires it. Logits are read through L2 (they may come from other
+// CTAs of the same kernel).
 // Mixture weights from the unbiased logits of the K chosen experts: sigmoid
 // of each ("Inside Kolibri 1", routing section) or, with KMOE_SCORE_SOFTMAX,
 // a softmax over the K ("Kolibri 1 Deep Dive", routing formulation).
@@ -99,46 +109,60 @@ template <int NPL>
 __device__ __forceinline__ void topk_warp(const float *lr, const float *__restrict__ bias, int E, int K, int score,
                                           int32_t *idx_row, float *w_row)
 {
-    float lsel[8];                    // lane 0: unbiased logits of the chosen experts (K <= 8)
+    // Unbiased logits of the chosen experts (K <= 8). Up to 512 experts they
+    // travel with their scores through the selection; beyond that lane 0
+    // reads them back (registers would spill).
+    constexpr bool kCarry = NPL <= 16;
+    float lsel[8];
     const int lane = threadIdx.x & 31;
-    float s[NPL];
+    int key[NPL];
+    float l[kCarry ? NPL : 1];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = i * 32 + lane;
-        s[i] = e < E ? __ldcg(lr + e) + bias[e] : -FLT_MAX;
+        const float li = e < E ? __ldcg(lr + e) : 0.f;
+        if (kCarry) l[i] = li;
+        key[i] = e < E ? score_key(li + bias[e]) : INT_MIN;
     }
-    for (int k = 0; k < K; ++k) {
-        float bv = -INFINITY;
-        int be = INT_MAX;
 #pragma unroll
-        for (int i = 0; i < NPL; ++i)        // ascending e inside a lane: '>' keeps the lowest
-            if (s[i] > bv) { bv = s[i]; be = i * 32 + lane; }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-        }
+    for (int k = 0; k < 8; ++k) {
+        if (k >= K) break;
+        // best of this lane (ascending e: '>' keeps the lowest index on ties),
+        // then the warp's largest key and the lowest expert holding it
+        int bk = INT_MIN, be = INT_MAX;
+        float bl = 0.f;
 #pragma unroll
         for (int i = 0; i < NPL; ++i)
-            if (i * 32 + lane == be) s[i] = -INFINITY;
-        if (lane == 0) {   // be < E whenever K <= E and the scores are finite
-            const int e = be < E ? be : E - 1;
-            idx_row[k] = e;
-            lsel[k] = __ldcg(lr + e);
-        }
+            if (key[i] > bk) { bk = key[i]; be = i * 32 + lane; if (kCarry) bl = l[i]; }
+        const int mk = __reduce_max_sync(0xffffffffu, bk);
+        const int me = __reduce_min_sync(0xffffffffu, bk == mk ? be : INT_MAX);
+        const int e = me < E ? me : E - 1;     // me < E whenever K <= E and the scores are finite
+        const float wl = kCarry ? __shfl_sync(0xffffffffu, bl, me & 31) : 0.f;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+            if (i * 32 + lane == me) key[i] = INT_MIN;
+        lsel[k] = kCarry ? wl : (lane == 0 ? __ldcg(lr + e) : 0.f);
+        if (lane == 0) idx_row[k] = e;
     }
     if (lane == 0) {
         if (score == KMOE_SCORE_SOFTMAX) {
             float mx = -INFINITY, sum = 0.f;
-            for (int k = 0; k < K; ++k) mx = fmaxf(mx, lsel[k]);
-            for (int k = 0; k < K; ++k) {
-                lsel[k] = expf(lsel[k] - mx);
-                sum += lsel[k];
-            }
-            for (int k = 0; k < K; ++k) w_row[k] = lsel[k] / sum;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k < K) mx = fmaxf(mx, lsel[k]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k < K) {
+                    lsel[k] = expf(lsel[k] - mx);
+                    sum += lsel[k];
+                }
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k < K) w_row[k] = lsel[k] / sum;
         } else {
-            for (int k = 0; k < K; ++k) w_row[k] = sigmoidf_(lsel[k]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k < K) w_row[k] = sigmoidf_(lsel[k]);
         }
     }
 }
@@ -176,21 +200,34 @@ kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, in
 // dispatch permutation run as one launch of CTAs of 32 warps. Each CTA owns
 // kRouteEPC experts: the bulk-copy engine brings their FP32 router rows and a
 // chunk of up to 32 token rows into shared memory. Warp w handles tokens
-// 4*(w%8) .. 4*(w%8)+3 of the chunk over column quarter w/8, so every router
-// weight read from shared memory feeds four tokens; the four quarter sums of
-// a logit are added in a fixed order. The last CTA to finish (a ticket in
+// 8*(w%4) .. 8*(w%4)+7 of the chunk over column part w/4 (one eighth of d),
+// four columns per lane and step, so every router weight read from shared
+// memory feeds eight tokens and no load has a bank conflict; the eight part
+// sums of a logit are added in a fixed order. The last CTA to finish (a ticket in
 // the workspace status area, zeroed before the launch) then selects the top K
 // of every token (one warp per token) and builds the permutation with 32-warp
 // ballot masks, reusing its shared memory.
 constexpr int kRouteEPC = 3;
 constexpr int kRouteThreads = 1024;
 constexpr int kRouteWarps = kRouteThreads / 32;
-constexpr int kRouteTPW = 4;                          // tokens per warp
-constexpr int kRouteTG = 8;                           // token groups per chunk
-constexpr int kRouteCQ = kRouteWarps / kRouteTG;      // column parts (4)
+constexpr int kRouteTPW = 8;                          // tokens per warp
+constexpr int kRouteTG = 4;                           // token groups per chunk
+constexpr int kRouteCQ = kRouteWarps / kRouteTG;      // column parts (8)
 constexpr int kRouteChunkMax = kRouteTPW * kRouteTG;  // 32 tokens per chunk
 constexpr int kRouteSmemMax = 200 * 1024;
 constexpr long long kRouteWaitLimit = 1LL << 32;
+
+__device__ __forceinline__ void load4(const float *p, float (&o)[4])
+{
+    const float4 v = *reinterpret_cast<const float4 *>(p);
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+__device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&o)[4])
+{
+    const uint2 v = *reinterpret_cast<const uint2 *>(p);
+    o[0] = __uint_as_float(v.x << 16); o[1] = __uint_as_float(v.x & 0xffff0000u);
+    o[2] = __uint_as_float(v.y << 16); o[3] = __uint_as_float(v.y & 0xffff0000u);
+}
 
 template <class XT, int NPL>
 __global__ void __launch_bounds__(kRouteThreads, 1)
@@ -241,25 +278,23 @@ route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const 
 #pragma unroll
             for (int e = 0; e < kRouteEPC; ++e) acc[a][e] = 0.f;
         if (t0 < nt) {
-            for (int j = cq * qd + lane * 8; j < (cq + 1) * qd; j += 256) {
-                float wv[kRouteEPC][8];
+            for (int j = cq * qd + lane * 4; j < (cq + 1) * qd; j += 128) {
+                float wv[kRouteEPC][4];
 #pragma unroll
                 for (int e = 0; e < kRouteEPC; ++e) {
-                    if (e < ne) load8(wsm + e * d + j, wv[e]);
-                    else {
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) wv[e][q] = 0.f;
-                    }
+                    const float4 v = e < ne ? *reinterpret_cast<const float4 *>(wsm + e * d + j)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                    wv[e][0] = v.x; wv[e][1] = v.y; wv[e][2] = v.z; wv[e][3] = v.w;
                 }
 #pragma unroll
                 for (int a = 0; a < kRouteTPW; ++a) {
                     if (t0 + a < nt) {
-                        float xv[8];
-                        load8(xsm + (size_t)(t0 + a) * d + j, xv);
+                        float xv[4];
+                        load4(xsm + (size_t)(t0 + a) * d + j, xv);
 #pragma unroll
                         for (int e = 0; e < kRouteEPC; ++e)
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) acc[a][e] = fmaf(xv[q], wv[e][q], acc[a][e]);
+                            for (int q = 0; q < 4; ++q) acc[a][e] = fmaf(xv[q], wv[e][q], acc[a][e]);
                     }
                 }
             }
@@ -294,7 +329,10 @@ route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const 
     for (int t = warp; t < N; t += kRouteWarps)
         topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, score, idx + (size_t)t * K, wout + (size_t)t * K);
     __syncthreads();
-    permute_small_block<kRouteWarps>(idx, N, K, E, counts, offsets, perm, inv, reinterpret_cast<uint32_t *>(sm_raw));
+    // ballot masks only as wide as the batch: one warp's worth for decode-sized batches
+    uint32_t *mask = reinterpret_cast<uint32_t *>(sm_raw);
+    if (N <= 32) permute_small_block<1>(idx, N, K, E, counts, offsets, perm, inv, mask);
+    else permute_small_block<kChunkWarps>(idx, N, K, E, counts, offsets, perm, inv, mask);
     if (threadIdx.x == 0) *ticket = 0;
 }
 
