@@ -40,11 +40,11 @@
 // time share the expert's token rows in L2.
 //
 // E4M3 weights ("Inside Kolibri 1", FP8 section: 128 x 128 blocks, one FP32
-// scale per block) take the same kernels with four more warps: warp 9 brings
-// the E4M3 bytes by TMA into a four-deep staging ring (16 KB per k-block),
-// and converter warps 10-13 decode them (hardware e4m3x2 -> f16x2), multiply
-// by the FP32 scale of the block, round to BF16 and write the swizzled tile
-// the MMA reads. Activations stay BF16, so the tensor cores see BF16 x BF16
+// scale per block) take the same kernels with eight more warps: warp 9
+// brings the E4M3 bytes by TMA into a four-deep staging ring (16 KB per
+// k-block), and converter warps 10-17 (one thread per weight row) decode
+// them (hardware e4m3x2 -> f16x2), multiply by the FP32 scale of the block,
+// round to BF16 and write the swizzled tile the MMA reads. Activations stay BF16, so the tensor cores see BF16 x BF16
 // with FP32 accumulation, and the weights cross HBM at one byte each.
 #include "common.cuh"
 #include "sm100.cuh"
@@ -71,8 +71,9 @@ __host__ __device__ constexpr int ring_bytes(bool fp8)
 constexpr int kMmaWarp = 4;
 constexpr int kProdWarp = 5;                 // token producers: warps 5-8
 constexpr int kWProdWarp = 9;                // weight producer
-constexpr int kConvWarp = 10;                // E4M3 only: warps 10-13
-__host__ __device__ constexpr int threads_of(bool fp8) { return (fp8 ? 14 : 10) * 32; }
+constexpr int kConvWarp = 10;                // E4M3 only: warps 10-17
+constexpr int kConvThreads = 256;            // one converter thread per weight row of a tile
+__host__ __device__ constexpr int threads_of(bool fp8) { return (fp8 ? 18 : 10) * 32; }
 constexpr int kMaxGroups = 1025;
 constexpr int kTQ = 4;                       // tile queue depth
 constexpr long long kWaitLimit = 1LL << 32;  // SM cycles (about 2 s)
@@ -312,12 +313,12 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             mbar_init(&tail->aempty[s], 1);
         }
         for (int s = 0; s < kBS; ++s) {
-            mbar_init(&tail->bfull[s], kFp8 ? 128 : 1);   // E4M3: the 128 converter threads
+            mbar_init(&tail->bfull[s], kFp8 ? kConvThreads : 1);   // E4M3: the converter threads
             mbar_init(&tail->bempty[s], 1);
         }
         for (int s = 0; s < kSStages; ++s) {
             mbar_init(&tail->sfull[s], 1);
-            mbar_init(&tail->sempty[s], 128);
+            mbar_init(&tail->sempty[s], kConvThreads);
         }
         mbar_init(&tail->tfull, 1);
         mbar_init(&tail->tempty[0], 128);
@@ -326,7 +327,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         for (int s = 0; s < kTQ; ++s) {
             mbar_init(&tail->tqfull[s], 1);
             // readers: token producers (up: 128, down: 1), the MMA thread, 128 epilogue threads, converters
-            mbar_init(&tail->tqempty[s], (kUp ? 128 : 1) + 1 + 128 + (kFp8 ? 128 : 0));
+            mbar_init(&tail->tqempty[s], (kUp ? 128 : 1) + 1 + 128 + (kFp8 ? kConvThreads : 0));
         }
         tail->abort = 0;
         fence_mbar_init();
@@ -352,7 +353,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
 
     if (kFp8 && warp >= kConvWarp) {
         // ------------------------------------------- E4M3 -> BF16 converters
-        const int q = threadIdx.x - kConvWarp * 32;          // rows q and q + 128 of the B tile
+        const int q = threadIdx.x - kConvWarp * 32;          // row q of the B tile
         uint32_t it = 0;
         bool ok = true;
         for (uint32_t tq = 0; ok; ++tq) {
@@ -381,8 +382,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                 }
                 const uint8_t *B8 = ring_s + (size_t)ss * kB8Tile;
                 uint8_t *Bs = ring_b + (size_t)sb * kBTile;
-                convert_row(B8 + q * kBK, Bs, q, sc0);
-                convert_row(B8 + (q + 128) * kBK, Bs, q + 128, sc1);
+                convert_row(B8 + q * kBK, Bs, q, q < 128 ? sc0 : sc1);
                 mbar_arrive(&tail->sempty[ss]);      // staging slot read
                 fence_proxy_async();                 // converted rows visible to the tensor cores
                 mbar_arrive(&tail->bfull[sb]);
