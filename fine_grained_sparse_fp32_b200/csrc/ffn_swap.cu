@@ -566,10 +566,16 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                         // token tile 0 carries the first weight tile's block scale, tile 1 the second's
                         const uint64_t b0 = sw128_kmajor_desc(smem_u32(convb + (size_t)cs * 2 * C::BTile));
                         const uint64_t b1 = sw128_kmajor_desc(smem_u32(convb + (size_t)(cs * 2 + 1) * C::BTile));
+                        // all k-steps of one accumulator before the other: an MMA
+                        // that switches accumulators costs nearly twice as much
 #pragma unroll
                         for (int k = 0; k < C::BK / 16; ++k) {
                             const uint64_t ko = (uint64_t)(((k >> 2) * C::Panel + (k & 3) * 32) >> 4);
                             umma_f16_tmem_a(dg, at + k * 8, b0 + ko, id, (kb | k) != 0);
+                        }
+#pragma unroll
+                        for (int k = 0; k < C::BK / 16; ++k) {
+                            const uint64_t ko = (uint64_t)(((k >> 2) * C::Panel + (k & 3) * 32) >> 4);
                             umma_f16_tmem_a(du, at + 64 + k * 8, b1 + ko, id, (kb | k) != 0);
                         }
                         umma_commit(&T->cempty[cs]);
@@ -581,10 +587,11 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                         const uint64_t a0 = sw128_kmajor_desc(sa), a1 = sw128_kmajor_desc(sa + kATile);
                         const uint64_t bd = sw128_kmajor_desc(sa + 2 * kATile);
 #pragma unroll
-                        for (int k = 0; k < C::BK / 16; ++k) {
+                        for (int k = 0; k < C::BK / 16; ++k)
                             umma_bf16(dg, a0 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), id, (kb | k) != 0);
+#pragma unroll
+                        for (int k = 0; k < C::BK / 16; ++k)
                             umma_bf16(du, a1 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), id, (kb | k) != 0);
-                        }
                         umma_commit(&T->empty[s]);
                     }
                 }
