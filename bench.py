@@ -157,13 +157,22 @@ def run_config(cfg, steps, warmup, rank, world, seed=0, use_graph=True):
     stream.synchronize()
     distinct = float(np.mean([(c > 0).sum().item() for c in counts]))
 
+    # One graph per step, and one graph holding a whole cycle of ROTATE
+    # consecutive steps (the way a model's forward pass replays many layer
+    # calls from a single graph); the timed loop replays cycles and fills any
+    # remainder with single steps, so it runs exactly `steps` layer calls.
     graphs = []
+    cycle = None
     if use_graph:
         for i in range(ROTATE):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 lay.forward(xs[i], y=ys[i], counts=counts[i], stream=stream)
             graphs.append(g)
+        cycle = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cycle, stream=stream):
+            for i in range(ROTATE):
+                lay.forward(xs[i], y=ys[i], counts=counts[i], stream=stream)
 
     def step(i):
         if use_graph:
@@ -171,9 +180,18 @@ def run_config(cfg, steps, warmup, rank, world, seed=0, use_graph=True):
         else:
             lay.forward(xs[i % ROTATE], y=ys[i % ROTATE], counts=counts[i % ROTATE], stream=stream)
 
+    def run_steps(n, single=False):
+        i = 0
+        while i < n:
+            if cycle is not None and not single and n - i >= ROTATE:
+                cycle.replay()
+                i += ROTATE
+            else:
+                step(i)
+                i += 1
+
     with torch.cuda.stream(stream):
-        for i in range(warmup):
-            step(i)
+        run_steps(warmup)
     torch.cuda.synchronize()
     barrier(world)
     clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
@@ -183,13 +201,23 @@ def run_config(cfg, steps, warmup, rank, world, seed=0, use_graph=True):
     barrier(world)
     with torch.cuda.stream(stream):
         t0.record(stream)
-        for i in range(steps):
-            step(i)
+        run_steps(steps)
         t1.record(stream)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
     clk = clocks.stop() if clocks else None
     ms_max = all_max(ms, world)
+
+    # the same steps replayed one graph per step (reported beside the main number)
+    single_ms = None
+    if cycle is not None:
+        barrier(world)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            run_steps(steps, single=True)
+            t1.record(stream)
+        torch.cuda.synchronize()
+        single_ms = all_max(t0.elapsed_time(t1), world) / steps
 
     # per-kernel-group timing of the dominant step (grouped FFN), decomposed calls
     ffn_ms = time_grouped_ffn(layer, xs, stream, steps=max(20, min(steps, 400)))
@@ -197,7 +225,7 @@ def run_config(cfg, steps, warmup, rank, world, seed=0, use_graph=True):
     # end to end: pinned host x -> device, layer, device y -> pinned host
     e2e_ms = time_e2e(lay, cfg, xs, stream, steps=max(20, min(steps, 400)), warmup=max(3, warmup // 4))
     alg = algorithmic(cfg, distinct)
-    return {"ms_per_step": ms_max / steps, "clocks": clk, "distinct": distinct, "alg": alg,
+    return {"ms_per_step": ms_max / steps, "single_graph_ms": single_ms, "clocks": clk, "distinct": distinct, "alg": alg,
             "ffn_ms": ffn_ms, "e2e_ms": e2e_ms}
 
 
@@ -394,7 +422,7 @@ def main():
                        "tokens_per_gpu": dec.N, "parallelism": f"replicas x{world} (no collective)",
                        "l2": "inputs larger than L2: ~%.2f GB of expert weights per step, %d rotating token batches"
                              % (alg["expert_weight_bytes"] / 1e9, ROTATE),
-                       "cuda_graph": not args.no_graph},
+                       "cuda_graph": (f"{ROTATE} consecutive layer calls per graph" if not args.no_graph else False)},
             "roofline": {"bound": "hbm", "kernel": "moe_grouped_ffn: ffn_swap_kernel (up and down units, one launch)",
                          "achieved": ffn_gbs, "peak": hbm, "unit": "GB/s", "frac": ffn_gbs / hbm,
                          "traffic": kernel_traffic("decode"), "peak_kind": peak_kind + " burst",
@@ -404,6 +432,7 @@ def main():
                     "h2d_bytes_per_step": r["e2e_ms"]["h2d"], "d2h_bytes_per_step": r["e2e_ms"]["d2h"]},
             "gpu_launches": launches_per_step(dec) * args.steps,
             "clocks": r["clocks"],
+            "ms_per_step_one_graph_per_step": r["single_graph_ms"],
             "distinct_experts_per_step": r["distinct"],
         }
         if pre is not None:

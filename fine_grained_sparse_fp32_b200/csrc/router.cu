@@ -299,13 +299,25 @@ route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const 
                 }
             }
         }
+        // Reduce the 24 partial sums across the warp in one transposing
+        // butterfly (31 shuffles instead of 24 x 5): at the level with offset
+        // o every lane keeps one half of its values and sends the other, so
+        // lane i ends up holding the warp total of value i.
+        static_assert(kRouteTPW * kRouteEPC <= 32, "one value per lane");
+        float v[32];
 #pragma unroll
-        for (int a = 0; a < kRouteTPW; ++a)
+        for (int i = 0; i < 32; ++i) v[i] = i < kRouteTPW * kRouteEPC ? acc[i / kRouteEPC][i % kRouteEPC] : 0.f;
 #pragma unroll
-            for (int e = 0; e < kRouteEPC; ++e) {
-                const float v = warp_sum(acc[a][e]);
-                if (lane == 0) red[cq][t0 + a][e] = v;
+        for (int o = 16; o >= 1; o >>= 1) {
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int j = 0; j < o; ++j) {
+                const float send = upper ? v[j] : v[j + o];
+                const float keep = upper ? v[j + o] : v[j];
+                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
             }
+        }
+        if (lane < kRouteTPW * kRouteEPC) red[cq][t0 + lane / kRouteEPC][lane % kRouteEPC] = v[0];
         __syncthreads();
         if (threadIdx.x < nt * ne) {
             const int t = threadIdx.x / ne, e = threadIdx.x - t * ne;
