@@ -42,6 +42,8 @@ combine_kernel(const YI *__restrict__ y_perm, const YI *__restrict__ y_shared,
                const float *__restrict__ w, const int32_t *__restrict__ inv, int N, int K, int d,
                YO *__restrict__ y)
 {
+    pdl_wait();
+    pdl_trigger();
     const int t = blockIdx.x;
     const int c = (blockIdx.y * kCombineThreads + threadIdx.x) * 8;
     if (c >= d) return;
@@ -104,6 +106,8 @@ combine_bulk_kernel(const __nv_bfloat16 *__restrict__ y_perm, const __nv_bfloat1
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_wait();
+    pdl_trigger();
     // thread 0 issues the rows of this block's i-th token into stage i % kBulkStages
     auto issue = [&](int i) {
         const int t = blockIdx.x + i * gridDim.x;
@@ -203,20 +207,20 @@ kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dt
         const bf *yp = static_cast<const bf *>(y_perm), *ys = static_cast<const bf *>(y_shared);
         if (y_dtype == KMOE_F32) {
             cudaFuncSetAttribute(combine_bulk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsm);
-            combine_bulk_kernel<float><<<grid, kBulkThreads, bsm, st>>>(yp, ys, w, inv, N, K, d, static_cast<float *>(y), err,
-                                                                        hr, gp, eps);
+            launch_pdl(combine_bulk_kernel<float>, grid, kBulkThreads, bsm, st, yp, ys, w, inv, N, K, d,
+                       static_cast<float *>(y), err, hr, gp, eps);
         } else {
             cudaFuncSetAttribute(combine_bulk_kernel<bf>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsm);
-            combine_bulk_kernel<bf><<<grid, kBulkThreads, bsm, st>>>(yp, ys, w, inv, N, K, d, static_cast<bf *>(y), err,
-                                                                     hr, gp, eps);
+            launch_pdl(combine_bulk_kernel<bf>, grid, kBulkThreads, bsm, st, yp, ys, w, inv, N, K, d,
+                       static_cast<bf *>(y), err, hr, gp, eps);
         }
         return check_launch("combine");
     }
     dim3 grid(N, (d / 8 + kCombineThreads - 1) / kCombineThreads);
 #define KMOE_COMB(YI, YO)                                                                            \
-    combine_kernel<YI, YO><<<grid, kCombineThreads, 0, st>>>(                                        \
-        static_cast<const YI *>(y_perm), static_cast<const YI *>(y_shared), w, inv, N, K, d,          \
-        static_cast<YO *>(y))
+    launch_pdl(combine_kernel<YI, YO>, grid, kCombineThreads, 0, st,                                 \
+               static_cast<const YI *>(y_perm), static_cast<const YI *>(y_shared), w, inv, N, K, d,  \
+               static_cast<YO *>(y))
     if (y_in_dtype == KMOE_F32) {
         if (y_dtype == KMOE_F32) KMOE_COMB(float, float);
         else KMOE_COMB(float, bf);

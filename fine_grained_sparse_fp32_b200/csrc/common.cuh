@@ -21,6 +21,32 @@ void clear_error();
 // Checks the last launch; on failure records the CUDA error string.
 kmoe_status check_launch(const char *what);
 
+// Programmatic dependent launch. The kernels of a layer call are launched
+// with launch_pdl, so each may start (its prologue: barriers, tensor memory,
+// descriptor prefetch) while the previous kernel on the stream is still
+// finishing. Every such kernel calls pdl_wait() before it reads anything an
+// earlier kernel wrote (the wait returns once that kernel has completed and
+// its writes are visible), then pdl_trigger() so that the next kernel can
+// be scheduled. Without a programmatic predecessor both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr{};
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);   // errors surface in check_launch
+}
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Carves 256-byte aligned pieces out of a caller-provided workspace.

@@ -371,7 +371,6 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
         T->abort = 0;
         fence_mbar_init();
     }
-    if (warp == kSchedWarp) build_prefix(T->pre, T->off, a);
     if (warp == 0) {
         tmem_alloc(&T->tmem_base, C::TmemCols);
         tmem_relinquish();
@@ -381,6 +380,9 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
         if (a.has_shared) { prefetch_map(&maps.g_s); prefetch_map(&maps.u_s); prefetch_map(&maps.d_s); }
         prefetch_map(&maps.xg); prefetch_map(&maps.hb);
     }
+    pdl_wait();               // routing (offsets, permutation) and x come from earlier kernels
+    pdl_trigger();
+    if (warp == kSchedWarp) build_prefix(T->pre, T->off, a);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -815,7 +817,7 @@ static void launch_cfg(const Maps &m, const Args &a, cudaStream_t st)
     static_assert(smem <= (size_t)kSmemLimit, "shared memory per CTA");
     auto k = ffn_swap_kernel<kFp8, kNT>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<swap_sm_count(), C::Warps * 32, smem, st>>>(m, a);
+    launch_pdl(k, swap_sm_count(), C::Warps * 32, smem, st, m, a);
 }
 
 kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,

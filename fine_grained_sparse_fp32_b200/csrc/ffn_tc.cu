@@ -332,7 +332,6 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         tail->abort = 0;
         fence_mbar_init();
     }
-    if (warp == kMmaWarp) build_prefix(tail->pre, a);
     if (warp == 0) {
         tmem_alloc(&tail->tmem_base, 512);
         tmem_relinquish();
@@ -343,6 +342,9 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         if (kUp) { prefetch_map(&maps.b1_routed); prefetch_map(&maps.b1_shared); }
         else prefetch_map(&maps.a);
     }
+    pdl_wait();               // routing, x and (down) H come from earlier kernels
+    pdl_trigger();
+    if (warp == kMmaWarp) build_prefix(tail->pre, a);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -656,7 +658,7 @@ static kmoe_status run_tc(const TcMaps &up, const TcMaps &dn, TcArgs a, int d, i
     a.s0_shared = sh.sg;
     a.s1_shared = sh.su;
     a.tile_ctr = sync;
-    ffn_tc_kernel<true, kFp8><<<grid, threads_of(kFp8), smem, st>>>(up, a);
+    launch_pdl(ffn_tc_kernel<true, kFp8>, grid, threads_of(kFp8), smem, st, up, a);
     kmoe_status s = check_launch("ffn_up_tc");
     if (s != KMOE_OK) return s;
     a.kblocks = I / kBK;
@@ -668,7 +670,7 @@ static kmoe_status run_tc(const TcMaps &up, const TcMaps &dn, TcArgs a, int d, i
     a.s0_shared = sh.sd;
     a.s1_shared = nullptr;
     a.tile_ctr = sync + 1;
-    ffn_tc_kernel<false, kFp8><<<grid, threads_of(kFp8), smem, st>>>(dn, a);
+    launch_pdl(ffn_tc_kernel<false, kFp8>, grid, threads_of(kFp8), smem, st, dn, a);
     return check_launch("ffn_down_tc");
 }
 

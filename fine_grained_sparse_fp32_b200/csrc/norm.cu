@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(kNormThreads)
 rmsnorm_bf16_kernel(const __nv_bfloat16 *__restrict__ h, const __nv_bfloat16 *__restrict__ gamma, float eps, int d,
                     __nv_bfloat16 *__restrict__ x)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float red[kNormThreads / 32];
     __shared__ float scale;
     const __nv_bfloat16 *row = h + (size_t)blockIdx.x * d;
@@ -56,7 +58,7 @@ rmsnorm_bf16_kernel(const __nv_bfloat16 *__restrict__ h, const __nv_bfloat16 *__
 kmoe_status launch_rmsnorm(const __nv_bfloat16 *h, const __nv_bfloat16 *gamma, float eps, int N, int d,
                            __nv_bfloat16 *x, cudaStream_t st)
 {
-    rmsnorm_bf16_kernel<<<N, kNormThreads, 0, st>>>(h, gamma, eps, d, x);
+    launch_pdl(rmsnorm_bf16_kernel, N, kNormThreads, 0, st, h, gamma, eps, d, x);
     return check_launch("rmsnorm");
 }
 

@@ -16,6 +16,8 @@ namespace kmoe {
 __global__ void __launch_bounds__(kChunk)
 chunk_hist_kernel(const int32_t *__restrict__ idx, int N, int K, int E, int32_t *__restrict__ hist)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint32_t mask[];
     build_masks(idx, N, K, E, blockIdx.x, mask);
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -32,6 +34,8 @@ __global__ void __launch_bounds__(1024)
 scan_kernel(int32_t *__restrict__ hist, int chunks, int E, int32_t *__restrict__ counts,
             int32_t *__restrict__ offsets)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int tmp[32];
     const int e = threadIdx.x;
     int total = 0;
@@ -56,6 +60,8 @@ __global__ void __launch_bounds__(kChunk)
 scatter_kernel(const int32_t *__restrict__ idx, int N, int K, int E,
                const int32_t *__restrict__ base, int32_t *__restrict__ perm, int32_t *__restrict__ inv)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint32_t mask[];
     build_masks(idx, N, K, E, blockIdx.x, mask);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -76,6 +82,8 @@ permute_single_kernel(const int32_t *__restrict__ idx, int N, int K, int E,
                       int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                       int32_t *__restrict__ perm, int32_t *__restrict__ inv)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint32_t mask[];
     permute_small_block(idx, N, K, E, counts, offsets, perm, inv, mask);
 }
@@ -94,19 +102,20 @@ kmoe_status launch_permute(const int32_t *idx, int N, int K, int E, int32_t *cou
     if (N <= kChunk) {
         const size_t smem = mask_bytes + sizeof(int) * E;
         cudaFuncSetAttribute(permute_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        permute_single_kernel<<<1, kChunk, smem, st>>>(idx, N, K, E, counts, offsets, perm, inv);
+        launch_pdl(permute_single_kernel, 1, kChunk, smem, st, idx, N, K, E, counts, offsets, perm, inv);
         return check_launch("permute_single");
     }
     const int chunks = (N + kChunk - 1) / kChunk;
     cudaFuncSetAttribute(chunk_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mask_bytes);
     cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mask_bytes);
-    chunk_hist_kernel<<<chunks, kChunk, mask_bytes, st>>>(idx, N, K, E, hist);
+    launch_pdl(chunk_hist_kernel, chunks, kChunk, mask_bytes, st, idx, N, K, E, hist);
     kmoe_status s = check_launch("permute_hist");
     if (s != KMOE_OK) return s;
-    scan_kernel<<<1, 1024, 0, st>>>(hist, chunks, E, counts, offsets);
+    launch_pdl(scan_kernel, 1, 1024, 0, st, hist, chunks, E, counts, offsets);
     s = check_launch("permute_scan");
     if (s != KMOE_OK) return s;
-    scatter_kernel<<<chunks, kChunk, mask_bytes, st>>>(idx, N, K, E, hist, perm, inv);
+    launch_pdl(scatter_kernel, chunks, kChunk, mask_bytes, st, idx, N, K, E,
+               static_cast<const int32_t *>(hist), perm, inv);
     return check_launch("permute_scatter");
 }
 

@@ -30,6 +30,8 @@ __global__ void __launch_bounds__(kRouterThreads)
 router_logits_kernel(const XT *__restrict__ x, const float *__restrict__ w, int N, int d, int E,
                      float *__restrict__ logits)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ float4 smem_f4[];
     float *wsm = reinterpret_cast<float *>(smem_f4);   // [EPC][d]
     const int e0 = blockIdx.x * kRouterEPC;
@@ -75,11 +77,11 @@ kmoe_status launch_router_logits(const void *x, int x_dtype, const float *w_rout
     size_t smem = sizeof(float) * kRouterEPC * d;
     if (x_dtype == KMOE_F32) {
         cudaFuncSetAttribute(router_logits_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        router_logits_kernel<float><<<grid, kRouterThreads, smem, st>>>(
+        launch_pdl(router_logits_kernel<float>, grid, kRouterThreads, smem, st,
             static_cast<const float *>(x), w_router, N, d, E, logits);
     } else {
         cudaFuncSetAttribute(router_logits_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        router_logits_kernel<__nv_bfloat16><<<grid, kRouterThreads, smem, st>>>(
+        launch_pdl(router_logits_kernel<__nv_bfloat16>, grid, kRouterThreads, smem, st,
             static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E, logits);
     }
     return check_launch("router_logits");
@@ -172,6 +174,8 @@ __global__ void __launch_bounds__(256)
 topk_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int N, int E, int K, int score,
             int32_t *__restrict__ idx, float *__restrict__ wout)
 {
+    pdl_wait();
+    pdl_trigger();
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= N) return;
     topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, score, idx + (size_t)t * K, wout + (size_t)t * K);
@@ -183,7 +187,7 @@ kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, in
     const int warps = 8;
     dim3 grid((N + warps - 1) / warps);
     const int npl = (E + 31) / 32;
-#define KMOE_TOPK(n) topk_kernel<n><<<grid, warps * 32, 0, st>>>(logits, bias, N, E, K, score, idx, w)
+#define KMOE_TOPK(n) launch_pdl(topk_kernel<n>, grid, warps * 32, 0, st, logits, bias, N, E, K, score, idx, w)
     if (npl <= 2) KMOE_TOPK(2);
     else if (npl <= 4) KMOE_TOPK(4);
     else if (npl <= 8) KMOE_TOPK(8);
@@ -256,6 +260,8 @@ route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const 
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_wait();
+    pdl_trigger();
     uint32_t phase = 0;
     for (int c0 = 0; c0 < N; c0 += chunk) {
         const int nt = min(chunk, N - c0);
@@ -363,7 +369,8 @@ kmoe_status launch_route_small(const void *x, int x_dtype, const float *w_router
     do {                                                                                                    \
         auto k = route_small_kernel<XT, n>;                                                                 \
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                    \
-        k<<<grid, kRouteThreads, smem, st>>>(static_cast<const XT *>(x), w_router, bias, N, d, E, K, score,   \
+        launch_pdl(k, grid, kRouteThreads, smem, st, static_cast<const XT *>(x), w_router, bias, N, d, E, K,  \
+                   score,                                                                                  \
                                              chunk,                                                          \
                                              w_bytes, logits, idx, w, counts, offsets, perm, inv, status);   \
     } while (0)

@@ -60,6 +60,8 @@ constexpr size_t kRSmem = 1024 + (size_t)kRStages * kRStage + sizeof(RouterTail)
 __global__ void __launch_bounds__(256)
 router_split_kernel(const float *__restrict__ w, int n, __nv_bfloat16 *__restrict__ out)
 {
+    pdl_wait();
+    pdl_trigger();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
         const float v = w[i];
         const __nv_bfloat16 a = __float2bfloat16_rn(v);
@@ -108,6 +110,9 @@ router_tc_kernel(const __grid_constant__ RouterMaps maps, int N, int d, int E, f
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_wait();
+    pdl_trigger();
+
     const uint32_t tmem = tail->tmem_base;
 
     if (warp == kRProdWarp) {
@@ -234,7 +239,7 @@ kmoe_status launch_router_tc(const __nv_bfloat16 *x, const float *w_router, int 
                              __nv_bfloat16 *w_split, float *logits, int *err, cudaStream_t st)
 {
     const int n = E * d;
-    router_split_kernel<<<(n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184, 256, 0, st>>>(w_router, n, w_split);
+    launch_pdl(router_split_kernel, (n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184, 256, 0, st, w_router, n, w_split);
     kmoe_status s = check_launch("router_split");
     if (s != KMOE_OK) return s;
     RouterMaps maps{};
@@ -242,7 +247,7 @@ kmoe_status launch_router_tc(const __nv_bfloat16 *x, const float *w_router, int 
         return fail(KMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (router)");
     cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRSmem);
     dim3 grid((N + kRBM - 1) / kRBM, (E + kRBN - 1) / kRBN);
-    router_tc_kernel<<<grid, kRThreads, kRSmem, st>>>(maps, N, d, E, logits, err);
+    launch_pdl(router_tc_kernel, grid, kRThreads, kRSmem, st, maps, N, d, E, logits, err);
     return check_launch("router_tc");
 }
 
