@@ -136,8 +136,8 @@ def launches_per_step(cfg):
     """Kernels of this library that one moe_forward launches (mirrors abi.cu's dispatch)."""
     if cfg.N <= 256:
         if cfg.x_dtype == "bf16" and cfg.w_dtype in ("bf16", "e4m3"):
-            return 3        # fused router+top-K+permute, swap-AB FFN (up and down), combine
-        return 4            # fused router+top-K+permute, ffn up, ffn down, combine
+            return 5        # router logits, top-K, permute, swap-AB FFN (up and down), combine
+        return 6            # router logits, top-K, permute, ffn up, ffn down, combine
     router = 2 if (cfg.x_dtype == "bf16" and cfg.N >= 512) else 1   # split + tcgen05 router | SIMT router
     return router + 1 + 3 + 2 + 1   # + top-K, permute (hist, scan, scatter), ffn up, ffn down, combine
 

@@ -175,7 +175,7 @@ static kmoe_status clear_status(int *status, cudaStream_t st, size_t bytes = kSt
     return KMOE_OK;
 }
 
-constexpr int kFusedRouteTokens = 256;   // routing, top-K and dispatch in one launch up to here
+constexpr int kSmallRouteTokens = 256;   // small-batch router (bulk-copied token rows) up to here
 
 static kmoe_status check_score(int score)
 {
@@ -217,18 +217,16 @@ static kmoe_status forward_path(const void *x, int x_dtype, int N, int d, int E,
     int32_t *idx = topk_idx_out ? topk_idx_out : L.idx;
     float *w = topk_w_out ? topk_w_out : L.w;
     int32_t *counts = counts_out ? counts_out : L.counts;
-    if (N <= kFusedRouteTokens) {
-        KMOE_TRY(launch_route_small(x, x_dtype, w_router, bias, N, d, E, K, score, L.logits, idx, w, counts, L.offsets,
-                                    L.perm, L.inv, L.status, st));
-    } else {
-        if (x_dtype == KMOE_BF16 && N >= kTcRouterTokens)
-            KMOE_TRY(launch_router_tc(static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E, L.w_split, L.logits,
-                                      L.status, st));
-        else
-            KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, L.logits, st));
-        KMOE_TRY(launch_topk(L.logits, bias, N, E, K, score, idx, w, st));
-        KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st));
-    }
+    // logits, then top-K (one warp per token), then the dispatch permutation
+    if (N <= kSmallRouteTokens)
+        KMOE_TRY(launch_router_small(x, x_dtype, w_router, N, d, E, L.logits, L.status, st));
+    else if (x_dtype == KMOE_BF16 && N >= kTcRouterTokens)
+        KMOE_TRY(launch_router_tc(static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E, L.w_split, L.logits,
+                                  L.status, st));
+    else
+        KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, L.logits, st));
+    KMOE_TRY(launch_topk(L.logits, bias, N, E, K, score, idx, w, st));
+    KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st));
     const ExpertPtrs r = ptrs(routed);
     ExpertPtrs s{};
     if (shared) s = ptrs(shared);

@@ -159,11 +159,10 @@ kmoe_status launch_router_logits(const void *x, int x_dtype, const float *w_rout
 kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, int K, int score,
                         int32_t *idx, float *w, cudaStream_t st);
 
-// Router + top-K + permutation in one launch for N <= 256 (status[4] is a
-// ticket that must be zero before the launch).
-kmoe_status launch_route_small(const void *x, int x_dtype, const float *w_router, const float *bias, int N,
-                               int d, int E, int K, int score, float *logits, int32_t *idx, float *w, int32_t *counts,
-                               int32_t *offsets, int32_t *perm, int32_t *inv, int *status, cudaStream_t st);
+// Router logits for N <= 256 (128 CTAs, three experts each); status is the
+// device status word for a bounded wait that gives up.
+kmoe_status launch_router_small(const void *x, int x_dtype, const float *w_router, int N, int d, int E,
+                                float *logits, int *status, cudaStream_t st);
 
 // Tensor-core FP32 router (x in BF16): W_r split into three BF16 terms in
 // `w_split` (router_tc_ws_bytes), logits [N, E] written out.

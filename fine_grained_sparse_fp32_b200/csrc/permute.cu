@@ -76,7 +76,8 @@ scatter_kernel(const int32_t *__restrict__ idx, int N, int K, int E,
     }
 }
 
-// N <= 256: everything in one CTA (decode batches).
+// N <= 256: everything in one CTA (decode batches); W ballot-mask words per expert.
+template <int W>
 __global__ void __launch_bounds__(kChunk)
 permute_single_kernel(const int32_t *__restrict__ idx, int N, int K, int E,
                       int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
@@ -85,7 +86,7 @@ permute_single_kernel(const int32_t *__restrict__ idx, int N, int K, int E,
     pdl_wait();
     pdl_trigger();
     extern __shared__ uint32_t mask[];
-    permute_small_block(idx, N, K, E, counts, offsets, perm, inv, mask);
+    permute_small_block<W>(idx, N, K, E, counts, offsets, perm, inv, mask);
 }
 
 size_t permute_ws_bytes(int N, int E)
@@ -101,8 +102,15 @@ kmoe_status launch_permute(const int32_t *idx, int N, int K, int E, int32_t *cou
     const size_t mask_bytes = sizeof(uint32_t) * kChunkWarps * E;
     if (N <= kChunk) {
         const size_t smem = mask_bytes + sizeof(int) * E;
-        cudaFuncSetAttribute(permute_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        launch_pdl(permute_single_kernel, 1, kChunk, smem, st, idx, N, K, E, counts, offsets, perm, inv);
+        if (N <= 32) {
+            launch_pdl(permute_single_kernel<1>, 1, kChunk, sizeof(uint32_t) * 2 * E, st, idx, N, K, E, counts,
+                       offsets, perm, inv);
+        } else {
+            cudaFuncSetAttribute(permute_single_kernel<kChunkWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+            launch_pdl(permute_single_kernel<kChunkWarps>, 1, kChunk, smem, st, idx, N, K, E, counts, offsets, perm,
+                       inv);
+        }
         return check_launch("permute_single");
     }
     const int chunks = (N + kChunk - 1) / kChunk;

@@ -198,19 +198,17 @@ kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, in
     return check_launch("topk");
 }
 
-// ------------------------------------------------ fused small-batch routing
+// ------------------------------------------------- small-batch router logits
 //
-// For N <= 256 tokens (decode) the router, the top-K selection and the
-// dispatch permutation run as one launch of CTAs of 32 warps. Each CTA owns
-// kRouteEPC experts: the bulk-copy engine brings their FP32 router rows and a
-// chunk of up to 32 token rows into shared memory. Warp w handles tokens
-// 8*(w%4) .. 8*(w%4)+7 of the chunk over column part w/4 (one eighth of d),
-// four columns per lane and step, so every router weight read from shared
-// memory feeds eight tokens and no load has a bank conflict; the eight part
-// sums of a logit are added in a fixed order. The last CTA to finish (a ticket in
-// the workspace status area, zeroed before the launch) then selects the top K
-// of every token (one warp per token) and builds the permutation with 32-warp
-// ballot masks, reusing its shared memory.
+// For N <= 256 tokens (decode) the logits come from 128 CTAs of 32 warps.
+// Each CTA owns kRouteEPC experts: the bulk-copy engine brings their FP32
+// router rows and a chunk of up to 32 token rows into shared memory. Warp w
+// handles tokens 8*(w%4) .. 8*(w%4)+7 of the chunk over column part w/4 (one
+// eighth of d), four columns per lane and step, so every router weight read
+// from shared memory feeds eight tokens and no load has a bank conflict; the
+// eight part sums of a logit are added in a fixed order. Top-K and the
+// dispatch permutation follow as separate dependent launches (one warp per
+// token, then one CTA), which keeps the selection off a single SM.
 constexpr int kRouteEPC = 3;
 constexpr int kRouteThreads = 1024;
 constexpr int kRouteWarps = kRouteThreads / 32;
@@ -233,18 +231,15 @@ __device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&o)[4])
     o[2] = __uint_as_float(v.y << 16); o[3] = __uint_as_float(v.y & 0xffff0000u);
 }
 
-template <class XT, int NPL>
+template <class XT>
 __global__ void __launch_bounds__(kRouteThreads, 1)
-route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
-                   int N, int d, int E, int K, int score, int chunk, int x_off, float *__restrict__ logits,
-                   int32_t *__restrict__ idx, float *__restrict__ wout, int32_t *__restrict__ counts,
-                   int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv,
-                   int *status)
+router_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, int N, int d, int E, int chunk, int x_off,
+                    float *__restrict__ logits, int *status)
 {
     using namespace sm100;
     extern __shared__ __align__(128) uint8_t sm_raw[];
     __shared__ __align__(8) uint64_t bar;
-    __shared__ int last, abort_flag;
+    __shared__ int abort_flag;
     __shared__ float red[kRouteCQ][kRouteChunkMax][kRouteEPC];
     float *wsm = reinterpret_cast<float *>(sm_raw);
     XT *xsm = reinterpret_cast<XT *>(sm_raw + x_off);
@@ -253,7 +248,6 @@ route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tg = warp % kRouteTG, cq = warp / kRouteTG;
     const int qd = d / kRouteCQ;                     // columns per part (d % 128 == 0)
-    int *ticket = status + 4;
     if (threadIdx.x == 0) {
         mbar_init(&bar, 1);
         abort_flag = 0;
@@ -334,60 +328,31 @@ route_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, const 
         }
         __syncthreads();
     }
-    if (abort_flag) {            // a copy never landed: let it finish (bounded) and leave
-        if (threadIdx.x == 0) mbar_wait_drain(&bar, phase ^ 1, kRouteWaitLimit);
-        return;
-    }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    for (int t = warp; t < N; t += kRouteWarps)
-        topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, score, idx + (size_t)t * K, wout + (size_t)t * K);
-    __syncthreads();
-    // ballot masks only as wide as the batch: one warp's worth for decode-sized batches
-    uint32_t *mask = reinterpret_cast<uint32_t *>(sm_raw);
-    if (N <= 32) permute_small_block<1>(idx, N, K, E, counts, offsets, perm, inv, mask);
-    else permute_small_block<kChunkWarps>(idx, N, K, E, counts, offsets, perm, inv, mask);
-    if (threadIdx.x == 0) *ticket = 0;
+    if (abort_flag && threadIdx.x == 0)   // a copy never landed: let it finish (bounded) and leave
+        mbar_wait_drain(&bar, phase ^ 1, kRouteWaitLimit);
 }
 
-kmoe_status launch_route_small(const void *x, int x_dtype, const float *w_router, const float *bias, int N,
-                               int d, int E, int K, int score, float *logits, int32_t *idx, float *w, int32_t *counts,
-                               int32_t *offsets, int32_t *perm, int32_t *inv, int *status, cudaStream_t st)
+
+kmoe_status launch_router_small(const void *x, int x_dtype, const float *w_router, int N, int d, int E,
+                                float *logits, int *status, cudaStream_t st)
 {
-    if (N > kChunk) return fail(KMOE_ERR_UNSUPPORTED, "fused routing: N=%d > %d", N, kChunk);
+    if (N > kChunk) return fail(KMOE_ERR_UNSUPPORTED, "small-batch router: N=%d > %d", N, kChunk);
     const int xb = x_dtype == KMOE_F32 ? 4 : 2;
     const int w_bytes = ((kRouteEPC * d * 4) + 127) / 128 * 128;
     const int chunk = std::min(std::min(N, kRouteChunkMax), std::max(1, (kRouteSmemMax - w_bytes) / (d * xb)));
-    const size_t smem = std::max((size_t)w_bytes + (size_t)chunk * d * xb, (size_t)(kRouteWarps + 1) * E * 4);
+    const size_t smem = (size_t)w_bytes + (size_t)chunk * d * xb;
     const int grid = (E + kRouteEPC - 1) / kRouteEPC;
-    const int npl = (E + 31) / 32;
-#define KMOE_ROUTE(XT, n)                                                                                   \
-    do {                                                                                                    \
-        auto k = route_small_kernel<XT, n>;                                                                 \
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                    \
-        launch_pdl(k, grid, kRouteThreads, smem, st, static_cast<const XT *>(x), w_router, bias, N, d, E, K,  \
-                   score,                                                                                  \
-                                             chunk,                                                          \
-                                             w_bytes, logits, idx, w, counts, offsets, perm, inv, status);   \
-    } while (0)
-#define KMOE_ROUTE_X(n)                                   \
-    do {                                                  \
-        if (x_dtype == KMOE_F32) KMOE_ROUTE(float, n);    \
-        else KMOE_ROUTE(__nv_bfloat16, n);                \
-    } while (0)
-    if (npl <= 2) KMOE_ROUTE_X(2);
-    else if (npl <= 4) KMOE_ROUTE_X(4);
-    else if (npl <= 8) KMOE_ROUTE_X(8);
-    else if (npl <= 12) KMOE_ROUTE_X(12);
-    else if (npl <= 16) KMOE_ROUTE_X(16);
-    else KMOE_ROUTE_X(32);
-#undef KMOE_ROUTE_X
-#undef KMOE_ROUTE
-    return check_launch("route_small");
+    if (x_dtype == KMOE_F32) {
+        cudaFuncSetAttribute(router_small_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        launch_pdl(router_small_kernel<float>, grid, kRouteThreads, smem, st, static_cast<const float *>(x), w_router,
+                   N, d, E, chunk, w_bytes, logits, status);
+    } else {
+        cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        launch_pdl(router_small_kernel<__nv_bfloat16>, grid, kRouteThreads, smem, st,
+                   static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E, chunk, w_bytes, logits, status);
+    }
+    return check_launch("router_small");
 }
 
 }  // namespace kmoe
