@@ -139,7 +139,9 @@ def launches_per_step(cfg):
             return 5        # router logits, top-K, permute, swap-AB FFN (up and down), combine
         return 6            # router logits, top-K, permute, ffn up, ffn down, combine
     router = 2 if (cfg.x_dtype == "bf16" and cfg.N >= 512) else 1   # split + tcgen05 router | SIMT router
-    return router + 1 + 3 + 2 + 1   # + top-K, permute (hist, scan, scatter), ffn up, ffn down, combine
+    chunks = (cfg.N + 255) // 256
+    permute = 1 if chunks <= 64 else 2      # scatter with the scan folded in | scan, scatter (top-K counts)
+    return router + 1 + permute + 2 + 1     # + top-K, permute, ffn up, ffn down, combine
 
 
 # --------------------------------------------------------------- GPU arm

@@ -176,6 +176,7 @@ static kmoe_status clear_status(int *status, cudaStream_t st, size_t bytes = kSt
 }
 
 constexpr int kSmallRouteTokens = 256;   // small-batch router (bulk-copied token rows) up to here
+constexpr int kChunkTokens = 256;        // the dispatch works in chunks of this many tokens
 
 static kmoe_status check_score(int score)
 {
@@ -217,7 +218,11 @@ static kmoe_status forward_path(const void *x, int x_dtype, int N, int d, int E,
     int32_t *idx = topk_idx_out ? topk_idx_out : L.idx;
     float *w = topk_w_out ? topk_w_out : L.w;
     int32_t *counts = counts_out ? counts_out : L.counts;
-    // logits, then top-K (one warp per token), then the dispatch permutation
+    // logits, then top-K (one warp per token), then the dispatch permutation;
+    // above one chunk the top-K kernel also counts the chunk histograms
+    const bool chunked = N > kChunkTokens;
+    if (chunked && cudaMemsetAsync(L.hist, 0, permute_ws_bytes(N, E), st) != cudaSuccess)
+        return check_launch("histogram memset");
     if (N <= kSmallRouteTokens)
         KMOE_TRY(launch_router_small(x, x_dtype, w_router, N, d, E, L.logits, L.status, st));
     else if (x_dtype == KMOE_BF16 && N >= kTcRouterTokens)
@@ -225,8 +230,8 @@ static kmoe_status forward_path(const void *x, int x_dtype, int N, int d, int E,
                                   L.status, st));
     else
         KMOE_TRY(launch_router_logits(x, x_dtype, w_router, N, d, E, L.logits, st));
-    KMOE_TRY(launch_topk(L.logits, bias, N, E, K, score, idx, w, st));
-    KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st));
+    KMOE_TRY(launch_topk(L.logits, bias, N, E, K, score, idx, w, st, chunked ? L.hist : nullptr));
+    KMOE_TRY(launch_permute(idx, N, K, E, counts, L.offsets, L.perm, L.inv, L.hist, st, chunked));
     const ExpertPtrs r = ptrs(routed);
     ExpertPtrs s{};
     if (shared) s = ptrs(shared);

@@ -156,8 +156,10 @@ namespace kmoe {
 
 kmoe_status launch_router_logits(const void *x, int x_dtype, const float *w_router, int N, int d,
                                  int E, float *logits, cudaStream_t st);
+// hist (may be NULL): per-chunk expert histogram [ceil(N / 256), E], zero on
+// entry, counted by the top-K kernel for the dispatch that follows.
 kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, int K, int score,
-                        int32_t *idx, float *w, cudaStream_t st);
+                        int32_t *idx, float *w, cudaStream_t st, int32_t *hist = nullptr);
 
 // Router logits for N <= 256 (128 CTAs, three experts each); status is the
 // device status word for a bounded wait that gives up.
@@ -172,9 +174,11 @@ kmoe_status launch_router_tc(const __nv_bfloat16 *x, const float *w_router, int 
 constexpr int kTcRouterTokens = 512;
 
 size_t permute_ws_bytes(int N, int E);
+// hist_ready: hist already holds the chunk histograms (counted by the top-K
+// kernel), so the histogram pass is skipped.
 kmoe_status launch_permute(const int32_t *idx, int N, int K, int E, int32_t *counts,
                            int32_t *offsets, int32_t *perm, int32_t *inv, int32_t *hist,
-                           cudaStream_t st);
+                           cudaStream_t st, bool hist_ready = false);
 
 kmoe_status launch_ffn_stream(const void *x, int x_dtype, int N, int d, int I, int E, int K,
                               const int32_t *perm, const int32_t *offsets, int w_dtype,

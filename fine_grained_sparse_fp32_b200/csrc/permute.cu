@@ -76,6 +76,61 @@ scatter_kernel(const int32_t *__restrict__ idx, int N, int K, int E,
     }
 }
 
+// Pass 3 with the scan folded in, for up to kScanChunks chunks: every CTA
+// sums the chunk histograms itself, in chunk order (the same sums the scan
+// pass forms), so no separate scan launch is needed; CTA 0 also writes
+// counts and offsets.
+constexpr int kScanChunks = 64;
+
+__global__ void __launch_bounds__(kChunk)
+scatter_scan_kernel(const int32_t *__restrict__ idx, int N, int K, int E, int chunks,
+                    const int32_t *__restrict__ hist, int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                    int32_t *__restrict__ perm, int32_t *__restrict__ inv)
+{
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ uint32_t mask[];               // kChunkWarps * E ballot words, then E row bases
+    int *base = reinterpret_cast<int *>(mask + kChunkWarps * E);
+    __shared__ int tmp[32];
+    __shared__ int round_total;
+    const int c = blockIdx.x;
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+        const int e = e0 + threadIdx.x;
+        int total = 0, before = 0;
+        if (e < E)
+            for (int q = 0; q < chunks; ++q) {
+                const int v = hist[(size_t)q * E + e];
+                before += q < c ? v : 0;
+                total += v;
+            }
+        const int excl = block_exclusive_scan(e < E ? total : 0, tmp);
+        if (e < E) {
+            base[e] = carry + excl + before;
+            if (c == 0) {
+                counts[e] = total;
+                offsets[e] = carry + excl;
+            }
+        }
+        if (threadIdx.x == blockDim.x - 1) round_total = excl + total;
+        __syncthreads();
+        carry += round_total;
+        __syncthreads();
+    }
+    if (c == 0 && threadIdx.x == 0) offsets[E] = carry;
+    build_masks(idx, N, K, E, c, mask);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = c * kChunk + threadIdx.x;
+    if (t >= N) return;
+    for (int k = 0; k < K; ++k) {
+        const int e = idx[(size_t)t * K + k];
+        if ((unsigned)e >= (unsigned)E) continue;
+        const int pos = base[e] + rank_in_chunk(mask, E, e, warp, lane);
+        perm[pos] = t;
+        inv[(size_t)t * K + k] = pos;
+    }
+}
+
 // N <= 256: everything in one CTA (decode batches); W ballot-mask words per expert.
 template <int W>
 __global__ void __launch_bounds__(kChunk)
@@ -97,7 +152,7 @@ size_t permute_ws_bytes(int N, int E)
 
 kmoe_status launch_permute(const int32_t *idx, int N, int K, int E, int32_t *counts,
                            int32_t *offsets, int32_t *perm, int32_t *inv, int32_t *hist,
-                           cudaStream_t st)
+                           cudaStream_t st, bool hist_ready)
 {
     const size_t mask_bytes = sizeof(uint32_t) * kChunkWarps * E;
     if (N <= kChunk) {
@@ -114,11 +169,21 @@ kmoe_status launch_permute(const int32_t *idx, int N, int K, int E, int32_t *cou
         return check_launch("permute_single");
     }
     const int chunks = (N + kChunk - 1) / kChunk;
+    if (hist_ready && chunks <= kScanChunks) {
+        const size_t smem = mask_bytes + sizeof(int) * E;
+        cudaFuncSetAttribute(scatter_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        launch_pdl(scatter_scan_kernel, chunks, kChunk, smem, st, idx, N, K, E, chunks,
+                   static_cast<const int32_t *>(hist), counts, offsets, perm, inv);
+        return check_launch("permute_scatter_scan");
+    }
     cudaFuncSetAttribute(chunk_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mask_bytes);
     cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mask_bytes);
-    launch_pdl(chunk_hist_kernel, chunks, kChunk, mask_bytes, st, idx, N, K, E, hist);
-    kmoe_status s = check_launch("permute_hist");
-    if (s != KMOE_OK) return s;
+    kmoe_status s;
+    if (!hist_ready) {
+        launch_pdl(chunk_hist_kernel, chunks, kChunk, mask_bytes, st, idx, N, K, E, hist);
+        s = check_launch("permute_hist");
+        if (s != KMOE_OK) return s;
+    }
     launch_pdl(scan_kernel, 1, 1024, 0, st, hist, chunks, E, counts, offsets);
     s = check_launch("permute_scan");
     if (s != KMOE_OK) return s;

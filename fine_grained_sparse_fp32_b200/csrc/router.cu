@@ -109,7 +109,7 @@ __device__ __forceinline__ int score_key(float s)
 // a softmax over the K ("Kolibri 1 Deep Dive", routing formulation).
 template <int NPL>
 __device__ __forceinline__ void topk_warp(const float *lr, const float *__restrict__ bias, int E, int K, int score,
-                                          int32_t *idx_row, float *w_row)
+                                          int32_t *idx_row, float *w_row, int32_t *hist_row = nullptr)
 {
     // Unbiased logits of the chosen experts (K <= 8). Up to 512 experts they
     // travel with their scores through the selection; beyond that lane 0
@@ -144,7 +144,10 @@ __device__ __forceinline__ void topk_warp(const float *lr, const float *__restri
         for (int i = 0; i < NPL; ++i)
             if (i * 32 + lane == me) key[i] = INT_MIN;
         lsel[k] = kCarry ? wl : (lane == 0 ? __ldcg(lr + e) : 0.f);
-        if (lane == 0) idx_row[k] = e;
+        if (lane == 0) {
+            idx_row[k] = e;
+            if (hist_row) atomicAdd(hist_row + e, 1);   // integer counts: exact in any order
+        }
     }
     if (lane == 0) {
         if (score == KMOE_SCORE_SOFTMAX) {
@@ -172,22 +175,23 @@ __device__ __forceinline__ void topk_warp(const float *lr, const float *__restri
 template <int NPL>
 __global__ void __launch_bounds__(256)
 topk_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int N, int E, int K, int score,
-            int32_t *__restrict__ idx, float *__restrict__ wout)
+            int32_t *__restrict__ idx, float *__restrict__ wout, int32_t *__restrict__ hist)
 {
     pdl_wait();
     pdl_trigger();
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= N) return;
-    topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, score, idx + (size_t)t * K, wout + (size_t)t * K);
+    topk_warp<NPL>(logits + (size_t)t * E, bias, E, K, score, idx + (size_t)t * K, wout + (size_t)t * K,
+                   hist ? hist + (size_t)(t / kChunk) * E : nullptr);
 }
 
 kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, int K, int score,
-                        int32_t *idx, float *w, cudaStream_t st)
+                        int32_t *idx, float *w, cudaStream_t st, int32_t *hist)
 {
     const int warps = 8;
     dim3 grid((N + warps - 1) / warps);
     const int npl = (E + 31) / 32;
-#define KMOE_TOPK(n) launch_pdl(topk_kernel<n>, grid, warps * 32, 0, st, logits, bias, N, E, K, score, idx, w)
+#define KMOE_TOPK(n) launch_pdl(topk_kernel<n>, grid, warps * 32, 0, st, logits, bias, N, E, K, score, idx, w, hist)
     if (npl <= 2) KMOE_TOPK(2);
     else if (npl <= 4) KMOE_TOPK(4);
     else if (npl <= 8) KMOE_TOPK(8);
