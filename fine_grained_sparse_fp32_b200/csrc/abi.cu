@@ -419,6 +419,7 @@ kmoe_status moe_block_forward(const void *h, int N, int d, int E, int K, int I, 
     if (routed->dtype != KMOE_BF16 && routed->dtype != KMOE_E4M3_B128)
         return fail(KMOE_ERR_UNSUPPORTED, "block: routed weights must be BF16 or E4M3 with 128x128 scales");
     if (!(eps >= 0.f) || eps > 1.f) return fail(KMOE_ERR_INVALID_ARG, "eps=%g: must be in [0, 1]", (double)eps);
+    if (d % 256) return fail(KMOE_ERR_UNSUPPORTED, "block: d=%d must be a multiple of 256", d);
     const size_t row_smem = (size_t)(K + (shared ? 1 : 0)) * d * 2;
     if (2 * row_smem > 100 * 1024)
         return fail(KMOE_ERR_UNSUPPORTED, "block: (K + 1) * d = %zu BF16 values per token exceed the combine's "

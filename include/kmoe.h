@@ -223,7 +223,7 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
  * before its h_out element is written, by the same thread) but must not
  * overlap it otherwise. x_out: optional device [N, d] BF16 output of the
  * normalised layer input x (NULL keeps it in the workspace). Routed (and shared) weights must be BF16 or E4M3
- * with 128 x 128 scales (KMOE_ERR_UNSUPPORTED otherwise), and
+ * with 128 x 128 scales and d a multiple of 256 (KMOE_ERR_UNSUPPORTED otherwise), and
  * (K + 1) * d <= 25600 BF16 values must fit the combine's staging buffer
  * (K + 1 counts the shared expert). Other arguments and outputs as in
  * moe_forward. ws: at least moe_block_workspace_size() bytes; its first 4

@@ -143,3 +143,11 @@ def test_block_forward_checks_arguments_on_the_host(lib):
     small = lib.moe_block_forward(a, 32, 2560, 384, 6, 512, 0, a, a, 1e-6, a, a, ctypes.byref(bf), None, a,
                                   None, None, None, None, a, 1024, None)
     assert small == kmoe.KMOE_ERR_WORKSPACE
+
+
+def test_block_forward_needs_d_multiple_of_256(lib):
+    a = ctypes.c_void_p(1 << 20)
+    bf = kmoe.Experts(a, a, a, None, None, None, kmoe.KMOE_BF16)
+    st = lib.moe_block_forward(a, 32, 2688, 384, 6, 512, 0, a, a, 1e-6, a, a, ctypes.byref(bf), ctypes.byref(bf), a,
+                               None, None, None, None, a, 1 << 40, None)
+    assert st == kmoe.KMOE_ERR_UNSUPPORTED and b"256" in lib.moe_last_error()
