@@ -7,7 +7,10 @@
 // is a pure function of the indices, so every output is bit-exact and
 // independent of scheduling: no atomics decide a position. Per-chunk
 // ballot masks (permute_dev.cuh) give chunk histograms and in-chunk ranks;
-// chunk histograms are scanned per expert in chunk order.
+// chunk histograms are scanned per expert in chunk order. Inside a layer
+// call the top-K kernel counts the chunk histograms instead (integer
+// atomics, exact in any order), and up to 64 chunks the scatter kernel
+// forms the scan itself.
 #include "permute_dev.cuh"
 
 namespace kmoe {
