@@ -29,7 +29,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from fine_grained_sparse_fp32_b200 import _build, kmoe  # noqa: E402
-from fine_grained_sparse_fp32_b200.inputs import CONFIGS, make_block_inputs, make_inputs, make_x  # noqa: E402
+from fine_grained_sparse_fp32_b200.inputs import (CONFIGS, expected_distinct_experts, make_block_inputs,  # noqa: E402
+                                                  make_inputs, make_x)
 
 METRIC = "MoE-layer tokens/s at 1 B200 (decode N=32, prefill N=8192); % of HBM/tensor roofline"
 ROTATE = 8           # distinct token batches cycled through the timed steps
@@ -420,11 +421,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "decode layer N=32 d=2560 E=384 top-6+1 shared I=512, BF16 experts, FP32 router",
-                       "tokens_per_gpu": dec.N, "parallelism": f"replicas x{world} (no collective)",
-                       "l2": "inputs larger than L2: ~%.2f GB of expert weights per step, %d rotating token batches"
-                             % (alg["expert_weight_bytes"] / 1e9, ROTATE),
-                       "cuda_graph": (f"{ROTATE} consecutive layer calls per graph" if not args.no_graph else False)},
+            "config": decode_config(world, args.no_graph),
             "roofline": {"bound": "hbm", "kernel": "moe_grouped_ffn: ffn_swap_kernel (up and down units, one launch)",
                          "achieved": ffn_gbs, "peak": hbm, "unit": "GB/s", "frac": ffn_gbs / hbm,
                          "traffic": kernel_traffic("decode"), "peak_kind": peak_kind + " burst",
@@ -504,6 +501,17 @@ def run_capture(name, calls):
         raise SystemExit(f"device status {status}")
 
 
+def decode_config(world, no_graph=False):
+    """The workload description both arms report (the GPU arm and the oracle)."""
+    cfg = CONFIGS["decode"]
+    w = algorithmic(cfg, expected_distinct_experts(cfg))["expert_weight_bytes"]
+    return {"workload": "decode layer N=32 d=2560 E=384 top-6+1 shared I=512, BF16 experts, FP32 router",
+            "tokens_per_gpu": cfg.N, "parallelism": f"replicas x{world} (no collective)",
+            "l2": "inputs larger than L2: ~%.2f GB of expert weights per step (expected), %d rotating token "
+                  "batches" % (w / 1e9, ROTATE),
+            "cuda_graph": (f"{ROTATE} consecutive layer calls per graph" if not no_graph else False)}
+
+
 def run_reference(args, world, rank):
     """The oracle on the host cores, on this arm's metric and workload."""
     if rank != 0:
@@ -517,7 +525,8 @@ def run_reference(args, world, rank):
     sample = max(1, min(cfg.N, 1600 // max(args.steps, 1)))
     rows = np.arange(sample, dtype=np.int32)
     nt = min(oracle.max_threads(), sample)
-    oracle.layer(host, rows=rows[:1], nthreads=1)
+    for _ in range(args.warmup):
+        oracle.layer(host, rows=rows, nthreads=nt)
     times = []
     for _ in range(args.steps):
         t = time.perf_counter()
@@ -528,7 +537,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": len(times), "warmup": args.warmup, "ms_per_step": per_token * cfg.N * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "decode layer N=32 d=2560 E=384 top-6+1 shared I=512, BF16 experts, FP32 router"},
+            "config": decode_config(world, args.no_graph),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nt, "kind": "oracle",
                              "sample": f"{sample} of the {cfg.N} decode tokens per step, whole layer in double"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
