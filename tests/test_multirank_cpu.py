@@ -56,3 +56,25 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.all_max(1.5, 1) == 1.5
     assert bench.whole_job_tokens_per_s(32, 1, 0.5) == pytest.approx(64000.0)
+
+
+def test_launch_counts_follow_the_dispatch_in_abi():
+    """gpu_launches is a claim: one layer call launches exactly these kernels (abi.cu forward_path)."""
+    import bench
+    from fine_grained_sparse_fp32_b200.inputs import CONFIGS
+    # router logits, top-K, dispatch (one CTA), swap-AB FFN, combine
+    assert bench.launches_per_step(CONFIGS["decode"]) == 5
+    assert bench.launches_per_step(CONFIGS["fp8_decode"]) == 5
+    # FP32 tiny layer: router logits, top-K, dispatch, streaming FFN up + down, combine
+    assert bench.launches_per_step(CONFIGS["tiny"]) == 6
+    # split + tensor-core router, top-K (with chunk histograms), scatter with the scan, FFN up + down, combine
+    assert bench.launches_per_step(CONFIGS["prefill"]) == 7
+    assert bench.launches_per_step(CONFIGS["fp8_prefill"]) == 7
+    # more than 64 chunks: scan and scatter are separate launches
+    assert bench.launches_per_step(CONFIGS["skew"]) == 8
+
+
+def test_both_bench_arms_report_the_same_workload():
+    import bench
+    a, b = bench.decode_config(1), bench.decode_config(1)
+    assert a == b and a["tokens_per_gpu"] == 32 and "GB of expert weights" in a["l2"]
