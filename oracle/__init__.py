@@ -42,6 +42,8 @@ def lib():
         _lib = ctypes.CDLL(build())
         _lib.oracle_e4m3_to_double.restype = ctypes.c_double
         _lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        _lib.oracle_float_to_e4m3.restype = ctypes.c_uint8
+        _lib.oracle_float_to_e4m3.argtypes = [ctypes.c_float]
         _lib.oracle_permute.restype = ctypes.c_int
         _lib.oracle_max_threads.restype = ctypes.c_int
     return _lib
@@ -186,5 +188,47 @@ def block(inp, h, gamma_pre, gamma_post, eps: float, rows=None, nthreads: int = 
     return {"h_out": h_out, "x": x, "m": m, "idx": ora["idx"], "g": ora["g"], "margin": ora["margin"], "rows": rws}
 
 
+def float_to_e4m3(values) -> np.ndarray:
+    """E4M3 codes (round to nearest even, saturated to +-448) of float32 values."""
+    v = np.asarray(values, dtype=np.float32).ravel()
+    return np.array([lib().oracle_float_to_e4m3(float(x)) for x in v], dtype=np.uint8).reshape(np.shape(values))
+
+
+def quant_1x128(x):
+    """Dynamic FP8 quantisation of BF16 rows in groups of 128 columns.
+
+    Returns (codes uint8 [rows, cols], scales float32 [rows, cols / 128])."""
+    xb = np.ascontiguousarray(_bits(x), dtype=np.uint16)
+    rows, cols = xb.shape
+    codes = np.empty((rows, cols), dtype=np.uint8)
+    scales = np.empty((rows, cols // 128), dtype=np.float32)
+    lib().oracle_quant_1x128(rows, cols, _p(xb), _p(codes), _p(scales))
+    return codes, scales
+
+
+def layer_a8(inp, rows=None, nthreads: int = 1, score: str = "sigmoid"):
+    """The layer with E4M3 weights and activations quantised in 1 x 128 groups (x for
+    gate/up, H for down); routing on x as stored. Returns dict(y, idx, g, margin, rows)."""
+    cfg = inp["cfg"]
+    if cfg.w_dtype != "e4m3" or cfg.x_dtype != "bf16":
+        raise ValueError("FP8 activations need BF16 x and E4M3 weights")
+    xb = np.ascontiguousarray(_bits(inp["x"]), dtype=np.uint16)
+    N = xb.shape[0]
+    rows = np.arange(N, dtype=np.int32) if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    wr = np.ascontiguousarray(_bits(inp["w_router"]), dtype=np.float32)
+    b = np.ascontiguousarray(_bits(inp["bias"]), dtype=np.float32)
+    wg, wu, wd, sg, su, sd = _weights(inp)
+    n = len(rows)
+    y = np.empty((n, cfg.d), dtype=np.float64)
+    idx = np.empty((n, cfg.K), dtype=np.int32)
+    g = np.empty((n, cfg.K), dtype=np.float64)
+    margin = np.empty(n, dtype=np.float64)
+    lib().oracle_layer_a8(N, cfg.d, cfg.E, cfg.K, cfg.I, _p(xb), _p(wr), _p(b), _p(wg), _p(wu), _p(wd),
+                          _p(sg), _p(su), _p(sd), n, _p(rows), SCORES[score], _p(y), _p(idx), _p(g), _p(margin),
+                          nthreads)
+    return {"y": y, "idx": idx, "g": g, "margin": margin, "rows": rows}
+
+
 __all__ = ["build", "lib", "max_threads", "e4m3_to_double", "router_logits", "select",
-           "permute", "expert_outputs", "layer", "rmsnorm_bf16", "block", "F32", "BF16", "E4M3"]
+           "permute", "expert_outputs", "layer", "rmsnorm_bf16", "block", "float_to_e4m3", "quant_1x128",
+           "layer_a8", "F32", "BF16", "E4M3"]

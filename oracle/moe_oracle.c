@@ -34,8 +34,8 @@
  *
  * Parity pins: every function here is pinned by the CPU tests in
  * tests/test_oracle.py (brute-force top-k, library sort, numpy float64
- * matmul, the 256 E4M3 codes against torch, closed forms and hand-computed
- * cases).
+ * matmul, the 256 E4M3 codes and the E4M3 encoder against torch, closed
+ * forms and hand-computed cases).
  */
 #include <math.h>
 #include <stdint.h>
@@ -391,5 +391,159 @@ void oracle_post_residual(int N, int d, int n_rows, const int32_t *rows, const u
         for (int j = 0; j < d; ++j)
             h_out[r * d + j] = bf16_bits_to_double(h[(int64_t)rows[r] * d + j]) + m[r * d + j] * s *
                                bf16_bits_to_double(g_post[j]);
+    }
+}
+
+/* ----------------------------------------------------------------------
+ * FP8 activations ("Inside Kolibri 1", section "The FP8 path is explicitly
+ * mixed precision": activations are quantised dynamically in groups of
+ * 1 x 128; the weights are E4M3 in 128 x 128 blocks with FP32 scales).
+ *
+ * Readings where the page is silent:
+ *   - a group is 128 consecutive columns of one row of a GEMM input (x for
+ *     the gate and up projections, H for the down projection);
+ *   - its scale is s = amax / 448 in FP32 (448 = the largest E4M3 value),
+ *     s = 1 for an all-zero group, used as computed (never rounded to 2^k,
+ *     like the weight scales);
+ *   - a code is E4M3(v), v = x / s computed in FP32, rounded to nearest with
+ *     ties to even and saturated to +-448; the code decision is taken in
+ *     FP32, the precision a kernel computes it in;
+ *   - H is rounded to BF16 before it is quantised, as the layer stores H;
+ *   - the GEMMs are exact: for each 128-column block kb,
+ *       out += s_act[kb] * s_w[kb] * sum_k E4M3(q_act[k]) * E4M3(q_w[k]),
+ *     summed in index order in double.
+ * ---------------------------------------------------------------------- */
+
+/* E4M3 code of a finite float: round to nearest, ties to even, saturate to
+ * +-448. Codes: sign bit 7, exponent bits 6..3 (bias 7; 0 = subnormal),
+ * mantissa bits 2..0; subnormals are m * 2^-9. */
+uint8_t oracle_float_to_e4m3(float v)
+{
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs((double)v);
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -6)) {                          /* below the smallest normal: quantum 2^-9 */
+        const double m = nearbyint(ldexp(a, 9));       /* 0 .. 8; 8 is the smallest normal 2^-6 */
+        return (uint8_t)(sign | (uint8_t)m);
+    }
+    int e;
+    frexp(a, &e);                                      /* a = f * 2^e, 0.5 <= f < 1: a in [2^(e-1), 2^e) */
+    int ex = e - 1;                                    /* unbiased exponent, ex >= -6 */
+    double m = nearbyint(ldexp(a, 3 - ex));            /* significand in eighths: 8 .. 16 */
+    if (m == 16.0) {
+        m = 8.0;
+        ex += 1;
+    }
+    if (ex > 8 || (ex == 8 && m > 14.0)) return (uint8_t)(sign | 0x7E);   /* saturate: 1.75 * 2^8 = 448 */
+    return (uint8_t)(sign | (uint8_t)((ex + 7) << 3) | (uint8_t)(m - 8.0));
+}
+
+/* Quantises `rows` rows of `cols` BF16 values in groups of 128 columns:
+ * codes [rows, cols], scales [rows, cols / 128]. */
+void oracle_quant_1x128(int rows, int cols, const uint16_t *x, uint8_t *codes, float *scales)
+{
+    const int groups = cols / OR_BLOCK;
+    for (int r = 0; r < rows; ++r)
+        for (int g = 0; g < groups; ++g) {
+            const int64_t base = (int64_t)r * cols + (int64_t)g * OR_BLOCK;
+            float amax = 0.0f;
+            for (int k = 0; k < OR_BLOCK; ++k) {
+                const float v = fabsf((float)bf16_bits_to_double(x[base + k]));
+                if (v > amax) amax = v;
+            }
+            const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+            scales[(int64_t)r * groups + g] = s;
+            for (int k = 0; k < OR_BLOCK; ++k)
+                codes[base + k] = oracle_float_to_e4m3((float)bf16_bits_to_double(x[base + k]) / s);
+        }
+}
+
+/* One SwiGLU expert `g` (E4M3 weights) on one token whose row is quantised:
+ * xq [d] codes with xs [d / 128] scales. H is formed in double, rounded to
+ * BF16, quantised in 1 x 128 groups, and the down projection runs on those
+ * codes. `hb` (I BF16), `hq` (I codes), `hs` (I / 128 scales) are scratch. */
+static void expert_ffn_a8(int d, int I, const uint8_t *xq, const float *xs, int64_t g,
+                          const uint8_t *wg, const uint8_t *wu, const uint8_t *wd,
+                          const float *sg, const float *su, const float *sd,
+                          uint16_t *hb, uint8_t *hq, float *hs, double *out)
+{
+    const int db = d / OR_BLOCK, ib = I / OR_BLOCK;
+    for (int i = 0; i < I; ++i) {
+        double a = 0.0, b = 0.0;
+        for (int kb = 0; kb < db; ++kb) {
+            double pa = 0.0, pb = 0.0;
+            for (int k = kb * OR_BLOCK; k < (kb + 1) * OR_BLOCK; ++k) {
+                const double xv = oracle_e4m3_to_double(xq[k]);
+                const int64_t wi = (g * I + i) * (int64_t)d + k;
+                pa += xv * oracle_e4m3_to_double(wg[wi]);
+                pb += xv * oracle_e4m3_to_double(wu[wi]);
+            }
+            const int64_t si = (g * ib + i / OR_BLOCK) * (int64_t)db + kb;
+            a += (double)xs[kb] * (double)sg[si] * pa;
+            b += (double)xs[kb] * (double)su[si] * pb;
+        }
+        hb[i] = double_to_bf16_rne(a * sigmoid(a) * b);
+    }
+    oracle_quant_1x128(1, I, hb, hq, hs);
+    for (int j = 0; j < d; ++j) {
+        double acc = 0.0;
+        for (int kb = 0; kb < ib; ++kb) {
+            double p = 0.0;
+            for (int k = kb * OR_BLOCK; k < (kb + 1) * OR_BLOCK; ++k)
+                p += oracle_e4m3_to_double(hq[k]) * oracle_e4m3_to_double(wd[(g * d + j) * (int64_t)I + k]);
+            acc += (double)hs[kb] * (double)sd[(g * db + j / OR_BLOCK) * (int64_t)ib + kb] * p;
+        }
+        out[j] = acc;
+    }
+}
+
+/* The whole layer with FP8 activations, for tokens rows[0 .. n_rows-1]:
+ * the router and the top-K see x as stored (BF16); each expert sees x
+ * quantised in 1 x 128 groups, and its down projection sees H quantised the
+ * same way. E4M3 weights only. Outputs as oracle_layer_score. */
+void oracle_layer_a8(int N, int d, int E, int K, int I,
+                     const uint16_t *x, const float *w_router, const float *bias,
+                     const uint8_t *wg, const uint8_t *wu, const uint8_t *wd,
+                     const float *sg, const float *su, const float *sd,
+                     int n_rows, const int32_t *rows, int score,
+                     double *y, int32_t *idx_out, double *g_out, double *margin_out, int nthreads)
+{
+    int r;
+    (void)N;
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic)
+    for (r = 0; r < n_rows; ++r) {
+        const int64_t t = rows[r];
+        double *l = (double *)malloc((size_t)E * sizeof(double));
+        double *f = (double *)malloc((size_t)d * sizeof(double));
+        uint8_t *xq = (uint8_t *)malloc((size_t)d);
+        float *xs = (float *)malloc((size_t)(d / OR_BLOCK) * sizeof(float));
+        uint16_t *hb = (uint16_t *)malloc((size_t)I * sizeof(uint16_t));
+        uint8_t *hq = (uint8_t *)malloc((size_t)I);
+        float *hs = (float *)malloc((size_t)(I / OR_BLOCK) * sizeof(float));
+        double *yr = y + (int64_t)r * d;
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j)
+                acc += bf16_bits_to_double(x[t * d + j]) * (double)w_router[(int64_t)e * d + j];
+            l[e] = acc;
+        }
+        oracle_select_score(1, E, K, l, bias, score, idx_out + (int64_t)r * K, g_out + (int64_t)r * K,
+                            margin_out + r);
+        oracle_quant_1x128(1, d, x + t * d, xq, xs);
+        expert_ffn_a8(d, I, xq, xs, E, wg, wu, wd, sg, su, sd, hb, hq, hs, yr);
+        for (int k = 0; k < K; ++k) {
+            const int e = idx_out[(int64_t)r * K + k];
+            const double gk = g_out[(int64_t)r * K + k];
+            expert_ffn_a8(d, I, xq, xs, e, wg, wu, wd, sg, su, sd, hb, hq, hs, f);
+            for (int j = 0; j < d; ++j)
+                yr[j] += gk * f[j];
+        }
+        free(hs);
+        free(hq);
+        free(hb);
+        free(xs);
+        free(xq);
+        free(f);
+        free(l);
     }
 }

@@ -328,3 +328,102 @@ def test_layer_shape_matches_printed_weight_counts():
     assert cfg.E + 1 == g["experts_total_per_block"]
     assert round((cfg.K + 1) * cfg.expert_weights / 1e5) / 10 == g["touched_per_token_per_block"] / 1e6
     assert round((cfg.E + 1) * cfg.expert_weights / 1e7) / 100 == g["all_experts_per_block"] / 1e9
+
+
+# ------------------------------------------------ FP8 activations (1 x 128)
+# "Inside Kolibri 1", section "The FP8 path is explicitly mixed precision":
+# activations are quantised dynamically in groups of 1 x 128.
+
+def _e4m3_values(codes):
+    return np.array([oracle.e4m3_to_double(int(c)) for c in np.ravel(codes)]).reshape(np.shape(codes))
+
+
+def test_float_to_e4m3_matches_torch_rounding():
+    """Round to nearest even on the E4M3 grid, the same codes as torch's float8_e4m3fn cast."""
+    rng = np.random.default_rng(11)
+    v = np.concatenate([rng.uniform(-448, 448, 4000), rng.normal(0, 1, 4000), rng.normal(0, 2 ** -7, 2000),
+                        rng.uniform(-2 ** -6, 2 ** -6, 2000)]).astype(np.float32)
+    ours = oracle.float_to_e4m3(v)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_float_to_e4m3_round_trips_midpoints_and_saturates():
+    finite = [c for c in range(256) if (c & 0x7F) != 0x7F]
+    for c in finite:                                   # every finite code decodes and re-encodes to itself
+        assert int(oracle.float_to_e4m3(np.float32(oracle.e4m3_to_double(c)))) == c
+    for c in range(0, 0x7E):                           # halfway between neighbours: the even mantissa wins
+        lo, hi = oracle.e4m3_to_double(c), oracle.e4m3_to_double(c + 1)
+        want = c if c % 2 == 0 else c + 1
+        assert int(oracle.float_to_e4m3(np.float32((lo + hi) / 2))) == want
+    assert oracle.float_to_e4m3(np.float32([470.0, -1e6, 448.0])).tolist() == [0x7E, 0xFE, 0x7E]
+
+
+def test_quant_1x128_exact_groups_and_error_bound():
+    rng = np.random.default_rng(12)
+    # groups built as E4M3 values times 2^k with one element at +-448: quantised exactly, scale 2^k
+    codes = rng.integers(0, 0x7E, size=(3, 384)).astype(np.uint8) | (rng.integers(0, 2, size=(3, 384)) << 7).astype(np.uint8)
+    codes[:, ::128] = 0x7E
+    k = rng.integers(-8, 3, size=(3, 3))
+    vals = _e4m3_values(codes) * np.repeat(2.0 ** k, 128, axis=1)
+    q, s = oracle.quant_1x128(_bf16_bits(vals))
+    assert np.array_equal(s, (2.0 ** k).astype(np.float32))
+    assert np.array_equal(_e4m3_values(q), _e4m3_values(codes))
+    # random BF16 rows: each group's largest magnitude maps to +-448, every value within half an E4M3 step
+    x = _bf16_bits(rng.normal(0, 1.5, size=(4, 256)))
+    xv = _bf16_values(x)
+    q, s = oracle.quant_1x128(x)
+    deq = _e4m3_values(q) * np.repeat(s.astype(np.float64), 128, axis=1)
+    for r in range(4):
+        for g in range(2):
+            seg = slice(128 * g, 128 * g + 128)
+            j = int(np.argmax(np.abs(xv[r, seg])))
+            assert int(q[r, seg][j]) & 0x7F == 0x7E
+    bound = np.maximum(np.abs(xv) * 2.0 ** -4, np.repeat(s.astype(np.float64), 128, axis=1) * 2.0 ** -10)
+    assert np.all(np.abs(deq - xv) <= bound * (1 + 1e-6))
+    zq, zs = oracle.quant_1x128(_bf16_bits(np.zeros((1, 128))))
+    assert zs.tolist() == [[1.0]] and not zq.any()
+
+
+def _a8_layer(d=256, I=128, E=8, K=2, N=6, seed=3):
+    cfg = LayerConfig("a8", N, d, E, K, I, "bf16", "e4m3")
+    return make_inputs(cfg, seed=seed)
+
+
+def test_layer_a8_routes_like_the_bf16_layer_and_stays_close():
+    inp = _a8_layer()
+    a8 = oracle.layer_a8(inp)
+    ref = oracle.layer(inp)
+    assert np.array_equal(a8["idx"], ref["idx"]) and np.allclose(a8["g"], ref["g"])
+    err = np.abs(a8["y"] - ref["y"]).max(axis=1) / np.abs(ref["y"]).max(axis=1)
+    # E4M3 activations carry 3 mantissa bits: a few percent, but not zero (quantisation is applied)
+    assert np.all(err < 0.15) and np.all(err > 1e-4)
+    zero = dict(inp, x=torch.zeros_like(inp["x"]))
+    assert not oracle.layer_a8(zero)["y"].any()
+
+
+def test_layer_a8_hand_computed_case():
+    """d = I = 128, one routed and the shared expert, identical: W_g and W_u read column 0 only,
+    W_d is all ones. Then g_i = u_i = a for every i, H = bf16(SiLU(a) a) in one 128-group (scale
+    H / 448, every code 448), and each expert outputs 128 * 448 * fl32(H / 448) on every column."""
+    d = I = 128
+    cfg = LayerConfig("hand", 1, d, 1, 1, I, "bf16", "e4m3")
+    a = 448.0 * 2.0 ** -8                              # exact in E4M3 with scale 2^-8
+    x = torch.zeros((1, d), dtype=torch.bfloat16)
+    x[0, 0] = a
+    one = 0x38                                         # E4M3 code of 1.0
+    wg = torch.zeros((2, I, d), dtype=torch.uint8)
+    wg[:, :, 0] = one
+    wd = torch.full((2, d, I), one, dtype=torch.uint8)
+    ones = torch.ones((2, 1, 1), dtype=torch.float32)
+    inp = {"cfg": cfg, "x": x, "w_router": torch.full((1, d), 0.5, dtype=torch.float32),
+           "bias": torch.zeros(1, dtype=torch.float32), "w_gate": wg, "w_up": wg.clone(), "w_down": wd,
+           "s_gate": ones, "s_up": ones.clone(), "s_down": ones.clone()}
+    out = oracle.layer_a8(inp)
+    h = float(_bf16_values(_bf16_bits([a / (1.0 + math.exp(-a)) * a]))[0])
+    s_h = float(np.float32(h) / np.float32(448.0))
+    f = 128 * 448.0 * s_h
+    logit = a * 0.5
+    g = 1.0 / (1.0 + math.exp(-logit))
+    assert out["idx"].tolist() == [[0]]
+    assert np.allclose(out["y"], (1.0 + g) * f, rtol=1e-12, atol=0)
