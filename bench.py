@@ -43,7 +43,7 @@ ROTATE = 8           # distinct token batches cycled through the timed steps
 # of those files, and a changed kernel reports no traffic until re-measured.
 TRAFFIC_SOURCES = ("fine_grained_sparse_fp32_b200/csrc/ffn_swap.cu", "fine_grained_sparse_fp32_b200/csrc/sm100.cuh",
                    "fine_grained_sparse_fp32_b200/csrc/common.cuh")
-TRAFFIC = {"25433d8f1e3f6487": {"decode": (1206.09 + 1.33) * 1e6, "fp8_decode": (603.35 + 0.93) * 1e6}}
+TRAFFIC = {"ca66eb03684632f2": {"decode": (1206.10 + 1.14) * 1e6, "fp8_decode": (603.34 + 0.84) * 1e6}}
 
 
 def kernel_traffic(layer):

@@ -442,6 +442,19 @@ kmoe_status moe_block_forward(const void *h, int N, int d, int E, int K, int I, 
                         topk_idx_out, topk_w_out, counts_out, L, h, gamma_post, eps, st);
 }
 
+kmoe_status moe_quant_1x128(const void *x, int rows, int cols, uint8_t *codes, float *scales, void *stream)
+{
+    clear_error();
+    if (rows < 0) return fail(KMOE_ERR_INVALID_ARG, "rows=%d must be >= 0", rows);
+    if (cols < 128 || cols % 128) return fail(KMOE_ERR_UNSUPPORTED, "cols=%d: must be a positive multiple of 128", cols);
+    if (rows == 0) return KMOE_OK;
+    KMOE_TRY(check_ptr(x, "x"));
+    KMOE_TRY(check_ptr(codes, "codes"));
+    KMOE_TRY(check_ptr(scales, "scales"));
+    return launch_quant_1x128(static_cast<const __nv_bfloat16 *>(x), rows, cols, codes, scales,
+                              static_cast<cudaStream_t>(stream));
+}
+
 kmoe_status moe_device_status(const void *ws, int *status, void *stream)
 {
     clear_error();

@@ -211,6 +211,11 @@ kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dt
                            int y_dtype, int *err, cudaStream_t st, const void *h_res = nullptr,
                            const void *g_post = nullptr, float eps = 0.f);
 
+// Dynamic FP8 quantisation of BF16 rows in groups of 128 columns: codes
+// [rows, cols] (E4M3), scales [rows, cols / 128] (FP32).
+kmoe_status launch_quant_1x128(const __nv_bfloat16 *x, int rows, int cols, uint8_t *codes, float *scales,
+                               cudaStream_t st);
+
 // x = bf16(h / sqrt(mean(h^2) + eps) * gamma), row by row.
 kmoe_status launch_rmsnorm(const __nv_bfloat16 *h, const __nv_bfloat16 *gamma, float eps, int N, int d,
                            __nv_bfloat16 *x, cudaStream_t st);

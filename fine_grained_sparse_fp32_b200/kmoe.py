@@ -22,8 +22,8 @@ SCORES = {"sigmoid": 0, "softmax": 1}     # kmoe_score
 FFN_STATUS_BYTES = (64 + 1088) * 4
 
 EXPORTS = ["moe_workspace_size", "moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn",
-           "moe_combine", "moe_forward", "moe_block_workspace_size", "moe_block_forward", "moe_device_status",
-           "moe_last_error", "moe_abi_version"]
+           "moe_combine", "moe_forward", "moe_block_workspace_size", "moe_block_forward", "moe_quant_1x128",
+           "moe_device_status", "moe_last_error", "moe_abi_version"]
 
 
 class KmoeError(RuntimeError):
@@ -68,9 +68,10 @@ def load(path: str | None = None):
     lib.moe_block_workspace_size.argtypes = [i, i, i, i, i, i]
     lib.moe_block_forward.argtypes = [vp, i, i, i, i, i, i, vp, vp, ctypes.c_float, vp, vp,
                                       ctypes.POINTER(Experts), ctypes.POINTER(Experts), vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.moe_quant_1x128.argtypes = [vp, i, i, vp, vp, vp]
     lib.moe_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
     for f in ("moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn", "moe_combine",
-              "moe_forward", "moe_block_forward", "moe_device_status"):
+              "moe_forward", "moe_block_forward", "moe_quant_1x128", "moe_device_status"):
         getattr(lib, f).restype = i
     if lib.moe_abi_version() != 2:
         raise RuntimeError("libkmoe ABI version mismatch")
@@ -308,3 +309,14 @@ def moe_block_forward(h, layer, gamma_pre, gamma_post, eps: float, with_outputs=
     out = lay.block_forward(h, gamma_pre, gamma_post, eps, h_out=h_out, topk_idx=idx, topk_w=w, counts=counts,
                             x_out=x, stream=stream)
     return out, x, idx, w, counts
+
+
+def moe_quant_1x128(x, codes=None, scales=None, stream=None):
+    """E4M3 codes (uint8 [rows, cols]) and FP32 scales ([rows, cols / 128]) of BF16 x."""
+    rows, cols = x.shape
+    if codes is None:
+        codes = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((rows, cols // 128), dtype=torch.float32, device=x.device)
+    _check(load().moe_quant_1x128(_ptr(x), rows, cols, _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales

@@ -239,6 +239,20 @@ kmoe_status moe_block_forward(const void *h, int N, int d, int E, int K, int I, 
                               void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Dynamic FP8 quantisation of activations ("Inside Kolibri 1", FP8 section:
+ * activations are quantised dynamically in groups of 1 x 128). For each row
+ * and each group of 128 consecutive columns:
+ *   scales[r][g] = amax / 448 in FP32 (1 for an all-zero group)
+ *   codes[r][c]  = E4M3(x[r][c] / scales[r][c / 128]), the quotient in FP32,
+ *                  rounded to nearest even and saturated to +-448
+ * x device [rows, cols] BF16; codes device [rows, cols] bytes (E4M3, sign
+ * bit 7, exponent bias 7); scales device [rows, cols / 128] FP32. cols must
+ * be a multiple of 128. rows == 0 is a no-op.
+ */
+kmoe_status moe_quant_1x128(const void *x, int rows, int cols, uint8_t *codes, float *scales,
+                            void *stream);
+
+/*
  * Device status word. moe_forward, moe_block_forward and moe_grouped_ffn clear the first 4
  * bytes of `ws` when they are enqueued; a tensor-core kernel whose pipeline
  * wait gives up (after about two seconds, which only a fault elsewhere can

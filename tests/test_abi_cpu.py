@@ -151,3 +151,11 @@ def test_block_forward_needs_d_multiple_of_256(lib):
     st = lib.moe_block_forward(a, 32, 2688, 384, 6, 512, 0, a, a, 1e-6, a, a, ctypes.byref(bf), ctypes.byref(bf), a,
                                None, None, None, None, a, 1 << 40, None)
     assert st == kmoe.KMOE_ERR_UNSUPPORTED and b"256" in lib.moe_last_error()
+
+
+def test_quant_1x128_checks_arguments_on_the_host(lib):
+    a = ctypes.c_void_p(1 << 20)
+    assert lib.moe_quant_1x128(a, 4, 200, a, a, None) == kmoe.KMOE_ERR_UNSUPPORTED
+    assert lib.moe_quant_1x128(a, -1, 128, a, a, None) == kmoe.KMOE_ERR_INVALID_ARG
+    assert lib.moe_quant_1x128(a, 4, 128, None, a, None) == kmoe.KMOE_ERR_INVALID_ARG
+    assert lib.moe_quant_1x128(None, 0, 128, None, None, None) == kmoe.KMOE_OK

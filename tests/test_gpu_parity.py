@@ -399,3 +399,21 @@ def test_block_forward_zero_tokens():
     blk = make_block_inputs(dev["cfg"], seed=3, device="cuda")
     out = kmoe.moe_block_forward(blk["h"][:0], dev, blk["gamma_pre"], blk["gamma_post"], BLOCK_EPS)
     assert out.shape == (0, 2560)
+
+
+# ------------------------------------------- FP8 activations: quantiser
+@pytest.mark.parametrize("rows,cols,std", [(1, 128, 1.0), (33, 2560, 2.0), (300, 512, 1e-3), (7, 6144, 30.0)])
+def test_quant_1x128_is_bit_exact(rows, cols, std):
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(rows * 7 + cols)
+    x = torch.empty((rows, cols), device="cuda").normal_(0.0, std, generator=gen)
+    x[0, :128] = 0.0                                   # an all-zero group
+    if cols >= 256:                                    # one large value over tiny ones: subnormal codes
+        x[0, 128:256] *= 1e-4
+        x[0, 128] = 10.0 * std
+    x = x.to(torch.bfloat16)
+    codes, scales = kmoe.moe_quant_1x128(x)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.quant_1x128(x.cpu())
+    assert np.array_equal(codes.cpu().numpy(), oc)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), os_.view(np.uint32))
