@@ -9,7 +9,10 @@
 - Expert FFN and combine: a hand-computed d = I = 1 layer, numpy float64 SwiGLU
   on a non-square expert, and the closed forms (x = 0, zero routed down
   projection, identical experts).
-- FP8 block scales: the E4M3 layer equals the FP32 layer on the decoded weights.
+- FP8 block scales: the E4M3 layer equals the FP32 layer on the decoded weights,
+  and closed forms on weights whose every code is 1.0 with a distinct scale per
+  128 x 128 block (several blocks along both axes, non-square), for both the
+  BF16-activation and the FP8-activation expert.
 - Shapes: the weight counts printed on the pages.
 """
 import itertools
@@ -294,11 +297,13 @@ def test_bias_forcing_selects_the_same_six_everywhere():
         np.testing.assert_allclose(g[t], 1.0 / (1.0 + np.exp(-l[t, idx[t]])), rtol=1e-15)
 
 
-def test_fp8_layer_equals_f32_layer_on_decoded_weights():
-    cfg = LayerConfig("q", 16, 256, 8, 6, 128, "f32", "e4m3")
+@pytest.mark.parametrize("d,I", [(256, 128), (384, 256)])
+def test_fp8_layer_equals_f32_layer_on_decoded_weights(d, I):
+    """At (384, 256) every matrix has several scale blocks along both axes and is not square."""
+    cfg = LayerConfig("q", 16, d, 8, 6, I, "f32", "e4m3")
     q = make_inputs(cfg, seed=10)
     f = dict(q)
-    f["cfg"] = LayerConfig("f", 16, 256, 8, 6, 128, "f32", "f32")
+    f["cfg"] = LayerConfig("f", 16, d, 8, 6, I, "f32", "f32")
     for w, s in (("w_gate", "s_gate"), ("w_up", "s_up"), ("w_down", "s_down")):
         vals = q[w].view(torch.float8_e4m3fn).to(torch.float64)          # [G, R, C]
         sc = q[s].double().repeat_interleave(128, 1).repeat_interleave(128, 2)
@@ -427,3 +432,89 @@ def test_layer_a8_hand_computed_case():
     g = 1.0 / (1.0 + math.exp(-logit))
     assert out["idx"].tolist() == [[0]]
     assert np.allclose(out["y"], (1.0 + g) * f, rtol=1e-12, atol=0)
+
+
+# ------------------------------------------------ FP8 block-scale indexing
+# "Inside Kolibri 1", FP8 section: one FP32 scale per 128 x 128 block, stored
+# [G, rows / 128, cols / 128]. With every E4M3 code equal to 1.0 (0x38) each
+# weight equals the scale of its block, and with x non-zero in one 128-column
+# block only, every projection reduces to a closed form in the scales. Each
+# block of each matrix of each expert gets its own scale, and the shapes have
+# several blocks along both axes (gate/up [256, 384]: 2 x 3, down [384, 256]:
+# 3 x 2), so reading a scale with rows and columns swapped, or from the wrong
+# expert, changes the result.
+
+def _blocky_layer(x_dtype, d=384, I=256, E=2):
+    G = E + 1
+    one = 0x38
+    cfg = LayerConfig("blocky", 1, d, E, 1, I, x_dtype, "e4m3")
+
+    def scales(rows, cols, base):
+        n = G * (rows // 128) * (cols // 128)
+        return torch.arange(base + 1, base + 1 + n, dtype=torch.float32).reshape(G, rows // 128, cols // 128) / 64
+
+    return {"cfg": cfg, "w_router": torch.zeros((E, d), dtype=torch.float32),
+            "bias": torch.tensor([0.0] * (E - 1) + [30.0], dtype=torch.float32),   # forces the last routed expert
+            "w_gate": torch.full((G, I, d), one, dtype=torch.uint8), "w_up": torch.full((G, I, d), one, dtype=torch.uint8),
+            "w_down": torch.full((G, d, I), one, dtype=torch.uint8),
+            "s_gate": scales(I, d, 0), "s_up": scales(I, d, 40), "s_down": scales(d, I, 80)}
+
+
+def _x_in_block(inp, kb, v, torch_dtype):
+    d = inp["cfg"].d
+    x = torch.zeros((1, d), dtype=torch.float32)
+    x[0, 128 * kb:128 * (kb + 1)] = v
+    return x.to(torch_dtype)
+
+
+def _bf16_rne(v: float) -> float:
+    """v rounded to 8 significant bits, ties to even (the BF16 grid; v normal and non-zero)."""
+    m, e = math.frexp(v)
+    return math.ldexp(round(math.ldexp(m, 8)), e - 8)
+
+
+@pytest.mark.parametrize("kb", [1, 2])
+def test_fp8_block_scales_closed_form_bf16_activations(kb):
+    """F_g(x) with x = v on columns of block kb only: a_i = 128 v s_g[g, i/128, kb] (same for the
+    up projection), h_i = SiLU(a_i) b_i, y_j = sum_ib s_d[g, j/128, ib] * sum_{i in ib} h_i."""
+    inp = _blocky_layer("bf16")
+    cfg = inp["cfg"]
+    v = 1.0 / 32
+    inp["x"] = _x_in_block(inp, kb, v, torch.bfloat16)
+    sg, su, sd = (inp[k].double().numpy() for k in ("s_gate", "s_up", "s_down"))
+    G = cfg.E + 1
+    got = oracle.expert_outputs(inp, np.zeros(G, dtype=np.int32), np.arange(G, dtype=np.int32))
+    for g in range(G):
+        a = 128 * v * np.repeat(sg[g, :, kb], 128)
+        b = 128 * v * np.repeat(su[g, :, kb], 128)
+        h = a / (1.0 + np.exp(-a)) * b
+        hb = h.reshape(cfg.I // 128, 128).sum(axis=1)
+        want = np.repeat(sd[g] @ hb, 128)
+        np.testing.assert_allclose(got[g], want, rtol=1e-13, atol=0)
+
+
+@pytest.mark.parametrize("kb", [1, 2])
+def test_fp8_block_scales_closed_form_fp8_activations(kb):
+    """The same weights with FP8 activations: x's block kb quantises to scale fl32(v / 448) and
+    codes 448, so a_i = fl32(v / 448) * s_g[g, i/128, kb] * 128 * 448; every 128-group of H is
+    constant (one gate row block), so it quantises to scale fl32(bf16(h) / 448) and codes 448, and
+    y_j = sum_ib s_h[ib] * s_d[g, j/128, ib] * 128 * 448. Routing is forced onto the last routed
+    expert (bias +30, zero router weights: g = sigmoid(0) = 1/2), so y = F_shared + F_last / 2."""
+    inp = _blocky_layer("bf16")
+    cfg = inp["cfg"]
+    v = 1.0 / 32
+    inp["x"] = _x_in_block(inp, kb, v, torch.bfloat16)
+    sg, su, sd = (inp[k].double().numpy() for k in ("s_gate", "s_up", "s_down"))
+    s_x = float(np.float32(v) / np.float32(448.0))
+
+    def expert(g):
+        a = s_x * sg[g, :, kb] * 128 * 448         # one value per gate row block
+        b = s_x * su[g, :, kb] * 128 * 448
+        h = [_bf16_rne(float(ai / (1.0 + math.exp(-ai)) * bi)) for ai, bi in zip(a, b)]
+        s_h = np.array([float(np.float32(hi) / np.float32(448.0)) for hi in h])
+        return np.repeat(sd[g] @ (s_h * 128 * 448), 128)
+
+    out = oracle.layer_a8(inp)
+    last = cfg.E - 1
+    assert out["idx"].tolist() == [[last]]
+    np.testing.assert_allclose(out["y"][0], expert(cfg.E) + 0.5 * expert(last), rtol=1e-13, atol=0)
