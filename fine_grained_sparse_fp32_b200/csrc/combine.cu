@@ -122,13 +122,17 @@ combine_bulk_kernel(const __nv_bfloat16 *__restrict__ y_perm, const __nv_bfloat1
     };
     if (threadIdx.x == 0)
         for (int i = 0; i < kBulkStages; ++i) issue(i);
+    int stop = -1;                                        // the token slot at which a wait gave up
     for (int i = 0;; ++i) {
         const int t = blockIdx.x + i * gridDim.x;
         if (t >= N) break;
         const int s = i % kBulkStages;
         // every thread reaches the vote each round, so a give-up is a uniform exit
         const bool ok = mbar_wait(&full[s], (i / kBulkStages) & 1, &abort_flag, err, kBulkWaitLimit);
-        if (!__syncthreads_and(ok)) break;
+        if (!__syncthreads_and(ok)) {
+            stop = i;
+            break;
+        }
         const uint8_t *rows = cb_smem + (size_t)s * stage_bytes;
         float g[8];
 #pragma unroll
@@ -183,8 +187,12 @@ combine_bulk_kernel(const __nv_bfloat16 *__restrict__ y_perm, const __nv_bfloat1
         __syncthreads();                                  // every thread is done with stage s
         if (threadIdx.x == 0) issue(i + kBulkStages);
     }
-    if (abort_flag && threadIdx.x == 0)                   // a copy never landed: let the others finish
-        for (int s = 0; s < kBulkStages; ++s) mbar_wait_drain(&full[s], 0, kBulkWaitLimit);
+    // A copy never landed: before the CTA exits, wait (bounded) for every
+    // token slot still in flight, i.e. the ones issued as stop .. stop +
+    // kBulkStages - 1, each on the phase its issue armed.
+    if (stop >= 0 && threadIdx.x == 0)
+        for (int j = stop; j < stop + kBulkStages; ++j)
+            if (blockIdx.x + j * gridDim.x < N) mbar_wait_drain(&full[j % kBulkStages], (j / kBulkStages) & 1, kBulkWaitLimit);
 }
 
 static size_t bulk_smem(int K, int d, bool shared) { return (size_t)kBulkStages * (K + (shared ? 1 : 0)) * d * 2; }

@@ -34,7 +34,9 @@ static int32_t *g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_permute_scratch on the current device. In host code
 // the symbol's name is only a host-side stand-in, so the address is looked
-// up once per device (with that device current) and cached.
+// up once per device (with that device current) and cached for the life of
+// the process; the cache assumes the primary context of the device is not
+// torn down (cudaDeviceReset) while the library is in use.
 static kmoe_status scratch_on_current_device(int32_t **out)
 {
     int dev = -1;

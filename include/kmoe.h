@@ -153,7 +153,10 @@ kmoe_status moe_permute(const int32_t *topk_idx, int N, int K, int E,
  * ceil(N / 256) * E > 262144 (e.g. N > 65536 at E = 1024), are rejected with
  * KMOE_ERR_UNSUPPORTED. The first call on a device looks up the array's
  * device address (once per device, with that device current); make that
- * first call before any stream capture. All calls on a GPU share the array:
+ * first call before any stream capture. The address is then kept for the
+ * life of the process: it assumes the device's primary context lives as
+ * long, so do not call this entry point after a cudaDeviceReset (or another
+ * teardown of the primary context) in the same process. All calls on a GPU share the array:
  * calls whose kernels may overlap on the GPU (different streams without
  * ordering) race and give wrong results, so order them on one stream. The
  * array keeps the last call's contents; each call overwrites every entry it
@@ -247,7 +250,8 @@ kmoe_status moe_block_forward(const void *h, int N, int d, int E, int K, int I, 
  *                  rounded to nearest even and saturated to +-448
  * x device [rows, cols] BF16; codes device [rows, cols] bytes (E4M3, sign
  * bit 7, exponent bias 7); scales device [rows, cols / 128] FP32. cols must
- * be a multiple of 128. rows == 0 is a no-op.
+ * be a multiple of 128. rows == 0 is a no-op. Every x must be finite: a
+ * group holding an Inf or a NaN gets an unspecified scale and codes.
  */
 kmoe_status moe_quant_1x128(const void *x, int rows, int cols, uint8_t *codes, float *scales,
                             void *stream);

@@ -47,7 +47,7 @@ def threads():
 
 # ----------------------------------------------------------------- router
 @pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("decode", 300), ("decode", 1),
-                                    ("skew", 2048), ("decode", 513), ("prefill", None)])
+                                    ("skew", 2048), ("decode", 513), ("prefill", None), ("skew", None)])
 def test_router_topk_matches_oracle(name, N):
     dev, host = layer_inputs(name, N)
     cfg = host["cfg"]
@@ -276,11 +276,41 @@ def test_forward_full_size_sampled_tokens(name):
     _forward_and_compare(name, rows=rows, check_all_routing=True)
 
 
-def test_forward_skew_full_size_sampled_tokens():
-    cfg = CONFIGS["skew"]
+def test_forward_skew_full_size():
+    """The skewed layer (N = 65536) at full size: routing of every token against the oracle's
+    router and selection, counts against the oracle's counting sort of the GPU's own (validated)
+    indices, the workload's skew itself, and the outputs and mixture weights of 160 tokens that
+    include tokens routed to the busiest expert and to the least busy non-empty one."""
+    dev, host = layer_inputs("skew")
+    cfg = host["cfg"]
+    y, idx, w, counts = kmoe.moe_forward(dev["x"], dev, with_outputs=True)
+    torch.cuda.synchronize()
+    idx_g, w_g = idx.cpu().numpy(), w.cpu().double().numpy()
+    l_all = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
+    i_all, g_all, _ = oracle.select(l_all, host["bias"], cfg.K)
+    _, differ = check_routing(idx_g, i_all, biased_scores(l_all, host["bias"]), cfg.K)
+    c_gpu = counts.cpu().numpy()
+    np.testing.assert_array_equal(c_gpu, oracle.permute(idx_g, cfg.E)[0])
+    c_ora = np.bincount(i_all.ravel(), minlength=cfg.E)
+    top = np.sort(c_ora)[::-1]
+    assert 0.45 <= top[:38].sum() / (cfg.N * cfg.K) <= 0.55            # ~half the slots on 10 % of experts
+    assert (c_ora == 0).sum() >= 20                                      # the empty groups exist
+    heavy = int(np.argmax(c_ora))
+    light = int(np.where(c_ora > 0, c_ora, np.iinfo(np.int64).max).argmin())
     rng = np.random.default_rng(2)
-    rows = np.unique(np.concatenate([[0, cfg.N - 1], rng.integers(0, cfg.N, 24)])).astype(np.int32)
-    _forward_and_compare("skew", rows=rows, check_all_routing=False)
+    on = lambda e: np.nonzero((i_all == e).any(axis=1))[0]
+    rows = np.unique(np.concatenate([[0, cfg.N - 1], rng.choice(on(heavy), 64, replace=False), on(light)[:32],
+                                     rng.integers(0, cfg.N, 64)])).astype(np.int32)
+    assert len(rows) >= 128
+    ora = oracle.layer(host, rows=rows, nthreads=threads())
+    keep = np.array([r not in set(differ) for r in rows])
+    got = y[torch.from_numpy(rows).cuda().long()].float().cpu().numpy()
+    assert row_rel_err(got[keep], ora["y"][keep]) <= TOL[cfg.w_dtype]
+    for j, t in enumerate(rows):
+        if keep[j]:
+            want = dict(zip(ora["idx"][j].tolist(), ora["g"][j].tolist()))
+            for k in range(cfg.K):
+                assert abs(w_g[t, k] - want[int(idx_g[t, k])]) <= G_TOL
 
 
 @pytest.mark.parametrize("name,N", [("decode", None), ("prefill", 300), ("fp8_decode", 64)])

@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from fine_grained_sparse_fp32_b200 import _build, kmoe
 
 pytestmark = pytest.mark.gpu
@@ -54,3 +55,31 @@ def test_noalloc_permute_rejects_sizes_beyond_its_fixed_scratch():
         kmoe.moe_permute_noalloc(idx, 1024)
     assert exc.value.status == kmoe.KMOE_ERR_UNSUPPORTED
     assert "fixed array" in str(exc.value)
+
+
+def _spread_rows(seed, N, K, E):
+    """K distinct experts per token: a random start plus K evenly spaced offsets (cheap at large N)."""
+    base = np.random.default_rng(seed).integers(0, E, size=(N, 1))
+    return ((base + np.arange(K)[None, :] * (E // K)) % E).astype(np.int32)
+
+
+@pytest.mark.parametrize("N,E,K", [(65536, 1024, 8),    # ceil(N/256) * E == 262144: the array exactly full
+                                   (32, 384, 6), (256, 384, 6),   # single-CTA sizes (no scratch used)
+                                   (257, 384, 6)])               # the first size that uses chunk histograms
+def test_noalloc_permute_matches_the_oracle_directly(N, E, K):
+    idx = _spread_rows(N + E, N, K, E)
+    got = kmoe.moe_permute_noalloc(torch.from_numpy(idx).cuda(), E)
+    ref = kmoe.moe_permute(torch.from_numpy(idx).cuda(), E)
+    torch.cuda.synchronize()
+    for want, g, r in zip(oracle.permute(idx, E), got, ref):
+        np.testing.assert_array_equal(g.cpu().numpy().reshape(np.shape(want)), want)
+        assert torch.equal(g, r)
+
+
+def test_noalloc_permute_zero_tokens_writes_zero_counts_and_offsets():
+    E = 384
+    counts = torch.full((E,), 7, dtype=torch.int32, device="cuda")
+    offsets = torch.full((E + 1,), 7, dtype=torch.int32, device="cuda")
+    kmoe.moe_permute_noalloc(torch.empty((0, 6), dtype=torch.int32, device="cuda"), E, counts=counts, offsets=offsets)
+    torch.cuda.synchronize()
+    assert int(counts.abs().sum()) == 0 and int(offsets.abs().sum()) == 0
