@@ -115,13 +115,13 @@ def dist_env():
 
 
 def bytes_per_weight(cfg):
-    return {"f32": 4, "bf16": 2, "e4m3": 1}[cfg.w_dtype]
+    return {"f32": 4, "bf16": 2, "e4m3": 1, "e4m3_a8": 1}[cfg.w_dtype]
 
 
 def algorithmic(cfg, distinct_routed: float):
     """Algorithmic bytes and FLOPs of one layer call (intermediates excluded)."""
     per_expert = cfg.expert_weights * bytes_per_weight(cfg)
-    if cfg.w_dtype == "e4m3":
+    if cfg.fp8_weights:
         per_expert += 3 * (cfg.d // 128) * (cfg.I // 128) * 4
     xb = 4 if cfg.x_dtype == "f32" else 2
     weights = (distinct_routed + 1) * per_expert
@@ -135,14 +135,18 @@ def algorithmic(cfg, distinct_routed: float):
 
 def launches_per_step(cfg):
     """Kernels of this library that one moe_forward launches (mirrors abi.cu's dispatch)."""
+    if cfg.w_dtype == "e4m3_a8":
+        ffn = 2             # x quantiser, FP8 tensor-core FFN (up and down units, one launch)
+    elif cfg.x_dtype == "bf16" and cfg.w_dtype in ("bf16", "e4m3") and cfg.N < 256:
+        ffn = 1             # swap-AB FFN (up and down units, one launch)
+    else:
+        ffn = 2             # ffn up, ffn down
     if cfg.N <= 256:
-        if cfg.x_dtype == "bf16" and cfg.w_dtype in ("bf16", "e4m3"):
-            return 5        # router logits, top-K, permute, swap-AB FFN (up and down), combine
-        return 6            # router logits, top-K, permute, ffn up, ffn down, combine
+        return 3 + ffn + 1  # router logits, top-K, permute, FFN, combine
     router = 2 if (cfg.x_dtype == "bf16" and cfg.N >= 512) else 1   # split + tcgen05 router | SIMT router
     chunks = (cfg.N + 255) // 256
     permute = 1 if chunks <= 64 else 2      # scatter with the scan folded in | scan, scatter (top-K counts)
-    return router + 1 + permute + 2 + 1     # + top-K, permute, ffn up, ffn down, combine
+    return router + 1 + permute + ffn + 1   # + top-K, permute, FFN, combine
 
 
 # --------------------------------------------------------------- GPU arm
@@ -280,7 +284,8 @@ def time_grouped_ffn(layer, xs, stream, steps):
             idx, w = kmoe.moe_router_topk(x, layer["w_router"], layer["bias"], cfg.K, stream=stream)
             _, offsets, perm, _ = kmoe.moe_permute(idx, cfg.E, stream=stream)
             preps.append((x, perm, offsets))
-    ws = torch.empty(kmoe.FFN_STATUS_BYTES + (cfg.N * cfg.K + cfg.N) * cfg.I * 4, dtype=torch.uint8, device=dev)
+    ws = kmoe.workspace(cfg.N, cfg.d, cfg.E, cfg.K, cfg.I, kmoe.dtype_code(xs[0].dtype), kmoe.w_dtype_code(cfg.w_dtype),
+                        dev)
     adt = kmoe.act_dtype_for(cfg.w_dtype)
     y_perm = torch.empty((cfg.N * cfg.K, cfg.d), dtype=adt, device=dev)
     y_shared = torch.empty((cfg.N, cfg.d), dtype=adt, device=dev)
@@ -403,7 +408,9 @@ def main():
         pre = run_config(pcfg, psteps, max(3, args.warmup // 10), rank, world, use_graph=not args.no_graph)
         torch.cuda.empty_cache()
         if not args.no_extra:
-            for name, n_steps in (("fp8_decode", max(20, min(args.steps, 1000))), ("fp8_prefill", 50), ("skew", 10)):
+            for name, n_steps in (("fp8_decode", max(20, min(args.steps, 1000))), ("fp8_prefill", 50),
+                                  ("fp8a8_decode", max(20, min(args.steps, 1000))), ("fp8a8_prefill", 50),
+                                  ("skew", 10)):
                 extras[name] = run_config(CONFIGS[name], n_steps, 3, rank, world, use_graph=not args.no_graph)
                 torch.cuda.empty_cache()
             if not args.no_graph:
@@ -452,13 +459,17 @@ def main():
             xcfg = CONFIGS[name]
             xms = r_x["ms_per_step"]
             xalg = r_x["alg"]
+            # FP8 x FP8 MMAs: the measured BF16 peak times the nominal FP8 / BF16 ratio of 2
+            tc_peak = tflops * (2.0 if xcfg.w_dtype == "e4m3_a8" else 1.0)
             t_hbm = xalg["layer_bytes"] / (hbm * 1e9)
-            t_tc = xalg["flops"] / (tflops * 1e12)
+            t_tc = xalg["flops"] / (tc_peak * 1e12)
             line[name] = {
                 "value": whole_job_tokens_per_s(xcfg.N, world, xms), "unit": "tokens/s", "ms_per_step": xms,
                 "N": xcfg.N, "weights": xcfg.w_dtype, "distinct_experts_per_step": r_x["distinct"],
                 "roofline_time_ms": max(t_hbm, t_tc) * 1e3, "bound": "hbm" if t_hbm >= t_tc else "tensor",
                 "frac": max(t_hbm, t_tc) * 1e3 / xms, "tflops": xalg["flops"] / (xms / 1e3) / 1e12,
+                "tensor_peak_tflops": tc_peak,
+                "ffn_frac": xalg["ffn_bytes"] / (r_x["ffn_ms"] / 1e3) / 1e9 / hbm,
                 "ffn_ms": r_x["ffn_ms"], "ffn_gbs": xalg["ffn_bytes"] / (r_x["ffn_ms"] / 1e3) / 1e9,
                 "gpu_launches_per_step": launches_per_step(xcfg), "clocks": r_x["clocks"],
                 "traffic": kernel_traffic(name),

@@ -71,15 +71,20 @@ static kmoe_status check_act_dtype(int t, const char *name)
     return KMOE_OK;
 }
 
+// E4M3 weights with FP32 128 x 128 block scales (BF16 or FP8 activations).
+static bool fp8_weights(int w_dtype) { return w_dtype == KMOE_E4M3_B128 || w_dtype == KMOE_E4M3_B128_A8; }
+
+static bool known_w_dtype(int w_dtype) { return w_dtype == KMOE_F32 || w_dtype == KMOE_BF16 || fp8_weights(w_dtype); }
+
 static kmoe_status check_experts(const kmoe_experts *x, const char *name)
 {
     if (!x) return fail(KMOE_ERR_INVALID_ARG, "%s is NULL", name);
-    if (x->dtype != KMOE_F32 && x->dtype != KMOE_BF16 && x->dtype != KMOE_E4M3_B128)
+    if (x->dtype != KMOE_F32 && x->dtype != KMOE_BF16 && !fp8_weights(x->dtype))
         return fail(KMOE_ERR_UNSUPPORTED, "%s dtype %d unknown", name, x->dtype);
     KMOE_TRY(check_ptr(x->w_gate, "w_gate"));
     KMOE_TRY(check_ptr(x->w_up, "w_up"));
     KMOE_TRY(check_ptr(x->w_down, "w_down"));
-    if (x->dtype == KMOE_E4M3_B128) {
+    if (fp8_weights(x->dtype)) {
         KMOE_TRY(check_ptr(x->s_gate, "s_gate"));
         KMOE_TRY(check_ptr(x->s_up, "s_up"));
         KMOE_TRY(check_ptr(x->s_down, "s_down"));
@@ -90,7 +95,7 @@ static kmoe_status check_experts(const kmoe_experts *x, const char *name)
 static ExpertPtrs ptrs(const kmoe_experts *x)
 {
     ExpertPtrs p{x->w_gate, x->w_up, x->w_down, nullptr, nullptr, nullptr};
-    if (x->dtype == KMOE_E4M3_B128) {
+    if (fp8_weights(x->dtype)) {
         p.sg = x->s_gate;
         p.su = x->s_up;
         p.sd = x->s_down;
@@ -99,6 +104,44 @@ static ExpertPtrs ptrs(const kmoe_experts *x)
 }
 
 static size_t act_bytes(int w_dtype) { return w_dtype == KMOE_F32 ? 4 : 2; }
+
+// Bytes of one H element: the output dtype, or an E4M3 code with FP8 activations.
+static size_t h_bytes(int w_dtype) { return w_dtype == KMOE_E4M3_B128_A8 ? 1 : act_bytes(w_dtype); }
+
+// The grouped FFN's scratch after the status block: H [N*K + N, I] and, with
+// FP8 activations, H's scales [N*K + N, I / 128], x's codes [N, d] and x's
+// scales [N, d / 128].
+struct FfnScratch {
+    void *h;
+    float *hs;
+    uint8_t *xq;
+    float *xs;
+};
+
+static FfnScratch take_ffn_scratch(Carver &c, int N, int d, int K, int I, int w_dtype)
+{
+    const size_t R = (size_t)N * K + N;
+    FfnScratch f{};
+    f.h = c.take<char>(R * I * h_bytes(w_dtype));
+    if (w_dtype == KMOE_E4M3_B128_A8) {
+        f.hs = c.take<float>(R * (I / 128));
+        f.xq = c.take<uint8_t>((size_t)N * d);
+        f.xs = c.take<float>((size_t)N * (d / 128));
+    }
+    return f;
+}
+
+// Bytes of a moe_grouped_ffn workspace: the status block, then the scratch.
+static size_t ffn_ws_bytes(int N, int d, int K, int I, int w_dtype)
+{
+    Carver c(nullptr);
+    c.take<int>(kStatusInts);
+    take_ffn_scratch(c, N, d, K, I, w_dtype);
+    return c.used;
+}
+
+// Give-up limit of the pipeline waits of the kernels this thread launches.
+static long long wait_limit() { return kDefaultWaitLimit; }
 
 // Workspace of the whole forward; every entry point uses a prefix-compatible
 // subset (router: logits; permute: chunk histograms; grouped FFN: H).
@@ -109,7 +152,8 @@ struct Layout {
     float *w;
     int32_t *counts, *offsets, *perm, *inv, *hist;
     __nv_bfloat16 *w_split;
-    void *h, *y_perm, *y_shared;
+    FfnScratch ffn;
+    void *y_perm, *y_shared;
     __nv_bfloat16 *x_norm;   // sandwich block only: the normalised layer input
     size_t bytes;
 };
@@ -130,7 +174,7 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype, b
     L.inv = c.take<int32_t>((size_t)N * K);
     L.hist = reinterpret_cast<int32_t *>(c.take<char>(permute_ws_bytes(N, E)));
     L.w_split = c.take<__nv_bfloat16>(router_tc_ws_bytes(d, E) / sizeof(__nv_bfloat16));
-    L.h = c.take<char>(R * I * ab);
+    L.ffn = take_ffn_scratch(c, N, d, K, I, w_dtype);
     L.y_perm = c.take<char>((size_t)N * K * d * ab);
     L.y_shared = c.take<char>((size_t)N * d * ab);
     L.x_norm = block ? c.take<__nv_bfloat16>((size_t)N * d) : nullptr;
@@ -142,10 +186,13 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype, b
 // d % 256 == 0): below kTcMinTokens tokens the swap-AB tcgen05 kernel
 // (weights as M, 16-token chunks as N), from there the tokens-as-M tcgen05
 // kernel; FP32 activations or weights take the CUDA-core streaming kernel.
-enum FfnPath { kPathStream, kPathSwap, kPathTc };
+// FP8 activations (KMOE_E4M3_B128_A8) take the FP8 tensor-core kernel at
+// every batch size.
+enum FfnPath { kPathStream, kPathSwap, kPathTc, kPathA8 };
 
 static FfnPath ffn_path(int x_dtype, int w_dtype, int N, int d)
 {
+    if (w_dtype == KMOE_E4M3_B128_A8) return kPathA8;
     if (x_dtype != KMOE_BF16 || (w_dtype != KMOE_BF16 && w_dtype != KMOE_E4M3_B128) || d % 256) return kPathStream;
     return N < kTcMinTokens ? kPathSwap : kPathTc;
 }
@@ -154,9 +201,18 @@ static FfnPath ffn_path(int x_dtype, int w_dtype, int N, int d)
 // kSyncInts counters at kSyncOffset (all zeroed by clear_status).
 static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int E, int K, const int32_t *perm,
                            const int32_t *offsets, int w_dtype, const ExpertPtrs &r, const ExpertPtrs *s,
-                           void *h, void *y_perm, void *y_shared, int *status, cudaStream_t st)
+                           const FfnScratch &f, void *y_perm, void *y_shared, int *status, cudaStream_t st)
 {
     const FfnPath path = ffn_path(x_dtype, w_dtype, N, d);
+    void *h = f.h;
+    if (path == kPathA8) {
+        if (x_dtype != KMOE_BF16 || d % 256)
+            return fail(KMOE_ERR_UNSUPPORTED, "FP8 activations: x must be BF16 and d a multiple of 256");
+        KMOE_TRY(launch_quant_1x128(static_cast<const __nv_bfloat16 *>(x), N, d, f.xq, f.xs, st));
+        return launch_ffn_a8(f.xq, f.xs, N, d, I, E, K, perm, offsets, r, s, static_cast<uint8_t *>(h), f.hs,
+                             static_cast<__nv_bfloat16 *>(y_perm), static_cast<__nv_bfloat16 *>(y_shared), status,
+                             status + kSyncOffset, wait_limit(), st);
+    }
     if (path == kPathSwap)
         return launch_ffn_swap(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, w_dtype, r, s,
                                static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
@@ -236,7 +292,7 @@ static kmoe_status forward_path(const void *x, int x_dtype, int N, int d, int E,
     ExpertPtrs s{};
     if (shared) s = ptrs(shared);
     KMOE_TRY(run_ffn(x, x_dtype, N, d, I, E, K, L.perm, L.offsets, routed->dtype, r, shared ? &s : nullptr,
-                     L.h, L.y_perm, L.y_shared, L.status, st));
+                     L.ffn, L.y_perm, L.y_shared, L.status, st));
     const int yin = routed->dtype == KMOE_F32 ? KMOE_F32 : KMOE_BF16;
     return launch_combine(L.y_perm, shared ? L.y_shared : nullptr, yin, w, L.inv, N, K, d, y, y_dtype, L.status, st,
                           h_res, g_post, eps);
@@ -256,7 +312,7 @@ size_t moe_workspace_size(int N, int d, int E, int K, int I, int x_dtype, int w_
 {
     if (check_sizes(N, d, E, K, I) != KMOE_OK) return 0;
     if (check_act_dtype(x_dtype, "x") != KMOE_OK) return 0;
-    if (w_dtype != KMOE_F32 && w_dtype != KMOE_BF16 && w_dtype != KMOE_E4M3_B128) return 0;
+    if (!known_w_dtype(w_dtype)) return 0;
     clear_error();
     return layout(nullptr, N, d, E, K, I, w_dtype).bytes;
 }
@@ -347,16 +403,18 @@ kmoe_status moe_grouped_ffn(const void *x, int x_dtype, int N, int d, int I, int
     KMOE_TRY(check_ptr(y_perm, "y_perm"));
     if (shared) KMOE_TRY(check_ptr(y_shared, "y_shared"));
     KMOE_TRY(check_ptr(ws, "ws"));
-    const size_t need = kFfnStatusBytes + ((size_t)N * K + N) * I * act_bytes(routed->dtype);
+    const size_t need = ffn_ws_bytes(N, d, K, I, routed->dtype);
     if (ws_bytes < need) return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
     const ExpertPtrs r = ptrs(routed);
     ExpertPtrs s{};
     if (shared) s = ptrs(shared);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    int *status = static_cast<int *>(ws);
+    Carver c(ws);
+    int *status = c.take<int>(kStatusInts);
+    const FfnScratch f = take_ffn_scratch(c, N, d, K, I, routed->dtype);
     KMOE_TRY(clear_status(status, st, kFfnStatusBytes));
-    return run_ffn(x, x_dtype, N, d, I, E, K, perm_token, offsets, routed->dtype, r, shared ? &s : nullptr,
-                   static_cast<char *>(ws) + kFfnStatusBytes, y_perm, y_shared, status, st);
+    return run_ffn(x, x_dtype, N, d, I, E, K, perm_token, offsets, routed->dtype, r, shared ? &s : nullptr, f,
+                   y_perm, y_shared, status, st);
 }
 
 kmoe_status moe_combine(const void *y_perm, const void *y_shared, int y_in_dtype, const float *topk_w,
@@ -402,7 +460,7 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
 size_t moe_block_workspace_size(int N, int d, int E, int K, int I, int w_dtype)
 {
     if (check_sizes(N, d, E, K, I) != KMOE_OK) return 0;
-    if (w_dtype != KMOE_BF16 && w_dtype != KMOE_E4M3_B128) return 0;
+    if (w_dtype != KMOE_BF16 && !fp8_weights(w_dtype)) return 0;
     clear_error();
     return layout(nullptr, N, d, E, K, I, w_dtype, true).bytes;
 }
@@ -416,7 +474,7 @@ kmoe_status moe_block_forward(const void *h, int N, int d, int E, int K, int I, 
     clear_error();
     KMOE_TRY(check_forward(N, d, E, K, I, score, routed, shared, w_router, bias, topk_idx_out, topk_w_out, counts_out,
                            ws));
-    if (routed->dtype != KMOE_BF16 && routed->dtype != KMOE_E4M3_B128)
+    if (routed->dtype != KMOE_BF16 && !fp8_weights(routed->dtype))
         return fail(KMOE_ERR_UNSUPPORTED, "block: routed weights must be BF16 or E4M3 with 128x128 scales");
     if (!(eps >= 0.f) || eps > 1.f) return fail(KMOE_ERR_INVALID_ARG, "eps=%g: must be in [0, 1]", (double)eps);
     if (d % 256) return fail(KMOE_ERR_UNSUPPORTED, "block: d=%d must be a multiple of 256", d);

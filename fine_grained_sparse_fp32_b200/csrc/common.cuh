@@ -11,6 +11,11 @@
 
 namespace kmoe {
 
+// Default give-up limit of a pipeline wait, in SM clock cycles (about 2 s at
+// 1.9 GHz): far beyond any wait of a healthy launch. Waits that drain
+// in-flight copies after another wait gave up always use this limit.
+constexpr long long kDefaultWaitLimit = 1LL << 32;
+
 // ---------------------------------------------------------------- host side
 
 // Records a printf-style message as the calling thread's last error and
@@ -203,6 +208,16 @@ kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, 
                             const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
                             __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status,
                             int *sync, cudaStream_t st);
+
+// Grouped FFN with FP8 activations (E4M3 weights + FP32 128 x 128 block
+// scales; x given as E4M3 codes xq [N, d] with FP32 scales xs [N, d / 128];
+// H kept as codes hq [N*K + N, I] with scales hs [N*K + N, I / 128]; d % 256
+// == 0). `sync` as for launch_ffn_swap. wait_limit: SM cycles before a
+// pipeline wait gives up.
+kmoe_status launch_ffn_a8(const uint8_t *xq, const float *xs, int N, int d, int I, int E, int K, const int32_t *perm,
+                          const int32_t *offsets, const ExpertPtrs &routed, const ExpertPtrs *shared, uint8_t *hq,
+                          float *hs, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status, int *sync,
+                          long long wait_limit, cudaStream_t st);
 
 // err: device status word for a bounded wait that gives up (may be NULL).
 // h_res / g_post (BF16, NULL for the plain combine): y = h_res + RMSNorm(m) * g_post.

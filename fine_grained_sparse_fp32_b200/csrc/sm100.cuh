@@ -205,6 +205,20 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T with 8-bit float inputs (kind::f8f6f4;
+// the formats are in the instruction descriptor), FP32 accumulation. One
+// instruction covers K = 32 elements (32 bytes of each K-major row).
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]^T (kind::f16: A, B both F16 or both BF16).
 // A sits in tensor memory: lane i holds row i, two 16-bit elements per
 // 32-bit column, K increasing with the column.
@@ -293,6 +307,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N)
     return (1u << 4)                       // D format: F32
            | (1u << 7)                     // A format: BF16
            | (1u << 10)                    // B format: BF16
+           | ((uint32_t)(N >> 3) << 17)    // N / 8
+           | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// Instruction descriptor of tcgen05.mma kind::f8f6f4 with E4M3 A and B (format
+// code 0 for both, K-major), FP32 accumulator, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
+{
+    return (1u << 4)                       // D format: F32
+           | (0u << 7)                     // A format: E4M3
+           | (0u << 10)                    // B format: E4M3
            | ((uint32_t)(N >> 3) << 17)    // N / 8
            | ((uint32_t)(M >> 4) << 24);   // M / 16
 }

@@ -14,7 +14,7 @@ import torch
 from ._build import LIB
 
 KMOE_OK, KMOE_ERR_INVALID_ARG, KMOE_ERR_UNSUPPORTED, KMOE_ERR_CUDA, KMOE_ERR_WORKSPACE, KMOE_ERR_DEVICE = range(6)
-KMOE_F32, KMOE_BF16, KMOE_E4M3_B128 = 0, 1, 2
+KMOE_F32, KMOE_BF16, KMOE_E4M3_B128, KMOE_E4M3_B128_A8 = 0, 1, 2, 3
 SCORES = {"sigmoid": 0, "softmax": 1}     # kmoe_score
 
 # Bytes at the head of a moe_grouped_ffn workspace: the status word, tickets
@@ -73,7 +73,7 @@ def load(path: str | None = None):
     for f in ("moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn", "moe_combine",
               "moe_forward", "moe_block_forward", "moe_quant_1x128", "moe_device_status"):
         getattr(lib, f).restype = i
-    if lib.moe_abi_version() != 2:
+    if lib.moe_abi_version() != 3:
         raise RuntimeError("libkmoe ABI version mismatch")
     _lib = lib
     return lib
@@ -98,7 +98,7 @@ def dtype_code(t: torch.dtype) -> int:
 
 
 def w_dtype_code(name: str) -> int:
-    return {"f32": KMOE_F32, "bf16": KMOE_BF16, "e4m3": KMOE_E4M3_B128}[name]
+    return {"f32": KMOE_F32, "bf16": KMOE_BF16, "e4m3": KMOE_E4M3_B128, "e4m3_a8": KMOE_E4M3_B128_A8}[name]
 
 
 def act_dtype_for(w_dtype: str) -> torch.dtype:
@@ -189,8 +189,7 @@ def moe_grouped_ffn(x, layer, perm_token, offsets, with_shared=True, ws=None, st
         y_perm = torch.empty((N * K, d), dtype=adt, device=x.device)
         y_shared = torch.empty((N, d), dtype=adt, device=x.device) if with_shared else None
     if ws is None:
-        ws = torch.empty(FFN_STATUS_BYTES + (N * K + N) * I * (4 if adt == torch.float32 else 2), dtype=torch.uint8,
-                         device=x.device)
+        ws = workspace(N, d, E, K, I, dtype_code(x.dtype), w_dtype_code(cfg.w_dtype), x.device)
     routed = experts_of(layer, "routed")
     shared = experts_of(layer, "shared") if with_shared else None
     _check(load().moe_grouped_ffn(_ptr(x), dtype_code(x.dtype), N, d, I, E, K, _ptr(perm_token), _ptr(offsets),

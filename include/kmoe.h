@@ -65,9 +65,19 @@ typedef enum {
 } kmoe_score;
 
 typedef enum {
-    KMOE_F32 = 0,        /* IEEE binary32 */
-    KMOE_BF16 = 1,       /* bfloat16 */
-    KMOE_E4M3_B128 = 2   /* OCP E4M3 bytes + one FP32 scale per 128x128 block */
+    KMOE_F32 = 0,           /* IEEE binary32 */
+    KMOE_BF16 = 1,          /* bfloat16 */
+    KMOE_E4M3_B128 = 2,     /* OCP E4M3 bytes + one FP32 scale per 128x128 block */
+    KMOE_E4M3_B128_A8 = 3   /* expert weights only: stored exactly as KMOE_E4M3_B128, and
+                               the expert GEMMs run on FP8 activations ("Inside Kolibri 1",
+                               FP8 section: activations quantised dynamically in groups of
+                               1 x 128). x (BF16) is quantised per row and 128 columns:
+                               scale = amax / 448 in FP32 (1 for an all-zero group), code =
+                               E4M3(x / scale) with the quotient in FP32, round to nearest
+                               even, saturated; H is rounded to BF16 and quantised the same
+                               way before the down projection. Each 128-column K block's
+                               E4M3 x E4M3 partial sums (FP32) are scaled by both FP32
+                               block scales and added in FP32. Routing sees x as given. */
 } kmoe_dtype;
 
 /*
@@ -175,7 +185,11 @@ kmoe_status moe_permute_noalloc(const int32_t *topk_idx, int N, int K, int E,
  * intermediate SiLU(.)*up rounded to the output dtype.
  * x device [N, d] (x_dtype F32 or BF16). perm_token, offsets as produced by
  * moe_permute. Output dtype: FP32 when the weights are FP32, else BF16.
- * y_perm device [N*K, d]; y_shared device [N, d].
+ * y_perm device [N*K, d]; y_shared device [N, d]. With KMOE_E4M3_B128_A8
+ * weights the activations are FP8 (see kmoe_dtype): x must be BF16 and d a
+ * multiple of 256 (KMOE_ERR_UNSUPPORTED otherwise). ws: at least
+ * moe_workspace_size() bytes for these sizes and dtypes; its first 4 bytes
+ * are the status word read by moe_device_status.
  */
 kmoe_status moe_grouped_ffn(const void *x, int x_dtype, int N, int d, int I, int E, int K,
                             const int32_t *perm_token, const int32_t *offsets,
@@ -202,7 +216,9 @@ kmoe_status moe_combine(const void *y_perm, const void *y_shared, int y_in_dtype
  * (kmoe_score) picks the mixture weights.
  * y device [N, d] output of y_dtype (F32 or BF16). topk_idx_out [N, K],
  * topk_w_out [N, K] and counts_out [E] are optional device outputs (NULL to
- * skip). `shared` may be NULL (no shared expert).
+ * skip). `shared` may be NULL (no shared expert). Routed and shared weights
+ * have the same dtype; KMOE_E4M3_B128_A8 runs the expert GEMMs on FP8
+ * activations (BF16 x, d a multiple of 256), with routing on x as given.
  */
 kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, int I, int score,
                         const float *w_router, const float *bias,
@@ -226,7 +242,8 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
  * before its h_out element is written, by the same thread) but must not
  * overlap it otherwise. x_out: optional device [N, d] BF16 output of the
  * normalised layer input x (NULL keeps it in the workspace). Routed (and shared) weights must be BF16 or E4M3
- * with 128 x 128 scales and d a multiple of 256 (KMOE_ERR_UNSUPPORTED otherwise), and
+ * with 128 x 128 scales (KMOE_E4M3_B128 or KMOE_E4M3_B128_A8) and d a multiple of 256
+ * (KMOE_ERR_UNSUPPORTED otherwise), and
  * (K + 1) * d <= 25600 BF16 values must fit the combine's staging buffer
  * (K + 1 counts the shared expert). Other arguments and outputs as in
  * moe_forward. ws: at least moe_block_workspace_size() bytes; its first 4
@@ -272,7 +289,7 @@ const char *moe_last_error(void);
 
 /* ABI version of this header (bumped on incompatible change). */
 int moe_abi_version(void);
-#define KMOE_ABI_VERSION 2
+#define KMOE_ABI_VERSION 3
 
 #ifdef __cplusplus
 }

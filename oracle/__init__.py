@@ -21,7 +21,7 @@ _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 F32, BF16, E4M3 = 0, 1, 2
-_DT = {"f32": F32, "bf16": BF16, "e4m3": E4M3}
+_DT = {"f32": F32, "bf16": BF16, "e4m3": E4M3, "e4m3_a8": E4M3}   # e4m3_a8: E4M3 weights, stored alike
 
 _lib = None
 
@@ -120,7 +120,7 @@ def permute(idx, E: int):
 def _weights(inp):
     cfg = inp["cfg"]
     wg, wu, wd = _bits(inp["w_gate"]), _bits(inp["w_up"]), _bits(inp["w_down"])
-    if cfg.w_dtype == "e4m3":
+    if cfg.w_dtype in ("e4m3", "e4m3_a8"):
         sg, su, sd = (np.ascontiguousarray(_bits(inp[k]), dtype=np.float32) for k in ("s_gate", "s_up", "s_down"))
     else:
         sg = su = sd = None
@@ -210,7 +210,7 @@ def layer_a8(inp, rows=None, nthreads: int = 1, score: str = "sigmoid"):
     """The layer with E4M3 weights and activations quantised in 1 x 128 groups (x for
     gate/up, H for down); routing on x as stored. Returns dict(y, idx, g, margin, rows)."""
     cfg = inp["cfg"]
-    if cfg.w_dtype != "e4m3" or cfg.x_dtype != "bf16":
+    if cfg.w_dtype not in ("e4m3", "e4m3_a8") or cfg.x_dtype != "bf16":
         raise ValueError("FP8 activations need BF16 x and E4M3 weights")
     xb = np.ascontiguousarray(_bits(inp["x"]), dtype=np.uint16)
     N = xb.shape[0]
@@ -229,6 +229,22 @@ def layer_a8(inp, rows=None, nthreads: int = 1, score: str = "sigmoid"):
     return {"y": y, "idx": idx, "g": g, "margin": margin, "rows": rows}
 
 
+def expert_outputs_a8(inp, tokens, experts, nthreads: int = 1) -> np.ndarray:
+    """F_e(x_t) in double with FP8 activations (x and H quantised in 1 x 128 groups) for each
+    (t, e) pair; e == E is the shared expert. E4M3 weights and BF16 x only."""
+    cfg = inp["cfg"]
+    if cfg.w_dtype not in ("e4m3", "e4m3_a8") or cfg.x_dtype != "bf16":
+        raise ValueError("FP8 activations need BF16 x and E4M3 weights")
+    xb = np.ascontiguousarray(_bits(inp["x"]), dtype=np.uint16)
+    wg, wu, wd, sg, su, sd = _weights(inp)
+    tok = np.ascontiguousarray(tokens, dtype=np.int32)
+    ex = np.ascontiguousarray(experts, dtype=np.int32)
+    out = np.empty((len(tok), cfg.d), dtype=np.float64)
+    lib().oracle_expert_outputs_a8(cfg.d, cfg.I, _p(xb), _p(wg), _p(wu), _p(wd), _p(sg), _p(su), _p(sd),
+                                   len(tok), _p(tok), _p(ex), _p(out), nthreads)
+    return out
+
+
 __all__ = ["build", "lib", "max_threads", "e4m3_to_double", "router_logits", "select",
            "permute", "expert_outputs", "layer", "rmsnorm_bf16", "block", "float_to_e4m3", "quant_1x128",
-           "layer_a8", "F32", "BF16", "E4M3"]
+           "layer_a8", "expert_outputs_a8", "F32", "BF16", "E4M3"]

@@ -497,6 +497,34 @@ static void expert_ffn_a8(int d, int I, const uint8_t *xq, const float *xs, int6
     }
 }
 
+/* F_g(x_t) with FP8 activations for a list of (token, expert) pairs: the
+ * token's row is quantised in 1 x 128 groups and expert_ffn_a8 runs on it.
+ * x is [N, d] BF16; out is [n_pairs, d]; expert g indexes the stacked
+ * [G, ., .] E4M3 tensors. */
+void oracle_expert_outputs_a8(int d, int I, const uint16_t *x,
+                              const uint8_t *wg, const uint8_t *wu, const uint8_t *wd,
+                              const float *sg, const float *su, const float *sd,
+                              int n_pairs, const int32_t *tokens, const int32_t *experts,
+                              double *out, int nthreads)
+{
+    int p;
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic)
+    for (p = 0; p < n_pairs; ++p) {
+        uint8_t *xq = (uint8_t *)malloc((size_t)d);
+        float *xs = (float *)malloc((size_t)(d / OR_BLOCK) * sizeof(float));
+        uint16_t *hb = (uint16_t *)malloc((size_t)I * sizeof(uint16_t));
+        uint8_t *hq = (uint8_t *)malloc((size_t)I);
+        float *hs = (float *)malloc((size_t)(I / OR_BLOCK) * sizeof(float));
+        oracle_quant_1x128(1, d, x + (int64_t)tokens[p] * d, xq, xs);
+        expert_ffn_a8(d, I, xq, xs, experts[p], wg, wu, wd, sg, su, sd, hb, hq, hs, out + (int64_t)p * d);
+        free(hs);
+        free(hq);
+        free(hb);
+        free(xs);
+        free(xq);
+    }
+}
+
 /* The whole layer with FP8 activations, for tokens rows[0 .. n_rows-1]:
  * the router and the top-K see x as stored (BF16); each expert sees x
  * quantised in 1 x 128 groups, and its down projection sees H quantised the

@@ -14,7 +14,7 @@ from __future__ import annotations
 import numpy as np
 
 TIE_MARGIN = 1e-5
-TOL = {"f32": 1e-4, "bf16": 2e-2, "e4m3": 5e-2}
+TOL = {"f32": 1e-4, "bf16": 2e-2, "e4m3": 5e-2, "e4m3_a8": 5e-2}
 G_TOL = 1e-5          # mixture weights (FP32 logits through sigmoid)
 
 

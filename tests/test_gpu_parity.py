@@ -45,6 +45,17 @@ def threads():
     return oracle.max_threads()
 
 
+def expert_ref(host, tokens, experts):
+    """The oracle's expert outputs under the config's activation precision."""
+    f = oracle.expert_outputs_a8 if host["cfg"].w_dtype == "e4m3_a8" else oracle.expert_outputs
+    return f(host, tokens, experts, nthreads=threads())
+
+
+def layer_ref(host, rows=None, score="sigmoid"):
+    f = oracle.layer_a8 if host["cfg"].w_dtype == "e4m3_a8" else oracle.layer
+    return f(host, rows=rows, nthreads=threads(), score=score)
+
+
 # ----------------------------------------------------------------- router
 @pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("decode", 300), ("decode", 1),
                                     ("skew", 2048), ("decode", 513), ("prefill", None), ("skew", None)])
@@ -132,7 +143,9 @@ def test_permute_all_tokens_on_the_same_experts():
 # ------------------------------------------------------------ grouped FFN
 @pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("fp8_decode", None), ("decode", 200),
                                     ("fp8_decode", 130), ("prefill", 256), ("prefill", 300), ("prefill", 1000),
-                                    ("fp8_prefill", 300), ("fp8_prefill", 777)])
+                                    ("fp8_prefill", 300), ("fp8_prefill", 777), ("fp8a8_decode", None),
+                                    ("fp8a8_decode", 1), ("fp8a8_decode", 255), ("fp8a8_prefill", 256),
+                                    ("fp8a8_prefill", 1000)])
 def test_grouped_ffn_matches_oracle(name, N):
     dev, host = layer_inputs(name, N)
     cfg = host["cfg"]
@@ -145,16 +158,17 @@ def test_grouped_ffn_matches_oracle(name, N):
     rng = np.random.default_rng(0)
     rows = np.unique(np.concatenate([[0, cfg.N * cfg.K - 1], rng.integers(0, cfg.N * cfg.K, 48)]))
     expert_of_row = np.searchsorted(offsets, rows, side="right") - 1
-    ref = oracle.expert_outputs(host, perm[rows], expert_of_row, nthreads=threads())
+    ref = expert_ref(host, perm[rows], expert_of_row)
     got = y_perm[torch.from_numpy(rows).cuda().long()].float().cpu().numpy()
     assert row_rel_err(got, ref) <= TOL[cfg.w_dtype]
     toks = np.unique(np.concatenate([[0, cfg.N - 1], rng.integers(0, cfg.N, 16)]))
-    ref_s = oracle.expert_outputs(host, toks, np.full(len(toks), cfg.E), nthreads=threads())
+    ref_s = expert_ref(host, toks, np.full(len(toks), cfg.E))
     got_s = y_shared[torch.from_numpy(toks).cuda().long()].float().cpu().numpy()
     assert row_rel_err(got_s, ref_s) <= TOL[cfg.w_dtype]
 
 
-@pytest.mark.parametrize("name,N", [("decode", 200), ("fp8_decode", 200), ("decode", 33)])
+@pytest.mark.parametrize("name,N", [("decode", 200), ("fp8_decode", 200), ("decode", 33), ("fp8a8_decode", 200),
+                                    ("fp8a8_prefill", 600)])
 def test_grouped_ffn_crowded_experts(name, N):
     """Every token on the same six experts: groups of N rows, several 32-row
     token chunks per expert on the small-batch path, and 378 empty groups."""
@@ -167,15 +181,15 @@ def test_grouped_ffn_crowded_experts(name, N):
     torch.cuda.synchronize()
     rows = np.unique(np.concatenate([[0, cfg.N * cfg.K - 1], np.arange(0, cfg.N * cfg.K, 7)]))
     expert_of_row = np.searchsorted(offsets, rows, side="right") - 1
-    ref = oracle.expert_outputs(host, perm[rows], expert_of_row, nthreads=threads())
+    ref = expert_ref(host, perm[rows], expert_of_row)
     got = y_perm[torch.from_numpy(rows).cuda().long()].float().cpu().numpy()
     assert row_rel_err(got, ref) <= TOL[cfg.w_dtype]
     toks = np.arange(cfg.N)
-    ref_s = oracle.expert_outputs(host, toks, np.full(len(toks), cfg.E), nthreads=threads())
+    ref_s = expert_ref(host, toks, np.full(len(toks), cfg.E))
     assert row_rel_err(y_shared.float().cpu().numpy(), ref_s) <= TOL[cfg.w_dtype]
 
 
-@pytest.mark.parametrize("name", ["decode", "fp8_decode", "prefill"])
+@pytest.mark.parametrize("name", ["decode", "fp8_decode", "prefill", "fp8a8_decode", "fp8a8_prefill"])
 def test_grouped_ffn_without_shared_expert(name):
     dev, host = layer_inputs(name, 40 if name != "prefill" else 300)
     cfg = host["cfg"]
@@ -188,7 +202,7 @@ def test_grouped_ffn_without_shared_expert(name):
     assert y_shared is None
     rows = np.arange(0, cfg.N * cfg.K, 5)
     expert_of_row = np.searchsorted(offsets, rows, side="right") - 1
-    ref = oracle.expert_outputs(host, perm[rows], expert_of_row, nthreads=threads())
+    ref = expert_ref(host, perm[rows], expert_of_row)
     got = y_perm[torch.from_numpy(rows).cuda().long()].float().cpu().numpy()
     assert row_rel_err(got, ref) <= TOL[cfg.w_dtype]
 
@@ -241,7 +255,7 @@ def _forward_and_compare(name, N=None, rows=None, check_all_routing=True):
     idx_g = idx.cpu().numpy()
     if rows is None:
         rows = np.arange(cfg.N, dtype=np.int32)
-    ora = oracle.layer(host, rows=rows, nthreads=threads())
+    ora = layer_ref(host, rows=rows)
     # routing on the compared rows (oracle logits recomputed for them)
     xr = host["x"][torch.from_numpy(rows).long()]
     l_rows = oracle.router_logits(xr, cfg.x_dtype, host["w_router"], nthreads=threads())
@@ -263,12 +277,13 @@ def _forward_and_compare(name, N=None, rows=None, check_all_routing=True):
 
 
 @pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("fp8_decode", None),
-                                    ("prefill", 300), ("fp8_prefill", 259), ("decode", 1)])
+                                    ("prefill", 300), ("fp8_prefill", 259), ("decode", 1), ("fp8a8_decode", None),
+                                    ("fp8a8_decode", 1), ("fp8a8_prefill", 259)])
 def test_forward_matches_oracle_all_tokens(name, N):
     _forward_and_compare(name, N)
 
 
-@pytest.mark.parametrize("name", ["prefill", "fp8_prefill"])
+@pytest.mark.parametrize("name", ["prefill", "fp8_prefill", "fp8a8_prefill"])
 def test_forward_full_size_sampled_tokens(name):
     cfg = CONFIGS[name]
     rng = np.random.default_rng(1)
@@ -328,7 +343,7 @@ def test_forward_softmax_score_matches_oracle(name, N):
 
 
 def test_forward_is_deterministic():
-    for name, N in (("decode", None), ("prefill", 300)):
+    for name, N in (("decode", None), ("prefill", 300), ("fp8a8_decode", None), ("fp8a8_prefill", 300)):
         dev, _ = layer_inputs(name, N)
         a = kmoe.moe_forward(dev["x"], dev, with_outputs=True)
         b = kmoe.moe_forward(dev["x"], dev, with_outputs=True)
@@ -337,7 +352,7 @@ def test_forward_is_deterministic():
 
 
 def test_device_status_is_clear_after_a_forward():
-    for name, N in (("decode", None), ("prefill", 300)):
+    for name, N in (("decode", None), ("prefill", 300), ("fp8a8_decode", None), ("fp8a8_prefill", 300)):
         dev, _ = layer_inputs(name, N)
         cfg = dev["cfg"]
         lay = kmoe.Layer(dev, cfg.N)

@@ -518,3 +518,7 @@ def test_fp8_block_scales_closed_form_fp8_activations(kb):
     last = cfg.E - 1
     assert out["idx"].tolist() == [[last]]
     np.testing.assert_allclose(out["y"][0], expert(cfg.E) + 0.5 * expert(last), rtol=1e-13, atol=0)
+    G = cfg.E + 1
+    per = oracle.expert_outputs_a8(inp, np.zeros(G, dtype=np.int32), np.arange(G, dtype=np.int32))
+    for g in range(G):
+        np.testing.assert_allclose(per[g], expert(g), rtol=1e-13, atol=0)
