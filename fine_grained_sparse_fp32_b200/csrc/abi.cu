@@ -140,8 +140,10 @@ static size_t ffn_ws_bytes(int N, int d, int K, int I, int w_dtype)
     return c.used;
 }
 
-// Give-up limit of the pipeline waits of the kernels this thread launches.
-static long long wait_limit() { return kDefaultWaitLimit; }
+// Give-up limit of the pipeline waits of the FFN kernels this thread
+// launches (moe_set_wait_limit; 0 = the default).
+static thread_local long long g_wait_limit = 0;
+static long long wait_limit() { return g_wait_limit > 0 ? g_wait_limit : kDefaultWaitLimit; }
 
 // Workspace of the whole forward; every entry point uses a prefix-compatible
 // subset (router: logits; permute: chunk histograms; grouped FFN: H).
@@ -216,11 +218,11 @@ static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int 
     if (path == kPathSwap)
         return launch_ffn_swap(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, w_dtype, r, s,
                                static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
-                               static_cast<__nv_bfloat16 *>(y_shared), status, status + kSyncOffset, st);
+                               static_cast<__nv_bfloat16 *>(y_shared), status, status + kSyncOffset, wait_limit(), st);
     if (path == kPathTc)
         return launch_ffn_tc(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, w_dtype, r, s,
                              static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
-                             static_cast<__nv_bfloat16 *>(y_shared), status, status + kSyncOffset, st);
+                             static_cast<__nv_bfloat16 *>(y_shared), status, status + kSyncOffset, wait_limit(), st);
     return launch_ffn_stream(x, x_dtype, N, d, I, E, K, perm, offsets, w_dtype, r, s, h, y_perm, y_shared, st);
 }
 
@@ -511,6 +513,14 @@ kmoe_status moe_quant_1x128(const void *x, int rows, int cols, uint8_t *codes, f
     KMOE_TRY(check_ptr(scales, "scales"));
     return launch_quant_1x128(static_cast<const __nv_bfloat16 *>(x), rows, cols, codes, scales,
                               static_cast<cudaStream_t>(stream));
+}
+
+kmoe_status moe_set_wait_limit(long long cycles)
+{
+    clear_error();
+    if (cycles < 0) return fail(KMOE_ERR_INVALID_ARG, "wait limit %lld cycles must be >= 0", cycles);
+    g_wait_limit = cycles;
+    return KMOE_OK;
 }
 
 kmoe_status moe_device_status(const void *ws, int *status, void *stream)

@@ -116,7 +116,8 @@ combine_bulk_kernel(const __nv_bfloat16 *__restrict__ y_perm, const __nv_bfloat1
         uint8_t *dst = cb_smem + (size_t)s * stage_bytes;
         mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
         for (int k = 0; k < K; ++k)
-            bulk_load(dst + (size_t)k * row_bytes, y_perm + (size_t)inv[(size_t)t * K + k] * d, (uint32_t)row_bytes,
+            bulk_load(dst + (size_t)k * row_bytes,
+                      y_perm + (size_t)checked_index(inv[(size_t)t * K + k], 0, N * K, err) * d, (uint32_t)row_bytes,
                       &full[s]);
         if (y_shared) bulk_load(dst + (size_t)K * row_bytes, y_shared + (size_t)t * d, (uint32_t)row_bytes, &full[s]);
     };

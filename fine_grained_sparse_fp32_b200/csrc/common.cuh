@@ -11,6 +11,47 @@
 
 namespace kmoe {
 
+// Index checks of the KMOE_DEBUG build (nvcc -DKMOE_DEBUG): a kernel that
+// reads a dispatch index outside its range (a token or dispatched row past the
+// batch, expert offsets that are not a monotone partition of the N*K rows)
+// records kErrIndex in the device status word and uses a safe index (or skips
+// the work) instead, so that no access leaves its buffer. Compiled out of the
+// release library.
+#ifdef KMOE_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+enum : int { kErrIndex = 3 };
+
+// Debug build: v if lo <= v < hi, else records kErrIndex in *err and returns lo.
+__device__ __forceinline__ int checked_index(int v, int lo, int hi, int *err)
+{
+    if constexpr (kDebugChecks) {
+        if (v < lo || v >= hi) {
+            if (err) atomicCAS(err, 0, kErrIndex);
+            return lo;
+        }
+    }
+    return v;
+}
+
+// Debug build: whether off[0..E] is 0, monotone and ends at rows (one warp;
+// records kErrIndex in *err otherwise). Always true in the release build.
+__device__ __forceinline__ bool offsets_ok(const int *off, int E, int rows, int *err)
+{
+    if constexpr (kDebugChecks) {
+        const int lane = threadIdx.x & 31;
+        bool bad = false;
+        for (int i = lane; i < E; i += 32) bad |= off[i] > off[i + 1];
+        if (lane == 0) bad |= off[0] != 0 || off[E] != rows;
+        bad = __any_sync(0xffffffffu, bad);
+        if (bad && lane == 0 && err) atomicCAS(err, 0, kErrIndex);
+        return !bad;
+    }
+    return true;
+}
+
 // Default give-up limit of a pipeline wait, in SM clock cycles (about 2 s at
 // 1.9 GHz): far beyond any wait of a healthy launch. Waits that drain
 // in-flight copies after another wait gave up always use this limit.
@@ -195,7 +236,7 @@ kmoe_status launch_ffn_stream(const void *x, int x_dtype, int N, int d, int I, i
 kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
                           const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
                           __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err, int *sync,
-                          cudaStream_t st);
+                          long long wait_limit, cudaStream_t st);
 
 // Batches of at least this many tokens take the tensor-core FFN.
 constexpr int kTcMinTokens = 256;
@@ -203,11 +244,13 @@ constexpr int kTcMinTokens = 256;
 // Swap-AB tensor-core FFN for small batches (BF16 activations; BF16 or
 // E4M3 + FP32 block-scale weights; d % 256 == 0). `sync` holds kSyncInts
 // counters that must be zero at launch (a unit counter and one per expert).
+// wait_limit (both tensor-core FFNs): SM cycles before a pipeline wait gives
+// up and the kernel writes status 1 and returns.
 constexpr int kSyncInts = 1088;
 kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
                             const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
                             __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status,
-                            int *sync, cudaStream_t st);
+                            int *sync, long long wait_limit, cudaStream_t st);
 
 // Grouped FFN with FP8 activations (E4M3 weights + FP32 128 x 128 block
 // scales; x given as E4M3 codes xq [N, d] with FP32 scales xs [N, d / 128];

@@ -23,16 +23,23 @@
 // K block, the chunk's codes (kNT rows x 128 bytes) the B operand; four
 // K = 32 MMAs per tile and block.
 //
-// Warp roles (one CTA per SM, persistent):
-//   warps 0-3  promotion: tcgen05.ld of each partial slot, scale and add into
-//              registers (thread = weight row of its quadrant), then the
-//              unit's epilogue (SwiGLU + H quantisation, or the BF16 output);
-//   warp  4    one thread issues tcgen05.mma / tcgen05.commit;
-//   warp  5    producer: TMA of the weight tiles (lane 0) and of the token
-//              codes (x rows gathered four at a time, or one box of H rows);
-//   warp  6    scheduler: claims units, resolves them into shared-memory
-//              slots, and before a down unit waits (bounded) for the up units
-//              of its expert.
+// Chunks hold kNT = 16, 32 or 64 token rows (the host picks one from the
+// expected rows per expert): a weight tile crosses shared memory once per
+// chunk, so larger batches take larger chunks.
+//
+// Warp roles (one CTA per SM, persistent), P = 4 promotion warps for chunks
+// of up to 32 rows and 8 for 64:
+//   warps 0..P-1  promotion: tcgen05.ld of each partial slot, scale and add
+//                 into registers (thread = weight row of its quadrant, warp
+//                 w & 3; with 8 warps, warp w >> 2 takes token columns
+//                 32 (w >> 2) ..), then the unit's epilogue (SwiGLU + H
+//                 quantisation, or the BF16 output);
+//   warp  P       one thread issues tcgen05.mma / tcgen05.commit;
+//   warp  P+1     producer: TMA of the weight tiles (lane 0) and of the token
+//                 codes (x rows gathered four at a time, or one box of H rows);
+//   warp  P+2     scheduler: claims units, resolves them into shared-memory
+//                 slots, and before a down unit waits (bounded) for the up
+//                 units of its expert.
 #include "common.cuh"
 #include "sm100.cuh"
 #include "swap_units.cuh"
@@ -52,21 +59,24 @@ constexpr int kM = 128;                 // weight rows per tile (MMA M)
 constexpr int kBK = 128;                // K columns per stage: one scale block of both operands
 constexpr int kATile = kM * kBK;        // 16 KB of E4M3 weights
 constexpr int kNU = 8;                  // unit slots
-constexpr int kNP = 8;                  // partial-sum slots in tensor memory
-constexpr int kMmaWarp = 4, kProdWarp = 5, kSchedWarp = 6, kWarps = 7;
-constexpr int kEpiThreads = 128;
 constexpr int kSmemLimit = 232448;      // 227 KB per CTA
 
 template <int kNT>
 struct Cfg {
+    static constexpr int TPW = kNT < 32 ? kNT : 32;      // token columns of one promotion warp
+    static constexpr int PWarps = 4 * (kNT / TPW);       // promotion warps: 4 lane quadrants x column groups
+    static constexpr int PThreads = 32 * PWarps;
+    static constexpr int MmaWarp = PWarps, ProdWarp = PWarps + 1, SchedWarp = PWarps + 2, Warps = PWarps + 3;
     static constexpr int BTile = kNT * kBK;              // token codes of one stage
     static constexpr int Stage = 2 * kATile + BTile;     // weight tile 0 | weight tile 1 | token codes
-    static constexpr int Stages = kNT <= 16 ? 6 : 5;
+    static constexpr int Stages = kNT == 16 ? 6 : kNT == 32 ? 5 : 4;
     static constexpr int PW = 2 * kNT;                   // one partial slot: tile 0 | tile 1
-    static constexpr int TmemCols = kNP * PW <= 256 ? 256 : 512;
-    static_assert(kNT == 16 || kNT == 32, "token chunk of 16 or 32 rows");
+    static constexpr int NP = 512 / PW < 8 ? 512 / PW : 8;   // partial slots in tensor memory
+    static constexpr int TmemCols = NP * PW <= 256 ? 256 : 512;
+    static constexpr int RPL = (kNT + 31) / 32;          // chunk rows per scheduler lane
+    static_assert(kNT == 16 || kNT == 32 || kNT == 64, "token chunk of 16, 32 or 64 rows");
     static_assert(Stage % 1024 == 0, "tiles on 1024-byte boundaries (128-byte swizzle atoms)");
-    static_assert(kNP * PW <= TmemCols, "tensor memory columns");
+    static_assert(NP * PW <= TmemCols, "tensor memory columns");
 };
 
 template <int kNT>
@@ -83,15 +93,15 @@ struct Slot {
 template <int kNT>
 struct Tail {
     uint64_t full[6], empty[6];
-    uint64_t pfull[kNP], pempty[kNP];
+    uint64_t pfull[8], pempty[8];
     uint64_t ufull[kNU], uempty[kNU];
     uint64_t drain, pstart;
     uint32_t tmem_base;
     int abort;
     Slot<kNT> slot[kNU];
-    alignas(16) uint32_t amax[4][32];        // up epilogue: each warp's |H| maximum per token (float bits)
-    alignas(16) uint8_t codes[kNT][128];     // up epilogue: the unit's H codes, token-major
-    alignas(16) uint16_t stage[4][16][32];   // down epilogue: 16 tokens x 32 features per warp
+    alignas(16) uint32_t amax[4][kNT];                        // up epilogue: |H| maximum per quadrant and token (float bits)
+    alignas(16) uint8_t codes[kNT][128];                      // up epilogue: the unit's H codes, token-major
+    alignas(16) uint16_t stage[Cfg<kNT>::PWarps][16][32];     // down epilogue: 16 tokens x 32 features per warp
     int pre[kMaxOrd + 1];
     int off[kMaxOrd + 1];
 };
@@ -152,11 +162,12 @@ __device__ __forceinline__ uint8_t e4m3_code(float v)
 using namespace a8;
 
 template <int kNT>
-__global__ void __launch_bounds__(kWarps * 32, 1)
+__global__ void __launch_bounds__(Cfg<kNT>::Warps * 32, 1)
 ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
 {
     using C = Cfg<kNT>;
-    constexpr int SA = C::Stages;
+    constexpr int SA = C::Stages, NP = C::NP, TPW = C::TPW;
+    constexpr int kMmaWarp = C::MmaWarp, kProdWarp = C::ProdWarp, kSchedWarp = C::SchedWarp;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Tail<kNT> *T = reinterpret_cast<Tail<kNT> *>(smem + (size_t)SA * C::Stage);
@@ -169,9 +180,9 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
             mbar_init(&T->full[s], 1);                   // TMA expect_tx: weights and token codes
             mbar_init(&T->empty[s], 1);                  // tcgen05.commit
         }
-        for (int p = 0; p < kNP; ++p) {
+        for (int p = 0; p < NP; ++p) {
             mbar_init(&T->pfull[p], 1);                  // tcgen05.commit
-            mbar_init(&T->pempty[p], kEpiThreads);       // every promotion thread has read the slot
+            mbar_init(&T->pempty[p], C::PThreads);       // every promotion thread has read the slot
         }
         for (int j = 0; j < kNU; ++j) {
             mbar_init(&T->ufull[j], 1);
@@ -225,8 +236,15 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
             const swp::Unit U = swp::decode(u, T->pre, T->off, a);
             const int row0 = U.G.row0 + U.m0;
             const size_t ge = U.G.shared ? 0 : (size_t)U.G.g;
-            int srcv = 0;                                  // one chunk row per lane (kNT <= 32)
-            if (lane < U.mc) srcv = U.up ? (U.G.shared ? row0 + lane - a.N * a.K : a.perm[row0 + lane]) : row0 + lane;
+            int srcv[C::RPL];                              // chunk rows lane, lane + 32
+#pragma unroll
+            for (int i = 0; i < C::RPL; ++i) {
+                const int n = lane + 32 * i;
+                srcv[i] = 0;
+                if (n < U.mc)
+                    srcv[i] = U.up ? (U.G.shared ? row0 + n - a.N * a.K : checked_index(a.perm[row0 + n], 0, a.N, a.err))
+                                   : row0 + n;
+            }
             swp::WarpScales w0, w1;
             if (U.up) {
                 const int nkb = a.d / kBK;
@@ -255,7 +273,9 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                 }
             }
             if (!__shfl_sync(0xffffffffu, good ? 1 : 0, 0)) break;
-            if (lane < U.mc) sl.src[lane] = srcv;
+#pragma unroll
+            for (int i = 0; i < C::RPL; ++i)
+                if (lane + 32 * i < U.mc) sl.src[lane + 32 * i] = srcv[i];
             sl.s[0][lane] = w0.lo;
             sl.s[1][lane] = w1.lo;
             if (lane < 16) { sl.s[0][lane + 32] = w0.hi; sl.s[1][lane + 32] = w1.hi; }
@@ -332,9 +352,9 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                 const uint32_t id = idesc_e4m3_f32(kM, sl.nmma);
                 bool ok = true;
                 for (int kb = 0; kb < kb_n; ++kb, ++it) {
-                    const int s = it % SA, p = it % kNP;
+                    const int s = it % SA, p = it % NP;
                     if (!mbar_wait(&T->full[s], (it / SA) & 1, abort, a.err, lim) ||
-                        !mbar_wait(&T->pempty[p], ((it / kNP) & 1) ^ 1, abort, a.err, lim)) {
+                        !mbar_wait(&T->pempty[p], ((it / NP) & 1) ^ 1, abort, a.err, lim)) {
                         ok = false;
                         break;
                     }
@@ -357,12 +377,13 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
             mbar_wait_drain(&T->drain, 0, kDefaultWaitLimit);
         }
         __syncwarp();
-    } else if (warp < 4) {
+    } else if (warp < C::PWarps) {
         // ------------------------------------------------- promotion, epilogue
-        // Thread = weight row quad * 32 + lane of the unit's tiles; lane n of
-        // each warp also carries token n's activation scale of the current K
-        // block (loaded two blocks ahead) and hands it out by shuffle.
-        const int quad = warp;
+        // Thread = weight row quad * 32 + lane of the unit's tiles, for the
+        // token columns c0 .. c0 + TPW - 1 of the chunk; lane n also carries
+        // token c0 + n's activation scale of the current K block (loaded two
+        // blocks ahead) and hands it out by shuffle.
+        const int quad = warp & 3, c0 = (warp >> 2) * TPW;
         uint32_t it = 0;
         for (int us = 0;; ++us) {
             const int j = us % kNU;
@@ -371,34 +392,41 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
             if (sl.u < 0) break;
             const bool up = sl.up, shared = sl.shared;
             const int mc = sl.mc, f0 = sl.f0, r0 = sl.row0, o = sl.o, kb_n = sl.kb;
-            const bool mine = lane < mc;
+            const int tok = c0 + lane;                     // this lane's token column (scales, epilogue)
+            const bool mine = lane < TPW && tok < mc;
             const int nkb = up ? a.d / kBK : a.I / kBK;
-            const float *sp = up ? a.xs + (size_t)(mine ? sl.src[lane] : 0) * nkb
-                                 : a.hs + (size_t)(r0 + (mine ? lane : 0)) * nkb;
+            const float *sp = up ? a.xs + (size_t)(mine ? sl.src[tok] : 0) * nkb
+                                 : a.hs + (size_t)(r0 + (mine ? tok : 0)) * nkb;
             float sx0 = mine ? ld_relaxed_f32(sp) : 0.f;
             float sx1 = mine && kb_n > 1 ? ld_relaxed_f32(sp + 1) : 0.f;
-            float acc0[kNT], acc1[kNT];
+            float acc0[TPW], acc1[TPW];
 #pragma unroll
-            for (int n = 0; n < kNT; ++n) acc0[n] = acc1[n] = 0.f;
+            for (int n = 0; n < TPW; ++n) acc0[n] = acc1[n] = 0.f;
             bool ok = true;
             for (int kb = 0; kb < kb_n; ++kb, ++it) {
                 const float sx2 = mine && kb + 2 < kb_n ? ld_relaxed_f32(sp + kb + 2) : 0.f;
-                const int p = it % kNP;
-                if (!mbar_wait(&T->pfull[p], (it / kNP) & 1, abort, a.err, lim)) { ok = false; break; }
+                const int p = it % NP;
+                if (!mbar_wait(&T->pfull[p], (it / NP) & 1, abort, a.err, lim)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t v0[kNT], v1[kNT];
-                const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + p * C::PW;
-                tmem_load<kNT>(ta, v0);
-                tmem_load<kNT>(ta + kNT, v1);
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(&T->pempty[p]);
+                const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + p * C::PW + c0;
                 const float w0 = sl.s[0][kb], w1 = sl.s[1][kb];
+                {
+                    uint32_t v[TPW];                       // tile 0 (gate or the first W_d rows)
+                    tmem_load<TPW>(ta, v);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int n = 0; n < kNT; ++n) {
-                    const float sn = __shfl_sync(0xffffffffu, sx0, n);
-                    acc0[n] = fmaf(__uint_as_float(v0[n]), w0 * sn, acc0[n]);
-                    acc1[n] = fmaf(__uint_as_float(v1[n]), w1 * sn, acc1[n]);
+                    for (int n = 0; n < TPW; ++n)
+                        acc0[n] = fmaf(__uint_as_float(v[n]), w0 * __shfl_sync(0xffffffffu, sx0, n), acc0[n]);
+                }
+                {
+                    uint32_t v[TPW];                       // tile 1 (up or the next W_d rows)
+                    tmem_load<TPW>(ta + kNT, v);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    mbar_arrive(&T->pempty[p]);
+#pragma unroll
+                    for (int n = 0; n < TPW; ++n)
+                        acc1[n] = fmaf(__uint_as_float(v[n]), w1 * __shfl_sync(0xffffffffu, sx0, n), acc1[n]);
                 }
                 sx0 = sx1;
                 sx1 = sx2;
@@ -406,36 +434,37 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
             if (!ok) break;
             if (up) {
                 // H = bf16(SiLU(gate) * up); each token's 128 features (this
-                // unit's rows) form one 1 x 128 group: scale = amax / 448,
-                // code = E4M3(h / scale), the quotient in FP32.
-                float hv[kNT];
+                // unit's rows, spread over the four lane quadrants) form one
+                // 1 x 128 group: scale = amax / 448, code = E4M3(h / scale),
+                // the quotient in FP32.
+                float hv[TPW];
 #pragma unroll
-                for (int n = 0; n < kNT; ++n) {
+                for (int n = 0; n < TPW; ++n) {
                     hv[n] = __bfloat162float(__float2bfloat16_rn(silu_mul(acc0[n], acc1[n])));
                     const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[n])));
-                    if (lane == n) T->amax[quad][n] = m;
+                    if (lane == n) T->amax[quad][c0 + n] = m;
                 }
-                swp::epi_sync<kEpiThreads>();
-                float s_l = 1.f;                           // lane n: scale of token n
-                if (lane < kNT) {
-                    const float am = fmaxf(fmaxf(__uint_as_float(T->amax[0][lane]), __uint_as_float(T->amax[1][lane])),
-                                           fmaxf(__uint_as_float(T->amax[2][lane]), __uint_as_float(T->amax[3][lane])));
+                swp::epi_sync<C::PThreads>();
+                float s_l = 1.f;                           // lane n: scale of token c0 + n
+                if (lane < TPW) {
+                    const float am = fmaxf(fmaxf(__uint_as_float(T->amax[0][tok]), __uint_as_float(T->amax[1][tok])),
+                                           fmaxf(__uint_as_float(T->amax[2][tok]), __uint_as_float(T->amax[3][tok])));
                     s_l = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
                 }
 #pragma unroll
-                for (int n = 0; n < kNT; ++n) {
+                for (int n = 0; n < TPW; ++n) {
                     const float sn = __shfl_sync(0xffffffffu, s_l, n);
-                    T->codes[n][quad * 32 + lane] = e4m3_code(__fdiv_rn(hv[n], sn));
+                    T->codes[c0 + n][quad * 32 + lane] = e4m3_code(__fdiv_rn(hv[n], sn));
                 }
-                swp::epi_sync<kEpiThreads>();
+                swp::epi_sync<C::PThreads>();
                 // 16-byte pieces: token n = i / 8, piece i % 8 of its 128 codes
-                for (int i = threadIdx.x; i < kNT * 8; i += kEpiThreads) {
+                for (int i = threadIdx.x; i < kNT * 8; i += C::PThreads) {
                     const int n = i >> 3, pc = i & 7;
                     if (n < mc)
                         *reinterpret_cast<uint4 *>(a.hq + (size_t)(r0 + n) * a.I + f0 + pc * 16) =
                             *reinterpret_cast<const uint4 *>(&T->codes[n][pc * 16]);
                 }
-                if (quad == 0 && mine) a.hs[(size_t)(r0 + lane) * (a.I / kBK) + f0 / kBK] = s_l;
+                if (quad == 0 && mine) a.hs[(size_t)(r0 + tok) * (a.I / kBK) + f0 / kBK] = s_l;
                 __threadfence();                           // H codes and scales visible before the count rises
             } else {
                 // Y = BF16 of the two tiles (features f0 .. f0+127, f0+128 ..
@@ -444,11 +473,11 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                 __nv_bfloat16 *dst = shared ? a.y_shared + (size_t)(r0 - a.N * a.K) * a.d
                                             : a.y_perm + (size_t)r0 * a.d;
                 dst += f0 + quad * 32;
-                uint16_t *stg = &T->stage[quad][0][0];
+                uint16_t *stg = &T->stage[warp][0][0];
 #pragma unroll
                 for (int t = 0; t < 2; ++t)
 #pragma unroll
-                    for (int half = 0; half < kNT / 16; ++half) {
+                    for (int half = 0; half < TPW / 16; ++half) {
 #pragma unroll
                         for (int n = 0; n < 16; ++n) {
                             const float v = t ? acc1[half * 16 + n] : acc0[half * 16 + n];
@@ -458,15 +487,15 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int idx = lane + 32 * hh, n = idx >> 2, pc = idx & 3;
-                            const int tok = half * 16 + n;
-                            if (tok < mc)
-                                *reinterpret_cast<uint4 *>(dst + t * kM + (size_t)tok * a.d + pc * 8) =
+                            const int tk = c0 + half * 16 + n;
+                            if (tk < mc)
+                                *reinterpret_cast<uint4 *>(dst + t * kM + (size_t)tk * a.d + pc * 8) =
                                     *reinterpret_cast<const uint4 *>(stg + n * 32 + pc * 8);
                         }
                         __syncwarp();
                     }
             }
-            swp::epi_sync<kEpiThreads>();                  // the slot and the staging areas are free
+            swp::epi_sync<C::PThreads>();                  // the slot and the staging areas are free
             if (threadIdx.x == 0) {
                 if (up) swp::red_release_add(a.up_done + o, 1);
                 mbar_arrive(&T->uempty[j]);
@@ -539,7 +568,7 @@ static kmoe_status launch_a8_cfg(const ExpertPtrs &routed, const ExpertPtrs &sh,
     static_assert(smem <= (size_t)kSmemLimit, "shared memory per CTA");
     auto k = ffn_a8_kernel<kNT>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    launch_pdl(k, a8_sm_count(), kWarps * 32, smem, st, m, a);
+    launch_pdl(k, a8_sm_count(), Cfg<kNT>::Warps * 32, smem, st, m, a);
     return check_launch("ffn_a8");
 }
 
@@ -571,9 +600,13 @@ kmoe_status launch_ffn_a8(const uint8_t *xq, const float *xs, int N, int d, int 
     a.has_shared = shared ? 1 : 0;
     a.n_ord = E + a.has_shared;
     a.sk = kBK;
-    // 16-row chunks while experts see a token or two, 32 rows for larger batches
-    // (each weight tile is then read by half as many chunks)
-    return N < kTcMinTokens ? launch_a8_cfg<16>(routed, sh, a, st) : launch_a8_cfg<32>(routed, sh, a, st);
+    // Chunk rows from the expected rows per routed expert, N * K / E: 16 while
+    // experts see a dozen tokens or fewer, then 32, then 64 (a weight tile
+    // crosses shared memory once per chunk).
+    const long long avg = (long long)N * K / E;
+    if (avg <= 12) return launch_a8_cfg<16>(routed, sh, a, st);
+    if (avg <= 32) return launch_a8_cfg<32>(routed, sh, a, st);
+    return launch_a8_cfg<64>(routed, sh, a, st);
 }
 
 }  // namespace kmoe

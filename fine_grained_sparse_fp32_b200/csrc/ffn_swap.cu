@@ -59,7 +59,7 @@ namespace swp {
 constexpr int kM = 128;                 // weight rows per tile (MMA M)
 constexpr int kATile = kM * 128;        // 16 KB: 128 rows x 128 bytes
 constexpr int kNU = 8;                  // unit-info slots
-constexpr long long kWaitLimit = 1LL << 32;   // SM cycles, about 2 s
+constexpr long long kWaitLimit = kDefaultWaitLimit;   // SM cycles, about 2 s: waits that drain after a give-up
 constexpr int kSmemLimit = 232448;            // 227 KB per CTA
 
 // Per configuration: kNT = token rows per unit at most (16 at decode, 128 at
@@ -146,6 +146,7 @@ struct Args {
     int *err;                         // device status word
     int *claim;                       // unit counter (zero at launch)
     int *up_done;                     // [groups] finished up units (zero at launch)
+    long long wait_limit;             // SM cycles before a pipeline wait gives up
     int N, K, E, d, I, has_shared, n_ord;
     int sk;                           // k per stage
     int nt;                           // token rows per unit at most
@@ -271,8 +272,8 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
         const int total = total_units(T->pre, a);
         for (int us = 0;; ++us) {
             const int j = us % kNU;
-            if (!mbar_wait(&T->uempty[j], ((us / kNU) & 1) ^ 1, abort, a.err, kWaitLimit)) break;
-            if (us > 0 && !mbar_wait(&T->pstart, (us - 1) & 1, abort, a.err, kWaitLimit)) break;
+            if (!mbar_wait(&T->uempty[j], ((us / kNU) & 1) ^ 1, abort, a.err, a.wait_limit)) break;
+            if (us > 0 && !mbar_wait(&T->pstart, (us - 1) & 1, abort, a.err, a.wait_limit)) break;
             int u = 0;
             if (lane == 0) u = atomicAdd(a.claim, 1);
             u = __shfl_sync(0xffffffffu, u, 0);
@@ -296,7 +297,8 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 const int n = lane + 32 * i;
                 srcv[i] = 0;
                 if (n < U.mc)
-                    srcv[i] = U.up ? (U.G.shared ? row0 + n - a.N * a.K : a.perm[row0 + n]) : row0 + n;
+                    srcv[i] = U.up ? (U.G.shared ? row0 + n - a.N * a.K : checked_index(a.perm[row0 + n], 0, a.N, a.err))
+                                   : row0 + n;
             }
             WarpScales w0, w1;
             w0.lo = w0.hi = w1.lo = w1.hi = 0.f;
@@ -331,7 +333,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 const long long t0 = clock64();
                 while (ld_acquire(a.up_done + U.o) < need) {
                     if (*abort) { good = false; break; }
-                    if (clock64() - t0 > kWaitLimit) {
+                    if (clock64() - t0 > a.wait_limit) {
                         *abort = 1;
                         atomicCAS(a.err, kErrNone, kErrWaitTimeout);
                         good = false;
@@ -370,7 +372,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
         bool ok = true;
         for (int us = 0;; ++us) {
             const int j = us % kNU;
-            if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+            if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, a.wait_limit)) { ok = false; break; }
             const Slot<kNT> &sl = T->slot[j];
             if (sl.u < 0) break;
             const bool up = sl.up, shared = sl.shared;
@@ -387,7 +389,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
             const uint32_t bbytes = (uint32_t)(up ? nmma : kNT) * 128 * NP;
             for (int kb = 0; kb < kb_n; ++kb, ++it) {
                 const int s = it % SA;
-                if (!mbar_wait(&T->empty[s], ((it / SA) & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                if (!mbar_wait(&T->empty[s], ((it / SA) & 1) ^ 1, abort, a.err, a.wait_limit)) { ok = false; break; }
                 uint8_t *A = smem + (size_t)s * C::Stage;
                 uint8_t *B = A + 2 * kATile;
                 if (lane == 0) {
@@ -418,13 +420,13 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
             uint32_t it = 0;
             for (int us = 0;; ++us) {
                 const int j = us % kNU;
-                if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, kWaitLimit)) break;
+                if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, a.wait_limit)) break;
                 const Slot<kNT> &sl = T->slot[j];
                 if (sl.u < 0) break;
                 const bool up = sl.up;
                 const int kb_n = sl.kb;
                 const int acc = us % C::NAcc;
-                if (!mbar_wait(&T->tempty[acc], ((us / C::NAcc) & 1) ^ 1, abort, a.err, kWaitLimit)) break;
+                if (!mbar_wait(&T->tempty[acc], ((us / C::NAcc) & 1) ^ 1, abort, a.err, a.wait_limit)) break;
                 tc_fence_after();
                 const uint32_t dg = tmem + acc * C::AccW;          // gate (or W_d) accumulator
                 const uint32_t du = dg + kNT;                      // up accumulator
@@ -433,7 +435,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 for (int kb = 0; kb < kb_n; ++kb, ++it) {
                     if (kFp8) {       // A: F16 in tensor memory (8 columns per k16); B: F16 panels
                         const int cs = it % C::ConvStages;
-                        if (!mbar_wait(&T->cfull[cs], (it / C::ConvStages) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                        if (!mbar_wait(&T->cfull[cs], (it / C::ConvStages) & 1, abort, a.err, a.wait_limit)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t at = tmem + C::AccCols + cs * C::ConvCols;
                         // token tile 0 carries the first weight tile's block scale, tile 1 the second's
@@ -454,7 +456,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                         umma_commit(&T->cempty[cs]);
                     } else {
                         const int s = it % SA;
-                        if (!mbar_wait(&T->full[s], (it / SA) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                        if (!mbar_wait(&T->full[s], (it / SA) & 1, abort, a.err, a.wait_limit)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t sa = smem_u32(smem + (size_t)s * C::Stage);
                         const uint64_t a0 = sw128_kmajor_desc(sa), a1 = sw128_kmajor_desc(sa + kATile);
@@ -486,14 +488,14 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
         uint16_t *stg = &T->stage[eg * 4 + quad][0][0];
         for (int us = 0;; ++us) {
             const int j = us % kNU;
-            if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, kWaitLimit)) break;
+            if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, a.wait_limit)) break;
             const Slot<kNT> &sl = T->slot[j];
             if (sl.u < 0) break;
             const bool up = sl.up, shared = sl.shared;
             const int mc = sl.mc, nmma = sl.nmma, f0 = sl.f0, r0 = sl.row0, o = sl.o;
             const float s0 = kFp8 ? sl.ref[0] : 1.f, s1 = kFp8 ? sl.ref[1] : 1.f;
             const int acc = us % C::NAcc;
-            if (!mbar_wait(&T->tfull[acc], (us / C::NAcc) & 1, abort, a.err, kWaitLimit)) break;
+            if (!mbar_wait(&T->tfull[acc], (us / C::NAcc) & 1, abort, a.err, a.wait_limit)) break;
             tc_fence_after();
             const uint32_t tg = tmem + ((uint32_t)(quad * 32) << 16) + acc * C::AccW;
             const int ld = up ? a.I : a.d;               // row stride of the output
@@ -558,7 +560,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
         bool ok = true;
         for (int us = 0; ok; ++us) {
             const int j = us % kNU;
-            if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, kWaitLimit)) break;
+            if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, a.wait_limit)) break;
             const Slot<kNT> &sl = T->slot[j];
             if (sl.u < 0) break;
             const bool up = sl.up;
@@ -570,8 +572,8 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 if ((int)(it % kConvGroups) != grp) continue;
                 const int s = it % SA, cs = it % C::ConvStages;
                 const float r0 = sl.s[0][kb] * inv0, r1 = sl.s[1][kb] * inv1;     // in [0, 1]
-                if (!mbar_wait(&T->full[s], (it / SA) & 1, abort, a.err, kWaitLimit) ||
-                    !mbar_wait(&T->cempty[cs], ((it / C::ConvStages) & 1) ^ 1, abort, a.err, kWaitLimit)) {
+                if (!mbar_wait(&T->full[s], (it / SA) & 1, abort, a.err, a.wait_limit) ||
+                    !mbar_wait(&T->cempty[cs], ((it / C::ConvStages) & 1) ^ 1, abort, a.err, a.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -694,7 +696,7 @@ static void launch_cfg(const Maps &m, const Args &a, cudaStream_t st)
 kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
                             const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
                             __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status,
-                            int *sync, cudaStream_t st)
+                            int *sync, long long wait_limit, cudaStream_t st)
 {
     constexpr int token_chunk = 16;
     if (E + 1 > kMaxOrd || E + 2 > kSyncInts) return fail(KMOE_ERR_UNSUPPORTED, "swap-AB FFN: too many experts");
@@ -720,6 +722,7 @@ kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, 
     a.err = status;
     a.claim = sync;
     a.up_done = sync + 1;
+    a.wait_limit = wait_limit;
     a.N = N; a.K = K; a.E = E; a.d = d; a.I = I;
     a.has_shared = shared ? 1 : 0;
     a.n_ord = E + a.has_shared;

@@ -76,7 +76,7 @@ constexpr int kConvThreads = 256;            // one converter thread per weight 
 __host__ __device__ constexpr int threads_of(bool fp8) { return (fp8 ? 18 : 10) * 32; }
 constexpr int kMaxGroups = 1025;
 constexpr int kTQ = 4;                       // tile queue depth
-constexpr long long kWaitLimit = 1LL << 32;  // SM cycles (about 2 s)
+constexpr long long kWaitLimit = kDefaultWaitLimit;   // SM cycles (about 2 s): waits that drain after a give-up
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w)
 {
@@ -107,6 +107,7 @@ struct TcArgs {
     const float *s0_routed, *s1_routed, *s0_shared, *s1_shared;
     int *err;
     int *tile_ctr;            // tiles claimed so far by all CTAs (zero at launch)
+    long long wait_limit;     // SM cycles before a pipeline wait gives up
 };
 
 struct SmemTail {
@@ -168,10 +169,10 @@ __device__ __forceinline__ int claim_to_tile(int c, int routed, int total)
 
 // The next tile of this CTA (or -1: no more, -2: a wait gave up), published
 // by the weight producer in the tile queue.
-__device__ __forceinline__ int tq_take(SmemTail *tail, uint32_t q, volatile int *abort, int *err)
+__device__ __forceinline__ int tq_take(SmemTail *tail, uint32_t q, volatile int *abort, int *err, long long limit)
 {
     const int s = q % kTQ;
-    if (!mbar_wait(&tail->tqfull[s], (q / kTQ) & 1, abort, err, kWaitLimit)) return -2;
+    if (!mbar_wait(&tail->tqfull[s], (q / kTQ) & 1, abort, err, limit)) return -2;
     const int t = reinterpret_cast<volatile int *>(tail->tq)[s];
     mbar_arrive(&tail->tqempty[s]);
     return t;
@@ -181,6 +182,11 @@ __device__ __forceinline__ int tq_take(SmemTail *tail, uint32_t q, volatile int 
 __device__ __forceinline__ void build_prefix(int *pre, const TcArgs &a)
 {
     const int lane = threadIdx.x & 31;
+    if (!offsets_ok(a.offsets, a.E, a.N * a.K, a.err)) {   // debug build: no tiles at all
+        for (int i = lane; i <= a.groups; i += 32) pre[i] = 0;
+        __syncwarp();
+        return;
+    }
     const int per = (a.groups + 31) / 32;
     const int g0 = lane * per;
     int sum = 0;
@@ -359,7 +365,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         uint32_t it = 0;
         bool ok = true;
         for (uint32_t tq = 0; ok; ++tq) {
-            const int t = tq_take(tail, tq, abort, a.err);
+            const int t = tq_take(tail, tq, abort, a.err, a.wait_limit);
             if (t < 0) break;
             const Tile T = decode_tile(t, tail->pre, a, bn);
             const size_t ge = T.shared ? 0 : (size_t)T.g;
@@ -377,8 +383,8 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                     sc0 = s0[si];
                     sc1 = s0[si + a.I / 128];
                 }
-                if (!mbar_wait(&tail->sfull[ss], (it / kSStages) & 1, abort, a.err, kWaitLimit) ||
-                    !mbar_wait(&tail->bempty[sb], ((it / kBS) & 1) ^ 1, abort, a.err, kWaitLimit)) {
+                if (!mbar_wait(&tail->sfull[ss], (it / kSStages) & 1, abort, a.err, a.wait_limit) ||
+                    !mbar_wait(&tail->bempty[sb], ((it / kBS) & 1) ^ 1, abort, a.err, a.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -407,7 +413,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                 const int c = atomicAdd(a.tile_ctr, 1);
                 const int t = c < total ? claim_to_tile(c, routed_tiles, total) : -1;
                 const int qs = tq % kTQ;
-                if (!mbar_wait(&tail->tqempty[qs], ((tq / kTQ) & 1) ^ 1, abort, a.err, kWaitLimit)) {
+                if (!mbar_wait(&tail->tqempty[qs], ((tq / kTQ) & 1) ^ 1, abort, a.err, a.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -422,7 +428,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                 const int r0 = kUp ? gi * a.I + T.n0 : gi * a.d + T.n0;
                 for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
                     const int s = it % S;
-                    if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                    if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort, a.err, a.wait_limit)) { ok = false; break; }
                     uint8_t *dst = ring + (size_t)s * bytes;
                     mbar_arrive_expect_tx(&full[s], bytes);
                     // rows 0-127: gate (up) or W_d rows n0..; rows 128-255: up rows n0.. or W_d rows n0+128..
@@ -447,23 +453,25 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             // instruction of a warp reads four whole 128-byte row segments.
             const int pw = p >> 5, pl = p & 31, pc = pl & 7;
             for (uint32_t tq = 0; ok; ++tq) {
-                const int t = tq_take(tail, tq, abort, a.err);
+                const int t = tq_take(tail, tq, abort, a.err, a.wait_limit);
                 if (t < 0) break;
                 const Tile T = decode_tile(t, tail->pre, a, bn);
                 int tok0[8], tok1[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int r = pw * 32 + 4 * j + (pl >> 3);
-                    tok0[j] = r >= T.rows ? -1 : T.shared ? T.row0 + r - a.N * a.K : a.perm[T.row0 + r];
+                    tok0[j] = r >= T.rows ? -1
+                              : T.shared  ? T.row0 + r - a.N * a.K
+                                          : checked_index(a.perm[T.row0 + r], 0, a.N, a.err);
                     tok1[j] = r + kBM >= T.rows ? -1
                               : T.shared        ? T.row0 + kBM + r - a.N * a.K
-                                                : a.perm[T.row0 + kBM + r];
+                                                : checked_index(a.perm[T.row0 + kBM + r], 0, a.N, a.err);
                 }
                 const int mt = T.two ? 2 : 1;
                 for (int kb = 0; kb < a.kblocks && ok; ++kb) {
                     for (int m = 0; m < mt; ++m, ++ia) {
                         const int sa = ia % kAS;
-                        if (!mbar_wait(&tail->aempty[sa], ((ia / kAS) & 1) ^ 1, abort, a.err, kWaitLimit)) {
+                        if (!mbar_wait(&tail->aempty[sa], ((ia / kAS) & 1) ^ 1, abort, a.err, a.wait_limit)) {
                             ok = false;
                             break;
                         }
@@ -482,14 +490,14 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             cp_async_wait_all();   // this thread's row copies have landed before it leaves
         } else if (p == 0) {
             for (uint32_t tq = 0; ok; ++tq) {
-                const int t = tq_take(tail, tq, abort, a.err);
+                const int t = tq_take(tail, tq, abort, a.err, a.wait_limit);
                 if (t < 0) break;
                 const Tile T = decode_tile(t, tail->pre, a, bn);
                 const int mt = T.two ? 2 : 1;
                 for (int kb = 0; kb < a.kblocks && ok; ++kb) {
                     for (int m = 0; m < mt; ++m, ++ia) {
                         const int sa = ia % kAS;
-                        if (!mbar_wait(&tail->aempty[sa], ((ia / kAS) & 1) ^ 1, abort, a.err, kWaitLimit)) {
+                        if (!mbar_wait(&tail->aempty[sa], ((ia / kAS) & 1) ^ 1, abort, a.err, a.wait_limit)) {
                             ok = false;
                             break;
                         }
@@ -515,7 +523,7 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             int hn = 0;
             bool ok = true;
             for (uint32_t tq = 0; ok; ++tq) {
-                const int t = tq_take(tail, tq, abort, a.err);
+                const int t = tq_take(tail, tq, abort, a.err, a.wait_limit);
                 if (t < 0) break;
                 const Tile T = decode_tile(t, tail->pre, a, bn);
                 const int h0 = hn, h1 = hn ^ 1;
@@ -523,13 +531,13 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                 const int mt = T.two ? 2 : 1;
                 for (int kb = 0; kb < a.kblocks && ok; ++kb, ++ib) {
                     const int sb = ib % kBS;
-                    if (!mbar_wait(&tail->bfull[sb], (ib / kBS) & 1, abort, a.err, kWaitLimit)) { ok = false; break; }
+                    if (!mbar_wait(&tail->bfull[sb], (ib / kBS) & 1, abort, a.err, a.wait_limit)) { ok = false; break; }
                     const uint64_t bd = sw128_kmajor_desc(smem_u32(ring_b + (size_t)sb * kBTile));
                     for (int m = 0; m < mt; ++m, ++ia) {
                         const int sa = ia % kAS, h = m ? h1 : h0;
-                        if (!mbar_wait(&tail->afull[sa], (ia / kAS) & 1, abort, a.err, kWaitLimit) ||
+                        if (!mbar_wait(&tail->afull[sa], (ia / kAS) & 1, abort, a.err, a.wait_limit) ||
                             (kb == 0 &&   // half h drained by the epilogue of its last use
-                             !mbar_wait(&tail->tempty[h], ((m ? c1 : c0) & 1) ^ 1, abort, a.err, kWaitLimit))) {
+                             !mbar_wait(&tail->tempty[h], ((m ? c1 : c0) & 1) ^ 1, abort, a.err, a.wait_limit))) {
                             ok = false;
                             break;
                         }
@@ -559,11 +567,11 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         int hn = 0;                       // the half rotation of the MMA thread, replayed
         const uint32_t stage = smem_u32(epi) + warp * 4096;
         for (;; ++at) {
-            const int t = tq_take(tail, at, abort, a.err);
+            const int t = tq_take(tail, at, abort, a.err, a.wait_limit);
             if (t < 0) break;
             const Tile T = decode_tile(t, tail->pre, a, bn);
             const int h0 = hn, h1 = hn ^ 1;
-            if (!mbar_wait(&tail->tfull, at & 1, abort, a.err, kWaitLimit)) break;
+            if (!mbar_wait(&tail->tfull, at & 1, abort, a.err, a.wait_limit)) break;
             tc_fence_after();
             const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
             epilogue_half<kUp>(tlane + h0 * kBN, T, a, 0, stage);
@@ -677,7 +685,7 @@ static kmoe_status run_tc(const TcMaps &up, const TcMaps &dn, TcArgs a, int d, i
 kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
                           const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
                           __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err, int *sync,
-                          cudaStream_t st)
+                          long long wait_limit, cudaStream_t st)
 {
     if (E + 1 > kMaxGroups) return fail(KMOE_ERR_UNSUPPORTED, "tensor-core FFN: too many experts");
     const bool fp8 = w_dtype == KMOE_E4M3_B128;
@@ -704,6 +712,7 @@ kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, in
     a.d = d;
     a.I = I;
     a.err = err;
+    a.wait_limit = wait_limit;
     if (fp8) return run_tc<true>(up, dn, a, d, I, sync, h, y_perm, y_shared, routed, sh, st);
     return run_tc<false>(up, dn, a, d, I, sync, h, y_perm, y_shared, routed, sh, st);
 }

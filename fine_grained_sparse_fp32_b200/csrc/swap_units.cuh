@@ -12,7 +12,7 @@
 //             W_d rows against the chunk's H rows.
 // Every kernel argument struct A used with these helpers has the fields
 // offsets, N, K, E, d, I, has_shared, n_ord (groups), nt (rows per chunk)
-// and sk (K columns per pipeline stage).
+// and sk (K columns per pipeline stage), and err (the device status word).
 #pragma once
 
 #include <cstdint>
@@ -58,6 +58,11 @@ __device__ void build_prefix(int *pre, int *off, const A &a)
     const int lane = threadIdx.x & 31;
     for (int i = lane; i <= a.E; i += 32) off[i] = a.offsets[i];
     __syncwarp();
+    if (!offsets_ok(off, a.E, a.N * a.K, a.err)) {     // debug build: no units at all
+        for (int i = lane; i <= a.n_ord; i += 32) pre[i] = 0;
+        __syncwarp();
+        return;
+    }
     const int per = (a.n_ord + 31) / 32;
     const int o0 = lane * per;
     int sum = 0;

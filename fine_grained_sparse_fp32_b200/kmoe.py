@@ -23,7 +23,7 @@ FFN_STATUS_BYTES = (64 + 1088) * 4
 
 EXPORTS = ["moe_workspace_size", "moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn",
            "moe_combine", "moe_forward", "moe_block_workspace_size", "moe_block_forward", "moe_quant_1x128",
-           "moe_device_status", "moe_last_error", "moe_abi_version"]
+           "moe_device_status", "moe_set_wait_limit", "moe_last_error", "moe_abi_version"]
 
 
 class KmoeError(RuntimeError):
@@ -43,11 +43,12 @@ _lib = None
 
 
 def load(path: str | None = None):
-    """Load libkmoe.so; raises if it has not been built."""
+    """Load libkmoe.so (or the library named by KMOE_LIBRARY, e.g. the KMOE_DEBUG build);
+    raises if it has not been built."""
     global _lib
     if _lib is not None:
         return _lib
-    path = path or LIB
+    path = path or os.environ.get("KMOE_LIBRARY") or LIB
     if not os.path.exists(path):
         raise RuntimeError(f"CUDA library {path} is missing: build it with __graft_entry__.build()")
     lib = ctypes.CDLL(path)
@@ -70,8 +71,9 @@ def load(path: str | None = None):
                                       ctypes.POINTER(Experts), ctypes.POINTER(Experts), vp, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_quant_1x128.argtypes = [vp, i, i, vp, vp, vp]
     lib.moe_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
+    lib.moe_set_wait_limit.argtypes = [ctypes.c_longlong]
     for f in ("moe_router_topk", "moe_permute", "moe_permute_noalloc", "moe_grouped_ffn", "moe_combine",
-              "moe_forward", "moe_block_forward", "moe_quant_1x128", "moe_device_status"):
+              "moe_forward", "moe_block_forward", "moe_quant_1x128", "moe_device_status", "moe_set_wait_limit"):
         getattr(lib, f).restype = i
     if lib.moe_abi_version() != 3:
         raise RuntimeError("libkmoe ABI version mismatch")
@@ -205,6 +207,11 @@ def moe_device_status(ws, stream=None) -> int:
     if rc not in (KMOE_OK, KMOE_ERR_DEVICE):
         _check(rc)
     return st.value
+
+
+def moe_set_wait_limit(cycles: int):
+    """Give-up limit (SM cycles) of the FFN kernels' pipeline waits for this host thread; 0 = default."""
+    _check(load().moe_set_wait_limit(int(cycles)))
 
 
 def moe_combine(y_perm, y_shared, topk_w, inv_pos, y_dtype=torch.bfloat16, out=None, stream=None):

@@ -284,6 +284,21 @@ kmoe_status moe_quant_1x128(const void *x, int rows, int cols, uint8_t *codes, f
  */
 kmoe_status moe_device_status(const void *ws, int *status, void *stream);
 
+/*
+ * Give-up limit of the pipeline waits in the tensor-core expert FFN kernels
+ * that later calls of the calling host thread launch (moe_grouped_ffn,
+ * moe_forward, moe_block_forward), in SM clock cycles; 0 restores the
+ * default of 2^32 cycles (about 2 s). This exists to test the failure path
+ * without faulting a GPU: with a limit far below what a wait normally takes,
+ * a kernel gives up, writes 1 to the workspace status word, lets its
+ * in-flight copies and MMAs finish (those waits always use the default
+ * limit), frees its tensor memory and returns; that call's outputs are then
+ * invalid, moe_device_status reports KMOE_ERR_DEVICE with status 1, and the
+ * next call with the default limit runs normally. cycles < 0 ->
+ * KMOE_ERR_INVALID_ARG. The setting is per host thread.
+ */
+kmoe_status moe_set_wait_limit(long long cycles);
+
 /* Message of the last error on the calling thread ("" after success). */
 const char *moe_last_error(void);
 

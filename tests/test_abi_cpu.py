@@ -159,3 +159,9 @@ def test_quant_1x128_checks_arguments_on_the_host(lib):
     assert lib.moe_quant_1x128(a, -1, 128, a, a, None) == kmoe.KMOE_ERR_INVALID_ARG
     assert lib.moe_quant_1x128(a, 4, 128, None, a, None) == kmoe.KMOE_ERR_INVALID_ARG
     assert lib.moe_quant_1x128(None, 0, 128, None, None, None) == kmoe.KMOE_OK
+
+
+def test_wait_limit_rejects_negative_and_restores_the_default(lib):
+    assert lib.moe_set_wait_limit(-1) == kmoe.KMOE_ERR_INVALID_ARG
+    assert lib.moe_set_wait_limit(1000) == kmoe.KMOE_OK
+    assert lib.moe_set_wait_limit(0) == kmoe.KMOE_OK

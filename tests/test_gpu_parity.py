@@ -145,7 +145,7 @@ def test_permute_all_tokens_on_the_same_experts():
                                     ("fp8_decode", 130), ("prefill", 256), ("prefill", 300), ("prefill", 1000),
                                     ("fp8_prefill", 300), ("fp8_prefill", 777), ("fp8a8_decode", None),
                                     ("fp8a8_decode", 1), ("fp8a8_decode", 255), ("fp8a8_prefill", 256),
-                                    ("fp8a8_prefill", 1000)])
+                                    ("fp8a8_prefill", 1000), ("fp8a8_prefill", 2500)])
 def test_grouped_ffn_matches_oracle(name, N):
     dev, host = layer_inputs(name, N)
     cfg = host["cfg"]
@@ -462,3 +462,34 @@ def test_quant_1x128_is_bit_exact(rows, cols, std):
     oc, os_ = oracle.quant_1x128(x.cpu())
     assert np.array_equal(codes.cpu().numpy(), oc)
     assert np.array_equal(scales.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+
+
+# ------------------------------------------------------ failure path
+@pytest.mark.parametrize("name,N", [("decode", None), ("fp8_decode", None), ("fp8a8_decode", None),
+                                    ("prefill", 300), ("fp8_prefill", 300), ("fp8a8_prefill", 300)])
+def test_a_wait_that_runs_out_reports_status_1_and_the_next_call_is_clean(name, N):
+    """With a give-up limit of 100 SM cycles (below any load's latency) the FFN kernels' pipeline
+    waits run out: the call leaves status 1 and returns; the GPU stays usable, and the next call
+    with the default limit on the same workspace reports 0 and matches the oracle."""
+    dev, host = layer_inputs(name, N)
+    cfg = host["cfg"]
+    l_ora = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
+    i_ora, _, _ = oracle.select(l_ora, host["bias"], cfg.K)
+    _, offsets, perm, _ = oracle.permute(i_ora, cfg.E)
+    perm_d, off_d = torch.from_numpy(perm).cuda(), torch.from_numpy(offsets).cuda()
+    ws = kmoe.workspace(cfg.N, cfg.d, cfg.E, cfg.K, cfg.I, kmoe.KMOE_BF16, kmoe.w_dtype_code(cfg.w_dtype))
+    try:
+        kmoe.moe_set_wait_limit(100)
+        kmoe.moe_grouped_ffn(dev["x"], dev, perm_d, off_d, ws=ws)
+        assert kmoe.moe_device_status(ws) == 1
+    finally:
+        kmoe.moe_set_wait_limit(0)
+    y_perm, y_shared = kmoe.moe_grouped_ffn(dev["x"], dev, perm_d, off_d, ws=ws)
+    assert kmoe.moe_device_status(ws) == 0
+    rows = np.arange(0, cfg.N * cfg.K, 7)
+    expert_of_row = np.searchsorted(offsets, rows, side="right") - 1
+    got = y_perm[torch.from_numpy(rows).cuda().long()].float().cpu().numpy()
+    assert row_rel_err(got, expert_ref(host, perm[rows], expert_of_row)) <= TOL[cfg.w_dtype]
+    toks = np.arange(0, cfg.N, 5)
+    got_s = y_shared[torch.from_numpy(toks).cuda().long()].float().cpu().numpy()
+    assert row_rel_err(got_s, expert_ref(host, toks, np.full(len(toks), cfg.E))) <= TOL[cfg.w_dtype]
