@@ -150,9 +150,11 @@ def launches_per_step(cfg):
 
 
 # --------------------------------------------------------------- GPU arm
-def run_config(cfg, steps, warmup, rank, world, seed=0, use_graph=True):
+def run_config(cfg, steps, warmup, rank, world, seed=0, use_graph=True, cpu_sample=0):
     dev = torch.device("cuda", torch.cuda.current_device())
     layer = make_inputs(cfg, seed=seed, device=dev)
+    # the oracle on the same layer, on a bounded token sample (host cores; rank 0 of a 1-GPU run only)
+    cpu = oracle_rates(cfg, layer, cpu_sample) if cpu_sample else None
     lay = kmoe.Layer(layer, cfg.N)
     xs = [make_x(cfg, seed=1000 * rank + 17 * i + 1, device=dev) for i in range(ROTATE)]
     ys = [torch.empty((cfg.N, cfg.d), dtype=torch.bfloat16, device=dev) for _ in range(ROTATE)]
@@ -233,7 +235,7 @@ def run_config(cfg, steps, warmup, rank, world, seed=0, use_graph=True):
     e2e_ms = time_e2e(lay, cfg, xs, stream, steps=max(20, min(steps, 400)), warmup=max(3, warmup // 4))
     alg = algorithmic(cfg, distinct)
     return {"ms_per_step": ms_max / steps, "single_graph_ms": single_ms, "clocks": clk, "distinct": distinct, "alg": alg,
-            "ffn_ms": ffn_ms, "e2e_ms": e2e_ms}
+            "ffn_ms": ffn_ms, "e2e_ms": e2e_ms, "cpu": cpu}
 
 
 def time_block(cfg, steps, warmup, seed=0):
@@ -351,19 +353,40 @@ def whole_job_tokens_per_s(tokens_per_rank, world, ms_max):
 
 
 # --------------------------------------------------------------- CPU oracle
-def cpu_baseline(cfg, n_tokens, seed=0, layer_host=None):
-    """The oracle, as it stands, on a bounded token sample of the workload."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_rates(cfg, layer, n_tokens):
+    """The oracle as it stands on the first n_tokens tokens of this workload, timed with all host
+    cores and with one thread (a quarter of the sample), in tokens/s. The skewed layer's sample
+    stands in for its 65,536 tokens: the rate is per token, and the full-layer time it implies is
+    an extrapolation, labelled so."""
     import oracle
     from fine_grained_sparse_fp32_b200.inputs import to_host
-    if layer_host is None:
-        layer_host = to_host(make_inputs(cfg, seed=seed, device="cpu" if not torch.cuda.is_available() else "cuda"))
-    rows = np.arange(min(n_tokens, cfg.N), dtype=np.int32)
+    host = to_host(layer)
+    fn = oracle.layer_a8 if cfg.w_dtype == "e4m3_a8" else oracle.layer
     nt = oracle.max_threads()
+    rows = np.arange(min(n_tokens, cfg.N), dtype=np.int32)
     t = time.perf_counter()
-    oracle.layer(layer_host, rows=rows, nthreads=nt)
-    dt = time.perf_counter() - t
-    return {"value": len(rows) / dt, "unit": "tokens/s", "cores": nt, "kind": "oracle",
-            "sample": f"{len(rows)} of the {cfg.N} tokens of the {cfg.name} layer, whole layer in double"}
+    fn(host, rows=rows, nthreads=nt)
+    all_cores = len(rows) / (time.perf_counter() - t)
+    rows1 = rows[: max(1, len(rows) // 4)]
+    t = time.perf_counter()
+    fn(host, rows=rows1, nthreads=1)
+    one = len(rows1) / (time.perf_counter() - t)
+    out = {"tokens_per_s_all_cores": all_cores, "tokens_per_s_1_thread": one, "cores": nt,
+           "sample": f"{len(rows)} of {cfg.N} tokens (all cores), {len(rows1)} (1 thread)"}
+    if cfg.N > len(rows):
+        out["full_layer_s_extrapolated"] = cfg.N / all_cores
+    return out
 
 
 # ------------------------------------------------------------------- main
@@ -398,20 +421,23 @@ def main():
 
     hbm, tflops, tflops_sus, peak_kind = peaks()
     dec = CONFIGS["decode"]
-    r = run_config(dec, args.steps, args.warmup, rank, world, use_graph=not args.no_graph)
+    cpu_n = args.cpu_tokens if (world == 1 and rank == 0) else 0
+    r = run_config(dec, args.steps, args.warmup, rank, world, use_graph=not args.no_graph, cpu_sample=cpu_n)
     pre = None
     extras = {}
     blocks = {}
     if not args.no_prefill:
         pcfg = CONFIGS["prefill"]
         psteps = max(10, min(args.steps // 10, 200))
-        pre = run_config(pcfg, psteps, max(3, args.warmup // 10), rank, world, use_graph=not args.no_graph)
+        pre = run_config(pcfg, psteps, max(3, args.warmup // 10), rank, world, use_graph=not args.no_graph,
+                         cpu_sample=cpu_n)
         torch.cuda.empty_cache()
         if not args.no_extra:
             for name, n_steps in (("fp8_decode", max(20, min(args.steps, 1000))), ("fp8_prefill", 50),
                                   ("fp8a8_decode", max(20, min(args.steps, 1000))), ("fp8a8_prefill", 50),
                                   ("skew", 10)):
-                extras[name] = run_config(CONFIGS[name], n_steps, 3, rank, world, use_graph=not args.no_graph)
+                extras[name] = run_config(CONFIGS[name], n_steps, 3, rank, world, use_graph=not args.no_graph,
+                                          cpu_sample=cpu_n)
                 torch.cuda.empty_cache()
             if not args.no_graph:
                 blocks = {"decode": time_block(dec, max(20, min(args.steps, 1000)), 10),
@@ -454,6 +480,7 @@ def main():
                 "tflops": palg["flops"] / (pms / 1e3) / 1e12, "tensor_frac": palg["flops"] / (pms / 1e3) / (tflops * 1e12),
                 "ffn_ms": pre["ffn_ms"], "clocks": pre["clocks"], "gpu_launches_per_step": launches_per_step(pcfg),
                 "e2e": {"value": pcfg.N * world / (pre["e2e_ms"]["ms"] / 1e3), "unit": "tokens/s"},
+                "cpu_oracle": pre["cpu"],
             }
         for name, r_x in extras.items():
             xcfg = CONFIGS[name]
@@ -473,6 +500,7 @@ def main():
                 "ffn_ms": r_x["ffn_ms"], "ffn_gbs": xalg["ffn_bytes"] / (r_x["ffn_ms"] / 1e3) / 1e9,
                 "gpu_launches_per_step": launches_per_step(xcfg), "clocks": r_x["clocks"],
                 "traffic": kernel_traffic(name),
+                "cpu_oracle": r_x["cpu"],
             }
         if blocks:
             base = {"decode": ms, "prefill": pre["ms_per_step"] if pre else None}
@@ -482,11 +510,11 @@ def main():
                        "value": CONFIGS[k].N * world / (v["ms_per_step"] / 1e3), "unit": "tokens/s",
                        "device_status": v["status"]} for k, v in blocks.items()},
             }
-        if world == 1:
-            try:
-                line["cpu_baseline"] = cpu_baseline(dec, args.cpu_tokens)
-            except Exception as exc:  # the baseline must never hide the GPU number
-                line["cpu_baseline"] = {"value": None, "error": str(exc)[:200]}
+        if world == 1 and r["cpu"]:
+            c = r["cpu"]
+            line["cpu_baseline"] = {"value": c["tokens_per_s_all_cores"], "unit": "tokens/s", "cores": c["cores"],
+                                    "kind": "oracle", "sample": c["sample"] + " of the decode layer, whole layer in double",
+                                    "value_1_thread": c["tokens_per_s_1_thread"], "cpu_model": cpu_model()}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

@@ -35,8 +35,10 @@
 //                 32 (w >> 2) ..), then the unit's epilogue (SwiGLU + H
 //                 quantisation, or the BF16 output);
 //   warp  P       one thread issues tcgen05.mma / tcgen05.commit;
-//   warp  P+1     producer: TMA of the weight tiles (lane 0) and of the token
-//                 codes (x rows gathered four at a time, or one box of H rows);
+//   warp  P+1     producer: TMA of the weight tiles and of the H codes (one
+//                 box of H rows, lane 0); an up unit's x-code rows are
+//                 gathered with cp.async, 8 lanes per 128-byte row, straight
+//                 into the swizzled layout, and complete on the stage barrier;
 //   warp  P+2     scheduler: claims units, resolves them into shared-memory
 //                 slots, and before a down unit waits (bounded) for the up
 //                 units of its expert.
@@ -115,7 +117,6 @@ __host__ __device__ constexpr size_t smem_bytes()
 struct Maps {
     CUtensorMap g_r, u_r, g_s, u_s;   // gate / up rows, routed and shared (128 rows x 128 bytes)
     CUtensorMap d_r, d_s;             // W_d rows
-    CUtensorMap xq;                   // x codes [N, d]: boxes of 1 row x 128 bytes (gathered four at a time)
     CUtensorMap hq;                   // H codes [N*K + N, I]: boxes of kNT rows x 128 bytes
 };
 
@@ -177,7 +178,7 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SA; ++s) {
-            mbar_init(&T->full[s], 1);                   // TMA expect_tx: weights and token codes
+            mbar_init(&T->full[s], 1 + 32);              // TMA expect_tx (lane 0) + every producer lane's cp.async
             mbar_init(&T->empty[s], 1);                  // tcgen05.commit
         }
         for (int p = 0; p < NP; ++p) {
@@ -200,7 +201,7 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
     if (warp == kProdWarp && lane == 0) {
         prefetch_map(&maps.g_r); prefetch_map(&maps.u_r); prefetch_map(&maps.d_r);
         if (a.has_shared) { prefetch_map(&maps.g_s); prefetch_map(&maps.u_s); prefetch_map(&maps.d_s); }
-        prefetch_map(&maps.xq); prefetch_map(&maps.hq);
+        prefetch_map(&maps.hq);
     }
     pdl_wait();               // routing, x codes and scales come from earlier kernels
     pdl_trigger();
@@ -297,8 +298,12 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
         }
     } else if (warp == kProdWarp) {
         // ------------------------------------------------------------ producer
+        // Lane l copies the 16-byte piece l % 8 of chunk rows 4j + l / 8, so
+        // that every cp.async instruction of the warp reads four whole
+        // 128-byte row segments; rows past the chunk are zero-filled.
         const uint64_t pol_w = policy_evict_first();    // routed weights: streamed once
         const uint64_t pol_k = policy_evict_last();     // token / H codes and the shared expert: reused
+        const int pc = lane & 7, rl = lane >> 3;
         uint32_t it = 0;
         bool ok = true;
         for (int us = 0;; ++us) {
@@ -308,34 +313,42 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
             if (sl.u < 0) break;
             const bool up = sl.up, shared = sl.shared;
             const int kb_n = sl.kb, wrow = sl.wrow, mc = sl.mc, nmma = sl.nmma, r0 = sl.row0;
-            const bool gl = up && 4 * lane < nmma;       // this lane gathers four token rows
-            int gr[4];
+            int tokr[kNT / 4];                           // token of chunk row 4j + rl, -1 past the chunk
 #pragma unroll
-            for (int q = 0; q < 4; ++q) gr[q] = 4 * lane + q < mc ? sl.src[4 * lane + q] : sl.src[0];
+            for (int q = 0; q < kNT / 4; ++q) tokr[q] = up && 4 * q + rl < mc ? sl.src[4 * q + rl] : -1;
             __syncwarp();
             if (lane == 0) mbar_arrive(&T->pstart);
-            if (!up) swp::fence_proxy_async_global();        // H codes written by other CTAs, seen through the scheduler
+            if (!up) swp::fence_proxy_async_global();   // H codes written by other CTAs, seen through the scheduler
             const CUtensorMap *m0 = up ? (shared ? &maps.g_s : &maps.g_r) : (shared ? &maps.d_s : &maps.d_r);
             const CUtensorMap *m1 = shared ? &maps.u_s : &maps.u_r;
             const uint64_t pw = shared ? pol_k : pol_w;
-            const uint32_t bbytes = (uint32_t)(up ? nmma : kNT) * kBK;
             for (int kb = 0; kb < kb_n; ++kb, ++it) {
                 const int s = it % SA;
                 if (!mbar_wait(&T->empty[s], ((it / SA) & 1) ^ 1, abort, a.err, lim)) { ok = false; break; }
                 uint8_t *A = smem + (size_t)s * C::Stage;
                 uint8_t *B = A + 2 * kATile;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&T->full[s], 2 * kATile + bbytes);
+                    mbar_arrive_expect_tx(&T->full[s], 2 * kATile + (up ? 0u : (uint32_t)kNT * kBK));
                     tma_load_2d_hint(A, m0, &T->full[s], kb * kBK, wrow, pw);
                     // second tile: the up rows of the same features, or the next 128 W_d rows
                     tma_load_2d_hint(A + kATile, up ? m1 : m0, &T->full[s], kb * kBK, up ? wrow : wrow + kM, pw);
                     if (!up) tma_load_2d_hint(B, &maps.hq, &T->full[s], kb * kBK, r0, pol_k);
                 }
-                __syncwarp();
-                if (gl) tma_gather4_hint(B + lane * 512, &maps.xq, &T->full[s], kb * kBK, gr[0], gr[1], gr[2], gr[3], pol_k);
+                if (up) {
+                    const uint32_t bdst = smem_u32(B);
+#pragma unroll
+                    for (int q = 0; q < kNT / 4; ++q)
+                        if (4 * q < nmma) {
+                            const int r = 4 * q + rl, tk = tokr[q];
+                            const uint8_t *src = a.xq + (size_t)(tk < 0 ? 0 : tk) * a.d + kb * kBK + pc * 16;
+                            cp_async16_hint(bdst + r * 128 + ((pc ^ (r & 7)) << 4), src, tk >= 0 ? 16u : 0u, pol_k);
+                        }
+                }
+                cp_async_arrive_noinc(&T->full[s]);       // the stage completes when these rows land
             }
             if (!ok) break;
         }
+        cp_async_wait_all();     // this lane's row copies have landed before it leaves
         if (!ok && lane == 0)    // let in-flight TMA loads land before the CTA exits
             for (uint32_t j = it > (uint32_t)SA ? it - SA : 0; j < it; ++j)
                 mbar_wait_drain(&T->full[j % SA], (j / SA) & 1, kDefaultWaitLimit);
@@ -560,8 +573,7 @@ static kmoe_status launch_a8_cfg(const ExpertPtrs &routed, const ExpertPtrs &sh,
                     code_map(&m.u_r, routed.wu, (uint64_t)a.E * a.I, a.d, kM) &&
                     code_map(&m.g_s, sh.wg, a.I, a.d, kM) && code_map(&m.u_s, sh.wu, a.I, a.d, kM) &&
                     code_map(&m.d_r, routed.wd, (uint64_t)a.E * a.d, a.I, kM) &&
-                    code_map(&m.d_s, sh.wd, a.d, a.I, kM) && code_map(&m.xq, a.xq, a.N, a.d, 1) &&
-                    code_map(&m.hq, a.hq, R, a.I, kNT);
+                    code_map(&m.d_s, sh.wd, a.d, a.I, kM) && code_map(&m.hq, a.hq, R, a.I, kNT);
     if (!ok) return fail(KMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     a.nt = kNT;
     constexpr size_t smem = smem_bytes<kNT>();
