@@ -36,26 +36,40 @@ METRIC = "MoE-layer tokens/s at 1 B200 (decode N=32, prefill N=8192); % of HBM/t
 ROTATE = 8           # distinct token batches cycled through the timed steps
 
 
-# DRAM bytes (read + write) per launch of the dominant decode kernel
-# (ffn_swap_kernel), from one ncu capture of `bench.py --capture <layer>`
-# (dram__bytes_read.sum + dram__bytes_write.sum, mean over 6 launches). They
-# hold only for the kernel sources they were measured on: the key is a hash
-# of those files, and a changed kernel reports no traffic until re-measured.
-TRAFFIC_SOURCES = ("fine_grained_sparse_fp32_b200/csrc/ffn_swap.cu", "fine_grained_sparse_fp32_b200/csrc/sm100.cuh",
-                   "fine_grained_sparse_fp32_b200/csrc/common.cuh")
-TRAFFIC = {"ca66eb03684632f2": {"decode": (1206.10 + 1.14) * 1e6, "fp8_decode": (603.34 + 0.84) * 1e6}}
+# DRAM bytes (read + write) per launch of each workload's FFN kernel(s), from
+# one ncu capture of `bench.py --capture <workload> --calls 4` (metrics
+# dram__bytes_read.sum and dram__bytes_write.sum, -k regex:ffn_, mean over the
+# 4 launches). They hold only for the kernel sources they were measured on:
+# each entry is keyed by a hash of those files, and a changed kernel reports
+# no traffic until it is measured again.
+TRAFFIC_SOURCES = {
+    "swap": ('fine_grained_sparse_fp32_b200/csrc/ffn_swap.cu', 'fine_grained_sparse_fp32_b200/csrc/swap_units.cuh', 'fine_grained_sparse_fp32_b200/csrc/sm100.cuh', 'fine_grained_sparse_fp32_b200/csrc/common.cuh'),
+    "a8": ('fine_grained_sparse_fp32_b200/csrc/ffn_a8.cu', 'fine_grained_sparse_fp32_b200/csrc/swap_units.cuh', 'fine_grained_sparse_fp32_b200/csrc/sm100.cuh', 'fine_grained_sparse_fp32_b200/csrc/common.cuh'),
+    "tc": ('fine_grained_sparse_fp32_b200/csrc/ffn_tc.cu', 'fine_grained_sparse_fp32_b200/csrc/sm100.cuh', 'fine_grained_sparse_fp32_b200/csrc/common.cuh'),
+}
+TRAFFIC = {
+    "decode": ("swap", "4d5ff5181bed47c9", (1195.6 + 1.7) * 1e6),
+    "fp8_decode": ("swap", "4d5ff5181bed47c9", (598.1 + 1.4) * 1e6),
+    "fp8a8_decode": ("a8", "90fdf62ea970a409", (598.1 + 1.3) * 1e6),
+    "fp8a8_prefill": ("a8", "90fdf62ea970a409", (1595.5 + 105.7) * 1e6),
+    "prefill": ("tc", "bf3858b93be7c4e5", (2210.4 + 39.7 + 1192.2 + 238.9) * 1e6),   # up + down kernel
+}
 
 
 def kernel_traffic(layer):
     import hashlib
+    entry = TRAFFIC.get(layer)
+    if entry is None:
+        return None
+    group, key, value = entry
     h = hashlib.sha256()
     try:
-        for f in TRAFFIC_SOURCES:
+        for f in TRAFFIC_SOURCES[group]:
             with open(os.path.join(ROOT, f), "rb") as fh:
                 h.update(fh.read())
     except OSError:
         return None
-    return TRAFFIC.get(h.hexdigest()[:16], {}).get(layer)
+    return value if h.hexdigest()[:16] == key else None
 
 
 def peaks():
@@ -481,6 +495,8 @@ def main():
                 "ffn_ms": pre["ffn_ms"], "clocks": pre["clocks"], "gpu_launches_per_step": launches_per_step(pcfg),
                 "e2e": {"value": pcfg.N * world / (pre["e2e_ms"]["ms"] / 1e3), "unit": "tokens/s"},
                 "cpu_oracle": pre["cpu"],
+                "traffic": kernel_traffic("prefill"),
+                "ffn_algorithmic_bytes": palg["ffn_bytes"],
             }
         for name, r_x in extras.items():
             xcfg = CONFIGS[name]
@@ -499,7 +515,7 @@ def main():
                 "ffn_frac": xalg["ffn_bytes"] / (r_x["ffn_ms"] / 1e3) / 1e9 / hbm,
                 "ffn_ms": r_x["ffn_ms"], "ffn_gbs": xalg["ffn_bytes"] / (r_x["ffn_ms"] / 1e3) / 1e9,
                 "gpu_launches_per_step": launches_per_step(xcfg), "clocks": r_x["clocks"],
-                "traffic": kernel_traffic(name),
+                "traffic": kernel_traffic(name), "ffn_algorithmic_bytes": xalg["ffn_bytes"],
                 "cpu_oracle": r_x["cpu"],
             }
         if blocks:
