@@ -36,8 +36,9 @@
 // 128-byte segments.
 // The up tile pairs 128 gate features with the same 128 up features (one
 // N = 256 MMA), so SiLU(g) * u is computed in registers. Tiles are
-// enumerated per expert as (n-tile, row pair), so CTAs running at the same
-// time share the expert's token rows in L2.
+// enumerated per expert as (row pair, n-tile), so CTAs running at the same
+// time share a row pair's token rows in L2, and the weights of an expert with
+// several row pairs are kept in L2 (evict-last) for its next row pair.
 //
 // E4M3 weights ("Inside Kolibri 1", FP8 section: 128 x 128 blocks, one FP32
 // scale per block) take the same kernels with eight more warps: warp 9
@@ -129,6 +130,7 @@ static_assert(tc_smem(false) <= 227 * 1024 && tc_smem(true) <= 227 * 1024, "shar
 struct Tile {
     int g, row0, rows, n0;
     bool shared, two;     // two: rows > 128 (second m-tile present)
+    bool reused;          // the group has several row pairs: its weight tiles are read again
 };
 
 __device__ __forceinline__ Tile decode_tile(int t, const int *pre, const TcArgs &a, int bn)
@@ -144,13 +146,16 @@ __device__ __forceinline__ Tile decode_tile(int t, const int *pre, const TcArgs 
     T.shared = T.g >= a.E;
     const int pcount = pre[T.g + 1] - pre[T.g];
     const int local = t - pre[T.g] * a.n_tiles;
-    const int nt = local / pcount, mp = local - nt * pcount;
+    // row pair major, n-tile minor: the n-tiles of one row pair are claimed
+    // side by side, so the CTAs running them share its token (or H) rows in L2
+    const int mp = local / a.n_tiles, nt = local - mp * a.n_tiles;
     int start, cnt;
     if (T.shared) { start = a.N * a.K; cnt = a.N; }
     else { start = a.offsets[T.g]; cnt = a.offsets[T.g + 1] - start; }
     T.row0 = start + mp * kPairRows;
     T.rows = min(kPairRows, cnt - mp * kPairRows);
     T.two = T.rows > kBM;
+    T.reused = pcount > 1;
     T.n0 = nt * bn;
     return T;
 }
@@ -409,8 +414,13 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             constexpr uint32_t bytes = kFp8 ? kB8Tile : kBTile;
             uint32_t it = 0;
             bool ok = true;
+            // The next tile is claimed while this tile's last k-blocks are issued
+            // (kClaimLead before its end), so the atomic's round trip overlaps
+            // the loads instead of sitting between two tiles.
+            constexpr int kClaimLead = 2;
+            int c_next = atomicAdd(a.tile_ctr, 1);
             for (uint32_t tq = 0; ok; ++tq) {
-                const int c = atomicAdd(a.tile_ctr, 1);
+                const int c = c_next;
                 const int t = c < total ? claim_to_tile(c, routed_tiles, total) : -1;
                 const int qs = tq % kTQ;
                 if (!mbar_wait(&tail->tqempty[qs], ((tq / kTQ) & 1) ^ 1, abort, a.err, a.wait_limit)) {
@@ -421,12 +431,16 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                 mbar_arrive(&tail->tqfull[qs]);
                 if (t < 0) break;
                 const Tile T = decode_tile(t, tail->pre, a, bn);
-                const uint64_t pol = T.shared ? pol_s : pol_w;
+                // weights read by one row pair are streamed once; an expert with
+                // several row pairs (and the shared expert) reads them again
+                const uint64_t pol = T.shared || T.reused ? pol_s : pol_w;
                 const CUtensorMap *m0 = T.shared ? &maps.b0_shared : &maps.b0_routed;
                 const CUtensorMap *m1 = T.shared ? &maps.b1_shared : &maps.b1_routed;
                 const int gi = T.shared ? 0 : T.g;
                 const int r0 = kUp ? gi * a.I + T.n0 : gi * a.d + T.n0;
+                const int claim_at = a.kblocks > kClaimLead ? a.kblocks - 1 - kClaimLead : 0;
                 for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                    if (kb == claim_at) c_next = atomicAdd(a.tile_ctr, 1);
                     const int s = it % S;
                     if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort, a.err, a.wait_limit)) { ok = false; break; }
                     uint8_t *dst = ring + (size_t)s * bytes;

@@ -18,14 +18,13 @@
 // memory, 2 x 192 columns), and the epilogue warps add the 20 partial sums in
 // FP32 registers on the CUDA cores, which brings the error back to ~1e-7.
 //
-// One CTA computes a 128-token x 192-expert tile: warp 9 loads by TMA
-// (128-byte swizzle) each 64-column block of x once into a 3-slot x ring and
-// the three weight-term tiles of that block into a 5-slot ring, one thread of
-// warp 8 issues tcgen05.mma (per 128-column round: 2 blocks of 64 x 3 terms,
-// the x tile of a block serving its three terms), warps 0-7 read each round's
-// partial sums out of tensor memory (warps w and w+4 share lane quadrant w%4
-// and split the 192 columns) and finally store the logits. The top-K
-// selection then runs on the stored logits.
+// One CTA computes a 128-token x 192-expert tile: warp 9 loads x and the
+// weight-term tiles by TMA (128-byte swizzle) into a 5-stage ring, one
+// thread of warp 8 issues tcgen05.mma (per 128-column round: 2 blocks of 64
+// x 3 terms), warps 0-7 read each round's partial sums out of tensor memory
+// (warps w and w+4 share lane quadrant w%4 and split the 192 columns) and
+// finally store the logits. The top-K selection then runs on the stored
+// logits.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -35,10 +34,10 @@ namespace kmoe {
 using namespace sm100;
 
 constexpr int kRBM = 128, kRBN = 192, kRBK = 64;
-constexpr int kRStages = 5;                 // weight-term tiles
-constexpr int kRXStages = 3;                // x tiles (one per 64-column block, used by its three terms)
+constexpr int kRStages = 5;
 constexpr int kRA = kRBM * kRBK * 2;        // 16 KB
-constexpr int kRB = kRBN * kRBK * 2;        // 24 KB (multiple of 1024)
+constexpr int kRB = kRBN * kRBK * 2;        // 24 KB
+constexpr int kRStage = kRA + kRB;          // 40 KB (multiple of 1024)
 constexpr int kRThreads = 10 * 32;
 constexpr int kRMmaWarp = 8, kRProdWarp = 9;
 constexpr int kRRoundBlocks = 2;            // 64-column blocks per fresh accumulator
@@ -51,12 +50,12 @@ struct RouterMaps {
 };
 
 struct RouterTail {
-    uint64_t full[kRStages], empty[kRStages], xfull[kRXStages], xempty[kRXStages], tfull[2], tempty[2], drain;
+    uint64_t full[kRStages], empty[kRStages], tfull[2], tempty[2], drain;
     uint32_t tmem_base;
     int abort;
 };
 
-constexpr size_t kRSmem = 1024 + (size_t)kRXStages * kRA + (size_t)kRStages * kRB + sizeof(RouterTail);
+constexpr size_t kRSmem = 1024 + (size_t)kRStages * kRStage + sizeof(RouterTail);
 
 __global__ void __launch_bounds__(256)
 router_split_kernel(const float *__restrict__ w, int n, __nv_bfloat16 *__restrict__ out)
@@ -81,9 +80,7 @@ router_tc_kernel(const __grid_constant__ RouterMaps maps, int N, int d, int E, f
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *xring = smem;                                        // kRXStages x 16 KB
-    uint8_t *wring = smem + (size_t)kRXStages * kRA;              // kRStages x 24 KB
-    RouterTail *tail = reinterpret_cast<RouterTail *>(wring + (size_t)kRStages * kRB);
+    RouterTail *tail = reinterpret_cast<RouterTail *>(smem + (size_t)kRStages * kRStage);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort = &tail->abort;
     const int m0 = blockIdx.x * kRBM, n0 = blockIdx.y * kRBN;
@@ -93,10 +90,6 @@ router_tc_kernel(const __grid_constant__ RouterMaps maps, int N, int d, int E, f
         for (int s = 0; s < kRStages; ++s) {
             mbar_init(&tail->full[s], 1);
             mbar_init(&tail->empty[s], 1);
-        }
-        for (int s = 0; s < kRXStages; ++s) {
-            mbar_init(&tail->xfull[s], 1);
-            mbar_init(&tail->xempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tail->tfull[b], 1);
@@ -125,28 +118,19 @@ router_tc_kernel(const __grid_constant__ RouterMaps maps, int N, int d, int E, f
     if (warp == kRProdWarp) {
         if (lane == 0) {
             const uint64_t pol = policy_evict_last();   // x and the weight terms are read by several CTAs
-            int i = 0, x_issued = 0;
+            int i = 0;
             for (; i < iters; ++i) {
-                const int kb = i / 3, term = i - kb * 3;
-                if (term == 0) {                        // the block's x tile, shared by its three terms
-                    const int xs = kb % kRXStages;
-                    if (!mbar_wait(&tail->xempty[xs], ((kb / kRXStages) & 1) ^ 1, abort, err, kRWaitLimit)) break;
-                    mbar_arrive_expect_tx(&tail->xfull[xs], kRA);
-                    tma_load_2d_hint(xring + (size_t)xs * kRA, &maps.x, &tail->xfull[xs], kb * kRBK, m0, pol);
-                    ++x_issued;
-                }
                 const int s = i % kRStages;
                 if (!mbar_wait(&tail->empty[s], ((i / kRStages) & 1) ^ 1, abort, err, kRWaitLimit)) break;
-                mbar_arrive_expect_tx(&tail->full[s], kRB);
-                tma_load_2d_hint(wring + (size_t)s * kRB, &maps.w, &tail->full[s], kb * kRBK, term * E + n0, pol);
+                const int kb = i / 3, term = i - kb * 3;
+                uint8_t *As = smem + (size_t)s * kRStage;
+                mbar_arrive_expect_tx(&tail->full[s], kRStage);
+                tma_load_2d_hint(As, &maps.x, &tail->full[s], kb * kRBK, m0, pol);
+                tma_load_2d_hint(As + kRA, &maps.w, &tail->full[s], kb * kRBK, term * E + n0, pol);
             }
-            if (i < iters) {   // aborted: let the loads already issued land
+            if (i < iters)     // aborted: let the loads already issued land
                 for (int j = i > kRStages ? i - kRStages : 0; j < i; ++j)
                     mbar_wait_drain(&tail->full[j % kRStages], (j / kRStages) & 1, kRWaitLimit);
-                const int kbs = x_issued;              // x blocks issued: 0 .. kbs - 1
-                for (int j = kbs > kRXStages ? kbs - kRXStages : 0; j < kbs; ++j)
-                    mbar_wait_drain(&tail->xfull[j % kRXStages], (j / kRXStages) & 1, kRWaitLimit);
-            }
         }
     } else if (warp == kRMmaWarp) {
         if (lane == 0) {
@@ -160,21 +144,16 @@ router_tc_kernel(const __grid_constant__ RouterMaps maps, int N, int d, int E, f
                     if (!mbar_wait(&tail->tempty[b], ((round >> 1) & 1) ^ 1, abort, err, kRWaitLimit)) { ok = false; break; }
                     tc_fence_after();
                 }
-                const int s = i % kRStages, kb = i / 3, term = i - kb * 3, xs = kb % kRXStages;
-                if ((term == 0 && !mbar_wait(&tail->xfull[xs], (kb / kRXStages) & 1, abort, err, kRWaitLimit)) ||
-                    !mbar_wait(&tail->full[s], (i / kRStages) & 1, abort, err, kRWaitLimit)) {
-                    ok = false;
-                    break;
-                }
+                const int s = i % kRStages;
+                if (!mbar_wait(&tail->full[s], (i / kRStages) & 1, abort, err, kRWaitLimit)) { ok = false; break; }
                 tc_fence_after();
-                const uint64_t ad = sw128_kmajor_desc(smem_u32(xring + (size_t)xs * kRA));
-                const uint64_t bd = sw128_kmajor_desc(smem_u32(wring + (size_t)s * kRB));
+                const uint64_t ad = sw128_kmajor_desc(smem_u32(smem + (size_t)s * kRStage));
+                const uint64_t bd = sw128_kmajor_desc(smem_u32(smem + (size_t)s * kRStage + kRA));
 #pragma unroll
                 for (int k = 0; k < kRBK / 16; ++k)
                     umma_bf16(tmem + b * kRBN, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc,
                               !(first && k == 0));
                 umma_commit(&tail->empty[s]);
-                if (term == 2) umma_commit(&tail->xempty[xs]);    // the x tile's three terms are issued
                 if (i % per_round == per_round - 1 || i == iters - 1) umma_commit(&tail->tfull[b]);
             }
             umma_commit(&tail->drain);
