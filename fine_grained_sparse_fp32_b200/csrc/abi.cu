@@ -266,7 +266,13 @@ static kmoe_status check_forward(int N, int d, int E, int K, int I, int score, c
 
 // Routing, dispatch, expert FFNs and combine of one layer call on laid-out
 // workspace L; with h_res set the combine also applies the post-norm and the
-// residual addition of the sandwich block.
+// residual addition of the sandwich block. The status block must be zero
+// before the first kernel that uses it: the caller clears it, except for
+// batches of the small-batch router (N <= kSmallRouteTokens), whose kernel
+// zeroes it itself (no memset between this call's kernels and the previous
+// call's, so the programmatic launch chain carries over).
+static bool router_zeroes_status(int N) { return N <= kSmallRouteTokens; }
+
 static kmoe_status forward_path(const void *x, int x_dtype, int N, int d, int E, int K, int I, int score,
                                 const float *w_router, const float *bias, const kmoe_experts *routed,
                                 const kmoe_experts *shared, void *y, int y_dtype, int32_t *topk_idx_out,
@@ -282,7 +288,7 @@ static kmoe_status forward_path(const void *x, int x_dtype, int N, int d, int E,
     if (chunked && cudaMemsetAsync(L.hist, 0, permute_ws_bytes(N, E), st) != cudaSuccess)
         return check_launch("histogram memset");
     if (N <= kSmallRouteTokens)
-        KMOE_TRY(launch_router_small(x, x_dtype, w_router, N, d, E, L.logits, L.status, st));
+        KMOE_TRY(launch_router_small(x, x_dtype, w_router, N, d, E, L.logits, L.status, st, kStatusInts));
     else if (x_dtype == KMOE_BF16 && N >= kTcRouterTokens)
         KMOE_TRY(launch_router_tc(static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E, L.w_split, L.logits,
                                   L.status, st));
@@ -454,7 +460,7 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
     // the base the Carver sees is 256-aligned by construction of the pieces
     const Layout L = layout(ws, N, d, E, K, I, routed->dtype);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    KMOE_TRY(clear_status(L.status, st, kFfnStatusBytes));
+    if (!router_zeroes_status(N)) KMOE_TRY(clear_status(L.status, st, kFfnStatusBytes));
     return forward_path(x, x_dtype, N, d, E, K, I, score, w_router, bias, routed, shared, y, y_dtype, topk_idx_out,
                         topk_w_out, counts_out, L, nullptr, nullptr, 0.f, st);
 }
@@ -494,7 +500,7 @@ kmoe_status moe_block_forward(const void *h, int N, int d, int E, int K, int I, 
     if (ws_bytes < need.bytes) return fail(KMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need.bytes);
     const Layout L = layout(ws, N, d, E, K, I, routed->dtype, true);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    KMOE_TRY(clear_status(L.status, st, kFfnStatusBytes));
+    if (!router_zeroes_status(N)) KMOE_TRY(clear_status(L.status, st, kFfnStatusBytes));
     __nv_bfloat16 *x = x_out ? static_cast<__nv_bfloat16 *>(x_out) : L.x_norm;
     KMOE_TRY(launch_rmsnorm(static_cast<const __nv_bfloat16 *>(h), static_cast<const __nv_bfloat16 *>(gamma_pre), eps,
                             N, d, x, st));

@@ -208,9 +208,11 @@ kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, in
                         int32_t *idx, float *w, cudaStream_t st, int32_t *hist = nullptr);
 
 // Router logits for N <= 256 (128 CTAs, three experts each); status is the
-// device status word for a bounded wait that gives up.
+// device status word for a bounded wait that gives up. With zero_ints > 0 the
+// kernel zeroes status[0 .. zero_ints) once the previous kernel on the stream
+// has finished (the layer call's status block, in place of a memset).
 kmoe_status launch_router_small(const void *x, int x_dtype, const float *w_router, int N, int d, int E,
-                                float *logits, int *status, cudaStream_t st);
+                                float *logits, int *status, cudaStream_t st, int zero_ints = 0);
 
 // Tensor-core FP32 router (x in BF16): W_r split into three BF16 terms in
 // `w_split` (router_tc_ws_bytes), logits [N, E] written out.

@@ -213,6 +213,10 @@ kmoe_status launch_topk(const float *logits, const float *bias, int N, int E, in
 // eight part sums of a logit are added in a fixed order. Top-K and the
 // dispatch permutation follow as separate dependent launches (one warp per
 // token, then one CTA), which keeps the selection off a single SM.
+// The router rows are layer weights that no earlier kernel writes, so their
+// copy is issued before the wait for the previous kernel; with zero_ints > 0
+// CTA 0 also zeroes the call's status block (status word and the FFN's
+// counters) once that kernel has finished, in place of a separate memset.
 constexpr int kRouteEPC = 3;
 constexpr int kRouteThreads = 1024;
 constexpr int kRouteWarps = kRouteThreads / 32;
@@ -238,11 +242,11 @@ __device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&o)[4])
 template <class XT>
 __global__ void __launch_bounds__(kRouteThreads, 1)
 router_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, int N, int d, int E, int chunk, int x_off,
-                    float *__restrict__ logits, int *status)
+                    float *__restrict__ logits, int *status, int zero_ints)
 {
     using namespace sm100;
     extern __shared__ __align__(128) uint8_t sm_raw[];
-    __shared__ __align__(8) uint64_t bar;
+    __shared__ __align__(8) uint64_t bar, wbar;
     __shared__ int abort_flag;
     __shared__ float red[kRouteCQ][kRouteChunkMax][kRouteEPC];
     float *wsm = reinterpret_cast<float *>(sm_raw);
@@ -254,24 +258,31 @@ router_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, int N
     const int qd = d / kRouteCQ;                     // columns per part (d % 128 == 0)
     if (threadIdx.x == 0) {
         mbar_init(&bar, 1);
+        mbar_init(&wbar, 1);
         abort_flag = 0;
         fence_mbar_init();
+        // the router rows do not come from the previous kernel: fetch them now
+        const uint32_t wbytes = (uint32_t)ne * d * 4;
+        mbar_arrive_expect_tx(&wbar, wbytes);
+        bulk_load(wsm, w + (size_t)e0 * d, wbytes, &wbar);
     }
     __syncthreads();
     pdl_wait();
     pdl_trigger();
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < zero_ints; i += blockDim.x) status[i] = 0;
     uint32_t phase = 0;
+    bool w_ok = true;
     for (int c0 = 0; c0 < N; c0 += chunk) {
         const int nt = min(chunk, N - c0);
         if (threadIdx.x == 0) {
             fence_proxy_async();      // earlier generic reads of xsm before the async overwrite
             const uint32_t xbytes = (uint32_t)nt * d * sizeof(XT);
-            const uint32_t wbytes = c0 == 0 ? (uint32_t)ne * d * 4 : 0u;
-            mbar_arrive_expect_tx(&bar, xbytes + wbytes);
-            if (wbytes) bulk_load(wsm, w + (size_t)e0 * d, wbytes, &bar);
+            mbar_arrive_expect_tx(&bar, xbytes);
             bulk_load(xsm, x + (size_t)c0 * d, xbytes, &bar);
         }
-        mbar_wait(&bar, phase, &abort_flag, status, kRouteWaitLimit);
+        if (c0 == 0) w_ok = mbar_wait(&wbar, 0, &abort_flag, status, kRouteWaitLimit);
+        if (w_ok) mbar_wait(&bar, phase, &abort_flag, status, kRouteWaitLimit);
         phase ^= 1;
         __syncthreads();
         if (abort_flag) break;
@@ -332,13 +343,15 @@ router_small_kernel(const XT *__restrict__ x, const float *__restrict__ w, int N
         }
         __syncthreads();
     }
-    if (abort_flag && threadIdx.x == 0)   // a copy never landed: let it finish (bounded) and leave
+    if (abort_flag && threadIdx.x == 0) {   // a copy never landed: let it finish (bounded) and leave
+        mbar_wait_drain(&wbar, 0, kRouteWaitLimit);
         mbar_wait_drain(&bar, phase ^ 1, kRouteWaitLimit);
+    }
 }
 
 
 kmoe_status launch_router_small(const void *x, int x_dtype, const float *w_router, int N, int d, int E,
-                                float *logits, int *status, cudaStream_t st)
+                                float *logits, int *status, cudaStream_t st, int zero_ints)
 {
     if (N > kChunk) return fail(KMOE_ERR_UNSUPPORTED, "small-batch router: N=%d > %d", N, kChunk);
     const int xb = x_dtype == KMOE_F32 ? 4 : 2;
@@ -349,12 +362,12 @@ kmoe_status launch_router_small(const void *x, int x_dtype, const float *w_route
     if (x_dtype == KMOE_F32) {
         cudaFuncSetAttribute(router_small_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         launch_pdl(router_small_kernel<float>, grid, kRouteThreads, smem, st, static_cast<const float *>(x), w_router,
-                   N, d, E, chunk, w_bytes, logits, status);
+                   N, d, E, chunk, w_bytes, logits, status, zero_ints);
     } else {
         cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
         launch_pdl(router_small_kernel<__nv_bfloat16>, grid, kRouteThreads, smem, st,
-                   static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E, chunk, w_bytes, logits, status);
+                   static_cast<const __nv_bfloat16 *>(x), w_router, N, d, E, chunk, w_bytes, logits, status, zero_ints);
     }
     return check_launch("router_small");
 }
