@@ -234,7 +234,8 @@ kmoe_status launch_ffn_stream(const void *x, int x_dtype, int N, int d, int I, i
                               void *h, void *y_perm, void *y_shared, cudaStream_t st);
 
 // Tensor-core grouped FFN (BF16 activations; BF16 or E4M3 + FP32 block-scale
-// weights; d % 256 == 0). `sync` holds two tile counters, zero at launch.
+// weights; d % 256 == 0). `sync` holds two tile counters and one finished-up-
+// tiles counter per group (E + 3 ints), zero at launch.
 kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
                           const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
                           __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err, int *sync,

@@ -400,7 +400,8 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
         uint32_t it = 0;
         for (int us = 0;; ++us) {
             const int j = us % kNU;
-            if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, lim)) break;
+            // the group's give-up decisions are votes (it meets at epi_sync later)
+            if (!bar_and(1, C::PThreads, mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, lim))) break;
             const Slot<kNT> &sl = T->slot[j];
             if (sl.u < 0) break;
             const bool up = sl.up, shared = sl.shared;
@@ -419,7 +420,10 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
             for (int kb = 0; kb < kb_n; ++kb, ++it) {
                 const float sx2 = mine && kb + 2 < kb_n ? ld_relaxed_f32(sp + kb + 2) : 0.f;
                 const int p = it % NP;
-                if (!mbar_wait(&T->pfull[p], (it / NP) & 1, abort, a.err, lim)) { ok = false; break; }
+                if (!bar_and(1, C::PThreads, mbar_wait(&T->pfull[p], (it / NP) & 1, abort, a.err, lim))) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + p * C::PW + c0;
                 const float w0 = sl.s[0][kb], w1 = sl.s[1][kb];

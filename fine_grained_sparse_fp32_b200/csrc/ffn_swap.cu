@@ -488,14 +488,16 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
         uint16_t *stg = &T->stage[eg * 4 + quad][0][0];
         for (int us = 0;; ++us) {
             const int j = us % kNU;
-            if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, a.wait_limit)) break;
+            // the group's give-up decisions are votes (it meets at epi_sync later)
+            if (!bar_and(1, C::EpiThreads, mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, a.wait_limit))) break;
             const Slot<kNT> &sl = T->slot[j];
             if (sl.u < 0) break;
             const bool up = sl.up, shared = sl.shared;
             const int mc = sl.mc, nmma = sl.nmma, f0 = sl.f0, r0 = sl.row0, o = sl.o;
             const float s0 = kFp8 ? sl.ref[0] : 1.f, s1 = kFp8 ? sl.ref[1] : 1.f;
             const int acc = us % C::NAcc;
-            if (!mbar_wait(&T->tfull[acc], (us / C::NAcc) & 1, abort, a.err, a.wait_limit)) break;
+            if (!bar_and(1, C::EpiThreads, mbar_wait(&T->tfull[acc], (us / C::NAcc) & 1, abort, a.err, a.wait_limit)))
+                break;
             tc_fence_after();
             const uint32_t tg = tmem + ((uint32_t)(quad * 32) << 16) + acc * C::AccW;
             const int ld = up ? a.I : a.d;               // row stride of the output

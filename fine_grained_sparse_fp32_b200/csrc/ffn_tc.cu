@@ -49,6 +49,7 @@
 // with FP32 accumulation, and the weights cross HBM at one byte each.
 #include "common.cuh"
 #include "sm100.cuh"
+#include "swap_units.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -108,6 +109,7 @@ struct TcArgs {
     const float *s0_routed, *s1_routed, *s0_shared, *s1_shared;
     int *err;
     int *tile_ctr;            // tiles claimed so far by all CTAs (zero at launch)
+    int *up_done;             // [groups] up tiles finished per group (zero before the up launch)
     long long wait_limit;     // SM cycles before a pipeline wait gives up
 };
 
@@ -353,7 +355,12 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         if (kUp) { prefetch_map(&maps.b1_routed); prefetch_map(&maps.b1_shared); }
         else prefetch_map(&maps.a);
     }
-    pdl_wait();               // routing, x and (down) H come from earlier kernels
+    // The up kernel waits for routing and x. The down kernel does not wait for
+    // the whole up grid: its CTAs start on SMs as up CTAs retire, stream W_d
+    // at once, and load a row pair's H only after every up tile of that
+    // expert has been counted in up_done (release / acquire at GPU scope).
+    // Routing itself finished before the up kernel passed its own wait.
+    if (kUp) pdl_wait();
     pdl_trigger();
     if (warp == kMmaWarp) build_prefix(tail->pre, a);
     tc_fence_before();
@@ -503,11 +510,29 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             }
             cp_async_wait_all();   // this thread's row copies have landed before it leaves
         } else if (p == 0) {
+            const int up_tiles_per_pair = a.I / (kBN / 2);
             for (uint32_t tq = 0; ok; ++tq) {
                 const int t = tq_take(tail, tq, abort, a.err, a.wait_limit);
                 if (t < 0) break;
                 const Tile T = decode_tile(t, tail->pre, a, bn);
                 const int mt = T.two ? 2 : 1;
+                // H of this expert is complete once all its up tiles are counted
+                const int need = (tail->pre[T.g + 1] - tail->pre[T.g]) * up_tiles_per_pair;
+                if (swp::ld_acquire(a.up_done + T.g) < need) {
+                    const long long t0 = clock64();
+                    while (swp::ld_acquire(a.up_done + T.g) < need) {
+                        if (*abort) { ok = false; break; }
+                        if (clock64() - t0 > a.wait_limit) {
+                            *abort = 1;
+                            atomicCAS(a.err, kErrNone, kErrWaitTimeout);
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(128);
+                    }
+                    if (!ok) break;
+                }
+                swp::fence_proxy_async_global();   // H written by other CTAs, read by TMA
                 for (int kb = 0; kb < a.kblocks && ok; ++kb) {
                     for (int m = 0; m < mt; ++m, ++ia) {
                         const int sa = ia % kAS;
@@ -581,11 +606,13 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
         int hn = 0;                       // the half rotation of the MMA thread, replayed
         const uint32_t stage = smem_u32(epi) + warp * 4096;
         for (;; ++at) {
-            const int t = tq_take(tail, at, abort, a.err, a.wait_limit);
+            // give-up decisions are votes of the four warps (they meet at a barrier per tile)
+            const int tt = tq_take(tail, at, abort, a.err, a.wait_limit);
+            const int t = bar_and(1, 128, tt != -2) ? tt : -2;
             if (t < 0) break;
             const Tile T = decode_tile(t, tail->pre, a, bn);
             const int h0 = hn, h1 = hn ^ 1;
-            if (!mbar_wait(&tail->tfull, at & 1, abort, a.err, a.wait_limit)) break;
+            if (!bar_and(1, 128, mbar_wait(&tail->tfull, at & 1, abort, a.err, a.wait_limit))) break;
             tc_fence_after();
             const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
             epilogue_half<kUp>(tlane + h0 * kBN, T, a, 0, stage);
@@ -597,6 +624,11 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
                 mbar_arrive(&tail->tempty[h1]);
             }
             hn = T.two ? h0 : h1;
+            if (kUp) {   // this tile's H rows are stored: count it for its expert
+                __threadfence();
+                swp::epi_sync<128>();
+                if (threadIdx.x == 0) swp::red_release_add(a.up_done + T.g, 1);
+            }
         }
     }
     tc_fence_before();
@@ -680,6 +712,7 @@ static kmoe_status run_tc(const TcMaps &up, const TcMaps &dn, TcArgs a, int d, i
     a.s0_shared = sh.sg;
     a.s1_shared = sh.su;
     a.tile_ctr = sync;
+    a.up_done = sync + 2;
     launch_pdl(ffn_tc_kernel<true, kFp8>, grid, threads_of(kFp8), smem, st, up, a);
     kmoe_status s = check_launch("ffn_up_tc");
     if (s != KMOE_OK) return s;
@@ -692,6 +725,7 @@ static kmoe_status run_tc(const TcMaps &up, const TcMaps &dn, TcArgs a, int d, i
     a.s0_shared = sh.sd;
     a.s1_shared = nullptr;
     a.tile_ctr = sync + 1;
+    a.up_done = sync + 2;
     launch_pdl(ffn_tc_kernel<false, kFp8>, grid, threads_of(kFp8), smem, st, dn, a);
     return check_launch("ffn_down_tc");
 }
@@ -701,7 +735,7 @@ kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, in
                           __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *err, int *sync,
                           long long wait_limit, cudaStream_t st)
 {
-    if (E + 1 > kMaxGroups) return fail(KMOE_ERR_UNSUPPORTED, "tensor-core FFN: too many experts");
+    if (E + 1 > kMaxGroups || E + 3 > kSyncInts) return fail(KMOE_ERR_UNSUPPORTED, "tensor-core FFN: too many experts");
     const bool fp8 = w_dtype == KMOE_E4M3_B128;
     const ExpertPtrs sh = shared ? *shared : routed;    // unused maps still need a valid base
     const long long R = (long long)N * K + N;

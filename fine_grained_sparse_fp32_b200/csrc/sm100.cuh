@@ -72,6 +72,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Vote over a named barrier: each of the `nthreads` threads that use barrier
+// `id` passes `p`, and every one of them gets the AND. A group of warps takes
+// its give-up decision after a bounded wait this way, so that no warp leaves
+// its loop while the others go on to a later barrier of the group (which
+// would then never complete).
+__device__ __forceinline__ bool bar_and(int id, int nthreads, bool p)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred a, b;\n\t"
+        "setp.ne.b32 a, %1, 0;\n\t"
+        "bar.red.and.pred b, %2, %3, a;\n\t"
+        "selp.u32 %0, 1, 0, b;\n\t}"
+        : "=r"(r)
+        : "r"(p ? 1u : 0u), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 // Plain bounded wait used while draining after an abort (no error recorded).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, long long limit)
 {
