@@ -320,6 +320,10 @@ def time_grouped_ffn(layer, xs, stream, steps):
 
 
 def time_e2e(lay, cfg, xs, stream, steps, warmup):
+    """End to end through Layer.forward: every step copies its token batch from pinned host memory
+    to the device, runs the layer and copies y back to pinned host memory, all inside the timed
+    region. Timed twice: with eager launches, and with each step (copy in, layer, copy out) replayed
+    from a CUDA graph, the way a serving loop replays a step. The graph figure is the reported one."""
     xb = 4 if cfg.x_dtype == "f32" else 2
     hx = [x.cpu().pin_memory() for x in xs]
     hy = torch.empty((cfg.N, cfg.d), dtype=torch.bfloat16).pin_memory()
@@ -331,18 +335,33 @@ def time_e2e(lay, cfg, xs, stream, steps, warmup):
         lay.forward(dx, y=dy, stream=stream)
         hy.copy_(dy, non_blocking=True)
 
+    def timed(run):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for i in range(steps):
+                run(i)
+            t1.record(stream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / steps
+
     with torch.cuda.stream(stream):
         for i in range(warmup):
             one(i)
     torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        t0.record(stream)
-        for i in range(steps):
+    eager = timed(one)
+    graphs = []
+    for i in range(len(hx)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
             one(i)
-        t1.record(stream)
+        graphs.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            graphs[i % len(graphs)].replay()
     torch.cuda.synchronize()
-    return {"ms": t0.elapsed_time(t1) / steps, "h2d": cfg.N * cfg.d * xb, "d2h": cfg.N * cfg.d * 2}
+    graphed = timed(lambda i: graphs[i % len(graphs)].replay())
+    return {"ms": graphed, "ms_eager": eager, "h2d": cfg.N * cfg.d * xb, "d2h": cfg.N * cfg.d * 2}
 
 
 def barrier(world):
@@ -475,6 +494,8 @@ def main():
                          "layer_achieved": layer_gbs, "layer_frac": layer_gbs / hbm,
                          "algorithmic_bytes_per_launch": alg["ffn_bytes"], "launch_ms": r["ffn_ms"]},
             "e2e": {"value": dec.N * world / (r["e2e_ms"]["ms"] / 1e3), "unit": "tokens/s",
+                    "how": "pinned host x -> device, layer, device y -> pinned host, each step one CUDA graph replay",
+                    "value_eager_launches": dec.N * world / (r["e2e_ms"]["ms_eager"] / 1e3),
                     "h2d_bytes_per_step": r["e2e_ms"]["h2d"], "d2h_bytes_per_step": r["e2e_ms"]["d2h"]},
             "gpu_launches": launches_per_step(dec) * args.steps,
             "clocks": r["clocks"],
