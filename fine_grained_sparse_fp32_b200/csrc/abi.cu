@@ -76,6 +76,15 @@ static bool fp8_weights(int w_dtype) { return w_dtype == KMOE_E4M3_B128 || w_dty
 
 static bool known_w_dtype(int w_dtype) { return w_dtype == KMOE_F32 || w_dtype == KMOE_BF16 || fp8_weights(w_dtype); }
 
+// FP8 activations need BF16 x and d % 256 == 0 (the FP8 FFN's down units);
+// checked on the host before anything is enqueued.
+static kmoe_status check_a8(int x_dtype, int d, int w_dtype)
+{
+    if (w_dtype == KMOE_E4M3_B128_A8 && (x_dtype != KMOE_BF16 || d % 256))
+        return fail(KMOE_ERR_UNSUPPORTED, "FP8 activations: x must be BF16 and d (%d) a multiple of 256", d);
+    return KMOE_OK;
+}
+
 static kmoe_status check_experts(const kmoe_experts *x, const char *name)
 {
     if (!x) return fail(KMOE_ERR_INVALID_ARG, "%s is NULL", name);
@@ -404,6 +413,7 @@ kmoe_status moe_grouped_ffn(const void *x, int x_dtype, int N, int d, int I, int
         KMOE_TRY(check_experts(shared, "shared"));
         if (shared->dtype != routed->dtype) return fail(KMOE_ERR_UNSUPPORTED, "shared and routed dtypes differ");
     }
+    KMOE_TRY(check_a8(x_dtype, d, routed->dtype));
     if (N == 0) return KMOE_OK;
     KMOE_TRY(check_ptr(x, "x"));
     KMOE_TRY(check_ptr(perm_token, "perm_token"));
@@ -452,6 +462,7 @@ kmoe_status moe_forward(const void *x, int x_dtype, int N, int d, int E, int K, 
     KMOE_TRY(check_act_dtype(y_dtype, "y"));
     KMOE_TRY(check_forward(N, d, E, K, I, score, routed, shared, w_router, bias, topk_idx_out, topk_w_out, counts_out,
                            ws));
+    KMOE_TRY(check_a8(x_dtype, d, routed->dtype));
     if (N == 0) return KMOE_OK;
     KMOE_TRY(check_ptr(x, "x"));
     KMOE_TRY(check_ptr(y, "y"));

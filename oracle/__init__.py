@@ -179,7 +179,8 @@ def block(inp, h, gamma_pre, gamma_post, eps: float, rows=None, nthreads: int = 
     hb = np.ascontiguousarray(_bits(h), dtype=np.uint16)
     N, d = hb.shape
     x = rmsnorm_bf16(hb, gamma_pre, eps)
-    ora = layer(dict(inp, x=x), rows=rows, nthreads=nthreads, score=score)
+    layer_fn = layer_a8 if inp["cfg"].w_dtype == "e4m3_a8" else layer      # FP8 activations: the 1 x 128 layer
+    ora = layer_fn(dict(inp, x=x), rows=rows, nthreads=nthreads, score=score)
     m = np.ascontiguousarray(ora["y"], dtype=np.float64)
     rws = ora["rows"]
     gp = np.ascontiguousarray(_bits(gamma_post), dtype=np.uint16)

@@ -165,3 +165,26 @@ def test_wait_limit_rejects_negative_and_restores_the_default(lib):
     assert lib.moe_set_wait_limit(-1) == kmoe.KMOE_ERR_INVALID_ARG
     assert lib.moe_set_wait_limit(1000) == kmoe.KMOE_OK
     assert lib.moe_set_wait_limit(0) == kmoe.KMOE_OK
+
+
+def test_fp8_activation_mode_is_sized_and_checked_on_the_host(lib):
+    """KMOE_E4M3_B128_A8: workspace sizes include the FP8 pieces, and FP32 x or a d that is not a
+    multiple of 256 is rejected before anything is enqueued (no GPU needed)."""
+    N, d, E, K, I = 32, 2560, 384, 6, 512
+    a8 = kmoe.moe_workspace_size(N, d, E, K, I, kmoe.KMOE_BF16, kmoe.KMOE_E4M3_B128_A8)
+    e4 = kmoe.moe_workspace_size(N, d, E, K, I, kmoe.KMOE_BF16, kmoe.KMOE_E4M3_B128)
+    # H as one-byte codes (instead of BF16) plus its scales, and x's codes and scales (each piece
+    # 256-byte aligned)
+    R = N * K + N
+    expected = -R * I + R * (I // 128) * 4 + N * d + N * (d // 128) * 4
+    assert a8 > 0 and abs((a8 - e4) - expected) <= 4 * 256
+    assert kmoe.moe_block_workspace_size(N, d, E, K, I, kmoe.KMOE_E4M3_B128_A8) > 0
+    aligned = ctypes.c_void_p(1 << 20)
+    ex = kmoe.Experts(aligned, aligned, aligned, aligned, aligned, aligned, kmoe.KMOE_E4M3_B128_A8)
+    for x_dtype, dd in ((kmoe.KMOE_F32, 2560), (kmoe.KMOE_BF16, 2688)):
+        st = lib.moe_forward(aligned, x_dtype, N, dd, E, K, I, 0, aligned, aligned, ctypes.byref(ex), ctypes.byref(ex),
+                             aligned, kmoe.KMOE_BF16, None, None, None, aligned, 1 << 40, None)
+        assert st == kmoe.KMOE_ERR_UNSUPPORTED and b"FP8 activations" in lib.moe_last_error()
+        st = lib.moe_grouped_ffn(aligned, x_dtype, N, dd, I, E, K, aligned, aligned, ctypes.byref(ex), None,
+                                 aligned, None, aligned, 1 << 40, None)
+        assert st == kmoe.KMOE_ERR_UNSUPPORTED

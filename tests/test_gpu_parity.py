@@ -328,13 +328,13 @@ def test_forward_skew_full_size():
                 assert abs(w_g[t, k] - want[int(idx_g[t, k])]) <= G_TOL
 
 
-@pytest.mark.parametrize("name,N", [("decode", None), ("prefill", 300), ("fp8_decode", 64)])
+@pytest.mark.parametrize("name,N", [("decode", None), ("prefill", 300), ("fp8_decode", 64), ("fp8a8_decode", 64)])
 def test_forward_softmax_score_matches_oracle(name, N):
     dev, host = layer_inputs(name, N)
     cfg = host["cfg"]
     y, idx, w, counts = kmoe.moe_forward(dev["x"], dev, with_outputs=True, score="softmax")
     torch.cuda.synchronize()
-    ora = oracle.layer(host, nthreads=threads(), score="softmax")
+    ora = layer_ref(host, score="softmax")
     l_all = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
     _, differ = check_routing(idx.cpu().numpy(), ora["idx"], biased_scores(l_all, host["bias"]), cfg.K)
     keep = np.array([t not in differ for t in range(cfg.N)])
@@ -409,7 +409,8 @@ def _check_block(name, N, rows=None, score="sigmoid"):
 
 
 @pytest.mark.parametrize("name,N", [("decode", None), ("decode", 1), ("decode", 300), ("fp8_decode", None),
-                                    ("fp8_decode", 200), ("prefill", 1024)])
+                                    ("fp8_decode", 200), ("prefill", 1024), ("fp8a8_decode", None),
+                                    ("fp8a8_prefill", 600)])
 def test_block_forward_matches_oracle(name, N):
     _check_block(name, N)
 
