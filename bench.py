@@ -49,7 +49,7 @@ TRAFFIC_SOURCES = {
 }
 TRAFFIC = {
     "decode": ("swap", "4d5ff5181bed47c9", (1195.6 + 1.7) * 1e6),
-    "fp8_decode": ("swap", "4d5ff5181bed47c9", (598.1 + 1.4) * 1e6),
+    "fp8_decode": ("a8", "90fdf62ea970a409", (598.1 + 1.4) * 1e6),
     "fp8a8_decode": ("a8", "90fdf62ea970a409", (598.1 + 1.3) * 1e6),
     "fp8a8_prefill": ("a8", "90fdf62ea970a409", (1595.5 + 105.7) * 1e6),
     "prefill": ("tc", "bf3858b93be7c4e5", (2210.4 + 39.7 + 1192.2 + 238.9) * 1e6),   # up + down kernel
@@ -147,11 +147,17 @@ def algorithmic(cfg, distinct_routed: float):
             "expert_weight_bytes": weights}
 
 
+def fp8_mma(cfg):
+    """Whether the layer's expert GEMMs run as FP8 x FP8 MMAs: FP8 activations, or E4M3 weights
+    with two-term BF16 activations below 256 tokens (mirrors abi.cu's dispatch)."""
+    return cfg.w_dtype == "e4m3_a8" or (cfg.w_dtype == "e4m3" and cfg.x_dtype == "bf16" and cfg.N < 256)
+
+
 def launches_per_step(cfg):
     """Kernels of this library that one moe_forward launches (mirrors abi.cu's dispatch)."""
-    if cfg.w_dtype == "e4m3_a8":
-        ffn = 2             # x quantiser, FP8 tensor-core FFN (up and down units, one launch)
-    elif cfg.x_dtype == "bf16" and cfg.w_dtype in ("bf16", "e4m3") and cfg.N < 256:
+    if fp8_mma(cfg):
+        ffn = 2             # x quantiser (one or two terms), FP8 tensor-core FFN (up and down units, one launch)
+    elif cfg.x_dtype == "bf16" and cfg.w_dtype == "bf16" and cfg.N < 256:
         ffn = 1             # swap-AB FFN (up and down units, one launch)
     else:
         ffn = 2             # ffn up, ffn down
@@ -524,7 +530,7 @@ def main():
             xms = r_x["ms_per_step"]
             xalg = r_x["alg"]
             # FP8 x FP8 MMAs: the measured BF16 peak times the nominal FP8 / BF16 ratio of 2
-            tc_peak = tflops * (2.0 if xcfg.w_dtype == "e4m3_a8" else 1.0)
+            tc_peak = tflops * (2.0 if fp8_mma(xcfg) else 1.0)
             t_hbm = xalg["layer_bytes"] / (hbm * 1e9)
             t_tc = xalg["flops"] / (tc_peak * 1e12)
             line[name] = {

@@ -117,13 +117,18 @@ static size_t act_bytes(int w_dtype) { return w_dtype == KMOE_F32 ? 4 : 2; }
 // Bytes of one H element: the output dtype, or an E4M3 code with FP8 activations.
 static size_t h_bytes(int w_dtype) { return w_dtype == KMOE_E4M3_B128_A8 ? 1 : act_bytes(w_dtype); }
 
+// Batches that run E4M3 weights on the FP8 tensor cores with two-term
+// (BF16-precision) activations: below kTcMinTokens tokens.
+static bool two_term(int w_dtype, int N) { return w_dtype == KMOE_E4M3_B128 && N < kTcMinTokens; }
+
 // The grouped FFN's scratch after the status block: H [N*K + N, I] and, with
 // FP8 activations, H's scales [N*K + N, I / 128], x's codes [N, d] and x's
-// scales [N, d / 128].
+// scales [N, d / 128]. In two-term mode H's two bytes per element are its
+// high and low code planes (each [N*K + N, I]) and x has low codes as well.
 struct FfnScratch {
     void *h;
     float *hs;
-    uint8_t *xq;
+    uint8_t *xq, *xl;
     float *xs;
 };
 
@@ -132,9 +137,10 @@ static FfnScratch take_ffn_scratch(Carver &c, int N, int d, int K, int I, int w_
     const size_t R = (size_t)N * K + N;
     FfnScratch f{};
     f.h = c.take<char>(R * I * h_bytes(w_dtype));
-    if (w_dtype == KMOE_E4M3_B128_A8) {
+    if (w_dtype == KMOE_E4M3_B128_A8 || two_term(w_dtype, N)) {
         f.hs = c.take<float>(R * (I / 128));
         f.xq = c.take<uint8_t>((size_t)N * d);
+        if (two_term(w_dtype, N)) f.xl = c.take<uint8_t>((size_t)N * d);
         f.xs = c.take<float>((size_t)N * (d / 128));
     }
     return f;
@@ -173,7 +179,6 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype, b
 {
     Carver c(ws);
     Layout L;
-    const size_t R = (size_t)N * K + N;
     const size_t ab = act_bytes(w_dtype);
     L.status = c.take<int>(kStatusInts);
     L.logits = c.take<float>((size_t)N * E);
@@ -195,16 +200,18 @@ static Layout layout(void *ws, int N, int d, int E, int K, int I, int w_dtype, b
 
 // Grouped FFN kernel for a batch (BF16 activations, BF16 or E4M3 weights,
 // d % 256 == 0): below kTcMinTokens tokens the swap-AB tcgen05 kernel
-// (weights as M, 16-token chunks as N), from there the tokens-as-M tcgen05
-// kernel; FP32 activations or weights take the CUDA-core streaming kernel.
-// FP8 activations (KMOE_E4M3_B128_A8) take the FP8 tensor-core kernel at
-// every batch size.
-enum FfnPath { kPathStream, kPathSwap, kPathTc, kPathA8 };
+// (weights as M, 16-token chunks as N) for BF16 weights and the FP8
+// tensor-core kernel in two-term mode for E4M3 weights, from there the
+// tokens-as-M tcgen05 kernel; FP32 activations or weights take the CUDA-core
+// streaming kernel. FP8 activations (KMOE_E4M3_B128_A8) take the FP8
+// tensor-core kernel at every batch size.
+enum FfnPath { kPathStream, kPathSwap, kPathTc, kPathA8, kPathTwo };
 
 static FfnPath ffn_path(int x_dtype, int w_dtype, int N, int d)
 {
     if (w_dtype == KMOE_E4M3_B128_A8) return kPathA8;
     if (x_dtype != KMOE_BF16 || (w_dtype != KMOE_BF16 && w_dtype != KMOE_E4M3_B128) || d % 256) return kPathStream;
+    if (two_term(w_dtype, N)) return kPathTwo;
     return N < kTcMinTokens ? kPathSwap : kPathTc;
 }
 
@@ -224,8 +231,16 @@ static kmoe_status run_ffn(const void *x, int x_dtype, int N, int d, int I, int 
                              static_cast<__nv_bfloat16 *>(y_perm), static_cast<__nv_bfloat16 *>(y_shared), status,
                              status + kSyncOffset, wait_limit(), st);
     }
+    if (path == kPathTwo) {
+        const size_t R = (size_t)N * K + N;
+        uint8_t *hq = static_cast<uint8_t *>(h), *hl = hq + R * I;
+        KMOE_TRY(launch_quant_1x128_split(static_cast<const __nv_bfloat16 *>(x), N, d, f.xq, f.xl, f.xs, st));
+        return launch_ffn_a8(f.xq, f.xs, N, d, I, E, K, perm, offsets, r, s, hq, f.hs,
+                             static_cast<__nv_bfloat16 *>(y_perm), static_cast<__nv_bfloat16 *>(y_shared), status,
+                             status + kSyncOffset, wait_limit(), st, f.xl, hl);
+    }
     if (path == kPathSwap)
-        return launch_ffn_swap(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, w_dtype, r, s,
+        return launch_ffn_swap(static_cast<const __nv_bfloat16 *>(x), N, d, I, E, K, perm, offsets, r, s,
                                static_cast<__nv_bfloat16 *>(h), static_cast<__nv_bfloat16 *>(y_perm),
                                static_cast<__nv_bfloat16 *>(y_shared), status, status + kSyncOffset, wait_limit(), st);
     if (path == kPathTc)

@@ -244,14 +244,14 @@ kmoe_status launch_ffn_tc(const __nv_bfloat16 *x, int N, int d, int I, int E, in
 // Batches of at least this many tokens take the tensor-core FFN.
 constexpr int kTcMinTokens = 256;
 
-// Swap-AB tensor-core FFN for small batches (BF16 activations; BF16 or
-// E4M3 + FP32 block-scale weights; d % 256 == 0). `sync` holds kSyncInts
+// Swap-AB tensor-core FFN for small batches (BF16 activations and weights;
+// d % 256 == 0). `sync` holds kSyncInts
 // counters that must be zero at launch (a unit counter and one per expert).
 // wait_limit (both tensor-core FFNs): SM cycles before a pipeline wait gives
 // up and the kernel writes status 1 and returns.
 constexpr int kSyncInts = 1088;
 kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
-                            const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
+                            const int32_t *offsets, const ExpertPtrs &routed, const ExpertPtrs *shared,
                             __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status,
                             int *sync, long long wait_limit, cudaStream_t st);
 
@@ -260,10 +260,14 @@ kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, 
 // H kept as codes hq [N*K + N, I] with scales hs [N*K + N, I / 128]; d % 256
 // == 0). `sync` as for launch_ffn_swap. wait_limit: SM cycles before a
 // pipeline wait gives up.
+// With xl / hl set (two-term mode, 16-row chunks): x and H are each held as
+// high and low E4M3 codes, x = s * (hi + lo / 16), which carries BF16
+// precision (E4M3 weights with BF16 activations on the FP8 tensor cores).
 kmoe_status launch_ffn_a8(const uint8_t *xq, const float *xs, int N, int d, int I, int E, int K, const int32_t *perm,
                           const int32_t *offsets, const ExpertPtrs &routed, const ExpertPtrs *shared, uint8_t *hq,
                           float *hs, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status, int *sync,
-                          long long wait_limit, cudaStream_t st);
+                          long long wait_limit, cudaStream_t st, const uint8_t *xl = nullptr,
+                          uint8_t *hl = nullptr);
 
 // err: device status word for a bounded wait that gives up (may be NULL).
 // h_res / g_post (BF16, NULL for the plain combine): y = h_res + RMSNorm(m) * g_post.
@@ -276,6 +280,11 @@ kmoe_status launch_combine(const void *y_perm, const void *y_shared, int y_in_dt
 // [rows, cols] (E4M3), scales [rows, cols / 128] (FP32).
 kmoe_status launch_quant_1x128(const __nv_bfloat16 *x, int rows, int cols, uint8_t *codes, float *scales,
                                cudaStream_t st);
+
+// Two E4M3 terms per value with the same group scale: x = s * (hi + lo / 16)
+// up to about 2^-8 of |x| (BF16-precision activations for the FP8 MMA).
+kmoe_status launch_quant_1x128_split(const __nv_bfloat16 *x, int rows, int cols, uint8_t *hi, uint8_t *lo,
+                                     float *scales, cudaStream_t st);
 
 // x = bf16(h / sqrt(mean(h^2) + eps) * gamma), row by row.
 kmoe_status launch_rmsnorm(const __nv_bfloat16 *h, const __nv_bfloat16 *gamma, float eps, int N, int d,

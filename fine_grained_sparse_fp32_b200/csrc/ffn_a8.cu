@@ -27,6 +27,14 @@
 // expected rows per expert): a weight tile crosses shared memory once per
 // chunk, so larger batches take larger chunks.
 //
+// Two-term mode (kTwo, 16-row chunks): the same kernel serves E4M3 weights
+// with BF16 activations. Every activation group is held as two E4M3 codes
+// with one scale, x = s * (hi + lo / 16) up to about 2^-8 of |x| (the size of
+// a BF16 rounding); the hi rows are B rows 0 .. 15 and the lo rows B rows
+// 16 .. 31 of one N = 32 operand, so a K block still takes four MMAs per
+// weight tile, and the promotion adds (P_hi + P_lo / 16) * s_w * s_x. H is
+// kept in the same two-term form between up and down.
+//
 // Warp roles (one CTA per SM, persistent), P = 4 promotion warps for chunks
 // of up to 32 rows and 8 for 64:
 //   warps 0..P-1  promotion: tcgen05.ld of each partial slot, scale and add
@@ -63,20 +71,22 @@ constexpr int kATile = kM * kBK;        // 16 KB of E4M3 weights
 constexpr int kNU = 8;                  // unit slots
 constexpr int kSmemLimit = 232448;      // 227 KB per CTA
 
-template <int kNT>
+template <int kNT, bool kTwo = false>
 struct Cfg {
     static constexpr int TPW = kNT < 32 ? kNT : 32;      // token columns of one promotion warp
     static constexpr int PWarps = 4 * (kNT / TPW);       // promotion warps: 4 lane quadrants x column groups
     static constexpr int PThreads = 32 * PWarps;
     static constexpr int MmaWarp = PWarps, ProdWarp = PWarps + 1, SchedWarp = PWarps + 2, Warps = PWarps + 3;
-    static constexpr int BTile = kNT * kBK;              // token codes of one stage
+    static constexpr int BRows = kTwo ? 2 * kNT : kNT;   // B operand rows: the chunk's codes (hi | lo)
+    static constexpr int BTile = BRows * kBK;            // token codes of one stage
     static constexpr int Stage = 2 * kATile + BTile;     // weight tile 0 | weight tile 1 | token codes
-    static constexpr int Stages = kNT == 16 ? 6 : kNT == 32 ? 5 : 4;
-    static constexpr int PW = 2 * kNT;                   // one partial slot: tile 0 | tile 1
+    static constexpr int Stages = kTwo ? 5 : kNT == 16 ? 6 : kNT == 32 ? 5 : 4;
+    static constexpr int PW = 2 * BRows;                 // one partial slot: tile 0 | tile 1
     static constexpr int NP = 512 / PW < 8 ? 512 / PW : 8;   // partial slots in tensor memory
     static constexpr int TmemCols = NP * PW <= 256 ? 256 : 512;
     static constexpr int RPL = (kNT + 31) / 32;          // chunk rows per scheduler lane
     static_assert(kNT == 16 || kNT == 32 || kNT == 64, "token chunk of 16, 32 or 64 rows");
+    static_assert(!kTwo || kNT == 16, "two-term operands with 16-row chunks");
     static_assert(Stage % 1024 == 0, "tiles on 1024-byte boundaries (128-byte swizzle atoms)");
     static_assert(NP * PW <= TmemCols, "tensor memory columns");
 };
@@ -92,7 +102,7 @@ struct Slot {
     int src[kNT];            // B row n: token (up) or dispatched row (down), n < mc
 };
 
-template <int kNT>
+template <int kNT, bool kTwo>
 struct Tail {
     uint64_t full[6], empty[6];
     uint64_t pfull[8], pempty[8];
@@ -102,29 +112,32 @@ struct Tail {
     int abort;
     Slot<kNT> slot[kNU];
     alignas(16) uint32_t amax[4][kNT];                        // up epilogue: |H| maximum per quadrant and token (float bits)
-    alignas(16) uint8_t codes[kNT][128];                      // up epilogue: the unit's H codes, token-major
+    alignas(16) uint8_t codes[kTwo ? 2 : 1][kNT][128];        // up epilogue: the unit's H codes (hi, lo), token-major
     alignas(16) uint16_t stage[Cfg<kNT>::PWarps][16][32];     // down epilogue: 16 tokens x 32 features per warp
     int pre[kMaxOrd + 1];
     int off[kMaxOrd + 1];
 };
 
-template <int kNT>
+template <int kNT, bool kTwo>
 __host__ __device__ constexpr size_t smem_bytes()
 {
-    return 1024 + (size_t)Cfg<kNT>::Stages * Cfg<kNT>::Stage + sizeof(Tail<kNT>);
+    return 1024 + (size_t)Cfg<kNT, kTwo>::Stages * Cfg<kNT, kTwo>::Stage + sizeof(Tail<kNT, kTwo>);
 }
 
 struct Maps {
     CUtensorMap g_r, u_r, g_s, u_s;   // gate / up rows, routed and shared (128 rows x 128 bytes)
     CUtensorMap d_r, d_s;             // W_d rows
     CUtensorMap hq;                   // H codes [N*K + N, I]: boxes of kNT rows x 128 bytes
+    CUtensorMap hl;                   // two-term mode: H low codes, same shape
 };
 
 struct Args {
-    const uint8_t *xq;                // x codes [N, d]
+    const uint8_t *xq;                // x codes [N, d] (two-term mode: the high codes)
+    const uint8_t *xl;                // two-term mode: x low codes [N, d]
     const float *xs;                  // x scales [N, d / 128]
     const int32_t *perm, *offsets;
-    uint8_t *hq;                      // H codes [N*K + N, I]
+    uint8_t *hq;                      // H codes [N*K + N, I] (two-term mode: the high codes)
+    uint8_t *hl;                      // two-term mode: H low codes [N*K + N, I]
     float *hs;                        // H scales [N*K + N, I / 128]
     __nv_bfloat16 *y_perm, *y_shared;
     const float *sg_r, *su_r, *sd_r, *sg_s, *su_s, *sd_s;   // weight block scales
@@ -162,16 +175,16 @@ __device__ __forceinline__ uint8_t e4m3_code(float v)
 
 using namespace a8;
 
-template <int kNT>
-__global__ void __launch_bounds__(Cfg<kNT>::Warps * 32, 1)
+template <int kNT, bool kTwo>
+__global__ void __launch_bounds__(Cfg<kNT, kTwo>::Warps * 32, 1)
 ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
 {
-    using C = Cfg<kNT>;
+    using C = Cfg<kNT, kTwo>;
     constexpr int SA = C::Stages, NP = C::NP, TPW = C::TPW;
     constexpr int kMmaWarp = C::MmaWarp, kProdWarp = C::ProdWarp, kSchedWarp = C::SchedWarp;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Tail<kNT> *T = reinterpret_cast<Tail<kNT> *>(smem + (size_t)SA * C::Stage);
+    Tail<kNT, kTwo> *T = reinterpret_cast<Tail<kNT, kTwo> *>(smem + (size_t)SA * C::Stage);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort = &T->abort;
     const long long lim = a.wait_limit;
@@ -202,6 +215,7 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
         prefetch_map(&maps.g_r); prefetch_map(&maps.u_r); prefetch_map(&maps.d_r);
         if (a.has_shared) { prefetch_map(&maps.g_s); prefetch_map(&maps.u_s); prefetch_map(&maps.d_s); }
         prefetch_map(&maps.hq);
+        if (kTwo) prefetch_map(&maps.hl);
     }
     pdl_wait();               // routing, x codes and scales come from earlier kernels
     pdl_trigger();
@@ -328,11 +342,14 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                 uint8_t *A = smem + (size_t)s * C::Stage;
                 uint8_t *B = A + 2 * kATile;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&T->full[s], 2 * kATile + (up ? 0u : (uint32_t)kNT * kBK));
+                    mbar_arrive_expect_tx(&T->full[s], 2 * kATile + (up ? 0u : (uint32_t)C::BRows * kBK));
                     tma_load_2d_hint(A, m0, &T->full[s], kb * kBK, wrow, pw);
                     // second tile: the up rows of the same features, or the next 128 W_d rows
                     tma_load_2d_hint(A + kATile, up ? m1 : m0, &T->full[s], kb * kBK, up ? wrow : wrow + kM, pw);
-                    if (!up) tma_load_2d_hint(B, &maps.hq, &T->full[s], kb * kBK, r0, pol_k);
+                    if (!up) {
+                        tma_load_2d_hint(B, &maps.hq, &T->full[s], kb * kBK, r0, pol_k);
+                        if (kTwo) tma_load_2d_hint(B + kNT * kBK, &maps.hl, &T->full[s], kb * kBK, r0, pol_k);
+                    }
                 }
                 if (up) {
                     const uint32_t bdst = smem_u32(B);
@@ -340,8 +357,13 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                     for (int q = 0; q < kNT / 4; ++q)
                         if (4 * q < nmma) {
                             const int r = 4 * q + rl, tk = tokr[q];
-                            const uint8_t *src = a.xq + (size_t)(tk < 0 ? 0 : tk) * a.d + kb * kBK + pc * 16;
-                            cp_async16_hint(bdst + r * 128 + ((pc ^ (r & 7)) << 4), src, tk >= 0 ? 16u : 0u, pol_k);
+                            const size_t off = (size_t)(tk < 0 ? 0 : tk) * a.d + kb * kBK + pc * 16;
+                            cp_async16_hint(bdst + r * 128 + ((pc ^ (r & 7)) << 4), a.xq + off, tk >= 0 ? 16u : 0u, pol_k);
+                            if (kTwo) {       // low codes: row kNT + r (kNT is a multiple of 8: same swizzle phase)
+                                const int r2 = kNT + r;
+                                cp_async16_hint(bdst + r2 * 128 + ((pc ^ (r2 & 7)) << 4), a.xl + off, tk >= 0 ? 16u : 0u,
+                                                pol_k);
+                            }
                         }
                 }
                 cp_async_arrive_noinc(&T->full[s]);       // the stage completes when these rows land
@@ -362,7 +384,8 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                 const Slot<kNT> &sl = T->slot[j];
                 if (sl.u < 0) break;
                 const int kb_n = sl.kb;
-                const uint32_t id = idesc_e4m3_f32(kM, sl.nmma);
+                // two-term: N covers the hi rows 0 .. kNT-1 and the lo rows kNT .. 2 kNT-1
+                const uint32_t id = idesc_e4m3_f32(kM, kTwo ? C::BRows : sl.nmma);
                 bool ok = true;
                 for (int kb = 0; kb < kb_n; ++kb, ++it) {
                     const int s = it % SA, p = it % NP;
@@ -375,7 +398,7 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                     const uint32_t sa = smem_u32(smem + (size_t)s * C::Stage);
                     const uint64_t a0 = sw128_kmajor_desc(sa), a1 = sw128_kmajor_desc(sa + kATile);
                     const uint64_t bd = sw128_kmajor_desc(sa + 2 * kATile);
-                    const uint32_t d0 = tmem + p * C::PW, d1 = d0 + kNT;
+                    const uint32_t d0 = tmem + p * C::PW, d1 = d0 + C::BRows;
                     // a fresh partial per K block; one accumulator's k-steps back to back
 #pragma unroll
                     for (int k = 0; k < kBK / 32; ++k) umma_f8(d0, a0 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), id, k);
@@ -427,23 +450,43 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                 tc_fence_after();
                 const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + p * C::PW + c0;
                 const float w0 = sl.s[0][kb], w1 = sl.s[1][kb];
-                {
-                    uint32_t v[TPW];                       // tile 0 (gate or the first W_d rows)
-                    tmem_load<TPW>(ta, v);
+                if constexpr (kTwo) {
+                    uint32_t vh[TPW], vl[TPW];             // tile 0: hi and lo products
+                    tmem_load<TPW>(ta, vh);
+                    tmem_load<TPW>(ta + kNT, vl);
                     tmem_ld_wait();
 #pragma unroll
                     for (int n = 0; n < TPW; ++n)
-                        acc0[n] = fmaf(__uint_as_float(v[n]), w0 * __shfl_sync(0xffffffffu, sx0, n), acc0[n]);
-                }
-                {
-                    uint32_t v[TPW];                       // tile 1 (up or the next W_d rows)
-                    tmem_load<TPW>(ta + kNT, v);
+                        acc0[n] = fmaf(fmaf(__uint_as_float(vl[n]), 0.0625f, __uint_as_float(vh[n])),
+                                       w0 * __shfl_sync(0xffffffffu, sx0, n), acc0[n]);
+                    tmem_load<TPW>(ta + C::BRows, vh);     // tile 1
+                    tmem_load<TPW>(ta + C::BRows + kNT, vl);
                     tmem_ld_wait();
                     tc_fence_before();
                     mbar_arrive(&T->pempty[p]);
 #pragma unroll
                     for (int n = 0; n < TPW; ++n)
-                        acc1[n] = fmaf(__uint_as_float(v[n]), w1 * __shfl_sync(0xffffffffu, sx0, n), acc1[n]);
+                        acc1[n] = fmaf(fmaf(__uint_as_float(vl[n]), 0.0625f, __uint_as_float(vh[n])),
+                                       w1 * __shfl_sync(0xffffffffu, sx0, n), acc1[n]);
+                } else {
+                    {
+                        uint32_t v[TPW];                   // tile 0 (gate or the first W_d rows)
+                        tmem_load<TPW>(ta, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int n = 0; n < TPW; ++n)
+                            acc0[n] = fmaf(__uint_as_float(v[n]), w0 * __shfl_sync(0xffffffffu, sx0, n), acc0[n]);
+                    }
+                    {
+                        uint32_t v[TPW];                   // tile 1 (up or the next W_d rows)
+                        tmem_load<TPW>(ta + kNT, v);
+                        tmem_ld_wait();
+                        tc_fence_before();
+                        mbar_arrive(&T->pempty[p]);
+#pragma unroll
+                        for (int n = 0; n < TPW; ++n)
+                            acc1[n] = fmaf(__uint_as_float(v[n]), w1 * __shfl_sync(0xffffffffu, sx0, n), acc1[n]);
+                    }
                 }
                 sx0 = sx1;
                 sx1 = sx2;
@@ -471,15 +514,25 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
 #pragma unroll
                 for (int n = 0; n < TPW; ++n) {
                     const float sn = __shfl_sync(0xffffffffu, s_l, n);
-                    T->codes[c0 + n][quad * 32 + lane] = e4m3_code(__fdiv_rn(hv[n], sn));
+                    const float y = __fdiv_rn(hv[n], sn);
+                    const uint8_t hc = e4m3_code(y);
+                    T->codes[0][c0 + n][quad * 32 + lane] = hc;
+                    if (kTwo) {       // lo = E4M3((y - hi) * 16)
+                        const float hd = __half2float(__half(__nv_cvt_fp8_to_halfraw(hc, __NV_E4M3)));
+                        T->codes[kTwo ? 1 : 0][c0 + n][quad * 32 + lane] = e4m3_code((y - hd) * 16.f);
+                    }
                 }
                 swp::epi_sync<C::PThreads>();
-                // 16-byte pieces: token n = i / 8, piece i % 8 of its 128 codes
+                // 16-byte pieces: token n = i / 8, piece i % 8 of its 128 codes (per plane)
                 for (int i = threadIdx.x; i < kNT * 8; i += C::PThreads) {
                     const int n = i >> 3, pc = i & 7;
-                    if (n < mc)
-                        *reinterpret_cast<uint4 *>(a.hq + (size_t)(r0 + n) * a.I + f0 + pc * 16) =
-                            *reinterpret_cast<const uint4 *>(&T->codes[n][pc * 16]);
+                    if (n < mc) {
+                        const size_t at = (size_t)(r0 + n) * a.I + f0 + pc * 16;
+                        *reinterpret_cast<uint4 *>(a.hq + at) = *reinterpret_cast<const uint4 *>(&T->codes[0][n][pc * 16]);
+                        if (kTwo)
+                            *reinterpret_cast<uint4 *>(a.hl + at) =
+                                *reinterpret_cast<const uint4 *>(&T->codes[kTwo ? 1 : 0][n][pc * 16]);
+                    }
                 }
                 if (quad == 0 && mine) a.hs[(size_t)(r0 + tok) * (a.I / kBK) + f0 / kBK] = s_l;
                 __threadfence();                           // H codes and scales visible before the count rises
@@ -568,7 +621,7 @@ static int a8_sm_count()
     return n;
 }
 
-template <int kNT>
+template <int kNT, bool kTwo = false>
 static kmoe_status launch_a8_cfg(const ExpertPtrs &routed, const ExpertPtrs &sh, Args a, cudaStream_t st)
 {
     const uint64_t R = (uint64_t)a.N * a.K + a.N;
@@ -577,21 +630,22 @@ static kmoe_status launch_a8_cfg(const ExpertPtrs &routed, const ExpertPtrs &sh,
                     code_map(&m.u_r, routed.wu, (uint64_t)a.E * a.I, a.d, kM) &&
                     code_map(&m.g_s, sh.wg, a.I, a.d, kM) && code_map(&m.u_s, sh.wu, a.I, a.d, kM) &&
                     code_map(&m.d_r, routed.wd, (uint64_t)a.E * a.d, a.I, kM) &&
-                    code_map(&m.d_s, sh.wd, a.d, a.I, kM) && code_map(&m.hq, a.hq, R, a.I, kNT);
+                    code_map(&m.d_s, sh.wd, a.d, a.I, kM) && code_map(&m.hq, a.hq, R, a.I, kNT) &&
+                    code_map(&m.hl, kTwo ? a.hl : a.hq, R, a.I, kNT);
     if (!ok) return fail(KMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     a.nt = kNT;
-    constexpr size_t smem = smem_bytes<kNT>();
+    constexpr size_t smem = smem_bytes<kNT, kTwo>();
     static_assert(smem <= (size_t)kSmemLimit, "shared memory per CTA");
-    auto k = ffn_a8_kernel<kNT>;
+    auto k = ffn_a8_kernel<kNT, kTwo>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    launch_pdl(k, a8_sm_count(), Cfg<kNT>::Warps * 32, smem, st, m, a);
+    launch_pdl(k, a8_sm_count(), Cfg<kNT, kTwo>::Warps * 32, smem, st, m, a);
     return check_launch("ffn_a8");
 }
 
 kmoe_status launch_ffn_a8(const uint8_t *xq, const float *xs, int N, int d, int I, int E, int K, const int32_t *perm,
                           const int32_t *offsets, const ExpertPtrs &routed, const ExpertPtrs *shared, uint8_t *hq,
                           float *hs, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status, int *sync,
-                          long long wait_limit, cudaStream_t st)
+                          long long wait_limit, cudaStream_t st, const uint8_t *xl, uint8_t *hl)
 {
     if (E + 1 > kMaxOrd || E + 2 > kSyncInts) return fail(KMOE_ERR_UNSUPPORTED, "FP8 FFN: too many experts");
     if (d % kFD || I % kF || d / kBK > 48 || I / kBK > 48)
@@ -599,10 +653,12 @@ kmoe_status launch_ffn_a8(const uint8_t *xq, const float *xs, int N, int d, int 
     const ExpertPtrs sh = shared ? *shared : routed;     // unused maps still need a valid base
     Args a{};
     a.xq = xq;
+    a.xl = xl;
     a.xs = xs;
     a.perm = perm;
     a.offsets = offsets;
     a.hq = hq;
+    a.hl = hl;
     a.hs = hs;
     a.y_perm = y_perm;
     a.y_shared = y_shared;
@@ -619,6 +675,10 @@ kmoe_status launch_ffn_a8(const uint8_t *xq, const float *xs, int N, int d, int 
     // Chunk rows from the expected rows per routed expert, N * K / E: 16 while
     // experts see a dozen tokens or fewer, then 32, then 64 (a weight tile
     // crosses shared memory once per chunk).
+    if (xl) {                 // two-term operands (BF16-precision activations): 16-row chunks
+        if (!hl) return fail(KMOE_ERR_INVALID_ARG, "FP8 FFN: two-term mode needs both low-code planes");
+        return launch_a8_cfg<16, true>(routed, sh, a, st);
+    }
     const long long avg = (long long)N * K / E;
     if (avg <= 12) return launch_a8_cfg<16>(routed, sh, a, st);
     if (avg <= 32) return launch_a8_cfg<32>(routed, sh, a, st);

@@ -32,19 +32,9 @@
 //   warp  4    one thread issues tcgen05.mma / tcgen05.commit;
 //   warp  5    producer: TMA loads of the weight tiles (lane 0), cp.async
 //              gathers of the token (or H) rows (all lanes);
-//   warp  6    scheduler;
-//   warps 7-14 E4M3 weights only: two groups of converters.
-// E4M3 weights ("Inside Kolibri 1", FP8 section: 128 x 128 blocks with one
-// FP32 scale each) arrive by TMA as bytes. Converter warps decode them
-// exactly to F16 (hardware e4m3x2 -> f16x2) and write the tiles straight
-// into tensor memory with tcgen05.st: the MMA takes A from tensor memory.
-// The block scale of a stage is one number per weight tile, so it goes on
-// the token tile instead: each weight tile gets its own F16 copy of the
-// token rows times s_kb / s_ref (its block's scale over the largest scale
-// of the row block, at most 1, so nothing overflows). The MMA is F16 x F16
-// with FP32 accumulation, and the epilogue multiplies by s_ref.
-// |x| must stay inside the F16 range (65504); a value outside it sets
-// device status 2.
+//   warp  6    scheduler.
+// BF16 weights only: small batches with E4M3 weights run on the FP8 tensor
+// cores (ffn_a8.cu, two-term activations).
 #include "common.cuh"
 #include "sm100.cuh"
 #include "swap_units.cuh"
@@ -62,35 +52,29 @@ constexpr int kNU = 8;                  // unit-info slots
 constexpr long long kWaitLimit = kDefaultWaitLimit;   // SM cycles, about 2 s: waits that drain after a give-up
 constexpr int kSmemLimit = 232448;            // 227 KB per CTA
 
-// Per configuration: kNT = token rows per unit at most (16 at decode, 128 at
-// prefill); E4M3 weights use 128-column stages (one scale block), BF16 64.
-template <bool kFp8, int kNT>
+// Per configuration: kNT = token rows per unit at most (16 are compiled).
+template <int kNT>
 struct Cfg {
-    static constexpr int BK = kFp8 ? 128 : 64;           // k per stage
+    static constexpr int BK = 64;                        // k per stage
     static constexpr int Panel = kNT * 128;              // one 64-column panel of a B tile
     static constexpr int BTile = kNT * BK * 2;           // token rows of a stage (16-bit)
     static constexpr int Stage = 2 * kATile + BTile;     // gate | up (or W_d) | tokens
     static constexpr int AccW = 2 * kNT;                 // accumulator slot: gate | up
     static constexpr int NAcc = 256 / kNT < 4 ? 256 / kNT : 4;
     static constexpr int AccCols = NAcc * AccW;
-    static constexpr int ConvStages = kFp8 ? 3 : 0;      // E4M3: decoded tiles in tensor memory
-    static constexpr int ConvCols = 128;                 // gate | up, 64 columns of F16 each
-    static constexpr int TmemCols = kFp8 ? 512 : (AccCols <= 128 ? 128 : AccCols <= 256 ? 256 : 512);
-    static constexpr int Stages = kFp8 ? 5 : (kNT <= 16 ? 6 : 4);
-    static constexpr int ConvB = ConvStages * 2 * BTile; // E4M3: F16 token tiles, one per weight tile
-    static constexpr int Ring = Stages * Stage + ConvB;
+    static constexpr int TmemCols = AccCols <= 128 ? 128 : AccCols <= 256 ? 256 : 512;
+    static constexpr int Stages = kNT <= 16 ? 6 : 4;
+    static constexpr int Ring = Stages * Stage;
     static constexpr int EpiGroups = kNT > 32 ? 2 : 1;   // groups of four epilogue warps
-    static constexpr int Warps = kFp8 ? 15 : (EpiGroups == 2 ? 11 : 7);
+    static constexpr int Warps = EpiGroups == 2 ? 11 : 7;
     static constexpr int EpiThreads = 128 * EpiGroups;
     static constexpr int W = kNT < 32 ? kNT : 32;        // accumulator columns an epilogue warp loads at once
     static_assert(kNT % 16 == 0 && kNT >= 16 && kNT <= 128, "token chunk");
-    static_assert(AccCols + ConvStages * ConvCols <= TmemCols && TmemCols <= 512, "tensor memory columns");
+    static_assert(AccCols <= TmemCols && TmemCols <= 512, "tensor memory columns");
 };
 
-// Warps 0-3 (and 7-10 when EpiGroups == 2) run the epilogue; E4M3
-// converters are warps 7-14.
-constexpr int kMmaWarp = 4, kProdWarp = 5, kSchedWarp = 6, kConvWarp = 7, kEpi2Warp = 7;
-constexpr int kConvGroups = 2;
+// Warps 0-3 (and 7-10 when EpiGroups == 2) run the epilogue.
+constexpr int kMmaWarp = 4, kProdWarp = 5, kSchedWarp = 6, kEpi2Warp = 7;
 
 // A unit as the scheduler warp resolved it: everything the other roles need,
 // so that none of them touches global memory to set a unit up.
@@ -101,15 +85,12 @@ struct Slot {
     int f0, mc, nmma, kb;    // first feature, token rows, MMA N, stages
     int row0;                // first dispatched row of the chunk
     int wrow;                // first weight row in the stacked weight matrix
-    float ref[2];            // E4M3: largest block scale of the rows (gate or W_d, up)
-    float s[2][48];          // E4M3: block scales of the rows along K (d / 128 <= 48)
     int src[kNT];            // B row n: token (up) or dispatched row (down), n < mc
 };
 
 template <int kNT>
 struct Tail {
     uint64_t full[6], empty[6];          // weight + token ring (Stages <= 6)
-    uint64_t cfull[3], cempty[3];        // E4M3: decoded stages
     uint64_t ufull[kNU], uempty[kNU];
     uint64_t tfull[4], tempty[4];
     uint64_t drain, pstart;              // pstart: the producer has started a unit
@@ -124,10 +105,10 @@ struct Tail {
 static_assert(offsetof(Tail<16>, stage) % 16 == 0 && offsetof(Tail<128>, stage) % 16 == 0, "16-byte staging");
 static_assert(sizeof(Tail<16>) % 16 == 0 && sizeof(Tail<128>) % 16 == 0, "tail size");
 
-template <bool kFp8, int kNT>
+template <int kNT>
 __host__ __device__ constexpr size_t smem_bytes()
 {
-    return 1024 + (size_t)Cfg<kFp8, kNT>::Ring + sizeof(Tail<kNT>);
+    return 1024 + (size_t)Cfg<kNT>::Ring + sizeof(Tail<kNT>);
 }
 
 struct Maps {
@@ -142,7 +123,6 @@ struct Args {
     const int32_t *perm, *offsets;
     __nv_bfloat16 *h;                 // [N*K + N, I]
     __nv_bfloat16 *y_perm, *y_shared;
-    const float *sg_r, *su_r, *sd_r, *sg_s, *su_s, *sd_s;   // E4M3 block scales
     int *err;                         // device status word
     int *claim;                       // unit counter (zero at launch)
     int *up_done;                     // [groups] finished up units (zero at launch)
@@ -152,71 +132,25 @@ struct Args {
     int nt;                           // token rows per unit at most
 };
 
-// Instruction descriptor of tcgen05.mma kind::f16: A and B both BF16 or both
-// F16 (K-major), FP32 accumulator, M x N.
-__host__ __device__ constexpr uint32_t idesc(int M, int N, bool bf16)
+// Instruction descriptor of tcgen05.mma kind::f16: A and B both BF16
+// (K-major), FP32 accumulator, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N)
 {
-    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
-}
-
-// Four E4M3 values (one 32-bit word, element 0 in the low byte) -> two F16x2
-// words, exactly (every E4M3 value is an F16 value).
-__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t &a, uint32_t &b)
-{
-    asm("{\n\t.reg .b16 l, h;\n\t"
-        "mov.b32 {l, h}, %2;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
-        : "=r"(a), "=r"(b)
-        : "r"(w));
-}
-
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
-{
-    uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-
-// Decodes one 128-byte E4M3 row (128-byte swizzle, row q of its tile)
-// exactly into 64 columns of F16 in tensor memory at `taddr` (this warp's
-// lanes).
-__device__ __forceinline__ void convert_row_tmem(const uint8_t *tile, int q, uint32_t taddr)
-{
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint32_t o[32];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const int c = half * 4 + c4;
-            const uint4 w = *reinterpret_cast<const uint4 *>(tile + q * 128 + ((c ^ (q & 7)) << 4));
-            const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                uint32_t lo, hi;
-                e4m3x4_to_f16(wd[h], o[c4 * 8 + 2 * h], o[c4 * 8 + 2 * h + 1]);
-            }
-        }
-        tmem_st32(taddr + half * 32, o);
-    }
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace swp
 
 using namespace swp;
 
-enum : int { kErrF16Range = 2 };
-
-template <bool kFp8, int kNT>
-__global__ void __launch_bounds__(Cfg<kFp8, kNT>::Warps * 32, 1)
+template <int kNT>
+__global__ void __launch_bounds__(Cfg<kNT>::Warps * 32, 1)
 ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
 {
-    using C = Cfg<kFp8, kNT>;
+    using C = Cfg<kNT>;
     constexpr int SA = C::Stages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *convb = smem + (size_t)SA * C::Stage;           // E4M3: F16 token tiles
     Tail<kNT> *T = reinterpret_cast<Tail<kNT> *>(smem + C::Ring);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort = &T->abort;
@@ -224,11 +158,7 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
     if (threadIdx.x == 0) {
         for (int s = 0; s < SA; ++s) {
             mbar_init(&T->full[s], 1);                   // TMA expect_tx (weights and token rows)
-            mbar_init(&T->empty[s], kFp8 ? 128 : 1);     // converters | tcgen05.commit
-        }
-        for (int s = 0; s < C::ConvStages; ++s) {
-            mbar_init(&T->cfull[s], 128);
-            mbar_init(&T->cempty[s], 1);
+            mbar_init(&T->empty[s], 1);                  // tcgen05.commit
         }
         for (int j = 0; j < kNU; ++j) {
             mbar_init(&T->ufull[j], 1);
@@ -288,7 +218,6 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
             }
             const Unit U = decode(u, T->pre, T->off, a);
             const int row0 = U.G.row0 + U.m0;
-            const size_t ge = U.G.shared ? 0 : (size_t)U.G.g;
             // every global load of the unit is issued before any is used: one round trip
             constexpr int RPL = (kNT + 31) / 32;         // rows per lane
             int srcv[RPL];
@@ -300,34 +229,12 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                     srcv[i] = U.up ? (U.G.shared ? row0 + n - a.N * a.K : checked_index(a.perm[row0 + n], 0, a.N, a.err))
                                    : row0 + n;
             }
-            WarpScales w0, w1;
-            w0.lo = w0.hi = w1.lo = w1.hi = 0.f;
-            if (kFp8) {
-                if (U.up) {
-                    const int nkb = a.d / 128;
-                    const size_t off = (ge * (a.I / 128) + U.f0 / 128) * nkb;
-                    w0.load((U.G.shared ? a.sg_s : a.sg_r) + off, nkb);
-                    w1.load((U.G.shared ? a.su_s : a.su_r) + off, nkb);
-                } else {        // the two row blocks of W_d
-                    const int nkb = a.I / 128;
-                    const float *sd = (U.G.shared ? a.sd_s : a.sd_r) + (ge * (a.d / 128) + U.f0 / 128) * nkb;
-                    w0.load(sd, nkb);
-                    w1.load(sd + nkb, nkb);
-                }
-            }
             const int need = (a.I / kF) * chunks_of(U.G.rows, a.nt);
             int done = need;
             if (!U.up && lane == 0) done = ld_acquire(a.up_done + U.o);
 #pragma unroll
             for (int i = 0; i < RPL; ++i)
                 if (lane + 32 * i < U.mc) sl.src[lane + 32 * i] = srcv[i];
-            if (kFp8) {
-                sl.s[0][lane] = w0.lo;
-                sl.s[1][lane] = w1.lo;
-                if (lane < 16) { sl.s[0][lane + 32] = w0.hi; sl.s[1][lane + 32] = w1.hi; }
-                const float r0 = w0.ref(), r1 = w1.ref();
-                if (lane == 0) { sl.ref[0] = r0; sl.ref[1] = r1; }
-            }
             bool good = true;
             if (lane == 0 && done < need) {       // the expert's H rows come from up units of any CTA
                 const long long t0 = clock64();
@@ -430,45 +337,24 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 tc_fence_after();
                 const uint32_t dg = tmem + acc * C::AccW;          // gate (or W_d) accumulator
                 const uint32_t du = dg + kNT;                      // up accumulator
-                const uint32_t id = idesc(kM, sl.nmma, !kFp8);
+                const uint32_t id = idesc_bf16(kM, sl.nmma);
                 bool ok = true;
                 for (int kb = 0; kb < kb_n; ++kb, ++it) {
-                    if (kFp8) {       // A: F16 in tensor memory (8 columns per k16); B: F16 panels
-                        const int cs = it % C::ConvStages;
-                        if (!mbar_wait(&T->cfull[cs], (it / C::ConvStages) & 1, abort, a.err, a.wait_limit)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint32_t at = tmem + C::AccCols + cs * C::ConvCols;
-                        // token tile 0 carries the first weight tile's block scale, tile 1 the second's
-                        const uint64_t b0 = sw128_kmajor_desc(smem_u32(convb + (size_t)cs * 2 * C::BTile));
-                        const uint64_t b1 = sw128_kmajor_desc(smem_u32(convb + (size_t)(cs * 2 + 1) * C::BTile));
-                        // all k-steps of one accumulator before the other: an MMA
-                        // that switches accumulators costs nearly twice as much
+                    const int s = it % SA;
+                    if (!mbar_wait(&T->full[s], (it / SA) & 1, abort, a.err, a.wait_limit)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + (size_t)s * C::Stage);
+                    const uint64_t a0 = sw128_kmajor_desc(sa), a1 = sw128_kmajor_desc(sa + kATile);
+                    const uint64_t bd = sw128_kmajor_desc(sa + 2 * kATile);
+                    // all k-steps of one accumulator before the other: an MMA
+                    // that switches accumulators costs nearly twice as much
 #pragma unroll
-                        for (int k = 0; k < C::BK / 16; ++k) {
-                            const uint64_t ko = (uint64_t)(((k >> 2) * C::Panel + (k & 3) * 32) >> 4);
-                            umma_f16_tmem_a(dg, at + k * 8, b0 + ko, id, (kb | k) != 0);
-                        }
+                    for (int k = 0; k < C::BK / 16; ++k)
+                        umma_bf16(dg, a0 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), id, (kb | k) != 0);
 #pragma unroll
-                        for (int k = 0; k < C::BK / 16; ++k) {
-                            const uint64_t ko = (uint64_t)(((k >> 2) * C::Panel + (k & 3) * 32) >> 4);
-                            umma_f16_tmem_a(du, at + 64 + k * 8, b1 + ko, id, (kb | k) != 0);
-                        }
-                        umma_commit(&T->cempty[cs]);
-                    } else {
-                        const int s = it % SA;
-                        if (!mbar_wait(&T->full[s], (it / SA) & 1, abort, a.err, a.wait_limit)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint32_t sa = smem_u32(smem + (size_t)s * C::Stage);
-                        const uint64_t a0 = sw128_kmajor_desc(sa), a1 = sw128_kmajor_desc(sa + kATile);
-                        const uint64_t bd = sw128_kmajor_desc(sa + 2 * kATile);
-#pragma unroll
-                        for (int k = 0; k < C::BK / 16; ++k)
-                            umma_bf16(dg, a0 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), id, (kb | k) != 0);
-#pragma unroll
-                        for (int k = 0; k < C::BK / 16; ++k)
-                            umma_bf16(du, a1 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), id, (kb | k) != 0);
-                        umma_commit(&T->empty[s]);
-                    }
+                    for (int k = 0; k < C::BK / 16; ++k)
+                        umma_bf16(du, a1 + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), id, (kb | k) != 0);
+                    umma_commit(&T->empty[s]);
                 }
                 if (!ok) break;
                 umma_commit(&T->tfull[acc]);
@@ -494,7 +380,6 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
             if (sl.u < 0) break;
             const bool up = sl.up, shared = sl.shared;
             const int mc = sl.mc, nmma = sl.nmma, f0 = sl.f0, r0 = sl.row0, o = sl.o;
-            const float s0 = kFp8 ? sl.ref[0] : 1.f, s1 = kFp8 ? sl.ref[1] : 1.f;
             const int acc = us % C::NAcc;
             if (!bar_and(1, C::EpiThreads, mbar_wait(&T->tfull[acc], (us / C::NAcc) & 1, abort, a.err, a.wait_limit)))
                 break;
@@ -520,14 +405,13 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                     if (up) tmem_ld16(tg + kNT + c, *reinterpret_cast<uint32_t(*)[16]>(u));
                 }
                 tmem_ld_wait();
-                const float sa = t ? s1 : s0;
                 __nv_bfloat16 *dt = dst + t * kM;
 #pragma unroll
                 for (int half = 0; half < W / 16; ++half) {
 #pragma unroll
                     for (int n = 0; n < 16; ++n) {
-                        const float gv = __uint_as_float(g[half * 16 + n]) * sa;
-                        const float val = up ? silu_mul(gv, __uint_as_float(u[half * 16 + n]) * s1) : gv;
+                        const float gv = __uint_as_float(g[half * 16 + n]);
+                        const float val = up ? silu_mul(gv, __uint_as_float(u[half * 16 + n])) : gv;
                         stg[n * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
                     }
                     __syncwarp();
@@ -550,72 +434,6 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
                 if (up) red_release_add(a.up_done + o, 1);
                 mbar_arrive(&T->uempty[j]);
             }
-        }
-    } else if (kFp8 && warp >= kConvWarp) {
-        // ---------------------------------------------------------- converters
-        // A warp reaches only its own quadrant of tensor-memory lanes, so the
-        // rows a thread converts are its lane in that quadrant (of the gate and
-        // of the up tile). Group `grp` takes the stages it with it % 2 == grp.
-        const int quad = warp & 3, grp = (warp - kConvWarp) / 4;
-        const int q = quad * 32 + lane;
-        uint32_t it = 0;
-        bool ok = true;
-        for (int us = 0; ok; ++us) {
-            const int j = us % kNU;
-            if (!mbar_wait(&T->ufull[j], (us / kNU) & 1, abort, a.err, a.wait_limit)) break;
-            const Slot<kNT> &sl = T->slot[j];
-            if (sl.u < 0) break;
-            const bool up = sl.up;
-            const int kb_n = sl.kb, nmma = sl.nmma;
-            const float inv0 = sl.ref[0] > 0.f ? 1.f / sl.ref[0] : 0.f;
-            const float inv1 = sl.ref[1] > 0.f ? 1.f / sl.ref[1] : 0.f;
-            bool range_ok = true;
-            for (int kb = 0; kb < kb_n; ++kb, ++it) {
-                if ((int)(it % kConvGroups) != grp) continue;
-                const int s = it % SA, cs = it % C::ConvStages;
-                const float r0 = sl.s[0][kb] * inv0, r1 = sl.s[1][kb] * inv1;     // in [0, 1]
-                if (!mbar_wait(&T->full[s], (it / SA) & 1, abort, a.err, a.wait_limit) ||
-                    !mbar_wait(&T->cempty[cs], ((it / C::ConvStages) & 1) ^ 1, abort, a.err, a.wait_limit)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t *A8 = smem + (size_t)s * C::Stage;
-                const uint8_t *Braw = A8 + 2 * kATile;
-                uint8_t *B0 = convb + (size_t)cs * 2 * C::BTile, *B1 = B0 + C::BTile;
-                const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16) + C::AccCols + cs * C::ConvCols;
-                convert_row_tmem(A8, q, tq);
-                convert_row_tmem(A8 + kATile, q, tq + 64);
-                // B: BF16 token (or H) rows times each weight tile's s_kb / s_ref, as F16
-                // at the same swizzled positions (a panel holds kNT rows of eight
-                // 16-byte chunks): the block scale rides on the small token tile
-                // instead of on every weight
-#pragma unroll
-                for (int i = 0; i < C::BTile / 16 / 128; ++i) {
-                    const int c16 = q + i * 128;
-                    if (((c16 % (kNT * 8)) >> 3) < nmma) {
-                        const uint4 w = *reinterpret_cast<const uint4 *>(Braw + c16 * 16);
-                        const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-                        uint32_t p0[4], p1[4];
-                        float mx = 0.f;
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float f0 = bf16_lo(wd[e]), f1 = bf16_hi(wd[e]);
-                            p0[e] = pack_f16x2(f0 * r0, f1 * r0);
-                            p1[e] = pack_f16x2(f0 * r1, f1 * r1);
-                            mx = fmaxf(mx, fmaxf(fabsf(f0), fabsf(f1)));
-                        }
-                        if (!(mx <= 65504.f)) range_ok = false;
-                        *reinterpret_cast<uint4 *>(B0 + c16 * 16) = make_uint4(p0[0], p0[1], p0[2], p0[3]);
-                        *reinterpret_cast<uint4 *>(B1 + c16 * 16) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
-                    }
-                }
-                tmem_st_wait();
-                fence_proxy_async();
-                tc_fence_before();
-                mbar_arrive(&T->cfull[cs]);
-                mbar_arrive(&T->empty[s]);
-            }
-            if (!range_ok) atomicCAS(a.err, kErrNone, kErrF16Range);
         }
     }
     tc_fence_before();
@@ -640,19 +458,17 @@ static PFN_cuTensorMapEncodeTiled_v12000 swap_encode_fn()
     return fn;
 }
 
-// Weight map over a row-major [rows, cols] matrix, box of 128 rows x 128
-// bytes (64 BF16 or 128 E4M3 columns), 128-byte swizzle: the layout the MMA
-// reads (BF16), and one the converters read without bank conflicts (E4M3).
-static bool weight_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, bool fp8)
+// BF16 weight map over a row-major [rows, cols] matrix, box of 128 rows x 64
+// columns, 128-byte swizzle: the layout the MMA reads.
+static bool weight_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols)
 {
     auto fn = swap_encode_fn();
     if (!fn) return false;
-    const uint64_t es = fp8 ? 1 : 2;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * es};
-    cuuint32_t box[2] = {(cuuint32_t)(128 / es), (cuuint32_t)kM};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kM};
     cuuint32_t estr[2] = {1, 1};
-    return fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base),
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base),
               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -684,32 +500,31 @@ static int swap_sm_count()
     return n;
 }
 
-template <bool kFp8, int kNT>
+template <int kNT>
 static void launch_cfg(const Maps &m, const Args &a, cudaStream_t st)
 {
-    using C = Cfg<kFp8, kNT>;
-    constexpr size_t smem = smem_bytes<kFp8, kNT>();
+    using C = Cfg<kNT>;
+    constexpr size_t smem = smem_bytes<kNT>();
     static_assert(smem <= (size_t)kSmemLimit, "shared memory per CTA");
-    auto k = ffn_swap_kernel<kFp8, kNT>;
+    auto k = ffn_swap_kernel<kNT>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     launch_pdl(k, swap_sm_count(), C::Warps * 32, smem, st, m, a);
 }
 
 kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, int K, const int32_t *perm,
-                            const int32_t *offsets, int w_dtype, const ExpertPtrs &routed, const ExpertPtrs *shared,
+                            const int32_t *offsets, const ExpertPtrs &routed, const ExpertPtrs *shared,
                             __nv_bfloat16 *h, __nv_bfloat16 *y_perm, __nv_bfloat16 *y_shared, int *status,
                             int *sync, long long wait_limit, cudaStream_t st)
 {
     constexpr int token_chunk = 16;
     if (E + 1 > kMaxOrd || E + 2 > kSyncInts) return fail(KMOE_ERR_UNSUPPORTED, "swap-AB FFN: too many experts");
     if (d % kFD || I % kF) return fail(KMOE_ERR_UNSUPPORTED, "swap-AB FFN: d %% 256, I %% 128 must be 0");
-    const bool fp8 = w_dtype == KMOE_E4M3_B128;
     const ExpertPtrs sh = shared ? *shared : routed;     // unused maps still need a valid base
     Maps m{};
-    const bool ok = weight_map(&m.g_r, routed.wg, (uint64_t)E * I, d, fp8) &&
-                    weight_map(&m.u_r, routed.wu, (uint64_t)E * I, d, fp8) &&
-                    weight_map(&m.g_s, sh.wg, I, d, fp8) && weight_map(&m.u_s, sh.wu, I, d, fp8) &&
-                    weight_map(&m.d_r, routed.wd, (uint64_t)E * d, I, fp8) && weight_map(&m.d_s, sh.wd, d, I, fp8) &&
+    const bool ok = weight_map(&m.g_r, routed.wg, (uint64_t)E * I, d) &&
+                    weight_map(&m.u_r, routed.wu, (uint64_t)E * I, d) &&
+                    weight_map(&m.g_s, sh.wg, I, d) && weight_map(&m.u_s, sh.wu, I, d) &&
+                    weight_map(&m.d_r, routed.wd, (uint64_t)E * d, I) && weight_map(&m.d_s, sh.wd, d, I) &&
                     act_map(&m.xg, x, N, d, 1) && act_map(&m.hb, h, (uint64_t)N * K + N, I, token_chunk);
     if (!ok) return fail(KMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     Args a{};
@@ -719,8 +534,6 @@ kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, 
     a.h = h;
     a.y_perm = y_perm;
     a.y_shared = y_shared;
-    a.sg_r = routed.sg; a.su_r = routed.su; a.sd_r = routed.sd;
-    a.sg_s = sh.sg; a.su_s = sh.su; a.sd_s = sh.sd;
     a.err = status;
     a.claim = sync;
     a.up_done = sync + 1;
@@ -728,10 +541,9 @@ kmoe_status launch_ffn_swap(const __nv_bfloat16 *x, int N, int d, int I, int E, 
     a.N = N; a.K = K; a.E = E; a.d = d; a.I = I;
     a.has_shared = shared ? 1 : 0;
     a.n_ord = E + a.has_shared;
-    a.sk = fp8 ? Cfg<true, 16>::BK : Cfg<false, 16>::BK;
+    a.sk = Cfg<token_chunk>::BK;
     a.nt = token_chunk;
-    if (fp8) launch_cfg<true, token_chunk>(m, a, st);
-    else launch_cfg<false, token_chunk>(m, a, st);
+    launch_cfg<token_chunk>(m, a, st);
     return check_launch("ffn_swap");
 }
 

@@ -71,6 +71,8 @@ kmoe_status launch_rmsnorm(const __nv_bfloat16 *h, const __nv_bfloat16 *gamma, f
     const int pieces = d / 256, grid = (N + kNormRowsPerCta - 1) / kNormRowsPerCta;
     if (d % 256)
         return fail(KMOE_ERR_UNSUPPORTED, "rmsnorm: d=%d must be a multiple of 256", d);
+    if (pieces > kNormMaxVec)
+        return fail(KMOE_ERR_UNSUPPORTED, "rmsnorm: d=%d must be at most %d", d, kNormMaxVec * 256);
 #define KMOE_NORM(V) launch_pdl(rmsnorm_bf16_kernel<V>, grid, kNormThreads, 0, st, h, gamma, eps, N, d, x)
     switch (pieces) {
     case 1: KMOE_NORM(1); break;
@@ -97,8 +99,8 @@ kmoe_status launch_rmsnorm(const __nv_bfloat16 *h, const __nv_bfloat16 *gamma, f
     case 22: KMOE_NORM(22); break;
     case 23: KMOE_NORM(23); break;
     case 24: KMOE_NORM(24); break;
-    default:
-        return fail(KMOE_ERR_UNSUPPORTED, "rmsnorm: d=%d must be at most 6144", d);
+    default:                  // d == 0
+        return fail(KMOE_ERR_UNSUPPORTED, "rmsnorm: d=%d must be positive", d);
     }
 #undef KMOE_NORM
     return check_launch("rmsnorm");

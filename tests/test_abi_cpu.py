@@ -161,6 +161,22 @@ def test_quant_1x128_checks_arguments_on_the_host(lib):
     assert lib.moe_quant_1x128(None, 0, 128, None, None, None) == kmoe.KMOE_OK
 
 
+def test_two_term_small_batches_are_sized_for_both_code_planes():
+    """E4M3 weights with BF16 x below 256 tokens run with two-term activations: H's two code planes
+    take the BF16 H's bytes, and H's scales plus x's high codes, low codes and scales come on top;
+    from 256 tokens the workspace is the BF16-weight one."""
+    d, E, K, I = 2560, 384, 6, 512
+    for N in (1, 32, 255):
+        e4 = kmoe.moe_workspace_size(N, d, E, K, I, kmoe.KMOE_BF16, kmoe.KMOE_E4M3_B128)
+        bf = kmoe.moe_workspace_size(N, d, E, K, I, kmoe.KMOE_BF16, kmoe.KMOE_BF16)
+        R = N * K + N
+        expected = R * (I // 128) * 4 + 2 * N * d + N * (d // 128) * 4
+        assert abs((e4 - bf) - expected) <= 4 * 256
+    for N in (256, 4096):
+        assert kmoe.moe_workspace_size(N, d, E, K, I, kmoe.KMOE_BF16, kmoe.KMOE_E4M3_B128) == \
+            kmoe.moe_workspace_size(N, d, E, K, I, kmoe.KMOE_BF16, kmoe.KMOE_BF16)
+
+
 def test_wait_limit_rejects_negative_and_restores_the_default(lib):
     assert lib.moe_set_wait_limit(-1) == kmoe.KMOE_ERR_INVALID_ARG
     assert lib.moe_set_wait_limit(1000) == kmoe.KMOE_OK
@@ -172,12 +188,12 @@ def test_fp8_activation_mode_is_sized_and_checked_on_the_host(lib):
     multiple of 256 is rejected before anything is enqueued (no GPU needed)."""
     N, d, E, K, I = 32, 2560, 384, 6, 512
     a8 = kmoe.moe_workspace_size(N, d, E, K, I, kmoe.KMOE_BF16, kmoe.KMOE_E4M3_B128_A8)
-    e4 = kmoe.moe_workspace_size(N, d, E, K, I, kmoe.KMOE_BF16, kmoe.KMOE_E4M3_B128)
+    bf = kmoe.moe_workspace_size(N, d, E, K, I, kmoe.KMOE_BF16, kmoe.KMOE_BF16)
     # H as one-byte codes (instead of BF16) plus its scales, and x's codes and scales (each piece
     # 256-byte aligned)
     R = N * K + N
     expected = -R * I + R * (I // 128) * 4 + N * d + N * (d // 128) * 4
-    assert a8 > 0 and abs((a8 - e4) - expected) <= 4 * 256
+    assert a8 > 0 and abs((a8 - bf) - expected) <= 4 * 256
     assert kmoe.moe_block_workspace_size(N, d, E, K, I, kmoe.KMOE_E4M3_B128_A8) > 0
     aligned = ctypes.c_void_p(1 << 20)
     ex = kmoe.Experts(aligned, aligned, aligned, aligned, aligned, aligned, kmoe.KMOE_E4M3_B128_A8)
