@@ -27,13 +27,14 @@
 // expected rows per expert): a weight tile crosses shared memory once per
 // chunk, so larger batches take larger chunks.
 //
-// Two-term mode (kTwo, 16-row chunks): the same kernel serves E4M3 weights
-// with BF16 activations. Every activation group is held as two E4M3 codes
+// Two-term mode (kTwo): the same kernel serves E4M3 weights with BF16
+// activations. Every activation group is held as two E4M3 codes
 // with one scale, x = s * (hi + lo / 16) up to about 2^-8 of |x| (the size of
-// a BF16 rounding); the hi rows are B rows 0 .. 15 and the lo rows B rows
-// 16 .. 31 of one N = 32 operand, so a K block still takes four MMAs per
-// weight tile, and the promotion adds (P_hi + P_lo / 16) * s_w * s_x. H is
-// kept in the same two-term form between up and down.
+// a BF16 rounding); the hi rows of a chunk are B rows 0 .. kNT-1 and the lo
+// rows B rows kNT .. 2 kNT-1 of one N = 2 kNT operand, so a K block still
+// takes four MMAs per weight tile, and the promotion adds
+// (P_hi + P_lo / 16) * s_w * s_x. H is kept in the same two-term form
+// between up and down.
 //
 // Warp roles (one CTA per SM, persistent), P = 4 promotion warps for chunks
 // of up to 32 rows and 8 for 64:
@@ -80,13 +81,12 @@ struct Cfg {
     static constexpr int BRows = kTwo ? 2 * kNT : kNT;   // B operand rows: the chunk's codes (hi | lo)
     static constexpr int BTile = BRows * kBK;            // token codes of one stage
     static constexpr int Stage = 2 * kATile + BTile;     // weight tile 0 | weight tile 1 | token codes
-    static constexpr int Stages = kTwo ? 5 : kNT == 16 ? 6 : kNT == 32 ? 5 : 4;
+    static constexpr int Stages = kTwo ? (kNT == 64 ? 3 : 5) : kNT == 16 ? 6 : kNT == 32 ? 5 : 4;
     static constexpr int PW = 2 * BRows;                 // one partial slot: tile 0 | tile 1
     static constexpr int NP = 512 / PW < 8 ? 512 / PW : 8;   // partial slots in tensor memory
     static constexpr int TmemCols = NP * PW <= 256 ? 256 : 512;
     static constexpr int RPL = (kNT + 31) / 32;          // chunk rows per scheduler lane
     static_assert(kNT == 16 || kNT == 32 || kNT == 64, "token chunk of 16, 32 or 64 rows");
-    static_assert(!kTwo || kNT == 16, "two-term operands with 16-row chunks");
     static_assert(Stage % 1024 == 0, "tiles on 1024-byte boundaries (128-byte swizzle atoms)");
     static_assert(NP * PW <= TmemCols, "tensor memory columns");
 };
@@ -450,7 +450,33 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                 tc_fence_after();
                 const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + p * C::PW + c0;
                 const float w0 = sl.s[0][kb], w1 = sl.s[1][kb];
-                if constexpr (kTwo) {
+                if constexpr (kTwo && TPW == 32) {
+                    // 32 columns per warp: hi and lo in turn through one register block
+                    const float w0l = 0.0625f * w0, w1l = 0.0625f * w1;
+                    uint32_t v[TPW];
+                    tmem_load<TPW>(ta, v);                 // tile 0, hi
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int n = 0; n < TPW; ++n)
+                        acc0[n] = fmaf(__uint_as_float(v[n]), w0 * __shfl_sync(0xffffffffu, sx0, n), acc0[n]);
+                    tmem_load<TPW>(ta + kNT, v);           // tile 0, lo
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int n = 0; n < TPW; ++n)
+                        acc0[n] = fmaf(__uint_as_float(v[n]), w0l * __shfl_sync(0xffffffffu, sx0, n), acc0[n]);
+                    tmem_load<TPW>(ta + C::BRows, v);      // tile 1, hi
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int n = 0; n < TPW; ++n)
+                        acc1[n] = fmaf(__uint_as_float(v[n]), w1 * __shfl_sync(0xffffffffu, sx0, n), acc1[n]);
+                    tmem_load<TPW>(ta + C::BRows + kNT, v);   // tile 1, lo
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    mbar_arrive(&T->pempty[p]);
+#pragma unroll
+                    for (int n = 0; n < TPW; ++n)
+                        acc1[n] = fmaf(__uint_as_float(v[n]), w1l * __shfl_sync(0xffffffffu, sx0, n), acc1[n]);
+                } else if constexpr (kTwo) {
                     uint32_t vh[TPW], vl[TPW];             // tile 0: hi and lo products
                     tmem_load<TPW>(ta, vh);
                     tmem_load<TPW>(ta + kNT, vl);
@@ -675,11 +701,13 @@ kmoe_status launch_ffn_a8(const uint8_t *xq, const float *xs, int N, int d, int 
     // Chunk rows from the expected rows per routed expert, N * K / E: 16 while
     // experts see a dozen tokens or fewer, then 32, then 64 (a weight tile
     // crosses shared memory once per chunk).
-    if (xl) {                 // two-term operands (BF16-precision activations): 16-row chunks
-        if (!hl) return fail(KMOE_ERR_INVALID_ARG, "FP8 FFN: two-term mode needs both low-code planes");
-        return launch_a8_cfg<16, true>(routed, sh, a, st);
-    }
     const long long avg = (long long)N * K / E;
+    if (xl) {                 // two-term operands (BF16-precision activations)
+        if (!hl) return fail(KMOE_ERR_INVALID_ARG, "FP8 FFN: two-term mode needs both low-code planes");
+        if (avg <= 12) return launch_a8_cfg<16, true>(routed, sh, a, st);
+        if (avg <= 32) return launch_a8_cfg<32, true>(routed, sh, a, st);
+        return launch_a8_cfg<64, true>(routed, sh, a, st);
+    }
     if (avg <= 12) return launch_a8_cfg<16>(routed, sh, a, st);
     if (avg <= 32) return launch_a8_cfg<32>(routed, sh, a, st);
     return launch_a8_cfg<64>(routed, sh, a, st);

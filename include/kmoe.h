@@ -183,6 +183,11 @@ kmoe_status moe_permute_noalloc(const int32_t *topk_idx, int N, int K, int E,
  *   y_shared[t] = F_shared(x[t])         (skipped when shared == NULL)
  * with F(x) = W_d (SiLU(W_g x) * (W_u x)), FP32 accumulation, and the
  * intermediate SiLU(.)*up rounded to the output dtype.
+ * With KMOE_E4M3_B128 weights, BF16 x, d a multiple of 256 and N < 256 the
+ * GEMMs run on the FP8 tensor cores: each 128-column group of a GEMM input
+ * row (x, and H before the down projection) is held as two E4M3 terms with
+ * one FP32 scale, v = s * (hi + lo / 16), within about 2^-8 of |v| (BF16's
+ * own rounding is 2^-9), over the whole BF16 range.
  * x device [N, d] (x_dtype F32 or BF16). perm_token, offsets as produced by
  * moe_permute. Output dtype: FP32 when the weights are FP32, else BF16.
  * y_perm device [N*K, d]; y_shared device [N, d]. With KMOE_E4M3_B128_A8

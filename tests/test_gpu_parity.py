@@ -10,7 +10,7 @@ import torch
 
 import oracle
 from fine_grained_sparse_fp32_b200 import _build, kmoe
-from fine_grained_sparse_fp32_b200.inputs import CONFIGS, make_block_inputs, make_inputs, to_host
+from fine_grained_sparse_fp32_b200.inputs import CONFIGS, LayerConfig, make_block_inputs, make_inputs, to_host
 from parity import G_TOL, TOL, biased_scores, check_routing, frob_rel_err, row_rel_err
 
 pytestmark = pytest.mark.gpu
@@ -142,7 +142,7 @@ def test_permute_all_tokens_on_the_same_experts():
 
 # ------------------------------------------------------------ grouped FFN
 @pytest.mark.parametrize("name,N", [("tiny", None), ("decode", None), ("fp8_decode", None), ("decode", 200),
-                                    ("fp8_decode", 130), ("prefill", 256), ("prefill", 300), ("prefill", 1000),
+                                    ("fp8_decode", 130), ("fp8_decode", 1), ("fp8_decode", 255), ("prefill", 256), ("prefill", 300), ("prefill", 1000),
                                     ("fp8_prefill", 300), ("fp8_prefill", 777), ("fp8a8_decode", None),
                                     ("fp8a8_decode", 1), ("fp8a8_decode", 255), ("fp8a8_prefill", 256),
                                     ("fp8a8_prefill", 1000), ("fp8a8_prefill", 2500)])
@@ -165,6 +165,29 @@ def test_grouped_ffn_matches_oracle(name, N):
     ref_s = expert_ref(host, toks, np.full(len(toks), cfg.E))
     got_s = y_shared[torch.from_numpy(toks).cuda().long()].float().cpu().numpy()
     assert row_rel_err(got_s, ref_s) <= TOL[cfg.w_dtype]
+
+
+@pytest.mark.parametrize("E,N,chunk", [(64, 200, 32), (16, 255, 64), (64, 40, 16)])
+def test_two_term_fp8_ffn_chunk_sizes(E, N, chunk):
+    """E4M3 weights with BF16 activations below 256 tokens take the FP8 tensor cores with two-term
+    activations; with few experts the expected rows per expert N*K/E pick 16-, 32- or 64-row chunks
+    (B operands of 32, 64 or 128 rows). Reduced layer (d = 512, I = 128) drawn on the host."""
+    cfg = LayerConfig(f"two_term_{E}_{N}", N, 512, E, 6, 128, "bf16", "e4m3")
+    avg = N * cfg.K // E
+    assert chunk == (16 if avg <= 12 else 32 if avg <= 32 else 64)
+    host = make_inputs(cfg, seed=5, device="cpu")
+    dev = {k: (v.to("cuda") if torch.is_tensor(v) else v) for k, v in host.items()}
+    l_ora = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
+    i_ora, _, _ = oracle.select(l_ora, host["bias"], cfg.K)
+    _, offsets, perm, _ = oracle.permute(i_ora, cfg.E)
+    y_perm, y_shared = kmoe.moe_grouped_ffn(dev["x"], dev, torch.from_numpy(perm).cuda(),
+                                            torch.from_numpy(offsets).cuda())
+    torch.cuda.synchronize()
+    rows = np.arange(cfg.N * cfg.K)
+    ref = expert_ref(host, perm, np.searchsorted(offsets, rows, side="right") - 1)
+    assert row_rel_err(y_perm.float().cpu().numpy(), ref) <= TOL["e4m3"]
+    ref_s = expert_ref(host, np.arange(cfg.N), np.full(cfg.N, cfg.E))
+    assert row_rel_err(y_shared.float().cpu().numpy(), ref_s) <= TOL["e4m3"]
 
 
 @pytest.mark.parametrize("name,N", [("decode", 200), ("fp8_decode", 200), ("decode", 33), ("fp8a8_decode", 200),
