@@ -48,11 +48,13 @@ TRAFFIC_SOURCES = {
     "tc": ('fine_grained_sparse_fp32_b200/csrc/ffn_tc.cu', 'fine_grained_sparse_fp32_b200/csrc/sm100.cuh', 'fine_grained_sparse_fp32_b200/csrc/common.cuh'),
 }
 TRAFFIC = {
-    "decode": ("swap", "4d5ff5181bed47c9", (1195.6 + 1.7) * 1e6),
-    "fp8_decode": ("a8", "90fdf62ea970a409", (598.1 + 1.4) * 1e6),
-    "fp8a8_decode": ("a8", "90fdf62ea970a409", (598.1 + 1.3) * 1e6),
-    "fp8a8_prefill": ("a8", "90fdf62ea970a409", (1595.5 + 105.7) * 1e6),
-    "prefill": ("tc", "bf3858b93be7c4e5", (2210.4 + 39.7 + 1192.2 + 238.9) * 1e6),   # up + down kernel
+    "decode": ("swap", "e5fcef145ca727b3", (1195.6 + 1.7) * 1e6),
+    "fp8_decode": ("a8", "89ce473296cdec8b", (598.1 + 1.5) * 1e6),
+    "fp8a8_decode": ("a8", "89ce473296cdec8b", (598.0 + 1.3) * 1e6),
+    "fp8a8_prefill": ("a8", "89ce473296cdec8b", (1591.9 + 104.6) * 1e6),
+    "prefill": ("tc", "4949badb10327177", (2221.8 + 40.9 + 1190.8 + 237.7) * 1e6),       # up + down kernel
+    "fp8_prefill": ("tc", "4949badb10327177", (1041.9 + 6.9 + 619.7 + 93.6) * 1e6),      # up + down kernel
+    "skew": ("tc", "4949badb10327177", (4254.5 + 461.2 + 1467.7 + 2298.0) * 1e6),        # up + down kernel
 }
 
 
