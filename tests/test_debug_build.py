@@ -48,8 +48,9 @@ CHILD = textwrap.dedent('''
                                       ws=ws)
         return yp, ys, kmoe.moe_device_status(ws)
 
-    # valid dispatch: status 0 and parity (swap-AB BF16, FP8 activations, tokens-as-M BF16)
-    for name, N in (("decode", 32), ("fp8a8_decode", 32), ("prefill", 300)):
+    # valid dispatch: status 0 and parity (swap-AB BF16, FP8 tensor cores with two-term and with FP8
+    # activations, tokens-as-M BF16)
+    for name, N in (("decode", 32), ("fp8_decode", 32), ("fp8a8_decode", 32), ("prefill", 300)):
         cfg, dev, host, offsets, perm = case(name, N)
         yp, ys, st = ffn(cfg, dev, perm, offsets)
         assert st == 0, (name, st)
@@ -68,6 +69,10 @@ CHILD = textwrap.dedent('''
     cfg, dev, host, offsets, perm = case("decode", 32)
     bad = perm.copy(); bad[5] = cfg.N + 1000
     assert ffn(cfg, dev, bad, offsets)[2] == 3
+    # the same on the FP8 tensor-core kernel (two-term activations)
+    cfg8, dev8, host8, offsets8, perm8 = case("fp8_decode", 32)
+    bad8 = perm8.copy(); bad8[7] = -5
+    assert ffn(cfg8, dev8, bad8, offsets8)[2] == 3
     # offsets that are not a monotone partition: no unit runs, status 3 (both FFN kernels)
     bad_off = offsets.copy(); bad_off[10], bad_off[11] = bad_off[11] + 3, bad_off[10]
     assert ffn(cfg, dev, perm, bad_off)[2] == 3
