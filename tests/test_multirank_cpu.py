@@ -64,7 +64,9 @@ def test_launch_counts_follow_the_dispatch_in_abi():
     from fine_grained_sparse_fp32_b200.inputs import CONFIGS
     # router logits, top-K, dispatch (one CTA), swap-AB FFN, combine
     assert bench.launches_per_step(CONFIGS["decode"]) == 5
-    assert bench.launches_per_step(CONFIGS["fp8_decode"]) == 5
+    # E4M3 weights: the x quantiser (two-term, or FP8 activations) before the FP8 tensor-core FFN
+    assert bench.launches_per_step(CONFIGS["fp8_decode"]) == 6
+    assert bench.launches_per_step(CONFIGS["fp8a8_decode"]) == 6
     # FP32 tiny layer: router logits, top-K, dispatch, streaming FFN up + down, combine
     assert bench.launches_per_step(CONFIGS["tiny"]) == 6
     # split + tensor-core router, top-K (with chunk histograms), scatter with the scan, FFN up + down, combine
