@@ -477,23 +477,22 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                     for (int n = 0; n < TPW; ++n)
                         acc1[n] = fmaf(__uint_as_float(v[n]), w1l * __shfl_sync(0xffffffffu, sx0, n), acc1[n]);
                 } else if constexpr (kTwo) {
-                    uint32_t vh[TPW], vl[TPW];             // tile 0: hi and lo products
-                    tmem_load<TPW>(ta, vh);
-                    tmem_load<TPW>(ta + kNT, vl);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int n = 0; n < TPW; ++n)
-                        acc0[n] = fmaf(fmaf(__uint_as_float(vl[n]), 0.0625f, __uint_as_float(vh[n])),
-                                       w0 * __shfl_sync(0xffffffffu, sx0, n), acc0[n]);
-                    tmem_load<TPW>(ta + C::BRows, vh);     // tile 1
-                    tmem_load<TPW>(ta + C::BRows + kNT, vl);
+                    // 16 columns per warp: the K block's four products (hi and lo
+                    // of both tiles) in one tensor-memory round trip
+                    uint32_t vh0[TPW], vl0[TPW], vh1[TPW], vl1[TPW];
+                    tmem_load<TPW>(ta, vh0);
+                    tmem_load<TPW>(ta + kNT, vl0);
+                    tmem_load<TPW>(ta + C::BRows, vh1);
+                    tmem_load<TPW>(ta + C::BRows + kNT, vl1);
                     tmem_ld_wait();
                     tc_fence_before();
                     mbar_arrive(&T->pempty[p]);
 #pragma unroll
-                    for (int n = 0; n < TPW; ++n)
-                        acc1[n] = fmaf(fmaf(__uint_as_float(vl[n]), 0.0625f, __uint_as_float(vh[n])),
-                                       w1 * __shfl_sync(0xffffffffu, sx0, n), acc1[n]);
+                    for (int n = 0; n < TPW; ++n) {
+                        const float sn = __shfl_sync(0xffffffffu, sx0, n);
+                        acc0[n] = fmaf(fmaf(__uint_as_float(vl0[n]), 0.0625f, __uint_as_float(vh0[n])), w0 * sn, acc0[n]);
+                        acc1[n] = fmaf(fmaf(__uint_as_float(vl1[n]), 0.0625f, __uint_as_float(vh1[n])), w1 * sn, acc1[n]);
+                    }
                 } else {
                     {
                         uint32_t v[TPW];                   // tile 0 (gate or the first W_d rows)
@@ -537,10 +536,13 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                                            fmaxf(__uint_as_float(T->amax[2][tok]), __uint_as_float(T->amax[3][tok])));
                     s_l = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
                 }
+                // two-term: h * (1 / s), whose last-bit difference from h / s
+                // the low code absorbs; FP8 activations: the exact quotient
+                const float r_l = kTwo ? __frcp_rn(s_l) : 1.f;
 #pragma unroll
                 for (int n = 0; n < TPW; ++n) {
-                    const float sn = __shfl_sync(0xffffffffu, s_l, n);
-                    const float y = __fdiv_rn(hv[n], sn);
+                    const float y = kTwo ? hv[n] * __shfl_sync(0xffffffffu, r_l, n)
+                                         : __fdiv_rn(hv[n], __shfl_sync(0xffffffffu, s_l, n));
                     const uint8_t hc = e4m3_code(y);
                     T->codes[0][c0 + n][quad * 32 + lane] = hc;
                     if (kTwo) {       // lo = E4M3((y - hi) * 16)
@@ -561,7 +563,6 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                     }
                 }
                 if (quad == 0 && mine) a.hs[(size_t)(r0 + tok) * (a.I / kBK) + f0 / kBK] = s_l;
-                __threadfence();                           // H codes and scales visible before the count rises
             } else {
                 // Y = BF16 of the two tiles (features f0 .. f0+127, f0+128 ..
                 // f0+255) through a per-warp 16 x 32 transpose, so that every
@@ -593,7 +594,12 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
             }
             swp::epi_sync<C::PThreads>();                  // the slot and the staging areas are free
             if (threadIdx.x == 0) {
-                if (up) swp::red_release_add(a.up_done + o, 1);
+                // the group's H codes and scales are ordered before this
+                // thread's fence by the barrier: one fence publishes them all
+                if (up) {
+                    __threadfence();
+                    swp::red_release_add(a.up_done + o, 1);
+                }
                 mbar_arrive(&T->uempty[j]);
             }
         }

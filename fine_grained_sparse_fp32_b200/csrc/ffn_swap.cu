@@ -428,10 +428,14 @@ ffn_swap_kernel(const __grid_constant__ Maps maps, const Args a)
             }
             tc_fence_before();
             mbar_arrive(&T->tempty[acc]);
-            if (up) __threadfence();                   // H visible before the expert's count is raised
             epi_sync<C::EpiThreads>();
             if (threadIdx.x == 0) {
-                if (up) red_release_add(a.up_done + o, 1);
+                // H visible before the expert's count is raised: the group's
+                // stores are ordered before this fence by the barrier
+                if (up) {
+                    __threadfence();
+                    red_release_add(a.up_done + o, 1);
+                }
                 mbar_arrive(&T->uempty[j]);
             }
         }

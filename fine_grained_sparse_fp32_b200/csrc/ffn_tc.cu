@@ -625,9 +625,13 @@ ffn_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a)
             }
             hn = T.two ? h0 : h1;
             if (kUp) {   // this tile's H rows are stored: count it for its expert
-                __threadfence();
+                // the barrier orders the group's stores before thread 0's
+                // fence, which publishes them before the count rises
                 swp::epi_sync<128>();
-                if (threadIdx.x == 0) swp::red_release_add(a.up_done + T.g, 1);
+                if (threadIdx.x == 0) {
+                    __threadfence();
+                    swp::red_release_add(a.up_done + T.g, 1);
+                }
             }
         }
     }
