@@ -4,6 +4,8 @@ Every test here needs a B200. Inputs are drawn on the device by the seeded
 generator and copied to the host for the oracle; no oracle input or expected
 value comes from the CUDA path.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -165,6 +167,29 @@ def test_grouped_ffn_matches_oracle(name, N):
     ref_s = expert_ref(host, toks, np.full(len(toks), cfg.E))
     got_s = y_shared[torch.from_numpy(toks).cuda().long()].float().cpu().numpy()
     assert row_rel_err(got_s, ref_s) <= TOL[cfg.w_dtype]
+
+
+@pytest.mark.parametrize("N", [32, 130])
+def test_two_term_activations_keep_bf16_precision(N):
+    """The two-term E4M3 form of x and H (error about 2^-8 of each value) keeps the E4M3-weight FFN
+    within the BF16 tolerance of the oracle's exact-BF16-activation expert outputs, and closer to
+    them than single-term FP8 activations on the same weights and tokens."""
+    dev, host = layer_inputs("fp8_decode", N)
+    cfg = host["cfg"]
+    l_ora = oracle.router_logits(host["x"], cfg.x_dtype, host["w_router"], nthreads=threads())
+    i_ora, _, _ = oracle.select(l_ora, host["bias"], cfg.K)
+    _, offsets, perm, _ = oracle.permute(i_ora, cfg.E)
+    y_perm, _ = kmoe.moe_grouped_ffn(dev["x"], dev, torch.from_numpy(perm).cuda(), torch.from_numpy(offsets).cuda())
+    torch.cuda.synchronize()
+    rows = np.arange(0, cfg.N * cfg.K, 3)
+    ref = expert_ref(host, perm[rows], np.searchsorted(offsets, rows, side="right") - 1)
+    err_two = row_rel_err(y_perm[torch.from_numpy(rows).cuda().long()].float().cpu().numpy(), ref)
+    assert err_two <= TOL["bf16"]
+    a8 = dict(dev, cfg=dataclasses.replace(cfg, w_dtype="e4m3_a8"))
+    y8, _ = kmoe.moe_grouped_ffn(dev["x"], a8, torch.from_numpy(perm).cuda(), torch.from_numpy(offsets).cuda())
+    torch.cuda.synchronize()
+    err_a8 = row_rel_err(y8[torch.from_numpy(rows).cuda().long()].float().cpu().numpy(), ref)
+    assert err_two < err_a8
 
 
 @pytest.mark.parametrize("E,N,chunk", [(64, 200, 32), (16, 255, 64), (64, 40, 16)])
