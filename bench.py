@@ -48,13 +48,13 @@ TRAFFIC_SOURCES = {
     "tc": ('fine_grained_sparse_fp32_b200/csrc/ffn_tc.cu', 'fine_grained_sparse_fp32_b200/csrc/sm100.cuh', 'fine_grained_sparse_fp32_b200/csrc/common.cuh'),
 }
 TRAFFIC = {
-    "decode": ("swap", "e5fcef145ca727b3", (1195.6 + 1.7) * 1e6),
-    "fp8_decode": ("a8", "89ce473296cdec8b", (598.1 + 1.5) * 1e6),
-    "fp8a8_decode": ("a8", "89ce473296cdec8b", (598.0 + 1.3) * 1e6),
-    "fp8a8_prefill": ("a8", "89ce473296cdec8b", (1591.9 + 104.6) * 1e6),
-    "prefill": ("tc", "4949badb10327177", (2221.8 + 40.9 + 1190.8 + 237.7) * 1e6),       # up + down kernel
-    "fp8_prefill": ("tc", "4949badb10327177", (1041.9 + 6.9 + 619.7 + 93.6) * 1e6),      # up + down kernel
-    "skew": ("tc", "4949badb10327177", (4254.5 + 461.2 + 1467.7 + 2298.0) * 1e6),        # up + down kernel
+    "decode": ("swap", "b063b24c9ff6ee47", 1197.2e6),
+    "fp8_decode": ("a8", "0c50598cd420e05b", 599.4e6),
+    "fp8a8_decode": ("a8", "0c50598cd420e05b", 599.4e6),
+    "fp8a8_prefill": ("a8", "0c50598cd420e05b", 1700.3e6),
+    "prefill": ("tc", "696ba858c73ac825", 3686.2e6),   # up + down kernel
+    "fp8_prefill": ("tc", "696ba858c73ac825", 1761.0e6),   # up + down kernel
+    "skew": ("tc", "696ba858c73ac825", 8472.8e6),   # up + down kernel
 }
 
 
