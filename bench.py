@@ -49,9 +49,9 @@ TRAFFIC_SOURCES = {
 }
 TRAFFIC = {
     "decode": ("swap", "b063b24c9ff6ee47", 1197.2e6),
-    "fp8_decode": ("a8", "0c50598cd420e05b", 599.4e6),
-    "fp8a8_decode": ("a8", "0c50598cd420e05b", 599.4e6),
-    "fp8a8_prefill": ("a8", "0c50598cd420e05b", 1700.3e6),
+    "fp8_decode": ("a8", "61c3a944c54b8a34", 599.4e6),
+    "fp8a8_decode": ("a8", "61c3a944c54b8a34", 599.4e6),
+    "fp8a8_prefill": ("a8", "61c3a944c54b8a34", 1695.5e6),
     "prefill": ("tc", "696ba858c73ac825", 3686.2e6),   # up + down kernel
     "fp8_prefill": ("tc", "696ba858c73ac825", 1761.0e6),   # up + down kernel
     "skew": ("tc", "696ba858c73ac825", 8472.8e6),   # up + down kernel

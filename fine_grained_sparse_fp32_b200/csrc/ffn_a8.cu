@@ -520,8 +520,10 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
             if (up) {
                 // H = bf16(SiLU(gate) * up); each token's 128 features (this
                 // unit's rows, spread over the four lane quadrants) form one
-                // 1 x 128 group: scale = amax / 448, code = E4M3(h / scale),
-                // the quotient in FP32.
+                // 1 x 128 group: scale = amax / 448, code = E4M3(h * (1 / scale))
+                // with the reciprocal and the product in FP32 (within 2^-23 of
+                // h / scale, so at most one code step away from E4M3(h / scale)
+                // when that quotient lies next to a rounding boundary).
                 float hv[TPW];
 #pragma unroll
                 for (int n = 0; n < TPW; ++n) {
@@ -536,13 +538,10 @@ ffn_a8_kernel(const __grid_constant__ Maps maps, const Args a)
                                            fmaxf(__uint_as_float(T->amax[2][tok]), __uint_as_float(T->amax[3][tok])));
                     s_l = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
                 }
-                // two-term: h * (1 / s), whose last-bit difference from h / s
-                // the low code absorbs; FP8 activations: the exact quotient
-                const float r_l = kTwo ? __frcp_rn(s_l) : 1.f;
+                const float r_l = __frcp_rn(s_l);
 #pragma unroll
                 for (int n = 0; n < TPW; ++n) {
-                    const float y = kTwo ? hv[n] * __shfl_sync(0xffffffffu, r_l, n)
-                                         : __fdiv_rn(hv[n], __shfl_sync(0xffffffffu, s_l, n));
+                    const float y = hv[n] * __shfl_sync(0xffffffffu, r_l, n);
                     const uint8_t hc = e4m3_code(y);
                     T->codes[0][c0 + n][quad * 32 + lane] = hc;
                     if (kTwo) {       // lo = E4M3((y - hi) * 16)

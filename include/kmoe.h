@@ -74,8 +74,11 @@ typedef enum {
                                1 x 128). x (BF16) is quantised per row and 128 columns:
                                scale = amax / 448 in FP32 (1 for an all-zero group), code =
                                E4M3(x / scale) with the quotient in FP32, round to nearest
-                               even, saturated; H is rounded to BF16 and quantised the same
-                               way before the down projection. Each 128-column K block's
+                               even, saturated; H is rounded to BF16 and quantised with the
+                               same scale rule before the down projection, its codes taken
+                               from h * (1 / scale) in FP32 (at most one code step from
+                               E4M3(h / scale), where that quotient lies within 2^-23 of a
+                               rounding boundary). Each 128-column K block's
                                E4M3 x E4M3 partial sums (FP32) are scaled by both FP32
                                block scales and added in FP32. Routing sees x as given. */
 } kmoe_dtype;
