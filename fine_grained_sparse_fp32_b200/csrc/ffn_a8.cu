@@ -1,5 +1,6 @@
-// Grouped SwiGLU expert FFN with FP8 activations: E4M3 x E4M3 on the
-// tcgen05 tensor cores (kind::f8f6f4), weights as the M operand.
+// Grouped SwiGLU expert FFN on the FP8 tensor cores: E4M3 x E4M3 tcgen05
+// MMAs (kind::f8f6f4), weights as the M operand, for E4M3 weights with FP8
+// activations, or with BF16 activations held as two E4M3 terms (below).
 //
 // "Inside Kolibri 1" (flozi.net), section "The FP8 path is explicitly mixed
 // precision": the weights are E4M3 in 128 x 128 blocks with one FP32 scale

@@ -142,7 +142,7 @@ __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n
 
 // The block scales of one row block, s[0 .. nkb-1] (nkb <= 48), loaded by a
 // whole warp at once: lane l holds s[l] in lo and s[l + 32] in hi (0 past
-// the end). ref() is their maximum (the F16 path's normaliser).
+// the end).
 struct WarpScales {
     float lo, hi;
     __device__ __forceinline__ void load(const float *s, int nkb)
@@ -150,13 +150,6 @@ struct WarpScales {
         const int l = threadIdx.x & 31;
         lo = l < nkb ? s[l] : 0.f;
         hi = l + 32 < nkb ? s[l + 32] : 0.f;
-    }
-    __device__ __forceinline__ float ref() const
-    {
-        float m = fmaxf(lo, hi);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        return m;
     }
 };
 
