@@ -48,13 +48,13 @@ TRAFFIC_SOURCES = {
     "tc": ('fine_grained_sparse_fp32_b200/csrc/ffn_tc.cu', 'fine_grained_sparse_fp32_b200/csrc/sm100.cuh', 'fine_grained_sparse_fp32_b200/csrc/common.cuh'),
 }
 TRAFFIC = {
-    "decode": ("swap", "b063b24c9ff6ee47", 1197.2e6),
-    "fp8_decode": ("a8", "61c3a944c54b8a34", 599.4e6),
-    "fp8a8_decode": ("a8", "61c3a944c54b8a34", 599.4e6),
-    "fp8a8_prefill": ("a8", "61c3a944c54b8a34", 1695.5e6),
-    "prefill": ("tc", "696ba858c73ac825", 3686.2e6),   # up + down kernel
-    "fp8_prefill": ("tc", "696ba858c73ac825", 1761.0e6),   # up + down kernel
-    "skew": ("tc", "696ba858c73ac825", 8472.8e6),   # up + down kernel
+    "decode": ("swap", "b6401135bdb7745e", 1197.4e6),
+    "fp8_decode": ("a8", "1dd307aeb0673877", 599.3e6),
+    "fp8a8_decode": ("a8", "1dd307aeb0673877", 599.2e6),
+    "fp8a8_prefill": ("a8", "1dd307aeb0673877", 1699.2e6),
+    "prefill": ("tc", "696ba858c73ac825", 3689.9e6),   # up + down kernel
+    "fp8_prefill": ("tc", "696ba858c73ac825", 1756.0e6),   # up + down kernel
+    "skew": ("tc", "696ba858c73ac825", 8471.2e6),   # up + down kernel
 }
 
 
