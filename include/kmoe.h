@@ -18,7 +18,9 @@
  * Conventions shared by every entry point:
  *   - Pointers marked "device" point to GPU global memory owned by the
  *     caller; the library never allocates or frees device memory and keeps
- *     no state between calls other than a per-thread error message.
+ *     no state between calls other than a per-thread error message and
+ *     give-up limit (moe_set_wait_limit); moe_permute_noalloc works in the
+ *     library's own static device array (see there).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is
  *     enqueued asynchronously; no entry point synchronises the device.
  *   - Matrices are dense row-major. Every device pointer must be 16-byte
